@@ -1,0 +1,526 @@
+/*
+ * nvfp4_oracle.c -- plain, slow CPU oracle for the NVFP4 quantizer, the MXFP8
+ * requantizer and the block-scaled GEMM.
+ *
+ * TEST INFRASTRUCTURE ONLY.  Only the test suite, the smoke check and the
+ * benchmark's CPU-baseline leg may load this library.  It shares no code,
+ * header, table or constant generator with the CUDA library: every value here
+ * is derived from the format definitions below, step by step.
+ *
+ * Sources (cited as "page, section"):
+ *   [asector] "Nvidia dobivaetsya uspekha s 4-bitnym formatom NVFP4"
+ *             (asector.ru), sections "NVFP4 and Blackwell" and
+ *             "Experiments and comparison with FP8".
+ *   [iitak]   "Thinking Machines uskorila obuchenie Inkling 2 Small
+ *             4-bitnymi chislami" (iitak.ru), sections "Details",
+ *             "How it works" and "But".
+ *   [hightech] "Novyi 4-bitnyi metod obucheniya BYaM ne ustupaet 8-bitnomu"
+ *             (hightech.plus, 2025-10-30).
+ *   Philox4x32-10: J. K. Salmon, M. A. Moraes, R. O. Dror, D. E. Shaw,
+ *             "Parallel random numbers: as easy as 1, 2, 3", SC'11.
+ *   MXFP8 scale rule: OCP Microscaling Formats (MX) v1.0 specification.
+ *
+ * Arithmetic: decisions that pick a code (block scale, element scaling) are
+ * taken in IEEE binary32, in the stated order, because the quantised code is
+ * an integer decided by floating point and both sides must decide it in the
+ * same precision.  Everything else (decode, nearest-code search, stochastic
+ * rounding fractions, dequantisation, GEMM) is done in binary64, where every
+ * intermediate is exact.  Build with -ffp-contract=off and without fast-math.
+ *
+ * Parity pins: the E2M1 table, RNE ties, the worked block-scale example, the
+ * stochastic-rounding example, 2D transpose invariance, the Hadamard closed
+ * form, Philox known-answer vectors and brute-force nearest search are pinned
+ * by the CPU tests.  "parity unpinned": the global-scale constant 2688 = 6*448,
+ * the Philox-to-element mapping, the Hadamard sign draw, the MXFP8 floor rule
+ * and the signed-zero convention are readings this build fixes; the pages do
+ * not determine them.
+ */
+#include <math.h>
+#include <stdint.h>
+#include <stdlib.h>
+#include <string.h>
+
+#define ORC_OK 0
+#define ORC_EINVAL 1
+
+/* ------------------------------------------------------------------------ */
+/* Philox4x32-10, written from the SC'11 definition: two 32x32->64 products  */
+/* per round, Weyl key schedule, ten rounds.                                 */
+/* ------------------------------------------------------------------------ */
+void orc_philox4x32_10(const uint32_t ctr[4], const uint32_t key[2], uint32_t out[4])
+{
+    uint32_t x0 = ctr[0], x1 = ctr[1], x2 = ctr[2], x3 = ctr[3];
+    uint32_t k0 = key[0], k1 = key[1];
+    for (int round = 0; round < 10; ++round) {
+        if (round > 0) {
+            k0 += 0x9E3779B9u; /* golden ratio */
+            k1 += 0xBB67AE85u; /* sqrt(3) - 1  */
+        }
+        uint64_t p0 = (uint64_t)0xD2511F53u * (uint64_t)x0;
+        uint64_t p1 = (uint64_t)0xCD9E8D57u * (uint64_t)x2;
+        uint32_t hi0 = (uint32_t)(p0 >> 32), lo0 = (uint32_t)p0;
+        uint32_t hi1 = (uint32_t)(p1 >> 32), lo1 = (uint32_t)p1;
+        uint32_t n0 = hi1 ^ x1 ^ k0;
+        uint32_t n1 = lo1;
+        uint32_t n2 = hi0 ^ x3 ^ k1;
+        uint32_t n3 = lo0;
+        x0 = n0; x1 = n1; x2 = n2; x3 = n3;
+    }
+    out[0] = x0; out[1] = x1; out[2] = x2; out[3] = x3;
+}
+
+/* Random 16-bit draw for element `idx` (position in the output's own
+ * row-major order) of Philox stream `stream`.  Counter = (idx/8 low, idx/8
+ * high, stream, offset), key = (seed low, seed high).  Element idx takes the
+ * (idx mod 2) half of word (idx mod 8)/2.  Streams: 0 NVFP4 rowwise, 1 NVFP4
+ * columnwise, 2 MXFP8, 3 Hadamard signs.  This mapping is the build's own
+ * reading: the pages name stochastic rounding but no generator. */
+uint16_t orc_sr_bits(uint64_t seed, uint32_t offset, uint32_t stream, uint64_t idx)
+{
+    uint64_t j = idx >> 3;
+    uint32_t ctr[4] = {(uint32_t)j, (uint32_t)(j >> 32), stream, offset};
+    uint32_t key[2] = {(uint32_t)seed, (uint32_t)(seed >> 32)};
+    uint32_t w[4];
+    orc_philox4x32_10(ctr, key, w);
+    uint32_t word = w[(idx & 7) >> 1];
+    return (uint16_t)((idx & 1) ? (word >> 16) : (word & 0xFFFFu));
+}
+
+/* ------------------------------------------------------------------------ */
+/* bf16 input                                                                */
+/* ------------------------------------------------------------------------ */
+static float bf16_to_float(uint16_t b)
+{
+    uint32_t u = (uint32_t)b << 16;
+    float f;
+    memcpy(&f, &u, 4);
+    return f;
+}
+
+/* ------------------------------------------------------------------------ */
+/* E2M1 element format [asector, "NVFP4 and Blackwell"]: 1 sign bit, 2      */
+/* exponent bits (bias 1), 1 mantissa bit; exponent 0 is subnormal.          */
+/* [iitak, "Details"]: 16 values from -6 to 6, e.g. 0.5, 1.5, 3, 4, not 5.   */
+/* ------------------------------------------------------------------------ */
+double orc_e2m1_decode(uint8_t code)
+{
+    int s = (code >> 3) & 1, e = (code >> 1) & 3, m = code & 1;
+    double mag = (e == 0) ? 0.5 * m : ldexp(1.0 + 0.5 * m, e - 1);
+    return s ? -mag : mag;
+}
+
+static double e2m1_mag(int m) { return orc_e2m1_decode((uint8_t)m); }
+
+/* Round-to-nearest-even onto the E2M1 grid with saturation at 6
+ * [asector, "NVFP4 and Blackwell": RNE is one of the tensor cores' modes].
+ * Plain nearest search over the eight magnitudes; a tie goes to the code whose
+ * mantissa bit is 0.  The sign bit is copied from y, also when the result is
+ * zero (reading: the pages say nothing about signed zero). */
+uint8_t orc_e2m1_rne(float y)
+{
+    double a = fabs((double)y);
+    if (a > 6.0) a = 6.0; /* saturate first: far-away distances lose precision */
+    int best = 0;
+    double bestd = INFINITY;
+    for (int m = 0; m < 8; ++m) {
+        double d = fabs(a - e2m1_mag(m));
+        if (d < bestd || (d == bestd && (m & 1) == 0)) {
+            best = m;
+            bestd = d;
+        }
+    }
+    return (uint8_t)((signbit(y) ? 8 : 0) | best);
+}
+
+/* Unbiased stochastic rounding onto the E2M1 grid [iitak, "How it works":
+ * 2.25 goes to 2 in three cases of four and to 3 in one].  For lo <= |y| < hi
+ * (adjacent grid magnitudes) the fraction f = (|y| - lo)/(hi - lo) is exact in
+ * binary64; t = floor(f * 2^16); the value rounds up iff u < t, so
+ * P(up) = t / 2^16.  |y| >= 6 saturates to 6. */
+uint8_t orc_e2m1_sr(float y, uint16_t u)
+{
+    uint8_t sign = signbit(y) ? 8 : 0;
+    double a = fabs((double)y);
+    if (a >= 6.0) return (uint8_t)(sign | 7);
+    int m = 0;
+    while (m < 7 && e2m1_mag(m + 1) <= a) ++m;
+    double lo = e2m1_mag(m), hi = e2m1_mag(m + 1);
+    double f = (a - lo) / (hi - lo);
+    uint32_t t = (uint32_t)floor(f * 65536.0);
+    int up = (uint32_t)u < t;
+    return (uint8_t)(sign | (m + up));
+}
+
+/* ------------------------------------------------------------------------ */
+/* E4M3 (FP8): 1 sign, 4 exponent bits (bias 7), 3 mantissa bits, exponent 0 */
+/* subnormal, no infinities, S.1111.111 is NaN; largest finite 448.  Used    */
+/* for the NVFP4 block scale (the build's choice: the pages' multiplier 9    */
+/* [iitak, "Details"] is not a power of two, so an E8M0 scale cannot hold    */
+/* it) and for MXFP8 elements.                                               */
+/* ------------------------------------------------------------------------ */
+double orc_e4m3_decode(uint8_t b)
+{
+    int s = (b >> 7) & 1, e = (b >> 3) & 15, m = b & 7;
+    if (e == 15 && m == 7) return NAN;
+    double mag = (e == 0) ? ldexp((double)m, -9) : ldexp(1.0 + m / 8.0, e - 7);
+    return s ? -mag : mag;
+}
+
+/* Round-to-nearest-even onto the finite E4M3 values, saturating (satfinite):
+ * magnitudes above 448 become 448, then a nearest search over all 127 finite
+ * magnitudes, ties to the code with an even mantissa (code bit 0 clear). */
+uint8_t orc_e4m3_rne_sat(double y)
+{
+    double a = fabs(y);
+    if (a > 448.0) a = 448.0; /* satfinite, explicit for very large inputs */
+    int best = 0;
+    double bestd = INFINITY;
+    for (int c = 0; c < 0x7F; ++c) {
+        double d = fabs(a - orc_e4m3_decode((uint8_t)c));
+        if (d < bestd || (d == bestd && (c & 1) == 0)) {
+            best = c;
+            bestd = d;
+        }
+    }
+    return (uint8_t)((signbit(y) ? 0x80 : 0) | best);
+}
+
+/* Stochastic rounding onto the E4M3 grid (optional MXFP8 mode), the same rule
+ * as orc_e2m1_sr on the E4M3 magnitudes; saturates at 448. */
+uint8_t orc_e4m3_sr_sat(double y, uint16_t u)
+{
+    uint8_t sign = signbit(y) ? 0x80 : 0;
+    double a = fabs(y);
+    if (a >= 448.0) return (uint8_t)(sign | 0x7E);
+    int c = 0;
+    while (c < 0x7E && orc_e4m3_decode((uint8_t)(c + 1)) <= a) ++c;
+    double lo = orc_e4m3_decode((uint8_t)c), hi = orc_e4m3_decode((uint8_t)(c + 1));
+    double f = (a - lo) / (hi - lo);
+    uint32_t t = (uint32_t)floor(f * 65536.0);
+    int up = (uint32_t)u < t;
+    return (uint8_t)(sign | (c + up));
+}
+
+/* ------------------------------------------------------------------------ */
+/* Random Hadamard transform [asector, "Experiments and comparison with     */
+/* FP8": random Hadamard transforms handle outlier gradients].  Size 16,     */
+/* v <- (1/4) H16 D v with H16 the Sylvester Hadamard matrix and D a random  */
+/* sign diagonal.                                                            */
+/* ------------------------------------------------------------------------ */
+
+/* Sign i (0..15) is -1 iff bit i of word 0 of Philox(counter (0,0,3,0),
+ * key = seed).  It depends on the seed only, so two tensors quantised with
+ * one seed share the transform and it cancels in the product. */
+void orc_rht_signs(uint64_t seed, float signs[16])
+{
+    uint32_t ctr[4] = {0, 0, 3, 0};
+    uint32_t key[2] = {(uint32_t)seed, (uint32_t)(seed >> 32)};
+    uint32_t w[4];
+    orc_philox4x32_10(ctr, key, w);
+    for (int i = 0; i < 16; ++i) signs[i] = ((w[0] >> i) & 1) ? -1.0f : 1.0f;
+}
+
+/* The transform in binary32 with a fixed order: sign flip (exact), then the
+ * butterfly stages h = 1, 2, 4, 8, each pair (i, i+h) with (i & h) == 0
+ * becoming (w_i + w_{i+h}, w_i - w_{i+h}) rounded to binary32, then the exact
+ * factor 1/4.  The unnormalised stages realise H16 (H16 H16^T = 16 I). */
+void orc_rht16(const float signs[16], const float in[16], float out[16])
+{
+    float w[16];
+    for (int i = 0; i < 16; ++i) w[i] = in[i] * signs[i];
+    for (int h = 1; h < 16; h <<= 1) {
+        for (int i = 0; i < 16; ++i) {
+            if (i & h) continue;
+            float a = w[i], b = w[i + h];
+            w[i] = a + b;
+            w[i + h] = a - b;
+        }
+    }
+    for (int i = 0; i < 16; ++i) out[i] = w[i] * 0.25f;
+}
+
+/* ------------------------------------------------------------------------ */
+/* Global (per-tensor) scale [asector, "NVFP4 and Blackwell": one local     */
+/* scale per 16-element block and one global scale per tensor].  Reading:    */
+/* the global encode scale maps the tensor amax onto 6 * 448 = 2688, the top */
+/* of E2M1 times the top of E4M3; S = 2688/amax and g = amax/2688, each one  */
+/* binary32 division.  amax = 0 gives S = g = 1.  S is capped at 2^118 (and  */
+/* g is then 2^-118) so that S divided by the smallest E4M3 scale stays      */
+/* finite for absurdly small tensors.                                        */
+/* ------------------------------------------------------------------------ */
+void orc_global_scale(float amax, float* S, float* g)
+{
+    const float cap = 0x1p118f;
+    if (amax == 0.0f) {
+        *S = 1.0f;
+        *g = 1.0f;
+        return;
+    }
+    float s = 2688.0f / amax;
+    if (!(s <= cap)) {
+        *S = cap;
+        *g = 0x1p-118f;
+        return;
+    }
+    *S = s;
+    *g = amax / 2688.0f;
+}
+
+/* ------------------------------------------------------------------------ */
+/* NVFP4 quantisation of one binary32 matrix v [n_rows, n_cols] along its    */
+/* rows (16-element blocks along n_cols).  The columnwise output is this     */
+/* same procedure applied to the transpose.                                  */
+/* ------------------------------------------------------------------------ */
+typedef struct {
+    int rounding;    /* 0 round-to-nearest-even, 1 stochastic */
+    int scaling;     /* 0 1D 16-element blocks, 1 2D 16x16 tiles */
+    int rht;         /* columnwise only: apply the 16-point RHT first */
+    uint64_t seed;
+    uint32_t offset;
+    int has_amax;    /* 1: use amax_row / amax_col instead of computing */
+    float amax_row, amax_col;
+} orc_qparams;
+
+static void quantize_matrix(const float* v, int64_t n_rows, int64_t n_cols, float amax,
+                            const orc_qparams* p, uint32_t stream, uint8_t* q,
+                            uint8_t* sf, float* g_out)
+{
+    float S, g;
+    orc_global_scale(amax, &S, &g);
+    *g_out = g;
+    int64_t nb = n_cols / 16;
+    for (int64_t r = 0; r < n_rows; ++r) {
+        for (int64_t b = 0; b < nb; ++b) {
+            /* block amax: 16 values (1D) or the whole 16x16 tile (2D) */
+            float amax_b = 0.0f;
+            int64_t r0 = p->scaling ? (r / 16) * 16 : r;
+            int64_t r1 = p->scaling ? r0 + 16 : r + 1;
+            for (int64_t rr = r0; rr < r1; ++rr)
+                for (int64_t c = b * 16; c < b * 16 + 16; ++c) {
+                    float a = fabsf(v[rr * n_cols + c]);
+                    if (a > amax_b) amax_b = a;
+                }
+            /* block scale [iitak, "Details": block max 54 -> 6 with multiplier
+             * 9]: s = (amax_b / 6) * S in binary32, rounded to E4M3 (RNE,
+             * satfinite; the rounding mode is the build's reading). */
+            float s = (amax_b / 6.0f) * S;
+            uint8_t sbyte = orc_e4m3_rne_sat((double)s);
+            float d = (float)orc_e4m3_decode(sbyte);
+            sf[r * nb + b] = sbyte;
+            float rs = (d != 0.0f) ? S / d : 0.0f;
+            for (int64_t c = b * 16; c < b * 16 + 16; ++c) {
+                float x = v[r * n_cols + c];
+                uint8_t code;
+                if (d == 0.0f) {
+                    code = signbit(x) ? 8 : 0;
+                } else {
+                    float y = x * rs;
+                    if (p->rounding == 0)
+                        code = orc_e2m1_rne(y);
+                    else
+                        code = orc_e2m1_sr(y, orc_sr_bits(p->seed, p->offset, stream,
+                                                          (uint64_t)(r * n_cols + c)));
+                }
+                /* pack: even element in the low nibble */
+                int64_t byte = (r * n_cols + c) / 2;
+                if ((c & 1) == 0)
+                    q[byte] = code;
+                else
+                    q[byte] = (uint8_t)(q[byte] | (code << 4));
+            }
+        }
+    }
+}
+
+/* x: bf16 [rows, ld] row-major.  direction 0 = rowwise (codes [rows, cols/2],
+ * scales [rows, cols/16], stream 0); 1 = columnwise = the rowwise procedure
+ * on x^T (codes [cols, rows/2], scales [cols, rows/16], stream 1), with the
+ * RHT applied to each 16-vector along rows first when p->rht is set.
+ * In 2D mode each 16x16 tile's scale byte is stored in every row's entry of
+ * that tile, so the scale tensors keep the 1D shapes. */
+int orc_nvfp4_quantize(const uint16_t* x, int64_t rows, int64_t cols, int64_t ld,
+                       int direction, const orc_qparams* p, uint8_t* q, uint8_t* sf,
+                       float* g)
+{
+    if (rows <= 0 || cols <= 0 || rows % 16 || cols % 16 || ld < cols) return ORC_EINVAL;
+    int64_t nr = direction ? cols : rows, nc = direction ? rows : cols;
+    float* v = (float*)malloc(sizeof(float) * (size_t)(nr * nc));
+    if (!v) return ORC_EINVAL;
+    for (int64_t r = 0; r < rows; ++r)
+        for (int64_t c = 0; c < cols; ++c) {
+            float xv = bf16_to_float(x[r * ld + c]);
+            if (direction)
+                v[c * rows + r] = xv;
+            else
+                v[r * cols + c] = xv;
+        }
+    if (direction && p->rht) {
+        float signs[16], in[16], out[16];
+        orc_rht_signs(p->seed, signs);
+        for (int64_t r = 0; r < nr; ++r)
+            for (int64_t b = 0; b < nc; b += 16) {
+                for (int i = 0; i < 16; ++i) in[i] = v[r * nc + b + i];
+                orc_rht16(signs, in, out);
+                for (int i = 0; i < 16; ++i) v[r * nc + b + i] = out[i];
+            }
+    }
+    float amax = 0.0f;
+    if (p->has_amax) {
+        amax = direction ? p->amax_col : p->amax_row;
+    } else {
+        for (int64_t i = 0; i < nr * nc; ++i) {
+            float a = fabsf(v[i]);
+            if (a > amax) amax = a;
+        }
+    }
+    quantize_matrix(v, nr, nc, amax, p, direction ? 1u : 0u, q, sf, g);
+    free(v);
+    return ORC_OK;
+}
+
+/* ------------------------------------------------------------------------ */
+/* MXFP8 [iitak, "How it works": the backward pass runs in MXFP8; "But":    */
+/* expert outputs travel at 8.25 bits per number = 8-bit elements plus one   */
+/* 8-bit scale per 32].  Scale rule from the OCP MX v1.0 specification:      */
+/* e = floor(log2(amax_32)) - 8 (8 = largest E4M3 exponent), clamped to      */
+/* [-127, 127], stored as the E8M0 byte e + 127; amax 0 gives e = -127.      */
+/* Elements are E4M3(x * 2^-e), RNE satfinite or stochastic (stream 2).      */
+/* direction 0: blocks along cols, codes [rows, cols], scales [rows, cols/32];*/
+/* direction 1: on x^T, codes [cols, rows], scales [cols, rows/32].          */
+/* ------------------------------------------------------------------------ */
+int orc_mxfp8_quantize(const uint16_t* x, int64_t rows, int64_t cols, int64_t ld,
+                       int direction, int rounding, uint64_t seed, uint32_t offset,
+                       uint8_t* q, uint8_t* e8)
+{
+    int64_t nr = direction ? cols : rows, nc = direction ? rows : cols;
+    if (rows <= 0 || cols <= 0 || nc % 32 || ld < cols) return ORC_EINVAL;
+    for (int64_t r = 0; r < nr; ++r) {
+        for (int64_t b = 0; b < nc / 32; ++b) {
+            double vals[32];
+            double amax = 0.0;
+            for (int i = 0; i < 32; ++i) {
+                int64_t c = b * 32 + i;
+                uint16_t raw = direction ? x[c * ld + r] : x[r * ld + c];
+                vals[i] = (double)bf16_to_float(raw);
+                if (fabs(vals[i]) > amax) amax = fabs(vals[i]);
+            }
+            int e;
+            if (amax == 0.0) {
+                e = -127;
+            } else {
+                int k;
+                frexp(amax, &k); /* amax = m 2^k, m in [0.5, 1): floor(log2) = k-1 */
+                e = (k - 1) - 8;
+                if (e < -127) e = -127;
+                if (e > 127) e = 127;
+            }
+            e8[r * (nc / 32) + b] = (uint8_t)(e + 127);
+            for (int i = 0; i < 32; ++i) {
+                double y = ldexp(vals[i], -e);
+                int64_t idx = r * nc + b * 32 + i;
+                q[idx] = rounding ? orc_e4m3_sr_sat(y, orc_sr_bits(seed, offset, 2, (uint64_t)idx))
+                                  : orc_e4m3_rne_sat(y);
+            }
+        }
+    }
+    return ORC_OK;
+}
+
+/* ------------------------------------------------------------------------ */
+/* Dequantisation: x_hat = e2m1(code) * d * g.  The binary64 form is exact;  */
+/* the binary32 form rounds once (code * d is exact in binary32).            */
+/* ------------------------------------------------------------------------ */
+void orc_nvfp4_dequant_f64(const uint8_t* q, const uint8_t* sf, float g, int64_t rows,
+                           int64_t cols, double* out)
+{
+    for (int64_t r = 0; r < rows; ++r)
+        for (int64_t c = 0; c < cols; ++c) {
+            uint8_t byte = q[(r * cols + c) / 2];
+            uint8_t code = (c & 1) ? (byte >> 4) : (byte & 15);
+            double d = orc_e4m3_decode(sf[r * (cols / 16) + c / 16]);
+            out[r * cols + c] = orc_e2m1_decode(code) * d * (double)g;
+        }
+}
+
+void orc_nvfp4_dequant_f32(const uint8_t* q, const uint8_t* sf, float g, int64_t rows,
+                           int64_t cols, float* out)
+{
+    for (int64_t r = 0; r < rows; ++r)
+        for (int64_t c = 0; c < cols; ++c) {
+            uint8_t byte = q[(r * cols + c) / 2];
+            uint8_t code = (c & 1) ? (byte >> 4) : (byte & 15);
+            float d = (float)orc_e4m3_decode(sf[r * (cols / 16) + c / 16]);
+            float cd = (float)orc_e2m1_decode(code) * d;
+            out[r * cols + c] = cd * g;
+        }
+}
+
+/* ------------------------------------------------------------------------ */
+/* Block-scaled GEMM reference [asector, "NVFP4 and Blackwell": the tensor  */
+/* cores compute with scaling and high-precision accumulation]:              */
+/*   D[i][j] = sum_k a_hat[i][k] * b_hat[j][k]  (binary64),                  */
+/* A [M, K] and B [N, K] both K-contiguous NVFP4 (codes + row-major 1D       */
+/* scales).  Also returns the tolerance basis sum_k |a_hat| |b_hat|.  Only   */
+/* the rows listed in `rows_sel` (n_sel of them) are computed; out is        */
+/* [n_sel, N].                                                               */
+/* ------------------------------------------------------------------------ */
+int orc_nvfp4_gemm_rows(const uint8_t* qa, const uint8_t* sfa, float ga, const uint8_t* qb,
+                        const uint8_t* sfb, float gb, int64_t M, int64_t N, int64_t K,
+                        const int64_t* rows_sel, int64_t n_sel, double* out, double* absout)
+{
+    if (K % 16) return ORC_EINVAL;
+    double* a = (double*)malloc(sizeof(double) * (size_t)K);
+    double* bt = (double*)malloc(sizeof(double) * (size_t)(N * K));
+    if (!a || !bt) {
+        free(a);
+        free(bt);
+        return ORC_EINVAL;
+    }
+    orc_nvfp4_dequant_f64(qb, sfb, gb, N, K, bt);
+    for (int64_t s = 0; s < n_sel; ++s) {
+        int64_t i = rows_sel[s];
+        if (i < 0 || i >= M) {
+            free(a);
+            free(bt);
+            return ORC_EINVAL;
+        }
+        orc_nvfp4_dequant_f64(qa + i * (K / 2), sfa + i * (K / 16), ga, 1, K, a);
+        for (int64_t j = 0; j < N; ++j) {
+            double acc = 0.0, aacc = 0.0;
+            for (int64_t k = 0; k < K; ++k) {
+                double pr = a[k] * bt[j * K + k];
+                acc += pr;
+                aacc += fabs(pr);
+            }
+            out[s * N + j] = acc;
+            absout[s * N + j] = aacc;
+        }
+    }
+    free(a);
+    free(bt);
+    return ORC_OK;
+}
+
+/* Grouped (MoE) form: rows [off[e], off[e+1]) of A multiply expert e's B
+ * (B stacked [G, N, K], per-expert gb[e]).  rows_sel lists global A rows. */
+int orc_nvfp4_grouped_gemm_rows(int G, const int64_t* off, const uint8_t* qa,
+                                const uint8_t* sfa, float ga, const uint8_t* qb,
+                                const uint8_t* sfb, const float* gb, int64_t N, int64_t K,
+                                const int64_t* rows_sel, int64_t n_sel, double* out,
+                                double* absout)
+{
+    for (int64_t s = 0; s < n_sel; ++s) {
+        int64_t i = rows_sel[s];
+        int e = -1;
+        for (int t = 0; t < G; ++t)
+            if (off[t] <= i && i < off[t + 1]) e = t;
+        if (e < 0) return ORC_EINVAL;
+        int64_t one = 0;
+        int rc = orc_nvfp4_gemm_rows(qa + i * (K / 2), sfa + i * (K / 16), ga,
+                                     qb + (int64_t)e * N * (K / 2),
+                                     sfb + (int64_t)e * N * (K / 16), gb[e], 1, N, K, &one, 1,
+                                     out + s * N, absout + s * N);
+        if (rc) return rc;
+    }
+    return ORC_OK;
+}
