@@ -1,0 +1,231 @@
+/*
+ * nvfp4.h -- C ABI of the B200 (sm_100a) NVFP4 quantizer and block-scaled GEMM.
+ *
+ * Format, as the pages state it:
+ *  - Elements are E2M1 (1 sign, 2 exponent, 1 mantissa bit), 16 values in
+ *    [-6, 6] (asector.ru, "Nvidia dobivaetsya uspekha s 4-bitnym formatom
+ *    NVFP4", section "NVFP4 and Blackwell"; iitak.ru, "Thinking Machines
+ *    uskorila obuchenie Inkling 2 Small 4-bitnymi chislami", section "Details").
+ *  - Two-level scaling: one local scale per 16-element block and one global
+ *    scale per tensor (asector, "NVFP4 and Blackwell").  The block scale is an
+ *    E4M3 byte (this library's choice: the worked multiplier 9 of iitak,
+ *    "Details", is not a power of two); the global scale is FP32.
+ *  - Optional 16x16 2D block scales for weights, invariant under transpose,
+ *    and a random Hadamard transform for outlier gradients (asector,
+ *    "Experiments and comparison with FP8"; iitak, "How it works").
+ *  - Round-to-nearest-even or unbiased stochastic rounding (asector, "NVFP4
+ *    and Blackwell"; iitak, "How it works": 2.25 -> 2 w.p. 3/4, 3 w.p. 1/4).
+ *  - MXFP8 requantisation for backward operands: E4M3 elements with one E8M0
+ *    scale per 32 (iitak, "How it works" and "But": 8.25 bits per number).
+ *
+ * Conventions shared by every call:
+ *  - Every tensor pointer is a DEVICE pointer owned by the caller.  The
+ *    library allocates no device memory; scratch comes from a caller-provided
+ *    workspace whose size the *_workspace_size helpers return.
+ *  - `stream` is a cudaStream_t passed as void* (NULL = legacy default
+ *    stream).  Calls only enqueue work and return; they never synchronise.
+ *  - The returned status reports argument and launch errors.  Errors the
+ *    device detects (a bounded wait that ran out, a gather index out of range)
+ *    are written to a status word in the workspace, which every call that is
+ *    given a workspace clears first; nvfp4_workspace_status() synchronises the
+ *    stream and returns the word of the last call that used that workspace.
+ *  - Matrices are row-major.  "Rowwise" quantisation blocks 16 consecutive
+ *    elements along a row; "columnwise" quantises the transpose, so its codes
+ *    are [cols, rows/2] and its 16-blocks run down a column of the input.
+ *  - Codes: two E2M1 nibbles per byte, the even element in the low nibble.
+ *  - Inputs must be finite; non-finite input gives unspecified codes.
+ */
+#ifndef NVFP4_H
+#define NVFP4_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    NVFP4_OK = 0,
+    NVFP4_ERR_INVALID_ARG = 1, /* null pointer, bad enum, inconsistent flags     */
+    NVFP4_ERR_SHAPE = 2,       /* size not a multiple of the block or tile       */
+    NVFP4_ERR_ALIGN = 3,       /* pointer or leading dimension not 16-byte aligned */
+    NVFP4_ERR_UNSUPPORTED = 4, /* no sm_100 device, or an unsupported combination */
+    NVFP4_ERR_CUDA = 5,        /* a CUDA runtime call failed                     */
+    NVFP4_ERR_TIMEOUT = 6,     /* device side: a bounded wait ran out            */
+    NVFP4_ERR_WORKSPACE = 7,   /* workspace missing or too small                 */
+    NVFP4_ERR_INDEX = 8        /* device side: a gather index was out of range   */
+} nvfp4_status;
+
+enum { NVFP4_RNE = 0, NVFP4_SR = 1 };                 /* rounding          */
+enum { NVFP4_1D16 = 0, NVFP4_2D16x16 = 1 };           /* block scaling     */
+enum { NVFP4_ROWWISE = 1, NVFP4_COLWISE = 2 };        /* output bitmask    */
+enum { NVFP4_SF_ROWMAJOR = 0, NVFP4_SF_MMA = 1 };     /* scale-byte layout */
+enum { NVFP4_OUT_F32 = 0, NVFP4_OUT_BF16 = 1 };       /* GEMM / dequant output */
+
+/*
+ * Scale-byte layouts.
+ *  NVFP4_SF_ROWMAJOR: scale of 16-block b of row r at sf[r * (K/16) + b],
+ *    where K is the length of the quantised rows (cols rowwise, rows
+ *    columnwise).  In 2D mode the byte of each 16x16 tile is stored in all 16
+ *    rows' entries, so the shapes stay those of 1D.
+ *  NVFP4_SF_MMA: the tiled layout the tensor cores read.  Rows are grouped in
+ *    blocks of 128 and 16-blocks in groups of 4 (64 elements); each group is a
+ *    512-byte atom, atoms ordered with the K group fastest:
+ *      offset = ((r/128) * (K/64) + b/4) * 512 + (r%32)*16 + ((r%128)/32)*4 + b%4.
+ *    Buffers must hold ceil(rows/128)*128 rows (bytes = nvfp4_sf_mma_bytes);
+ *    bytes of padding rows are not written.  K must be a multiple of 64.
+ *  With group_offsets (MoE layout), each group e's rows start a fresh
+ *    128-row block: row r of group e uses padded row
+ *    r - off[e] + sum_{e'<e} ceil((off[e'+1]-off[e'])/128)*128.
+ */
+
+/* Stochastic rounding draws 16 random bits per element from Philox4x32-10
+ * (Salmon et al., SC'11), key = seed, counter = (idx/8 low word, idx/8 high
+ * word, stream, offset), element idx taking 16-bit half (idx%2) of word
+ * (idx%8)/2.  idx is the element's position in the OUTPUT's row-major order;
+ * stream 0 = NVFP4 rowwise, 1 = NVFP4 columnwise, 2 = MXFP8.  The Hadamard
+ * signs are bits 0..15 of word 0 of Philox(counter (0,0,3,0), key = seed):
+ * they depend on the seed only, so two tensors quantised with one seed share
+ * the transform and it cancels in their product. */
+typedef struct {
+    int rounding;          /* NVFP4_RNE | NVFP4_SR (NVFP4 codes, both directions) */
+    int scaling;           /* NVFP4_1D16 | NVFP4_2D16x16                        */
+    int outputs;           /* NVFP4_ROWWISE | NVFP4_COLWISE bitmask (may be 0)  */
+    int rht_colwise;       /* 1: 16-point random Hadamard on columnwise vectors  */
+    int sf_layout;         /* NVFP4_SF_ROWMAJOR | NVFP4_SF_MMA                   */
+    uint64_t seed;         /* Philox key                                         */
+    uint32_t offset;       /* Philox counter word 3: selects a sub-stream        */
+    const float* amax_in;  /* optional device [2] = {amax rowwise, amax columnwise
+                              (after the Hadamard when rht_colwise)}; NULL = compute */
+    /* Gather (MoE): output row i reads input row row_index[i]; the input has
+     * src_rows rows.  NULL = identity (src_rows ignored). */
+    const int32_t* row_index;
+    int64_t src_rows;
+    /* MoE scale layout: device offsets [num_groups+1] of output rows; only with
+     * NVFP4_SF_MMA and the rowwise output.  NULL = dense. */
+    const int32_t* group_offsets;
+    int num_groups;
+    /* Optional MXFP8 copy produced in the same pass (E4M3 codes [rows, cols] /
+     * [cols, rows] with E8M0 scales per 32 along the block axis, row-major). */
+    int mx_outputs;        /* NVFP4_ROWWISE | NVFP4_COLWISE bitmask, 0 = none    */
+    int mx_rounding;       /* NVFP4_RNE | NVFP4_SR (stream 2)                    */
+    uint8_t* mx_q_row;
+    uint8_t* mx_sf_row;
+    uint8_t* mx_q_col;
+    uint8_t* mx_sf_col;
+} nvfp4_quant_params;
+
+/* Bytes of scale storage in NVFP4_SF_MMA layout for a [rows, k] operand. */
+size_t nvfp4_sf_mma_bytes(int64_t rows, int64_t k);
+
+/* Bytes of scale storage in NVFP4_SF_MMA layout for the grouped (MoE) layout:
+ * sum over groups of ceil(rows_e/128)*128 rows; bounded by
+ * (total_rows + 128*num_groups) rows, which this returns. */
+size_t nvfp4_sf_mma_grouped_bytes(int64_t total_rows, int num_groups, int64_t k);
+
+/* Workspace bytes nvfp4_quantize needs (global amax and the status word). */
+size_t nvfp4_quantize_workspace_size(int64_t rows, int64_t cols, const nvfp4_quant_params* p);
+
+/*
+ * nvfp4_quantize -- NVFP4 quantisation of a bf16 matrix x [rows, ld] (row-major,
+ * cols <= ld), rowwise and/or columnwise in one pass over the data, plus an
+ * optional MXFP8 copy.
+ *
+ * Steps (asector "NVFP4 and Blackwell" / "Experiments and comparison with
+ * FP8"; iitak "Details" / "How it works"):
+ *   amax (per direction; over the transformed values when rht_colwise),
+ *   S = 2688/amax and g = amax/2688 (FP32 divisions; amax 0 -> 1, 1; S capped
+ *   at 2^118 with g = 2^-118), block amax over 16 (1D) or 16x16 (2D),
+ *   scale byte = E4M3_RNE_satfinite((amax_b / 6) * S), d = its value,
+ *   y = x * (S / d), code = RNE or SR of y onto E2M1 (saturating at 6;
+ *   d = 0 gives +-0 codes).
+ *
+ * Outputs (NULL when that direction is not requested):
+ *   q_row  [rows, cols/2] codes,  sf_row scales,  g_row [1] FP32 decode scale;
+ *   q_col  [cols, rows/2] codes,  sf_col scales,  g_col [1].
+ * Shapes: rows, cols multiples of 16; MXFP8 needs its block axis a multiple
+ * of 32; NVFP4_SF_MMA needs the quantised length a multiple of 64.
+ * Alignment: x and ld*2 bytes 16-byte aligned; outputs 16-byte aligned.
+ * Returns NVFP4_ERR_SHAPE / _ALIGN / _INVALID_ARG / _WORKSPACE before any
+ * launch, NVFP4_ERR_CUDA if a launch fails.
+ */
+nvfp4_status nvfp4_quantize(const void* x_bf16, int64_t rows, int64_t cols, int64_t ld,
+                            const nvfp4_quant_params* p, uint8_t* q_row, uint8_t* sf_row,
+                            float* g_row, uint8_t* q_col, uint8_t* sf_col, float* g_col,
+                            void* workspace, size_t ws_bytes, void* stream);
+
+/*
+ * mxfp8_quantize -- MXFP8 (iitak, "How it works" and "But"): per 32-element
+ * block e = clamp(floor(log2 amax) - 8, -127, 127) (OCP MX v1.0 rule),
+ * E8M0 byte e + 127 (amax 0 -> byte 0), element = E4M3 of x * 2^-e, RNE
+ * satfinite or SR (Philox stream 2).
+ * directions: NVFP4_ROWWISE (codes [rows, cols], scales [rows, cols/32]) and/or
+ * NVFP4_COLWISE (codes [cols, rows], scales [cols, rows/32]).  The block axis
+ * must be a multiple of 32, the other a multiple of 16.
+ */
+nvfp4_status mxfp8_quantize(const void* x_bf16, int64_t rows, int64_t cols, int64_t ld,
+                            int directions, int rounding, uint64_t seed, uint32_t offset,
+                            uint8_t* q_row, uint8_t* e8_row, uint8_t* q_col, uint8_t* e8_col,
+                            void* stream);
+
+/*
+ * nvfp4_dequantize -- x_hat = (e2m1(code) * d) * g, the first product exact,
+ * one FP32 rounding, then (for NVFP4_OUT_BF16) RNE to bf16.
+ * q [rows, cols/2], sf in sf_layout, g device [1]; out [rows, cols].
+ */
+nvfp4_status nvfp4_dequantize(const uint8_t* q, const uint8_t* sf, const float* g, int64_t rows,
+                              int64_t cols, int sf_layout, int out_dtype, void* out,
+                              void* stream);
+
+/* Workspace bytes nvfp4_gemm / nvfp4_grouped_gemm need (status word). */
+size_t nvfp4_gemm_workspace_size(int64_t M, int64_t N, int64_t K);
+
+/*
+ * nvfp4_gemm -- block-scaled NVFP4 GEMM on the tcgen05 tensor cores
+ * (asector, "NVFP4 and Blackwell": scaled computation with high-precision
+ * accumulation):
+ *   D[i][j] = ga * gb * sum_k (e2m1(a_ik) * sa(i, k/16)) * (e2m1(b_jk) * sb(j, k/16))
+ * with FP32 accumulation.  "TN": A [M, K] and B [N, K] are both K-contiguous
+ * codes (qa [M, K/2], qb [N, K/2]); scales sfa / sfb in NVFP4_SF_MMA layout;
+ * ga, gb device FP32 [1].  D [M, ldd] FP32 or bf16 (RNE), row-major.
+ * Shapes: K a multiple of 256 (one pipeline stage), M and N multiples of 16;
+ * ldd >= N with ldd * element size a multiple of 16 bytes.
+ */
+nvfp4_status nvfp4_gemm(const uint8_t* qa, const uint8_t* sfa, const float* ga,
+                        const uint8_t* qb, const uint8_t* sfb, const float* gb, int64_t M,
+                        int64_t N, int64_t K, int out_dtype, void* D, int64_t ldd,
+                        void* workspace, size_t ws_bytes, void* stream);
+
+/*
+ * nvfp4_grouped_gemm -- MoE grouped form (iitak, "Details": NVFP4 in the
+ * expert layers): rows [off[e], off[e+1]) of the stacked A [total_rows, K]
+ * are multiplied by expert e's B_e [N, K]:
+ *   D[i][j] = ga * gb[e] * sum_k a_hat_ik b_hat_e,jk.
+ * group_offsets: device int32 [G+1], non-decreasing, off[0] = 0,
+ * off[G] = total_rows.  sfa in the grouped NVFP4_SF_MMA layout (see above);
+ * qb [G, N, K/2], sfb [G] consecutive NVFP4_SF_MMA blocks of N rows each,
+ * gb device [G].  D [total_rows, N] row-major.  The tile schedule is computed
+ * on the device from group_offsets: the host never reads the offsets.
+ */
+nvfp4_status nvfp4_grouped_gemm(int G, const int32_t* group_offsets, int64_t total_rows,
+                                const uint8_t* qa, const uint8_t* sfa, const float* ga,
+                                const uint8_t* qb, const uint8_t* sfb, const float* gb,
+                                int64_t N, int64_t K, int out_dtype, void* D, void* workspace,
+                                size_t ws_bytes, void* stream);
+
+/* Synchronise `stream` and return the device status word of a workspace
+ * (NVFP4_OK, NVFP4_ERR_TIMEOUT or NVFP4_ERR_INDEX); clears it. */
+nvfp4_status nvfp4_workspace_status(void* workspace, void* stream);
+
+/* Text of a status code (static storage). */
+const char* nvfp4_status_string(nvfp4_status s);
+
+/* Library version: major * 10000 + minor * 100 + patch. */
+int nvfp4_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* NVFP4_H */

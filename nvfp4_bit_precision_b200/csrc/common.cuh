@@ -1,0 +1,301 @@
+// common.cuh -- device helpers shared by the NVFP4 kernels (sm_100a only).
+//
+// Everything here is written for Blackwell: mbarrier-tracked bulk copies into
+// shared memory, hardware FP8/FP4 conversions, and bounded waits that give up
+// after a wall-clock limit instead of hanging the GPU.
+#pragma once
+
+#include <cuda_bf16.h>
+#include <cuda_fp16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "nvfp4.h"
+
+#if defined(__CUDA_ARCH__) && (__CUDA_ARCH__ < 1000)
+#error "this library targets sm_100a (B200) only"
+#endif
+
+namespace nvfp4 {
+
+// --------------------------------------------------------------------------
+// Bounded waits.  Every spin on an mbarrier gives up after this many
+// nanoseconds of %globaltimer, records NVFP4_ERR_TIMEOUT in the status word
+// and lets the kernel return normally.
+// --------------------------------------------------------------------------
+constexpr uint64_t kWaitLimitNs = 2000000000ull;  // 2 s
+
+__device__ __forceinline__ uint64_t global_timer_ns()
+{
+    uint64_t t;
+    asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+    return t;
+}
+
+__device__ __forceinline__ uint32_t smem_addr(const void* p)
+{
+    return static_cast<uint32_t>(__cvta_generic_to_shared(p));
+}
+
+__device__ __forceinline__ void mbar_init(uint64_t* bar, uint32_t count)
+{
+    asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_addr(bar)), "r"(count)
+                 : "memory");
+}
+
+// Make initialised barriers visible to the async (bulk copy / tensor core) proxy.
+__device__ __forceinline__ void fence_barrier_init()
+{
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+}
+
+__device__ __forceinline__ void fence_proxy_async_smem()
+{
+    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+
+__device__ __forceinline__ void mbar_arrive_expect_tx(uint64_t* bar, uint32_t bytes)
+{
+    asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(smem_addr(bar)),
+                 "r"(bytes)
+                 : "memory");
+}
+
+__device__ __forceinline__ void mbar_arrive(uint64_t* bar)
+{
+    asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_addr(bar)) : "memory");
+}
+
+__device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity)
+{
+    uint32_t ok;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(ok)
+        : "r"(smem_addr(bar)), "r"(parity)
+        : "memory");
+    return ok != 0;
+}
+
+// Wait for the phase with the given parity to complete; false after the limit.
+__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity)
+{
+    if (mbar_try_wait(bar, parity)) return true;
+    const uint64_t t0 = global_timer_ns();
+    while (true) {
+#pragma unroll 1
+        for (int i = 0; i < 32; ++i)
+            if (mbar_try_wait(bar, parity)) return true;
+        if (global_timer_ns() - t0 > kWaitLimitNs) return false;
+    }
+}
+
+// One-dimensional bulk copy global -> shared, completing on `bar`.
+// dst, src 16-byte aligned; bytes a multiple of 16.
+__device__ __forceinline__ void bulk_copy_g2s(void* dst, const void* src, uint32_t bytes,
+                                              uint64_t* bar)
+{
+    asm volatile(
+        "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
+            smem_addr(dst)),
+        "l"(src), "r"(bytes), "r"(smem_addr(bar))
+        : "memory");
+}
+
+__device__ __forceinline__ void record_status(uint32_t* status, uint32_t code)
+{
+    if (status) atomicCAS(status, 0u, code);
+}
+
+// --------------------------------------------------------------------------
+// Philox4x32-10 (Salmon, Moraes, Dror, Shaw, SC'11): two 32x32->64 products
+// per round, Weyl key schedule, ten rounds.
+// --------------------------------------------------------------------------
+struct U4 {
+    uint32_t x, y, z, w;
+};
+
+__device__ __forceinline__ U4 philox4x32_10(uint32_t c0, uint32_t c1, uint32_t c2, uint32_t c3,
+                                             uint32_t k0, uint32_t k1)
+{
+#pragma unroll
+    for (int r = 0; r < 10; ++r) {
+        const uint32_t lo0 = 0xD2511F53u * c0, hi0 = __umulhi(0xD2511F53u, c0);
+        const uint32_t lo1 = 0xCD9E8D57u * c2, hi1 = __umulhi(0xCD9E8D57u, c2);
+        const uint32_t n0 = hi1 ^ c1 ^ k0;
+        const uint32_t n2 = hi0 ^ c3 ^ k1;
+        c0 = n0;
+        c1 = lo1;
+        c2 = n2;
+        c3 = lo0;
+        k0 += 0x9E3779B9u;
+        k1 += 0xBB67AE85u;
+    }
+    return U4{c0, c1, c2, c3};
+}
+
+// Random bits for elements idx8*8 .. idx8*8+7 of one stream: element j takes
+// the 16-bit half (j % 2) of word j / 2.
+__device__ __forceinline__ U4 sr_block8(uint64_t seed, uint32_t offset, uint32_t stream,
+                                        uint64_t idx8)
+{
+    return philox4x32_10(static_cast<uint32_t>(idx8), static_cast<uint32_t>(idx8 >> 32), stream,
+                         offset, static_cast<uint32_t>(seed), static_cast<uint32_t>(seed >> 32));
+}
+
+__device__ __forceinline__ uint32_t u16_of(const U4& w, int j)
+{
+    const uint32_t word = (j >> 1) == 0 ? w.x : (j >> 1) == 1 ? w.y : (j >> 1) == 2 ? w.z : w.w;
+    return (j & 1) ? (word >> 16) : (word & 0xFFFFu);
+}
+
+// Hadamard sign bits: bit i set -> sign i is -1.  Word 0 of Philox(counter
+// (0,0,3,0), key = seed); depends on the seed only.
+__device__ __forceinline__ uint32_t rht_sign_bits(uint64_t seed)
+{
+    return philox4x32_10(0u, 0u, 3u, 0u, static_cast<uint32_t>(seed),
+                         static_cast<uint32_t>(seed >> 32))
+        .x;
+}
+
+// 16-point random-sign Hadamard in registers, fixed order: sign flip, then
+// butterfly stages h = 1, 2, 4, 8 with IEEE add/sub, then the exact factor 1/4.
+__device__ __forceinline__ void rht16(float (&v)[16], uint32_t signs)
+{
+#pragma unroll
+    for (int i = 0; i < 16; ++i)
+        v[i] = __uint_as_float(__float_as_uint(v[i]) ^ (((signs >> i) & 1u) << 31));
+#pragma unroll
+    for (int h = 1; h < 16; h <<= 1) {
+#pragma unroll
+        for (int i = 0; i < 16; ++i) {
+            if (i & h) continue;
+            const float a = v[i], b = v[i + h];
+            v[i] = __fadd_rn(a, b);
+            v[i + h] = __fsub_rn(a, b);
+        }
+    }
+#pragma unroll
+    for (int i = 0; i < 16; ++i) v[i] = __fmul_rn(v[i], 0.25f);
+}
+
+// --------------------------------------------------------------------------
+// Conversions (hardware, exact where stated).
+// --------------------------------------------------------------------------
+__device__ __forceinline__ float bf16_lo(uint32_t packed) { return __uint_as_float(packed << 16); }
+__device__ __forceinline__ float bf16_hi(uint32_t packed)
+{
+    return __uint_as_float(packed & 0xFFFF0000u);
+}
+
+// E4M3 round-to-nearest-even, saturating to +-448; returns the byte.
+__device__ __forceinline__ uint32_t e4m3_rne_sat(float v)
+{
+    uint16_t r;
+    asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;" : "=h"(r) : "f"(0.0f), "f"(v));
+    return r & 0xFFu;
+}
+
+// Two E4M3 bytes in one 16-bit value: hi -> upper byte, lo -> lower byte.
+__device__ __forceinline__ uint32_t e4m3x2_rne_sat(float hi, float lo)
+{
+    uint16_t r;
+    asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;" : "=h"(r) : "f"(hi), "f"(lo));
+    return r;
+}
+
+// Value of an E4M3 byte (exact).
+__device__ __forceinline__ float e4m3_value(uint32_t byte)
+{
+    uint32_t h2;
+    const uint16_t b = static_cast<uint16_t>(byte & 0xFFu);
+    asm("cvt.rn.f16x2.e4m3x2 %0, %1;" : "=r"(h2) : "h"(b));
+    return __half2float(__ushort_as_half(static_cast<unsigned short>(h2 & 0xFFFFu)));
+}
+
+// Eight floats -> eight E2M1 codes (RNE, saturating), packed with element 0 in
+// the low nibble of byte 0.
+__device__ __forceinline__ uint32_t e2m1x8_rne(const float* v)
+{
+    uint32_t out;
+    asm("{\n\t.reg .b8 b0, b1, b2, b3;\n\t"
+        "cvt.rn.satfinite.e2m1x2.f32 b0, %2, %1;\n\t"
+        "cvt.rn.satfinite.e2m1x2.f32 b1, %4, %3;\n\t"
+        "cvt.rn.satfinite.e2m1x2.f32 b2, %6, %5;\n\t"
+        "cvt.rn.satfinite.e2m1x2.f32 b3, %8, %7;\n\t"
+        "mov.b32 %0, {b0, b1, b2, b3};\n\t}"
+        : "=r"(out)
+        : "f"(v[0]), "f"(v[1]), "f"(v[2]), "f"(v[3]), "f"(v[4]), "f"(v[5]), "f"(v[6]),
+          "f"(v[7]));
+    return out;
+}
+
+// Stochastic rounding onto the E2M1 grid, returning the grid value (exact, so
+// a following RNE conversion only encodes it).  P(up) = floor(f * 2^16) / 2^16
+// with f the position of |y| between its two grid neighbours: the 16 bits of
+// the fraction that the grid drops are added to (0xFFFF - u) and the carry,
+// if any, rounds up.  Magnitudes below 1 are first lifted by 0.5 (truncating)
+// so that the grid step equals the float's kept-bit step.
+__device__ __forceinline__ float e2m1_sr_value(float y, uint32_t u16)
+{
+    const float a = fabsf(y);
+    const bool small = a < 1.0f;
+    const float a2 = small ? __fadd_rz(a, 0.5f) : a;
+    const uint32_t sh = (a2 < 1.0f) ? 7u : 6u;
+    const uint32_t noise = (0xFFFFu - u16) << sh;
+    const uint32_t mask = 0xFFFFFFFFu << (sh + 16u);
+    float r = __uint_as_float((__float_as_uint(a2) + noise) & mask);
+    r = small ? __fsub_rn(r, 0.5f) : r;
+    r = fminf(r, 6.0f);
+    return copysignf(r, y);
+}
+
+// Same rule on the E4M3 grid (3 kept mantissa bits, subnormal step 2^-9,
+// saturating at 448).
+__device__ __forceinline__ float e4m3_sr_value(float y, uint32_t u16)
+{
+    const float a = fabsf(y);
+    const float lift = 0.015625f;  // 2^-6, the smallest normal E4M3 value
+    const bool small = a < lift;
+    const float a2 = small ? __fadd_rz(a, lift) : a;
+    const uint32_t noise = (0xFFFFu - u16) << 4;
+    float r = __uint_as_float((__float_as_uint(a2) + noise) & 0xFFF00000u);
+    r = small ? __fsub_rn(r, lift) : r;
+    r = fminf(r, 448.0f);
+    return copysignf(r, y);
+}
+
+// --------------------------------------------------------------------------
+// Global scale: S = 2688/amax, g = amax/2688 (IEEE single divisions); amax 0
+// gives 1, 1; S is capped at 2^118 (g = 2^-118).
+// --------------------------------------------------------------------------
+__device__ __forceinline__ void global_scales(float amax, float& S, float& g)
+{
+    if (amax == 0.0f) {
+        S = 1.0f;
+        g = 1.0f;
+        return;
+    }
+    const float cap = 3.32306998946228968226e+35f;  // 2^118
+    const float s = __fdiv_rn(2688.0f, amax);
+    if (!(s <= cap)) {
+        S = cap;
+        g = 3.00926553346026563215e-36f;  // 2^-118
+        return;
+    }
+    S = s;
+    g = __fdiv_rn(amax, 2688.0f);
+}
+
+// Offset of scale byte (row r, 16-block b) in the tiled tensor-core layout of
+// an operand whose rows hold k16 = K/16 blocks: 128x4 atoms of 512 bytes,
+// atoms ordered with the K group fastest.
+__host__ __device__ __forceinline__ int64_t sf_mma_offset(int64_t r, int64_t b, int64_t k16)
+{
+    const int64_t atom = (r >> 7) * (k16 >> 2) + (b >> 2);
+    return atom * 512 + (r & 31) * 16 + ((r & 127) >> 5) * 4 + (b & 3);
+}
+
+}  // namespace nvfp4

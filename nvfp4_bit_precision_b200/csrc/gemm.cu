@@ -1,0 +1,572 @@
+// gemm.cu -- block-scaled NVFP4 GEMM and MoE grouped GEMM on the sm_100a
+// tensor cores (tcgen05, kind::mxf4nvf4, 16-element UE4M3 block scales).
+//
+// D[i][j] = ga * gb * sum_k (e2m1(a_ik) sa(i,k/16)) (e2m1(b_jk) sb(j,k/16)),
+// FP32 accumulation in tensor memory (asector.ru, "Nvidia dobivaetsya uspekha
+// s 4-bitnym formatom NVFP4", section "NVFP4 and Blackwell": the tensor cores
+// compute with scaling and high-precision accumulation; iitak.ru, "Thinking
+// Machines uskorila obuchenie Inkling 2 Small 4-bitnymi chislami", section
+// "Details": NVFP4 in the expert layers -> the grouped form).
+//
+// Structure (one persistent CTA per SM, 192 threads):
+//   warp 0      TMA producer: A/B tiles (128-byte swizzled, 4-bit codes packed
+//               two per byte) by cp.async.bulk.tensor, scale atoms by
+//               cp.async.bulk, into a 4-stage ring guarded by mbarriers.
+//   warp 1      one elected thread moves the stage's scale factors into tensor
+//               memory (tcgen05.cp 32x128b.warpx4) and issues 4 MMAs of
+//               128x256x64, then commits the stage back to the producer and,
+//               after the last K stage, the accumulator to the epilogue.
+//   warps 2..5  epilogue: tcgen05.ld of the 128x256 FP32 accumulator, times
+//               ga*gb, converted and stored to global memory.
+// Every mbarrier wait is bounded (2 s); a timeout sets the workspace status
+// word and the kernel winds down instead of hanging.
+#include <cudaTypedefs.h>
+
+#include <algorithm>
+#include <mutex>
+
+#include "common.cuh"
+
+namespace nvfp4 {
+
+constexpr int BM = 128;
+constexpr int BN = 256;
+constexpr int BK = 256;                    // elements per stage (128 bytes per row)
+constexpr int kGemmStages = 4;
+constexpr int kA_Bytes = BM * BK / 2;      // 16 KB
+constexpr int kB_Bytes = BN * BK / 2;      // 32 KB
+constexpr int kSFA_Bytes = BM * BK / 16;   // 2 KB: 4 atoms of 512 B
+constexpr int kSFB_Bytes = BN * BK / 16;   // 4 KB: 2 row blocks x 4 atoms
+constexpr int kStageBytes = kA_Bytes + kB_Bytes + kSFA_Bytes + kSFB_Bytes;
+constexpr int kGemmThreads = 192;
+constexpr int kTmemCols = 512;             // accumulator 256 + SFA 16 + SFB 32, rounded up
+constexpr int kTmemSFA = 256;
+constexpr int kTmemSFB = 256 + 16;
+constexpr int kMaxGemmGroups = 256;
+
+struct GemmArgs {
+    const uint8_t* sfa;
+    const uint8_t* sfb;
+    const float* ga;
+    const float* gb;
+    void* D;
+    int64_t M, N, K, ldd;
+    int bf16_out;
+    // grouped form
+    int grouped;
+    int G;
+    const int32_t* group_offsets;
+    int64_t total_rows;
+    uint32_t* status;
+};
+
+struct GemmShared {
+    uint64_t full[kGemmStages];
+    uint64_t empty[kGemmStages];
+    uint64_t acc_full;
+    uint64_t acc_empty;
+    uint32_t tmem_base;
+    int32_t total_tiles;
+    int32_t cum_tiles[kMaxGemmGroups + 1];
+    int32_t group_start[kMaxGemmGroups + 1];
+    int32_t group_sfblk[kMaxGemmGroups + 1];  // first padded 128-row scale block of a group
+};
+
+// ---------------------------------------------------------------- PTX wrappers
+__device__ __forceinline__ void tma_load_2d(void* dst, const CUtensorMap* map, int32_t x, int32_t y,
+                                            uint64_t* bar)
+{
+    asm volatile(
+        "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes [%0], "
+        "[%1, {%2, %3}], [%4];" ::"r"(smem_addr(dst)),
+        "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(smem_addr(bar))
+        : "memory");
+}
+
+__device__ __forceinline__ void tmem_alloc(uint32_t* dst_smem, uint32_t ncols)
+{
+    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
+                     smem_addr(dst_smem)),
+                 "r"(ncols)
+                 : "memory");
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+}
+
+__device__ __forceinline__ void tmem_dealloc(uint32_t taddr, uint32_t ncols)
+{
+    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(taddr), "r"(ncols)
+                 : "memory");
+}
+
+__device__ __forceinline__ void tc_fence_before() { asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory"); }
+__device__ __forceinline__ void tc_fence_after() { asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory"); }
+
+__device__ __forceinline__ void tc_commit(uint64_t* bar)
+{
+    asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(
+                     smem_addr(bar))
+                 : "memory");
+}
+
+// Shared-memory matrix descriptor: K-major operand, 128-byte swizzle, 8-row
+// groups 1024 bytes apart (start, LBO and SBO in 16-byte units; version 1).
+__device__ __forceinline__ uint64_t desc_sw128(const void* p)
+{
+    const uint64_t start = (smem_addr(p) >> 4) & 0x3FFFu;
+    return start | (1ull << 16) | (64ull << 32) | (1ull << 46) | (2ull << 61);
+}
+
+// Descriptor of one 512-byte scale atom: 32 rows of 16 bytes, no swizzle,
+// 8-row groups 128 bytes apart.
+__device__ __forceinline__ uint64_t desc_sf_atom(const void* p)
+{
+    const uint64_t start = (smem_addr(p) >> 4) & 0x3FFFu;
+    return start | (1ull << 16) | (8ull << 32) | (1ull << 46);
+}
+
+__device__ __forceinline__ void tc_cp_sf(uint32_t taddr, uint64_t desc)
+{
+    asm volatile("tcgen05.cp.cta_group::1.32x128b.warpx4 [%0], %1;" ::"r"(taddr), "l"(desc)
+                 : "memory");
+}
+
+// Instruction descriptor: kind::mxf4nvf4, A/B E2M1 (format 1), UE4M3 scales,
+// both K-major, M = 128, N = 256, dense, K = 64 per instruction.
+__host__ __device__ constexpr uint32_t make_idesc()
+{
+    return (1u << 7) | (1u << 10) | ((uint32_t)(BN >> 3) << 17) | ((uint32_t)(BM >> 4) << 24);
+}
+
+__device__ __forceinline__ void tc_mma(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc,
+                                       uint32_t idesc, uint32_t sfa_tmem, uint32_t sfb_tmem,
+                                       uint32_t accumulate)
+{
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::mxf4nvf4.block_scale.block16 [%0], %1, %2, %3, [%5], [%6], p;\n\t"
+        "}" ::"r"(d_tmem),
+        "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate), "r"(sfa_tmem), "r"(sfb_tmem)
+        : "memory");
+}
+
+#define TMEM_LD_32(taddr, r)                                                                       \
+    asm volatile("tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12," \
+                 "%13,%14,%15,%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, "  \
+                 "[%32];"                                                                          \
+                 : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]),         \
+                   "=r"(r[6]), "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]),       \
+                   "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15]), "=r"(r[16]), "=r"(r[17]),   \
+                   "=r"(r[18]), "=r"(r[19]), "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]),   \
+                   "=r"(r[24]), "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]),   \
+                   "=r"(r[30]), "=r"(r[31])                                                        \
+                 : "r"(taddr))
+
+__device__ __forceinline__ void tmem_ld_wait() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory"); }
+
+// ---------------------------------------------------------------- scheduling
+struct TileCoord {
+    int group;       // expert (0 when dense)
+    int64_t row0;    // first A row of the tile
+    int64_t row_end; // one past the last valid A row
+    int64_t sf_blk;  // 128-row scale block of the tile
+    int64_t n0;
+};
+
+__device__ __forceinline__ TileCoord tile_coord(const GemmArgs& a, const GemmShared* sh, int t)
+{
+    TileCoord c;
+    const int64_t tiles_n = (a.N + BN - 1) / BN;
+    if (!a.grouped) {
+        const int64_t tiles_m = (a.M + BM - 1) / BM;
+        const int64_t band = 8 * tiles_n;  // 8 M tiles share a band: B tiles reused from L2
+        const int64_t g = t / band, first_m = g * 8;
+        const int64_t gm = min((int64_t)8, tiles_m - first_m);
+        const int64_t r = t - g * band;
+        const int64_t mt = first_m + r % gm, nt = r / gm;
+        c.group = 0;
+        c.row0 = mt * BM;
+        c.row_end = a.M;
+        c.sf_blk = mt;
+        c.n0 = nt * BN;
+    } else {
+        int lo = 0, hi = a.G - 1;  // e with cum[e] <= t < cum[e+1]
+        while (lo < hi) {
+            const int mid = (lo + hi + 1) >> 1;
+            if (sh->cum_tiles[mid] <= t)
+                lo = mid;
+            else
+                hi = mid - 1;
+        }
+        const int64_t local = t - sh->cum_tiles[lo];
+        const int64_t mt = local / tiles_n, nt = local - mt * tiles_n;
+        c.group = lo;
+        c.row0 = sh->group_start[lo] + mt * BM;
+        c.row_end = sh->group_start[lo + 1];
+        c.sf_blk = sh->group_sfblk[lo] + mt;
+        c.n0 = nt * BN;
+    }
+    return c;
+}
+
+// ---------------------------------------------------------------- kernel
+__global__ void __launch_bounds__(kGemmThreads, 1)
+    gemm_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_constant__ CUtensorMap map_b,
+                GemmArgs a)
+{
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                               ~uintptr_t(1023));
+    GemmShared* sh = reinterpret_cast<GemmShared*>(smem + kGemmStages * kStageBytes);
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < kGemmStages; ++s) {
+            mbar_init(&sh->full[s], 1);
+            mbar_init(&sh->empty[s], 1);
+        }
+        mbar_init(&sh->acc_full, 1);
+        mbar_init(&sh->acc_empty, 4);
+        fence_barrier_init();
+        // tile table
+        const int64_t tiles_n = (a.N + BN - 1) / BN;
+        if (!a.grouped) {
+            sh->total_tiles = (int32_t)(((a.M + BM - 1) / BM) * tiles_n);
+        } else {
+            int32_t cum = 0, blk = 0;
+            for (int e = 0; e <= a.G; ++e) {
+                const int32_t st = a.group_offsets[e];
+                sh->group_start[e] = st;
+                sh->cum_tiles[e] = cum;
+                sh->group_sfblk[e] = blk;
+                if (e < a.G) {
+                    const int32_t cnt = a.group_offsets[e + 1] - st;
+                    const int32_t mt = cnt > 0 ? (cnt + BM - 1) / BM : 0;
+                    cum += mt * (int32_t)tiles_n;
+                    blk += mt;
+                }
+            }
+            sh->total_tiles = cum;
+        }
+    }
+    if (warp == 1) tmem_alloc(&sh->tmem_base, kTmemCols);
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = sh->tmem_base;
+    const int total = sh->total_tiles;
+    const int64_t kstages = a.K / BK;
+    const int64_t k64 = a.K / 64;  // scale atoms per 128-row block
+    bool failed = false;
+
+    if (warp == 0) {
+        // ------------------------------------------------ TMA producer
+        if (lane == 0) {
+            asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&map_a)) : "memory");
+            asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&map_b)) : "memory");
+            const int64_t n_blocks_valid = (a.N + 127) / 128;  // scale row blocks that exist
+            uint32_t it = 0;
+            for (int t = blockIdx.x; t < total && !failed; t += gridDim.x) {
+                const TileCoord c = tile_coord(a, sh, t);
+                const int64_t b_row0 = (int64_t)c.group * a.N + c.n0;
+                const int64_t nb0 = c.n0 / 128;
+                const int nsfb = (int)min((int64_t)2, n_blocks_valid - nb0);
+                const uint8_t* sfb_base = a.sfb + (int64_t)c.group * ((a.N + 127) / 128) * k64 * 512;
+                for (int64_t ks = 0; ks < kstages; ++ks, ++it) {
+                    const int s = (int)(it % kGemmStages);
+                    const uint32_t ph = (it / kGemmStages) & 1u;
+                    if (!mbar_wait(&sh->empty[s], ph ^ 1u)) {
+                        record_status(a.status, NVFP4_ERR_TIMEOUT);
+                        failed = true;
+                        break;
+                    }
+                    uint8_t* st = smem + s * kStageBytes;
+                    const uint32_t bytes = kA_Bytes + kB_Bytes + kSFA_Bytes + nsfb * (kSFB_Bytes / 2);
+                    mbar_arrive_expect_tx(&sh->full[s], bytes);
+                    tma_load_2d(st, &map_a, (int32_t)(ks * (BK / 2)), (int32_t)c.row0, &sh->full[s]);
+                    tma_load_2d(st + kA_Bytes, &map_b, (int32_t)(ks * (BK / 2)), (int32_t)b_row0,
+                                &sh->full[s]);
+                    // 4 consecutive scale atoms (K/64 groups ks*4 .. ks*4+3) per 128-row block
+                    bulk_copy_g2s(st + kA_Bytes + kB_Bytes, a.sfa + (c.sf_blk * k64 + ks * 4) * 512,
+                                  kSFA_Bytes, &sh->full[s]);
+                    for (int h = 0; h < nsfb; ++h)
+                        bulk_copy_g2s(st + kA_Bytes + kB_Bytes + kSFA_Bytes + h * (kSFB_Bytes / 2),
+                                      sfb_base + ((nb0 + h) * k64 + ks * 4) * 512, kSFB_Bytes / 2,
+                                      &sh->full[s]);
+                }
+            }
+        }
+    } else if (warp == 1) {
+        // ------------------------------------------------ MMA issuer
+        if (lane == 0) {
+            const uint32_t idesc = make_idesc();
+            uint32_t it = 0, tcount = 0;
+            for (int t = blockIdx.x; t < total && !failed; t += gridDim.x, ++tcount) {
+                // wait until the epilogue drained the accumulator of the previous tile
+                if (!mbar_wait(&sh->acc_empty, (tcount & 1u) ^ 1u)) {
+                    record_status(a.status, NVFP4_ERR_TIMEOUT);
+                    failed = true;
+                    break;
+                }
+                tc_fence_after();
+                for (int64_t ks = 0; ks < kstages; ++ks, ++it) {
+                    const int s = (int)(it % kGemmStages);
+                    const uint32_t ph = (it / kGemmStages) & 1u;
+                    if (!mbar_wait(&sh->full[s], ph)) {
+                        record_status(a.status, NVFP4_ERR_TIMEOUT);
+                        failed = true;
+                        break;
+                    }
+                    tc_fence_after();
+                    uint8_t* st = smem + s * kStageBytes;
+                    const uint8_t* sfa_s = st + kA_Bytes + kB_Bytes;
+                    const uint8_t* sfb_s = sfa_s + kSFA_Bytes;
+#pragma unroll
+                    for (int j = 0; j < 4; ++j) {
+                        tc_cp_sf(tmem + kTmemSFA + 4 * j, desc_sf_atom(sfa_s + j * 512));
+                        tc_cp_sf(tmem + kTmemSFB + 8 * j, desc_sf_atom(sfb_s + j * 512));
+                        tc_cp_sf(tmem + kTmemSFB + 8 * j + 4,
+                                 desc_sf_atom(sfb_s + kSFB_Bytes / 2 + j * 512));
+                    }
+                    const uint64_t ad = desc_sw128(st), bd = desc_sw128(st + kA_Bytes);
+#pragma unroll
+                    for (int j = 0; j < 4; ++j) {
+                        // +32 bytes (64 four-bit elements) along K inside the swizzled row
+                        tc_mma(tmem, ad + 2 * j, bd + 2 * j, idesc, tmem + kTmemSFA + 4 * j,
+                               tmem + kTmemSFB + 8 * j, (ks > 0 || j > 0) ? 1u : 0u);
+                    }
+                    tc_commit(&sh->empty[s]);  // stage free once these MMAs completed
+                }
+                if (failed) break;
+                tc_commit(&sh->acc_full);
+            }
+        }
+    } else {
+        // ------------------------------------------------ epilogue (warps 2..5)
+        const int quad = warp & 3;  // TMEM lanes 32*quad .. 32*quad+31
+        uint32_t tcount = 0;
+        for (int t = blockIdx.x; t < total; t += gridDim.x, ++tcount) {
+            const TileCoord c = tile_coord(a, sh, t);
+            const bool ok = mbar_wait(&sh->acc_full, tcount & 1u);
+            if (!ok) {
+                if (lane == 0) record_status(a.status, NVFP4_ERR_TIMEOUT);
+                break;
+            }
+            tc_fence_after();
+            const float alpha = __fmul_rn(a.ga[0], a.gb[c.group]);
+            const int64_t row = c.row0 + 32 * quad + lane;
+            const bool row_ok = row < c.row_end;
+            const uint32_t tbase = tmem + ((uint32_t)(32 * quad) << 16);
+            if (a.bf16_out) {
+                uint32_t packed[BN / 2];
+#pragma unroll
+                for (int ch = 0; ch < BN / 32; ++ch) {
+                    uint32_t r[32];
+                    TMEM_LD_32(tbase + 32 * ch, r);
+                    tmem_ld_wait();
+#pragma unroll
+                    for (int i = 0; i < 16; ++i) {
+                        const __nv_bfloat162 p = __floats2bfloat162_rn(
+                            __fmul_rn(__uint_as_float(r[2 * i]), alpha),
+                            __fmul_rn(__uint_as_float(r[2 * i + 1]), alpha));
+                        packed[16 * ch + i] = *reinterpret_cast<const uint32_t*>(&p);
+                    }
+                }
+                // accumulator drained: the next tile's MMAs may start
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&sh->acc_empty);
+                if (row_ok) {
+                    uint16_t* drow = static_cast<uint16_t*>(a.D) + row * a.ldd;
+#pragma unroll
+                    for (int v = 0; v < BN / 8; ++v) {
+                        const int64_t col = c.n0 + 8 * v;
+                        if (col < a.N)
+                            *reinterpret_cast<uint4*>(drow + col) =
+                                make_uint4(packed[4 * v], packed[4 * v + 1], packed[4 * v + 2],
+                                           packed[4 * v + 3]);
+                    }
+                }
+            } else {
+#pragma unroll 1
+                for (int ch = 0; ch < BN / 32; ++ch) {
+                    uint32_t r[32];
+                    TMEM_LD_32(tbase + 32 * ch, r);
+                    tmem_ld_wait();
+                    if (row_ok) {
+                        float* drow = static_cast<float*>(a.D) + row * a.ldd;
+#pragma unroll
+                        for (int v = 0; v < 8; ++v) {
+                            const int64_t col = c.n0 + 32 * ch + 4 * v;
+                            if (col < a.N)
+                                *reinterpret_cast<float4*>(drow + col) =
+                                    make_float4(__fmul_rn(__uint_as_float(r[4 * v]), alpha),
+                                                __fmul_rn(__uint_as_float(r[4 * v + 1]), alpha),
+                                                __fmul_rn(__uint_as_float(r[4 * v + 2]), alpha),
+                                                __fmul_rn(__uint_as_float(r[4 * v + 3]), alpha));
+                        }
+                    }
+                }
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&sh->acc_empty);
+            }
+        }
+    }
+
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    if (warp == 1) tmem_dealloc(tmem, kTmemCols);
+}
+
+// ---------------------------------------------------------------- host side
+static PFN_cuTensorMapEncodeTiled_v12000 encode_tiled()
+{
+    static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+    static std::once_flag once;
+    std::call_once(once, []() {
+        void* p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) ==
+                cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+    });
+    return fn;
+}
+
+// [rows, kbytes] uint8 matrix, box 128 bytes x box_rows, 128-byte swizzle.
+static bool make_map(CUtensorMap* m, const void* base, int64_t rows, int64_t kbytes, int box_rows)
+{
+    auto fn = encode_tiled();
+    if (!fn) return false;
+    cuuint64_t dims[2] = {(cuuint64_t)kbytes, (cuuint64_t)rows};
+    cuuint64_t strides[1] = {(cuuint64_t)kbytes};
+    cuuint32_t box[2] = {128u, (cuuint32_t)box_rows};
+    cuuint32_t estr[2] = {1u, 1u};
+    return fn(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void*>(base), dims, strides, box,
+              estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+              CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+static size_t gemm_smem_bytes() { return (size_t)kGemmStages * kStageBytes + sizeof(GemmShared) + 1024; }
+
+struct GemmDevice {
+    int sms = 0;
+    bool ok = false;
+};
+
+static GemmDevice& gemm_device(int dev)
+{
+    static GemmDevice infos[64];
+    static std::once_flag flags[64];
+    std::call_once(flags[dev & 63], [dev]() {
+        GemmDevice& d = infos[dev & 63];
+        cudaDeviceProp prop;
+        if (cudaGetDeviceProperties(&prop, dev) != cudaSuccess || prop.major != 10) return;
+        if (cudaFuncSetAttribute(gemm_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 (int)gemm_smem_bytes()) != cudaSuccess)
+            return;
+        d.sms = prop.multiProcessorCount;
+        d.ok = true;
+    });
+    return infos[dev & 63];
+}
+
+static bool al16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+constexpr size_t kGemmWorkspace = 256;
+
+}  // namespace nvfp4
+
+using namespace nvfp4;
+
+extern "C" size_t nvfp4_gemm_workspace_size(int64_t, int64_t, int64_t) { return kGemmWorkspace; }
+
+static nvfp4_status launch_gemm(const CUtensorMap& ma, const CUtensorMap& mb, GemmArgs& a,
+                                int64_t max_tiles, cudaStream_t st)
+{
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return NVFP4_ERR_CUDA;
+    GemmDevice& info = gemm_device(dev);
+    if (!info.ok) return NVFP4_ERR_UNSUPPORTED;
+    // the status word reports this call only
+    if (cudaMemsetAsync(a.status, 0, 4, st) != cudaSuccess) return NVFP4_ERR_CUDA;
+    const int grid = (int)std::max<int64_t>(1, std::min<int64_t>(max_tiles, info.sms));
+    gemm_kernel<<<grid, kGemmThreads, gemm_smem_bytes(), st>>>(ma, mb, a);
+    return cudaGetLastError() == cudaSuccess ? NVFP4_OK : NVFP4_ERR_CUDA;
+}
+
+extern "C" nvfp4_status nvfp4_gemm(const uint8_t* qa, const uint8_t* sfa, const float* ga,
+                                   const uint8_t* qb, const uint8_t* sfb, const float* gb,
+                                   int64_t M, int64_t N, int64_t K, int out_dtype, void* D,
+                                   int64_t ldd, void* workspace, size_t ws_bytes, void* stream)
+{
+    if (!qa || !sfa || !ga || !qb || !sfb || !gb || !D) return NVFP4_ERR_INVALID_ARG;
+    if (out_dtype != NVFP4_OUT_F32 && out_dtype != NVFP4_OUT_BF16) return NVFP4_ERR_INVALID_ARG;
+    if (M <= 0 || N <= 0 || K <= 0 || M % 16 || N % 16 || K % BK || ldd < N) return NVFP4_ERR_SHAPE;
+    if (M > (int64_t)1 << 31 || N > (int64_t)1 << 31) return NVFP4_ERR_SHAPE;
+    const int esz = out_dtype == NVFP4_OUT_BF16 ? 2 : 4;
+    if (!al16(qa) || !al16(qb) || !al16(sfa) || !al16(sfb) || !al16(D) || (ldd * esz) % 16)
+        return NVFP4_ERR_ALIGN;
+    if (!workspace || ws_bytes < kGemmWorkspace) return NVFP4_ERR_WORKSPACE;
+    if (!al16(workspace)) return NVFP4_ERR_ALIGN;
+    CUtensorMap ma, mb;
+    if (!make_map(&ma, qa, M, K / 2, BM) || !make_map(&mb, qb, N, K / 2, BN)) return NVFP4_ERR_CUDA;
+    GemmArgs a{};
+    a.sfa = sfa;
+    a.sfb = sfb;
+    a.ga = ga;
+    a.gb = gb;
+    a.D = D;
+    a.M = M;
+    a.N = N;
+    a.K = K;
+    a.ldd = ldd;
+    a.bf16_out = out_dtype == NVFP4_OUT_BF16;
+    a.grouped = 0;
+    a.G = 1;
+    a.status = static_cast<uint32_t*>(workspace) + 2;
+    const int64_t tiles = ((M + BM - 1) / BM) * ((N + BN - 1) / BN);
+    return launch_gemm(ma, mb, a, tiles, static_cast<cudaStream_t>(stream));
+}
+
+extern "C" nvfp4_status nvfp4_grouped_gemm(int G, const int32_t* group_offsets, int64_t total_rows,
+                                           const uint8_t* qa, const uint8_t* sfa, const float* ga,
+                                           const uint8_t* qb, const uint8_t* sfb, const float* gb,
+                                           int64_t N, int64_t K, int out_dtype, void* D,
+                                           void* workspace, size_t ws_bytes, void* stream)
+{
+    if (G < 1 || G > kMaxGemmGroups || !group_offsets || !qa || !sfa || !ga || !qb || !sfb ||
+        !gb || !D)
+        return NVFP4_ERR_INVALID_ARG;
+    if (out_dtype != NVFP4_OUT_F32 && out_dtype != NVFP4_OUT_BF16) return NVFP4_ERR_INVALID_ARG;
+    if (total_rows <= 0 || N <= 0 || K <= 0 || N % 128 || K % BK) return NVFP4_ERR_SHAPE;
+    if (total_rows > (int64_t)1 << 31 || (int64_t)G * N > (int64_t)1 << 31) return NVFP4_ERR_SHAPE;
+    if (!al16(qa) || !al16(qb) || !al16(sfa) || !al16(sfb) || !al16(D)) return NVFP4_ERR_ALIGN;
+    if (!workspace || ws_bytes < kGemmWorkspace) return NVFP4_ERR_WORKSPACE;
+    if (!al16(workspace)) return NVFP4_ERR_ALIGN;
+    CUtensorMap ma, mb;
+    if (!make_map(&ma, qa, total_rows, K / 2, BM) || !make_map(&mb, qb, (int64_t)G * N, K / 2, BN))
+        return NVFP4_ERR_CUDA;
+    GemmArgs a{};
+    a.sfa = sfa;
+    a.sfb = sfb;
+    a.ga = ga;
+    a.gb = gb;
+    a.D = D;
+    a.M = total_rows;
+    a.N = N;
+    a.K = K;
+    a.ldd = N;
+    a.bf16_out = out_dtype == NVFP4_OUT_BF16;
+    a.grouped = 1;
+    a.G = G;
+    a.group_offsets = group_offsets;
+    a.total_rows = total_rows;
+    a.status = static_cast<uint32_t*>(workspace) + 2;
+    // upper bound on tiles: every group may add one partial M tile
+    const int64_t tiles = ((total_rows + BM - 1) / BM + G) * (N / BN + 1);
+    return launch_gemm(ma, mb, a, tiles, static_cast<cudaStream_t>(stream));
+}

@@ -1,0 +1,830 @@
+// quantize.cu -- NVFP4 / MXFP8 quantisation and NVFP4 dequantisation on sm_100a.
+//
+// Two HBM-bound passes:
+//   1. amax_kernel: one read of the tensor, warp-shuffle max of |x| and, when
+//      the columnwise Hadamard is on, of |RHT(x)| over the columnwise
+//      16-vectors; one atomicMax per CTA on the float bit pattern.
+//   2. quant_kernel: a persistent grid walks 128x128 tiles in the reverse
+//      order of pass 1 (so the tail pass 1 left in L2 is read first).  One warp
+//      stages each tile into shared memory with mbarrier-tracked bulk copies
+//      (double-buffered); all eight warps then produce, from that one copy,
+//      the rowwise codes/scales, the columnwise (transposed, optionally
+//      Hadamard-rotated) codes/scales and the MXFP8 copies, with Philox
+//      stochastic rounding in registers and 8/16-byte vector stores.
+//
+// Format and steps: asector.ru, "Nvidia dobivaetsya uspekha s 4-bitnym
+// formatom NVFP4" ("NVFP4 and Blackwell": E2M1, 16-element local scale plus a
+// per-tensor scale, RNE and stochastic rounding; "Experiments and comparison
+// with FP8": 2D weight scales, random Hadamard transforms), and iitak.ru,
+// "Thinking Machines uskorila obuchenie Inkling 2 Small 4-bitnymi chislami"
+// ("Details": -54 -> -6 with multiplier 9; "How it works": transposed blocks,
+// 16x16 squares, random re-rounding, MXFP8 backward).
+#include <algorithm>
+#include <cstdio>
+#include <mutex>
+
+#include "common.cuh"
+
+namespace nvfp4 {
+
+constexpr int kTileRows = 128;
+constexpr int kTileCols = 128;
+constexpr int kPitch = kTileCols * 2 + 16;  // bytes per staged row (+16 breaks bank aliasing)
+constexpr int kTileBytes = kTileRows * kPitch;
+constexpr int kStages = 2;
+constexpr int kQuantThreads = 256;
+constexpr int kMaxGroups = 1024;
+
+struct QArgs {
+    const uint16_t* x;
+    int64_t rows, cols, ld;
+    int rounding, scaling, outputs, rht, sf_layout;
+    uint64_t seed;
+    uint32_t offset;
+    const float* amax_in;
+    const uint32_t* amax_ws;
+    const int32_t* row_index;
+    int64_t src_rows;
+    const int32_t* group_offsets;
+    int num_groups;
+    int mx_outputs, mx_rounding;
+    uint8_t *q_row, *sf_row;
+    float* g_row;
+    uint8_t *q_col, *sf_col;
+    float* g_col;
+    uint8_t *mx_q_row, *mx_sf_row, *mx_q_col, *mx_sf_col;
+    uint32_t* status;
+    int64_t tiles_c, n_tiles;
+};
+
+__device__ __forceinline__ uint4 ld_global_v4(const void* p)
+{
+    uint4 r;
+    asm volatile("ld.global.nc.v4.u32 {%0,%1,%2,%3}, [%4];"
+                 : "=r"(r.x), "=r"(r.y), "=r"(r.z), "=r"(r.w)
+                 : "l"(p));
+    return r;
+}
+
+__device__ __forceinline__ uint4 ld_shared_v4(const void* p)
+{
+    uint4 r;
+    asm volatile("ld.shared.v4.u32 {%0,%1,%2,%3}, [%4];"
+                 : "=r"(r.x), "=r"(r.y), "=r"(r.z), "=r"(r.w)
+                 : "r"(smem_addr(p)));
+    return r;
+}
+
+__device__ __forceinline__ uint32_t ld_shared_u16(const void* p)
+{
+    uint16_t r;
+    asm volatile("ld.shared.u16 %0, [%1];" : "=h"(r) : "r"(smem_addr(p)));
+    return r;
+}
+
+// Source row of output row r (gather); an out-of-range index is reported and
+// replaced by row 0 so that every access stays inside x.
+__device__ __forceinline__ int64_t source_row(const QArgs& a, int64_t r)
+{
+    if (!a.row_index) return r;
+    const int64_t s = a.row_index[r];
+    if (s < 0 || s >= a.src_rows) {
+        record_status(a.status, NVFP4_ERR_INDEX);
+        return 0;
+    }
+    return s;
+}
+
+__device__ __forceinline__ float warp_max16(float v)
+{
+#pragma unroll
+    for (int o = 1; o < 16; o <<= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, o));
+    return v;
+}
+
+// --------------------------------------------------------------------------
+// Pass 1: global amax.
+// --------------------------------------------------------------------------
+__global__ void __launch_bounds__(256) amax_kernel(QArgs a, uint32_t* amax_out)
+{
+    const uint32_t signs = a.rht ? rht_sign_bits(a.seed) : 0u;
+    float mr = 0.0f, mc = 0.0f;
+    const int64_t ncg = a.cols / 8;
+    const int64_t units = (a.rows / 16) * ncg;
+    for (int64_t u = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; u < units;
+         u += (int64_t)gridDim.x * blockDim.x) {
+        const int64_t rb = u / ncg, cg = u - rb * ncg;
+        uint4 raw[16];
+#pragma unroll
+        for (int i = 0; i < 16; ++i) {
+            const int64_t sr = source_row(a, rb * 16 + i);
+            raw[i] = ld_global_v4(a.x + sr * a.ld + cg * 8);
+        }
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+            float v[16];
+#pragma unroll
+            for (int i = 0; i < 16; ++i) {
+                const uint32_t w = (j >> 1) == 0 ? raw[i].x
+                                   : (j >> 1) == 1 ? raw[i].y
+                                   : (j >> 1) == 2 ? raw[i].z
+                                                   : raw[i].w;
+                v[i] = (j & 1) ? bf16_hi(w) : bf16_lo(w);
+                mr = fmaxf(mr, fabsf(v[i]));
+            }
+            if (a.rht) {
+                rht16(v, signs);
+#pragma unroll
+                for (int i = 0; i < 16; ++i) mc = fmaxf(mc, fabsf(v[i]));
+            }
+        }
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) {
+        mr = fmaxf(mr, __shfl_xor_sync(0xffffffffu, mr, o));
+        mc = fmaxf(mc, __shfl_xor_sync(0xffffffffu, mc, o));
+    }
+    __shared__ float red[2][8];
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    if (lane == 0) {
+        red[0][warp] = mr;
+        red[1][warp] = mc;
+    }
+    __syncthreads();
+    if (threadIdx.x == 0) {
+        for (int w = 1; w < (int)(blockDim.x >> 5); ++w) {
+            mr = fmaxf(mr, red[0][w]);
+            mc = fmaxf(mc, red[1][w]);
+        }
+        // non-negative floats order like their bit patterns
+        atomicMax(&amax_out[0], __float_as_uint(mr));
+        atomicMax(&amax_out[1], __float_as_uint(mc));
+    }
+}
+
+// --------------------------------------------------------------------------
+// Pass 2: fused quantisation of 128x128 tiles.
+// --------------------------------------------------------------------------
+struct QShared {
+    int32_t n_groups;
+    int32_t group_start[kMaxGroups + 1];   // output-row offsets
+    int32_t group_padded[kMaxGroups + 1];  // padded scale-row offsets
+};
+
+// Padded scale row of output row r (MoE layout); identity when dense.
+__device__ __forceinline__ int64_t padded_row(const QShared* sh, const QArgs& a, int64_t r)
+{
+    if (!a.group_offsets) return r;
+    int lo = 0, hi = sh->n_groups - 1;  // find e with start[e] <= r < start[e+1]
+    while (lo < hi) {
+        const int mid = (lo + hi + 1) >> 1;
+        if (sh->group_start[mid] <= r)
+            lo = mid;
+        else
+            hi = mid - 1;
+    }
+    return r - sh->group_start[lo] + sh->group_padded[lo];
+}
+
+__device__ __forceinline__ void issue_tile(const QArgs& a, int64_t tile, uint8_t* buf,
+                                           uint64_t* bar, int lane)
+{
+    const int64_t tr = tile / a.tiles_c, tc = tile - tr * a.tiles_c;
+    const int64_t r0 = tr * kTileRows, c0 = tc * kTileCols;
+    const int nrows = (int)(a.rows - r0 < kTileRows ? a.rows - r0 : kTileRows);
+    const uint32_t row_bytes = (uint32_t)(a.cols - c0 < kTileCols ? a.cols - c0 : kTileCols) * 2u;
+    if (lane == 0) mbar_arrive_expect_tx(bar, (uint32_t)nrows * row_bytes);
+    __syncwarp();
+    for (int i = lane; i < nrows; i += 32) {
+        const int64_t sr = source_row(a, r0 + i);
+        bulk_copy_g2s(buf + i * kPitch, a.x + sr * a.ld + c0, row_bytes, bar);
+    }
+}
+
+__device__ __forceinline__ void unpack8(const uint4& p, float* v)
+{
+    v[0] = bf16_lo(p.x);
+    v[1] = bf16_hi(p.x);
+    v[2] = bf16_lo(p.y);
+    v[3] = bf16_hi(p.y);
+    v[4] = bf16_lo(p.z);
+    v[5] = bf16_hi(p.z);
+    v[6] = bf16_lo(p.w);
+    v[7] = bf16_hi(p.w);
+}
+
+// Quantise one 16-value block given its (possibly 2D-reduced) amax.
+// Returns the scale byte; writes 8 code bytes to c0/c1.
+__device__ __forceinline__ uint32_t quant_block16(float (&v)[16], float amax_b, float S,
+                                                  bool sr, uint64_t seed, uint32_t offset,
+                                                  uint32_t stream, uint64_t idx, uint32_t& c0,
+                                                  uint32_t& c1)
+{
+    const float s = __fmul_rn(__fdiv_rn(amax_b, 6.0f), S);
+    const uint32_t byte = e4m3_rne_sat(s);
+    const float d = e4m3_value(byte);
+    const float r = (d != 0.0f) ? __fdiv_rn(S, d) : 0.0f;  // d = 0: every y is +-0
+#pragma unroll
+    for (int i = 0; i < 16; ++i) v[i] = __fmul_rn(v[i], r);
+    if (sr) {
+        const U4 w0 = sr_block8(seed, offset, stream, idx >> 3);
+        const U4 w1 = sr_block8(seed, offset, stream, (idx >> 3) + 1);
+#pragma unroll
+        for (int i = 0; i < 8; ++i) v[i] = e2m1_sr_value(v[i], u16_of(w0, i));
+#pragma unroll
+        for (int i = 0; i < 8; ++i) v[8 + i] = e2m1_sr_value(v[8 + i], u16_of(w1, i));
+    }
+    c0 = e2m1x8_rne(v);
+    c1 = e2m1x8_rne(v + 8);
+    return byte;
+}
+
+// MXFP8 of 32 values: returns the E8M0 byte, writes 32 code bytes to out[8].
+__device__ __forceinline__ uint32_t mx_block32(const float* v, bool sr, uint64_t seed,
+                                               uint32_t offset, uint64_t idx, uint32_t* out)
+{
+    float am = 0.0f;
+#pragma unroll
+    for (int i = 0; i < 32; ++i) am = fmaxf(am, fabsf(v[i]));
+    // floor(log2 amax) - 8 from the exponent field; subnormal or zero amax -> -127
+    const int ef = (int)((__float_as_uint(am) >> 23) & 0xFFu);
+    const int e = max(ef - 127 - 8, -127);
+    const float scale = __uint_as_float((uint32_t)(127 - e) << 23);  // 2^-e, exact
+    U4 w[4];
+    if (sr) {
+#pragma unroll
+        for (int q = 0; q < 4; ++q) w[q] = sr_block8(seed, offset, 2u, (idx >> 3) + q);
+    }
+#pragma unroll
+    for (int k = 0; k < 8; ++k) {
+        float y[4];
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+            y[i] = __fmul_rn(v[4 * k + i], scale);
+            if (sr) y[i] = e4m3_sr_value(y[i], u16_of(w[(4 * k + i) >> 3], (4 * k + i) & 7));
+        }
+        const uint32_t lo = e4m3x2_rne_sat(y[1], y[0]);
+        const uint32_t hi = e4m3x2_rne_sat(y[3], y[2]);
+        out[k] = lo | (hi << 16);
+    }
+    return (uint32_t)(e + 127);
+}
+
+__device__ __forceinline__ void store_codes32(uint8_t* dst, const uint32_t (&c)[8], bool vec16)
+{
+    if (vec16) {
+        reinterpret_cast<uint4*>(dst)[0] = make_uint4(c[0], c[1], c[2], c[3]);
+        reinterpret_cast<uint4*>(dst)[1] = make_uint4(c[4], c[5], c[6], c[7]);
+    } else {
+#pragma unroll
+        for (int i = 0; i < 4; ++i)
+            reinterpret_cast<uint2*>(dst)[i] = make_uint2(c[2 * i], c[2 * i + 1]);
+    }
+}
+
+__global__ void __launch_bounds__(kQuantThreads) quant_kernel(QArgs a)
+{
+    extern __shared__ __align__(128) uint8_t smem[];
+    uint8_t* tiles = smem;
+    uint64_t* bars = reinterpret_cast<uint64_t*>(smem + kStages * kTileBytes);
+    QShared* sh = reinterpret_cast<QShared*>(smem + kStages * kTileBytes + 64);
+
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < kStages; ++s) mbar_init(&bars[s], 1);
+        fence_barrier_init();
+    }
+    if (a.group_offsets) {
+        if (threadIdx.x == 0) {
+            sh->n_groups = a.num_groups;
+            int32_t pad = 0;
+            for (int e = 0; e <= a.num_groups; ++e) {
+                const int32_t st = a.group_offsets[e];
+                sh->group_start[e] = st;
+                sh->group_padded[e] = pad;
+                if (e < a.num_groups) {
+                    const int32_t cnt = a.group_offsets[e + 1] - st;
+                    pad += ((cnt + 127) / 128) * 128;
+                }
+            }
+        }
+    }
+    __syncthreads();
+
+    const bool nv_row = (a.outputs & NVFP4_ROWWISE) != 0;
+    const bool nv_col = (a.outputs & NVFP4_COLWISE) != 0;
+    const bool mx_row = (a.mx_outputs & NVFP4_ROWWISE) != 0;
+    const bool mx_col = (a.mx_outputs & NVFP4_COLWISE) != 0;
+    const bool sr = a.rounding == NVFP4_SR;
+    const bool mx_sr = a.mx_rounding == NVFP4_SR;
+    const bool two_d = a.scaling == NVFP4_2D16x16;
+    const bool mma_sf = a.sf_layout == NVFP4_SF_MMA;
+
+    float S_row = 1.0f, g_row = 1.0f, S_col = 1.0f, g_col = 1.0f;
+    if (nv_row || nv_col) {
+        float amax_r, amax_c;
+        if (a.amax_in) {
+            amax_r = a.amax_in[0];
+            amax_c = a.amax_in[1];
+        } else {
+            amax_r = __uint_as_float(a.amax_ws[0]);
+            amax_c = a.rht ? __uint_as_float(a.amax_ws[1]) : amax_r;
+        }
+        global_scales(amax_r, S_row, g_row);
+        global_scales(amax_c, S_col, g_col);
+        if (blockIdx.x == 0 && threadIdx.x == 0) {
+            if (nv_row) *a.g_row = g_row;
+            if (nv_col) *a.g_col = g_col;
+        }
+    }
+    const uint32_t signs = (nv_col && a.rht) ? rht_sign_bits(a.seed) : 0u;
+
+    const int64_t first = blockIdx.x;
+    const int64_t my_count =
+        first < a.n_tiles ? (a.n_tiles - first + gridDim.x - 1) / gridDim.x : 0;
+    auto tile_of = [&](int64_t k) { return a.n_tiles - 1 - (first + k * (int64_t)gridDim.x); };
+
+    if (warp == 0 && my_count > 0) issue_tile(a, tile_of(0), tiles, &bars[0], lane);
+
+    const bool q_row_vec = (a.cols % 32) == 0;
+    const bool q_col_vec = (a.rows % 32) == 0;
+    const bool sf_row_vec = mma_sf || (a.cols % 64) == 0;
+    const bool sf_col_vec = mma_sf || (a.rows % 64) == 0;
+
+    int64_t k = 0;
+    for (; k < my_count; ++k) {
+        const int stage = (int)(k & 1);
+        const uint32_t parity = (uint32_t)((k >> 1) & 1);
+        if (warp == 0 && k + 1 < my_count)
+            issue_tile(a, tile_of(k + 1), tiles + (stage ^ 1) * kTileBytes, &bars[stage ^ 1],
+                       lane);
+        const bool ok = mbar_wait(&bars[stage], parity);
+        if (__syncthreads_or(!ok)) {
+            if (threadIdx.x == 0) record_status(a.status, NVFP4_ERR_TIMEOUT);
+            break;
+        }
+        const uint8_t* T = tiles + stage * kTileBytes;
+        const int64_t tile = tile_of(k);
+        const int64_t tr = tile / a.tiles_c, tc = tile - tr * a.tiles_c;
+        const int64_t r0 = tr * kTileRows, c0 = tc * kTileCols;
+
+        // ---------------- rowwise: thread = (row, 64-column half) ----------
+        if (nv_row || mx_row) {
+            const int rl = 16 * warp + (lane & 15);
+            const int h = lane >> 4;
+            const int64_t rg = r0 + rl;
+            const bool rvalid = rg < a.rows;
+            const uint8_t* rowp = T + rl * kPitch + h * 128;
+            const int64_t cbase = c0 + 64 * h;
+            if (nv_row) {
+                uint32_t codes[8];
+                uint32_t sfw = 0;
+                bool all_valid = true;
+#pragma unroll
+                for (int blk = 0; blk < 4; ++blk) {
+                    const int64_t cg = cbase + 16 * blk;
+                    const bool valid = rvalid && cg < a.cols;
+                    all_valid &= valid;
+                    float v[16];
+                    if (valid) {
+                        unpack8(ld_shared_v4(rowp + blk * 32), v);
+                        unpack8(ld_shared_v4(rowp + blk * 32 + 16), v + 8);
+                    } else {
+#pragma unroll
+                        for (int i = 0; i < 16; ++i) v[i] = 0.0f;
+                    }
+                    float am = 0.0f;
+#pragma unroll
+                    for (int i = 0; i < 16; ++i) am = fmaxf(am, fabsf(v[i]));
+                    if (two_d) am = warp_max16(am);
+                    uint32_t cw0, cw1;
+                    const uint32_t byte = quant_block16(v, am, S_row, sr && valid, a.seed,
+                                                        a.offset, 0u,
+                                                        (uint64_t)(rg * a.cols + cg), cw0, cw1);
+                    codes[2 * blk] = cw0;
+                    codes[2 * blk + 1] = cw1;
+                    sfw |= byte << (8 * blk);
+                }
+                if (all_valid) {
+                    store_codes32(a.q_row + rg * (a.cols / 2) + cbase / 2, codes, q_row_vec);
+                    const int64_t b0 = cbase / 16;
+                    const int64_t off = mma_sf ? sf_mma_offset(padded_row(sh, a, rg), b0, a.cols / 16)
+                                               : rg * (a.cols / 16) + b0;
+                    if (sf_row_vec) {
+                        *reinterpret_cast<uint32_t*>(a.sf_row + off) = sfw;
+                    } else {
+#pragma unroll
+                        for (int blk = 0; blk < 4; ++blk) a.sf_row[off + blk] = (sfw >> (8 * blk)) & 0xFFu;
+                    }
+                } else if (rvalid) {
+#pragma unroll
+                    for (int blk = 0; blk < 4; ++blk) {
+                        const int64_t cg = cbase + 16 * blk;
+                        if (cg >= a.cols) continue;
+                        *reinterpret_cast<uint2*>(a.q_row + rg * (a.cols / 2) + cg / 2) =
+                            make_uint2(codes[2 * blk], codes[2 * blk + 1]);
+                        const int64_t off = mma_sf ? sf_mma_offset(padded_row(sh, a, rg), cg / 16, a.cols / 16)
+                                                   : rg * (a.cols / 16) + cg / 16;
+                        a.sf_row[off] = (sfw >> (8 * blk)) & 0xFFu;
+                    }
+                }
+            }
+            if (mx_row && rvalid) {
+#pragma unroll 1
+                for (int part = 0; part < 2; ++part) {
+                    const int64_t cg = cbase + 32 * part;
+                    if (cg >= a.cols) continue;
+                    float v[32];
+#pragma unroll
+                    for (int q = 0; q < 4; ++q) unpack8(ld_shared_v4(rowp + part * 64 + q * 16), v + 8 * q);
+                    uint32_t out[8];
+                    const uint32_t e8 = mx_block32(v, mx_sr, a.seed, a.offset,
+                                                   (uint64_t)(rg * a.cols + cg), out);
+                    uint4* dst = reinterpret_cast<uint4*>(a.mx_q_row + rg * a.cols + cg);
+                    dst[0] = make_uint4(out[0], out[1], out[2], out[3]);
+                    dst[1] = make_uint4(out[4], out[5], out[6], out[7]);
+                    a.mx_sf_row[rg * (a.cols / 32) + cg / 32] = (uint8_t)e8;
+                }
+            }
+        }
+
+        // ---------------- columnwise: thread = (column, 64-row half) --------
+        if (nv_col || mx_col) {
+            const int cl = 32 * (warp & 3) + lane;
+            const int hh = warp >> 2;
+            const int64_t cgl = c0 + cl;
+            const bool cvalid = cgl < a.cols;
+            const int64_t rbase = r0 + 64 * hh;
+            const uint8_t* colp = T + (64 * hh) * kPitch + cl * 2;
+            uint32_t codes[8];
+            uint32_t sfw = 0;
+            bool all_valid = true;
+#pragma unroll 1
+            for (int part = 0; part < 2; ++part) {
+                const int64_t rg0 = rbase + 32 * part;
+                float x[32];
+#pragma unroll
+                for (int i = 0; i < 32; ++i) {
+                    const bool ok = cvalid && (rg0 + i) < a.rows;
+                    x[i] = ok ? bf16_lo(ld_shared_u16(colp + (32 * part + i) * kPitch)) : 0.0f;
+                }
+                if (mx_col && cvalid && rg0 + 32 <= a.rows) {
+                    uint32_t out[8];
+                    const uint32_t e8 = mx_block32(x, mx_sr, a.seed, a.offset,
+                                                   (uint64_t)(cgl * a.rows + rg0), out);
+                    uint4* dst = reinterpret_cast<uint4*>(a.mx_q_col + cgl * a.rows + rg0);
+                    dst[0] = make_uint4(out[0], out[1], out[2], out[3]);
+                    dst[1] = make_uint4(out[4], out[5], out[6], out[7]);
+                    a.mx_sf_col[cgl * (a.rows / 32) + rg0 / 32] = (uint8_t)e8;
+                }
+                if (nv_col) {
+#pragma unroll
+                    for (int sub = 0; sub < 2; ++sub) {
+                        const int64_t rg = rg0 + 16 * sub;
+                        const bool valid = cvalid && rg < a.rows;
+                        all_valid &= valid;
+                        float v[16];
+#pragma unroll
+                        for (int i = 0; i < 16; ++i) v[i] = x[16 * sub + i];
+                        if (a.rht) rht16(v, signs);
+                        float am = 0.0f;
+#pragma unroll
+                        for (int i = 0; i < 16; ++i) am = fmaxf(am, fabsf(v[i]));
+                        if (two_d) am = warp_max16(am);
+                        uint32_t cw0, cw1;
+                        const uint32_t byte =
+                            quant_block16(v, am, S_col, sr && valid, a.seed, a.offset, 1u,
+                                          (uint64_t)(cgl * a.rows + rg), cw0, cw1);
+                        const int blk = 2 * part + sub;
+                        codes[2 * blk] = cw0;
+                        codes[2 * blk + 1] = cw1;
+                        sfw |= byte << (8 * blk);
+                    }
+                }
+            }
+            if (nv_col) {
+                if (all_valid) {
+                    store_codes32(a.q_col + cgl * (a.rows / 2) + rbase / 2, codes, q_col_vec);
+                    const int64_t b0 = rbase / 16;
+                    const int64_t off = mma_sf ? sf_mma_offset(cgl, b0, a.rows / 16)
+                                               : cgl * (a.rows / 16) + b0;
+                    if (sf_col_vec) {
+                        *reinterpret_cast<uint32_t*>(a.sf_col + off) = sfw;
+                    } else {
+#pragma unroll
+                        for (int blk = 0; blk < 4; ++blk) a.sf_col[off + blk] = (sfw >> (8 * blk)) & 0xFFu;
+                    }
+                } else if (cvalid) {
+#pragma unroll
+                    for (int blk = 0; blk < 4; ++blk) {
+                        const int64_t rg = rbase + 16 * blk;
+                        if (rg >= a.rows) continue;
+                        *reinterpret_cast<uint2*>(a.q_col + cgl * (a.rows / 2) + rg / 2) =
+                            make_uint2(codes[2 * blk], codes[2 * blk + 1]);
+                        const int64_t off = mma_sf ? sf_mma_offset(cgl, rg / 16, a.rows / 16)
+                                                   : cgl * (a.rows / 16) + rg / 16;
+                        a.sf_col[off] = (sfw >> (8 * blk)) & 0xFFu;
+                    }
+                }
+            }
+        }
+        __syncthreads();  // the stage may be refilled next iteration
+    }
+    // A copy issued for a tile this CTA did not consume (only after a timeout)
+    // must land before the CTA's shared memory goes away.
+    if (k < my_count && k + 1 < my_count && warp == 0) {
+        const int stage = (int)((k + 1) & 1);
+        (void)mbar_wait(&bars[stage], (uint32_t)(((k + 1) >> 1) & 1));
+    }
+}
+
+// --------------------------------------------------------------------------
+// Dequantisation: x_hat = (e2m1(code) * d) * g.
+// --------------------------------------------------------------------------
+__device__ __forceinline__ void e2m1x2_to_f32(uint32_t byte, float& lo, float& hi)
+{
+    uint32_t h2;
+    const uint16_t b = static_cast<uint16_t>(byte & 0xFFu);
+    asm("{\n\t.reg .b8 b0, b1;\n\tmov.b16 {b0, b1}, %1;\n\tcvt.rn.f16x2.e2m1x2 %0, b0;\n\t}"
+        : "=r"(h2)
+        : "h"(b));
+    lo = __half2float(__ushort_as_half(static_cast<unsigned short>(h2 & 0xFFFFu)));
+    hi = __half2float(__ushort_as_half(static_cast<unsigned short>(h2 >> 16)));
+}
+
+__global__ void __launch_bounds__(256) dequant_kernel(const uint8_t* q, const uint8_t* sf,
+                                                      const float* gp, int64_t rows, int64_t cols,
+                                                      int mma_sf, int bf16_out, void* out)
+{
+    const float g = *gp;
+    const int64_t nb = rows * (cols / 16);
+    for (int64_t blk = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; blk < nb;
+         blk += (int64_t)gridDim.x * blockDim.x) {
+        const int64_t r = blk / (cols / 16), b = blk - r * (cols / 16);
+        const uint2 c = *reinterpret_cast<const uint2*>(q + r * (cols / 2) + b * 8);
+        const int64_t off = mma_sf ? sf_mma_offset(r, b, cols / 16) : r * (cols / 16) + b;
+        const float d = e4m3_value(sf[off]);
+        float v[16];
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+            const uint32_t word = i < 4 ? c.x : c.y;
+            float lo, hi;
+            e2m1x2_to_f32((word >> (8 * (i & 3))) & 0xFFu, lo, hi);
+            v[2 * i] = __fmul_rn(__fmul_rn(lo, d), g);
+            v[2 * i + 1] = __fmul_rn(__fmul_rn(hi, d), g);
+        }
+        if (bf16_out) {
+            uint32_t w[8];
+#pragma unroll
+            for (int i = 0; i < 8; ++i) {
+                const __nv_bfloat162 p = __floats2bfloat162_rn(v[2 * i], v[2 * i + 1]);
+                w[i] = *reinterpret_cast<const uint32_t*>(&p);
+            }
+            uint4* dst = reinterpret_cast<uint4*>(static_cast<uint16_t*>(out) + r * cols + b * 16);
+            dst[0] = make_uint4(w[0], w[1], w[2], w[3]);
+            dst[1] = make_uint4(w[4], w[5], w[6], w[7]);
+        } else {
+            float4* dst = reinterpret_cast<float4*>(static_cast<float*>(out) + r * cols + b * 16);
+#pragma unroll
+            for (int i = 0; i < 4; ++i) dst[i] = make_float4(v[4 * i], v[4 * i + 1], v[4 * i + 2], v[4 * i + 3]);
+        }
+    }
+}
+
+// --------------------------------------------------------------------------
+// Host side.
+// --------------------------------------------------------------------------
+struct DeviceInfo {
+    int sms = 0;
+    int quant_blocks_per_sm = 0;
+    bool ok = false;
+};
+
+static size_t quant_smem_bytes() { return (size_t)kStages * kTileBytes + 64 + sizeof(QShared); }
+
+static DeviceInfo& device_info(int dev)
+{
+    static DeviceInfo infos[64];
+    static std::once_flag flags[64];
+    std::call_once(flags[dev & 63], [dev]() {
+        DeviceInfo& d = infos[dev & 63];
+        cudaDeviceProp prop;
+        if (cudaGetDeviceProperties(&prop, dev) != cudaSuccess) return;
+        if (prop.major != 10) return;
+        d.sms = prop.multiProcessorCount;
+        if (cudaFuncSetAttribute(quant_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 (int)quant_smem_bytes()) != cudaSuccess)
+            return;
+        int nb = 0;
+        if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&nb, quant_kernel, kQuantThreads,
+                                                          quant_smem_bytes()) != cudaSuccess ||
+            nb < 1)
+            return;
+        d.quant_blocks_per_sm = nb;
+        d.ok = true;
+    });
+    return infos[dev & 63];
+}
+
+static bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+constexpr size_t kQuantWorkspace = 256;
+
+}  // namespace nvfp4
+
+using namespace nvfp4;
+
+extern "C" size_t nvfp4_sf_mma_bytes(int64_t rows, int64_t k)
+{
+    if (rows <= 0 || k <= 0) return 0;
+    return (size_t)((rows + 127) / 128) * 128 * (size_t)(((k / 16) + 3) / 4) * 4;
+}
+
+extern "C" size_t nvfp4_sf_mma_grouped_bytes(int64_t total_rows, int num_groups, int64_t k)
+{
+    if (total_rows < 0 || num_groups <= 0 || k <= 0) return 0;
+    const int64_t padded = ((total_rows + 127) / 128) * 128 + 128 * (int64_t)num_groups;
+    return (size_t)padded * (size_t)(((k / 16) + 3) / 4) * 4;
+}
+
+extern "C" size_t nvfp4_quantize_workspace_size(int64_t, int64_t, const nvfp4_quant_params*)
+{
+    return kQuantWorkspace;
+}
+
+static nvfp4_status launch_quant(QArgs& a, bool need_amax, void* workspace, cudaStream_t st)
+{
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return NVFP4_ERR_CUDA;
+    DeviceInfo& info = device_info(dev);
+    if (!info.ok) return NVFP4_ERR_UNSUPPORTED;
+    a.tiles_c = (a.cols + kTileCols - 1) / kTileCols;
+    a.n_tiles = ((a.rows + kTileRows - 1) / kTileRows) * a.tiles_c;
+    if (workspace) {
+        // amax words (when computed) and the status word start at zero on every call
+        uint32_t* ws = static_cast<uint32_t*>(workspace);
+        if (cudaMemsetAsync(need_amax ? ws : ws + 2, 0, need_amax ? 12 : 4, st) != cudaSuccess)
+            return NVFP4_ERR_CUDA;
+    }
+    if (need_amax) {
+        uint32_t* amax = static_cast<uint32_t*>(workspace);
+        a.amax_ws = amax;
+        const int64_t units = (a.rows / 16) * (a.cols / 8);
+        const int64_t want = (units + 255) / 256;
+        const int blocks = (int)std::max<int64_t>(1, std::min<int64_t>(want, (int64_t)info.sms * 8));
+        amax_kernel<<<blocks, 256, 0, st>>>(a, amax);
+        if (cudaGetLastError() != cudaSuccess) return NVFP4_ERR_CUDA;
+    }
+    const int64_t grid = std::min<int64_t>(a.n_tiles, (int64_t)info.sms * info.quant_blocks_per_sm);
+    quant_kernel<<<(int)grid, kQuantThreads, quant_smem_bytes(), st>>>(a);
+    if (cudaGetLastError() != cudaSuccess) return NVFP4_ERR_CUDA;
+    return NVFP4_OK;
+}
+
+extern "C" nvfp4_status nvfp4_quantize(const void* x_bf16, int64_t rows, int64_t cols, int64_t ld,
+                                       const nvfp4_quant_params* p, uint8_t* q_row,
+                                       uint8_t* sf_row, float* g_row, uint8_t* q_col,
+                                       uint8_t* sf_col, float* g_col, void* workspace,
+                                       size_t ws_bytes, void* stream)
+{
+    if (!x_bf16 || !p) return NVFP4_ERR_INVALID_ARG;
+    if (rows <= 0 || cols <= 0 || rows % 16 || cols % 16 || ld < cols) return NVFP4_ERR_SHAPE;
+    if (!aligned16(x_bf16) || (ld * 2) % 16) return NVFP4_ERR_ALIGN;
+    if (p->rounding != NVFP4_RNE && p->rounding != NVFP4_SR) return NVFP4_ERR_INVALID_ARG;
+    if (p->mx_rounding != NVFP4_RNE && p->mx_rounding != NVFP4_SR) return NVFP4_ERR_INVALID_ARG;
+    if (p->scaling != NVFP4_1D16 && p->scaling != NVFP4_2D16x16) return NVFP4_ERR_INVALID_ARG;
+    if (p->sf_layout != NVFP4_SF_ROWMAJOR && p->sf_layout != NVFP4_SF_MMA) return NVFP4_ERR_INVALID_ARG;
+    if (p->outputs & ~3 || p->mx_outputs & ~3) return NVFP4_ERR_INVALID_ARG;
+    if (p->rht_colwise != 0 && p->rht_colwise != 1) return NVFP4_ERR_INVALID_ARG;
+    if (p->outputs == 0 && p->mx_outputs == 0) return NVFP4_ERR_INVALID_ARG;
+    const bool nv_row = p->outputs & NVFP4_ROWWISE, nv_col = p->outputs & NVFP4_COLWISE;
+    if (nv_row && (!q_row || !sf_row || !g_row)) return NVFP4_ERR_INVALID_ARG;
+    if (nv_col && (!q_col || !sf_col || !g_col)) return NVFP4_ERR_INVALID_ARG;
+    if ((nv_row && (!aligned16(q_row) || !aligned16(sf_row))) ||
+        (nv_col && (!aligned16(q_col) || !aligned16(sf_col))))
+        return NVFP4_ERR_ALIGN;
+    if (p->sf_layout == NVFP4_SF_MMA && ((nv_row && cols % 64) || (nv_col && rows % 64)))
+        return NVFP4_ERR_SHAPE;
+    if (p->mx_outputs & NVFP4_ROWWISE) {
+        if (cols % 32) return NVFP4_ERR_SHAPE;
+        if (!p->mx_q_row || !p->mx_sf_row) return NVFP4_ERR_INVALID_ARG;
+        if (!aligned16(p->mx_q_row)) return NVFP4_ERR_ALIGN;
+    }
+    if (p->mx_outputs & NVFP4_COLWISE) {
+        if (rows % 32) return NVFP4_ERR_SHAPE;
+        if (!p->mx_q_col || !p->mx_sf_col) return NVFP4_ERR_INVALID_ARG;
+        if (!aligned16(p->mx_q_col)) return NVFP4_ERR_ALIGN;
+    }
+    if (p->row_index && p->src_rows <= 0) return NVFP4_ERR_INVALID_ARG;
+    if (p->group_offsets) {
+        if (p->sf_layout != NVFP4_SF_MMA || !nv_row || p->num_groups < 1 ||
+            p->num_groups > kMaxGroups)
+            return NVFP4_ERR_INVALID_ARG;
+    }
+    const bool need_amax = (nv_row || nv_col) && !p->amax_in;
+    if (need_amax && (!workspace || ws_bytes < kQuantWorkspace)) return NVFP4_ERR_WORKSPACE;
+    if (workspace && !aligned16(workspace)) return NVFP4_ERR_ALIGN;
+
+    QArgs a{};
+    a.x = static_cast<const uint16_t*>(x_bf16);
+    a.rows = rows;
+    a.cols = cols;
+    a.ld = ld;
+    a.rounding = p->rounding;
+    a.scaling = p->scaling;
+    a.outputs = p->outputs;
+    a.rht = p->rht_colwise;
+    a.sf_layout = p->sf_layout;
+    a.seed = p->seed;
+    a.offset = p->offset;
+    a.amax_in = p->amax_in;
+    a.row_index = p->row_index;
+    a.src_rows = p->src_rows;
+    a.group_offsets = p->group_offsets;
+    a.num_groups = p->num_groups;
+    a.mx_outputs = p->mx_outputs;
+    a.mx_rounding = p->mx_rounding;
+    a.q_row = q_row;
+    a.sf_row = sf_row;
+    a.g_row = g_row;
+    a.q_col = q_col;
+    a.sf_col = sf_col;
+    a.g_col = g_col;
+    a.mx_q_row = p->mx_q_row;
+    a.mx_sf_row = p->mx_sf_row;
+    a.mx_q_col = p->mx_q_col;
+    a.mx_sf_col = p->mx_sf_col;
+    a.status = workspace ? static_cast<uint32_t*>(workspace) + 2 : nullptr;
+    return launch_quant(a, need_amax, workspace, static_cast<cudaStream_t>(stream));
+}
+
+extern "C" nvfp4_status mxfp8_quantize(const void* x_bf16, int64_t rows, int64_t cols, int64_t ld,
+                                       int directions, int rounding, uint64_t seed,
+                                       uint32_t offset, uint8_t* q_row, uint8_t* e8_row,
+                                       uint8_t* q_col, uint8_t* e8_col, void* stream)
+{
+    nvfp4_quant_params p{};
+    p.rounding = NVFP4_RNE;
+    p.mx_outputs = directions;
+    p.mx_rounding = rounding;
+    p.seed = seed;
+    p.offset = offset;
+    p.mx_q_row = q_row;
+    p.mx_sf_row = e8_row;
+    p.mx_q_col = q_col;
+    p.mx_sf_col = e8_col;
+    if (directions == 0 || (directions & ~3)) return NVFP4_ERR_INVALID_ARG;
+    return nvfp4_quantize(x_bf16, rows, cols, ld, &p, nullptr, nullptr, nullptr, nullptr, nullptr,
+                          nullptr, nullptr, 0, stream);
+}
+
+extern "C" nvfp4_status nvfp4_dequantize(const uint8_t* q, const uint8_t* sf, const float* g,
+                                         int64_t rows, int64_t cols, int sf_layout, int out_dtype,
+                                         void* out, void* stream)
+{
+    if (!q || !sf || !g || !out) return NVFP4_ERR_INVALID_ARG;
+    if (rows <= 0 || cols <= 0 || cols % 16) return NVFP4_ERR_SHAPE;
+    if (sf_layout != NVFP4_SF_ROWMAJOR && sf_layout != NVFP4_SF_MMA) return NVFP4_ERR_INVALID_ARG;
+    if (sf_layout == NVFP4_SF_MMA && cols % 64) return NVFP4_ERR_SHAPE;
+    if (out_dtype != NVFP4_OUT_F32 && out_dtype != NVFP4_OUT_BF16) return NVFP4_ERR_INVALID_ARG;
+    if ((reinterpret_cast<uintptr_t>(q) & 7u) || !aligned16(out)) return NVFP4_ERR_ALIGN;
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return NVFP4_ERR_CUDA;
+    DeviceInfo& info = device_info(dev);
+    if (!info.ok) return NVFP4_ERR_UNSUPPORTED;
+    const int64_t nb = rows * (cols / 16);
+    const int blocks = (int)std::max<int64_t>(1, std::min<int64_t>((nb + 255) / 256, (int64_t)info.sms * 8));
+    dequant_kernel<<<blocks, 256, 0, static_cast<cudaStream_t>(stream)>>>(
+        q, sf, g, rows, cols, sf_layout == NVFP4_SF_MMA, out_dtype == NVFP4_OUT_BF16, out);
+    return cudaGetLastError() == cudaSuccess ? NVFP4_OK : NVFP4_ERR_CUDA;
+}
+
+extern "C" nvfp4_status nvfp4_workspace_status(void* workspace, void* stream)
+{
+    if (!workspace) return NVFP4_ERR_INVALID_ARG;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    uint32_t v = 0;
+    uint32_t* word = static_cast<uint32_t*>(workspace) + 2;
+    if (cudaMemcpyAsync(&v, word, 4, cudaMemcpyDeviceToHost, st) != cudaSuccess) return NVFP4_ERR_CUDA;
+    if (cudaStreamSynchronize(st) != cudaSuccess) return NVFP4_ERR_CUDA;
+    if (v != 0 && cudaMemsetAsync(word, 0, 4, st) != cudaSuccess) return NVFP4_ERR_CUDA;
+    return static_cast<nvfp4_status>(v);
+}
+
+extern "C" const char* nvfp4_status_string(nvfp4_status s)
+{
+    switch (s) {
+    case NVFP4_OK: return "ok";
+    case NVFP4_ERR_INVALID_ARG: return "invalid argument";
+    case NVFP4_ERR_SHAPE: return "unsupported shape";
+    case NVFP4_ERR_ALIGN: return "pointer or leading dimension not 16-byte aligned";
+    case NVFP4_ERR_UNSUPPORTED: return "unsupported device or combination";
+    case NVFP4_ERR_CUDA: return "CUDA runtime error";
+    case NVFP4_ERR_TIMEOUT: return "device wait timed out";
+    case NVFP4_ERR_WORKSPACE: return "workspace missing or too small";
+    case NVFP4_ERR_INDEX: return "gather index out of range";
+    }
+    return "unknown status";
+}
+
+extern "C" int nvfp4_version(void) { return 100; }

@@ -36,7 +36,7 @@ class QParams(ctypes.Structure):
     _fields_ = [("rounding", ctypes.c_int), ("scaling", ctypes.c_int), ("rht", ctypes.c_int),
                 ("seed", ctypes.c_uint64), ("offset", ctypes.c_uint32),
                 ("has_amax", ctypes.c_int), ("amax_row", ctypes.c_float),
-                ("amax_col", ctypes.c_float)]
+                ("amax_col", ctypes.c_float), ("idx_base", ctypes.c_uint64)]
 
 
 def lib():
@@ -69,7 +69,9 @@ def lib():
                                          P, P, P]
         L.orc_nvfp4_quantize.restype = ctypes.c_int
         L.orc_mxfp8_quantize.argtypes = [P, i64, i64, i64, ctypes.c_int, ctypes.c_int, u64, u32,
-                                         P, P]
+                                         u64, P, P]
+        L.orc_amax.argtypes = [P, i64, i64, i64, ctypes.c_int, ctypes.c_int, u64]
+        L.orc_amax.restype = ctypes.c_float
         L.orc_mxfp8_quantize.restype = ctypes.c_int
         L.orc_nvfp4_dequant_f64.argtypes = [P, P, ctypes.c_float, i64, i64, P]
         L.orc_nvfp4_dequant_f32.argtypes = [P, P, ctypes.c_float, i64, i64, P]
@@ -146,9 +148,19 @@ def global_scale(amax: float) -> Tuple[float, float]:
 
 
 # ---------------------------------------------------------------- tensor pieces
+def amax(x_bf16: np.ndarray, direction: int, rht: int = 0, seed: int = 0) -> float:
+    """Tensor amax of one direction (over the Hadamard-rotated vectors when rht)."""
+    x = np.ascontiguousarray(x_bf16, dtype=np.uint16)
+    rows, cols = x.shape
+    v = float(lib().orc_amax(_p(x), rows, cols, cols, direction, rht, seed))
+    if v < 0:
+        raise ValueError("oracle amax: invalid arguments")
+    return v
+
+
 def nvfp4_quantize(x_bf16: np.ndarray, direction: int, rounding: int = 0, scaling: int = 0,
                    rht: int = 0, seed: int = 0, offset: int = 0,
-                   amax: Optional[Tuple[float, float]] = None):
+                   amax: Optional[Tuple[float, float]] = None, idx_base: int = 0):
     """Quantise a bf16 matrix (given as uint16 bit patterns, [rows, cols]).
 
     direction 0: rowwise -> codes [rows, cols/2], scales [rows, cols/16].
@@ -162,7 +174,8 @@ def nvfp4_quantize(x_bf16: np.ndarray, direction: int, rounding: int = 0, scalin
     sf = np.zeros((nr, nc // 16), dtype=np.uint8)
     g = np.zeros(1, dtype=np.float32)
     p = QParams(rounding, scaling, rht, seed, offset, 1 if amax is not None else 0,
-                amax[0] if amax is not None else 0.0, amax[1] if amax is not None else 0.0)
+                amax[0] if amax is not None else 0.0, amax[1] if amax is not None else 0.0,
+                idx_base)
     rc = lib().orc_nvfp4_quantize(_p(x), rows, cols, cols, direction, ctypes.byref(p), _p(q),
                                   _p(sf), _p(g))
     if rc != 0:
@@ -171,7 +184,7 @@ def nvfp4_quantize(x_bf16: np.ndarray, direction: int, rounding: int = 0, scalin
 
 
 def mxfp8_quantize(x_bf16: np.ndarray, direction: int, rounding: int = 0, seed: int = 0,
-                   offset: int = 0):
+                   offset: int = 0, idx_base: int = 0):
     """MXFP8: codes [rows, cols] + E8M0 [rows, cols/32] (direction 0) or on x^T (1)."""
     x = np.ascontiguousarray(x_bf16, dtype=np.uint16)
     rows, cols = x.shape
@@ -179,7 +192,7 @@ def mxfp8_quantize(x_bf16: np.ndarray, direction: int, rounding: int = 0, seed: 
     q = np.zeros((nr, nc), dtype=np.uint8)
     e8 = np.zeros((nr, nc // 32), dtype=np.uint8)
     rc = lib().orc_mxfp8_quantize(_p(x), rows, cols, cols, direction, rounding, seed, offset,
-                                  _p(q), _p(e8))
+                                  idx_base, _p(q), _p(e8))
     if rc != 0:
         raise ValueError("oracle mxfp8_quantize: invalid arguments")
     return q, e8

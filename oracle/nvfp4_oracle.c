@@ -279,6 +279,9 @@ typedef struct {
     uint32_t offset;
     int has_amax;    /* 1: use amax_row / amax_col instead of computing */
     float amax_row, amax_col;
+    uint64_t idx_base; /* added to every element index (Philox counter): lets a
+                          slice of a larger tensor draw the bits the full tensor
+                          would draw at those positions */
 } orc_qparams;
 
 static void quantize_matrix(const float* v, int64_t n_rows, int64_t n_cols, float amax,
@@ -319,7 +322,7 @@ static void quantize_matrix(const float* v, int64_t n_rows, int64_t n_cols, floa
                         code = orc_e2m1_rne(y);
                     else
                         code = orc_e2m1_sr(y, orc_sr_bits(p->seed, p->offset, stream,
-                                                          (uint64_t)(r * n_cols + c)));
+                                                          p->idx_base + (uint64_t)(r * n_cols + c)));
                 }
                 /* pack: even element in the low nibble */
                 int64_t byte = (r * n_cols + c) / 2;
@@ -330,6 +333,53 @@ static void quantize_matrix(const float* v, int64_t n_rows, int64_t n_cols, floa
             }
         }
     }
+}
+
+/* The matrix a direction quantises, in binary32: x (direction 0) or x^T
+ * (direction 1), with the RHT applied to each 16-vector along rows of x^T
+ * when rht is set.  Returns a malloc'd [nr, nc] array. */
+static float* direction_matrix(const uint16_t* x, int64_t rows, int64_t cols, int64_t ld,
+                               int direction, int rht, uint64_t seed)
+{
+    int64_t nr = direction ? cols : rows, nc = direction ? rows : cols;
+    float* v = (float*)malloc(sizeof(float) * (size_t)(nr * nc));
+    if (!v) return NULL;
+    for (int64_t r = 0; r < rows; ++r)
+        for (int64_t c = 0; c < cols; ++c) {
+            float xv = bf16_to_float(x[r * ld + c]);
+            if (direction)
+                v[c * rows + r] = xv;
+            else
+                v[r * cols + c] = xv;
+        }
+    if (direction && rht) {
+        float signs[16], in[16], out[16];
+        orc_rht_signs(seed, signs);
+        for (int64_t r = 0; r < nr; ++r)
+            for (int64_t b = 0; b < nc; b += 16) {
+                for (int i = 0; i < 16; ++i) in[i] = v[r * nc + b + i];
+                orc_rht16(signs, in, out);
+                for (int i = 0; i < 16; ++i) v[r * nc + b + i] = out[i];
+            }
+    }
+    return v;
+}
+
+/* Tensor amax of one direction: max |x|, or max |RHT(x)| over the columnwise
+ * vectors when rht is set. */
+float orc_amax(const uint16_t* x, int64_t rows, int64_t cols, int64_t ld, int direction, int rht,
+               uint64_t seed)
+{
+    if (rows <= 0 || cols <= 0 || rows % 16 || cols % 16 || ld < cols) return -1.0f;
+    float* v = direction_matrix(x, rows, cols, ld, direction, rht, seed);
+    if (!v) return -1.0f;
+    float amax = 0.0f;
+    for (int64_t i = 0; i < rows * cols; ++i) {
+        float a = fabsf(v[i]);
+        if (a > amax) amax = a;
+    }
+    free(v);
+    return amax;
 }
 
 /* x: bf16 [rows, ld] row-major.  direction 0 = rowwise (codes [rows, cols/2],
@@ -344,26 +394,8 @@ int orc_nvfp4_quantize(const uint16_t* x, int64_t rows, int64_t cols, int64_t ld
 {
     if (rows <= 0 || cols <= 0 || rows % 16 || cols % 16 || ld < cols) return ORC_EINVAL;
     int64_t nr = direction ? cols : rows, nc = direction ? rows : cols;
-    float* v = (float*)malloc(sizeof(float) * (size_t)(nr * nc));
+    float* v = direction_matrix(x, rows, cols, ld, direction, direction ? p->rht : 0, p->seed);
     if (!v) return ORC_EINVAL;
-    for (int64_t r = 0; r < rows; ++r)
-        for (int64_t c = 0; c < cols; ++c) {
-            float xv = bf16_to_float(x[r * ld + c]);
-            if (direction)
-                v[c * rows + r] = xv;
-            else
-                v[r * cols + c] = xv;
-        }
-    if (direction && p->rht) {
-        float signs[16], in[16], out[16];
-        orc_rht_signs(p->seed, signs);
-        for (int64_t r = 0; r < nr; ++r)
-            for (int64_t b = 0; b < nc; b += 16) {
-                for (int i = 0; i < 16; ++i) in[i] = v[r * nc + b + i];
-                orc_rht16(signs, in, out);
-                for (int i = 0; i < 16; ++i) v[r * nc + b + i] = out[i];
-            }
-    }
     float amax = 0.0f;
     if (p->has_amax) {
         amax = direction ? p->amax_col : p->amax_row;
@@ -390,7 +422,7 @@ int orc_nvfp4_quantize(const uint16_t* x, int64_t rows, int64_t cols, int64_t ld
 /* ------------------------------------------------------------------------ */
 int orc_mxfp8_quantize(const uint16_t* x, int64_t rows, int64_t cols, int64_t ld,
                        int direction, int rounding, uint64_t seed, uint32_t offset,
-                       uint8_t* q, uint8_t* e8)
+                       uint64_t idx_base, uint8_t* q, uint8_t* e8)
 {
     int64_t nr = direction ? cols : rows, nc = direction ? rows : cols;
     if (rows <= 0 || cols <= 0 || nc % 32 || ld < cols) return ORC_EINVAL;
@@ -418,7 +450,8 @@ int orc_mxfp8_quantize(const uint16_t* x, int64_t rows, int64_t cols, int64_t ld
             for (int i = 0; i < 32; ++i) {
                 double y = ldexp(vals[i], -e);
                 int64_t idx = r * nc + b * 32 + i;
-                q[idx] = rounding ? orc_e4m3_sr_sat(y, orc_sr_bits(seed, offset, 2, (uint64_t)idx))
+                q[idx] = rounding ? orc_e4m3_sr_sat(y, orc_sr_bits(seed, offset, 2,
+                                                                 idx_base + (uint64_t)idx))
                                   : orc_e4m3_rne_sat(y);
             }
         }

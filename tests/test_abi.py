@@ -1,0 +1,101 @@
+"""The C-ABI library loads, exports every function include/nvfp4.h declares, and
+rejects bad arguments on the host before any device work.  CPU only: the calls
+below fail validation before they would touch memory or a GPU."""
+import ctypes
+import os
+import re
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module")
+def nv():
+    import nvfp4_bit_precision_b200 as nv
+    return nv
+
+
+def declared_functions():
+    src = open(os.path.join(ROOT, "include", "nvfp4.h")).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    return sorted(set(re.findall(r"\b(\w+)\s*\(", src)) - {"if", "sizeof", "defined"})
+
+
+def test_exports_every_declared_function(nv):
+    names = declared_functions()
+    assert "nvfp4_quantize" in names and "nvfp4_grouped_gemm" in names
+    for n in names:
+        assert hasattr(nv._lib, n), n
+    assert set(nv.EXPORTED) <= set(names)
+
+
+def test_status_strings(nv):
+    assert nv.status_string(0) == "ok"
+    assert "timed out" in nv.status_string(6)
+    assert nv.nvfp4_version() >= 100
+
+
+def test_size_helpers(nv):
+    assert nv.nvfp4_sf_mma_bytes(128, 256) == 128 * 16
+    assert nv.nvfp4_sf_mma_bytes(130, 256) == 256 * 16
+    assert nv.nvfp4_sf_mma_grouped_bytes(300, 4, 512) == (384 + 512) * 32
+    assert nv.nvfp4_quantize_workspace_size() >= 16
+    assert nv.nvfp4_gemm_workspace_size() >= 16
+
+
+FAKE = 1 << 20  # a 16-byte aligned non-null address that validation never dereferences
+
+
+def q(nv, rows, cols, ld, p, ws=FAKE, outs=(FAKE,) * 6):
+    return nv._lib.nvfp4_quantize(FAKE, rows, cols, ld, ctypes.byref(p), *outs, ws, 256, None)
+
+
+def test_quantize_argument_errors(nv):
+    p = nv.QuantParams()
+    p.outputs = nv.NVFP4_ROWWISE
+    assert nv._lib.nvfp4_quantize(None, 16, 16, 16, ctypes.byref(p), *(FAKE,) * 6, FAKE, 256,
+                                  None) == 1
+    assert q(nv, 17, 16, 16, p) == 2                    # rows not a multiple of 16
+    assert q(nv, 16, 24, 24, p) == 2
+    assert q(nv, 16, 16, 8, p) == 2                     # ld < cols
+    assert nv._lib.nvfp4_quantize(FAKE + 2, 16, 16, 16, ctypes.byref(p), *(FAKE,) * 6, FAKE, 256,
+                                  None) == 3
+    assert q(nv, 16, 16, 20, p) == 3                    # ld * 2 not 16-byte aligned
+    p.rounding = 7
+    assert q(nv, 16, 16, 16, p) == 1
+    p.rounding = 0
+    p.sf_layout = nv.NVFP4_SF_MMA
+    assert q(nv, 16, 48, 48, p) == 2                    # tiled scales need K % 64
+    p.sf_layout = 0
+    assert q(nv, 16, 16, 16, p, ws=None) == 7           # amax needs the workspace
+    p.outputs = 0
+    assert q(nv, 16, 16, 16, p) == 1                    # nothing requested
+    p.mx_outputs = nv.NVFP4_COLWISE
+    assert q(nv, 16, 32, 32, p) == 2                    # MXFP8 columnwise needs rows % 32
+    p.mx_outputs = 0
+    p.outputs = nv.NVFP4_ROWWISE
+    p.group_offsets = FAKE
+    p.num_groups = 4
+    assert q(nv, 16, 64, 64, p) == 1                    # grouped layout needs tiled scales
+
+
+def test_gemm_argument_errors(nv):
+    L = nv._lib
+    args = (FAKE,) * 6
+    assert L.nvfp4_gemm(*args, 128, 128, 100, 0, FAKE, 128, FAKE, 256, None) == 2   # K % 256
+    assert L.nvfp4_gemm(*args, 100, 128, 256, 0, FAKE, 128, FAKE, 256, None) == 2   # M % 16
+    assert L.nvfp4_gemm(*args, 128, 128, 256, 0, FAKE, 120, FAKE, 256, None) == 2   # ldd < N
+    assert L.nvfp4_gemm(*args, 128, 128, 256, 1, FAKE, 132, FAKE, 256, None) == 3   # ldd align
+    assert L.nvfp4_gemm(*args, 128, 128, 256, 0, FAKE, 128, None, 0, None) == 7     # workspace
+    assert L.nvfp4_gemm(*args, 128, 128, 256, 5, FAKE, 128, FAKE, 256, None) == 1   # dtype
+    assert L.nvfp4_grouped_gemm(0, FAKE, 128, *args, 128, 256, 0, FAKE, FAKE, 256, None) == 1
+    assert L.nvfp4_grouped_gemm(4, FAKE, 128, *args, 100, 256, 0, FAKE, FAKE, 256, None) == 2
+
+
+def test_mxfp8_and_dequant_argument_errors(nv):
+    L = nv._lib
+    assert L.mxfp8_quantize(FAKE, 32, 32, 32, 0, 0, 0, 0, FAKE, FAKE, FAKE, FAKE, None) == 1
+    assert L.mxfp8_quantize(FAKE, 32, 48, 48, 1, 0, 0, 0, FAKE, FAKE, None, None, None) == 2
+    assert L.nvfp4_dequantize(FAKE, FAKE, FAKE, 16, 24, 0, 0, FAKE, None) == 2
+    assert L.nvfp4_dequantize(FAKE, FAKE, FAKE, 16, 32, 0, 3, FAKE, None) == 1

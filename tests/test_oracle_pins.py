@@ -492,3 +492,33 @@ def test_grouped_gemm_oracle_matches_dense(orc):
         e = 0 if i < 8 else 2
         Dd, _ = orc.nvfp4_gemm_rows(qa, sa, ga, qbs[e][0], qbs[e][1], qbs[e][2], rows_sel=[i])
         np.testing.assert_array_equal(D[s], Dd[0])
+
+
+# ------------------------------------------------------------------ sampled-parity mechanism
+def test_slices_with_amax_and_index_base_match_full(orc):
+    """A row (or column) slice quantised with the full tensor's amax and the slice's
+    element-index base reproduces that part of the full result, for SR and RHT too."""
+    rng = np.random.default_rng(17)
+    x = W.f32_to_bf16_bits(W.student_t(rng, (96, 64), 3.0, 1e-3))
+    R, C = x.shape
+    for direction, rht in ((0, 0), (1, 0), (1, 1)):
+        am = (orc.amax(x, 0), orc.amax(x, 1, rht=rht, seed=3))
+        qf, sff, gf = orc.nvfp4_quantize(x, direction, rounding=1, rht=rht, seed=3)
+        if direction == 0:
+            r0, r1 = 32, 64
+            qs, sfs, gs = orc.nvfp4_quantize(x[r0:r1], 0, rounding=1, seed=3, amax=am,
+                                             idx_base=r0 * C)
+            np.testing.assert_array_equal(qs, qf[r0:r1])
+            np.testing.assert_array_equal(sfs, sff[r0:r1])
+        else:
+            c0, c1 = 16, 48
+            qs, sfs, gs = orc.nvfp4_quantize(np.ascontiguousarray(x[:, c0:c1]), 1, rounding=1,
+                                             rht=rht, seed=3, amax=am, idx_base=c0 * R)
+            np.testing.assert_array_equal(qs, qf[c0:c1])
+            np.testing.assert_array_equal(sfs, sff[c0:c1])
+        assert gs == gf
+    q8, e8 = orc.mxfp8_quantize(x, 1, rounding=1, seed=4)
+    q8s, e8s = orc.mxfp8_quantize(np.ascontiguousarray(x[:, 32:64]), 1, rounding=1, seed=4,
+                                  idx_base=32 * R)
+    np.testing.assert_array_equal(q8s, q8[32:64])
+    np.testing.assert_array_equal(e8s, e8[32:64])
