@@ -357,6 +357,23 @@ def run_reference(args, rank, world):
     print(json.dumps(line), flush=True)
 
 
+# ----------------------------------------------------------------------------- ranks
+def max_over_ranks(times, world, device=None):
+    """Max of each timing over all ranks (the slowest replica sets the job time)."""
+    if world <= 1:
+        return [float(t) for t in times]
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([float(v) for v in times], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return [float(v) for v in t.cpu()]
+
+
+def job_tflops(flops_per_step, world, steps, ms):
+    """Whole-job throughput: every replica's GEMM FLOP over the slowest replica's time."""
+    return flops_per_step * world * steps / (ms / 1e3) / 1e12
+
+
 # ----------------------------------------------------------------------------- main
 def main():
     ap = argparse.ArgumentParser()
@@ -433,14 +450,9 @@ def main():
     barrier()
     ms_e2e = e0.elapsed_time(e1)
 
-    times = torch.tensor([ms, ms_e2e], dtype=torch.float64, device=dev)
-    if world > 1:
-        dist.all_reduce(times, op=dist.ReduceOp.MAX)
-    ms, ms_e2e = float(times[0]), float(times[1])
-
-    flops = step.flops() * world * args.steps
-    value = flops / (ms / 1e3) / 1e12
-    value_e2e = flops / (ms_e2e / 1e3) / 1e12
+    ms, ms_e2e = max_over_ranks([ms, ms_e2e], world, dev)
+    value = job_tflops(step.flops(), world, args.steps, ms)
+    value_e2e = job_tflops(step.flops(), world, args.steps, ms_e2e)
     pk = peaks()
     fp4_peak = 4.0 * pk["bf16_tflops_sustained"]
     gd = per_kernel["gemm_dense"]

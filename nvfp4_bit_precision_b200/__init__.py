@@ -22,12 +22,14 @@ from typing import Optional
 _HERE = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(_HERE, "libnvfp4.so")
 
-if not os.path.exists(LIB_PATH):
-    from . import build as _build
+from . import build as _build
+
+if _build.stale():
     try:
         _build.build()
     except Exception as exc:  # no nvcc / compile error: there is no CPU fallback
-        raise ImportError(f"{LIB_PATH} is missing and could not be built: {exc}") from exc
+        if not os.path.exists(LIB_PATH):
+            raise ImportError(f"{LIB_PATH} is missing and could not be built: {exc}") from exc
 
 _lib = ctypes.CDLL(LIB_PATH)
 

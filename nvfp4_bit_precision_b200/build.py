@@ -31,7 +31,8 @@ def _nvcc() -> str:
     return "nvcc"
 
 
-def _stale() -> bool:
+def stale() -> bool:
+    """True when the library is missing or older than a source or header."""
     if not os.path.exists(LIB):
         return True
     t = os.path.getmtime(LIB)
@@ -41,7 +42,7 @@ def _stale() -> bool:
 
 def build(force: bool = False, verbose: bool = False) -> str:
     """Compile the CUDA library if it is missing or older than its sources."""
-    if not force and not _stale():
+    if not force and not stale():
         return LIB
     tmp = LIB + f".tmp{os.getpid()}"
     cmd = [_nvcc(), *NVCC_FLAGS, "-I", INCLUDE, "-o", tmp,

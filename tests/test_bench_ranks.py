@@ -1,0 +1,48 @@
+"""The N>1 host path of bench.py: replicas report the max of their timings and the
+job throughput counts every replica's work.  Two gloo ranks on CPU."""
+import os
+import socket
+
+import pytest
+import torch.multiprocessing as mp
+
+
+def _free_port():
+    s = socket.socket()
+    s.bind(("127.0.0.1", 0))
+    port = s.getsockname()[1]
+    s.close()
+    return port
+
+
+def _rank_main(rank, world, port, out):
+    import torch.distributed as dist
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
+    dist.init_process_group("gloo", rank=rank, world_size=world)
+    import bench
+    ms = [10.0 + rank, 50.0 - 10 * rank]          # rank 0: (10, 50); rank 1: (11, 40)
+    got = bench.max_over_ranks(ms, world, "cpu")
+    out[rank] = got
+    dist.barrier()
+    dist.destroy_process_group()
+
+
+def test_max_over_ranks_gloo_world2():
+    ctx = mp.get_context("spawn")
+    mgr = ctx.Manager()
+    out = mgr.dict()
+    port = _free_port()
+    procs = [ctx.Process(target=_rank_main, args=(r, 2, port, out)) for r in range(2)]
+    for p in procs:
+        p.start()
+    for p in procs:
+        p.join(120)
+        assert p.exitcode == 0
+    assert out[0] == [11.0, 50.0] and out[1] == [11.0, 50.0]
+
+
+def test_job_throughput_counts_all_replicas():
+    import bench
+    assert bench.job_tflops(1e12, 1, 10, 1000.0) == pytest.approx(10.0)
+    assert bench.job_tflops(1e12, 4, 10, 1000.0) == pytest.approx(40.0)
+    assert bench.max_over_ranks([3.0, 4.0], 1) == [3.0, 4.0]
