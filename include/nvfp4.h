@@ -156,6 +156,37 @@ nvfp4_status nvfp4_quantize(const void* x_bf16, int64_t rows, int64_t cols, int6
                             void* workspace, size_t ws_bytes, void* stream);
 
 /*
+ * nvfp4_quantize_noalloc -- nvfp4_quantize for callers that cannot supply a
+ * workspace.  (The pages have no counterpart: this is an interface
+ * convenience, not part of the method.)
+ *
+ * Who needs it: code that may not allocate device memory at the point of the
+ * call -- for example a host framework whose GPU memory is entirely reserved
+ * by its own caching allocator, or a latency-critical path that must never
+ * reach cudaMalloc, which can synchronise the whole device.
+ *
+ * Behaviour: identical results to nvfp4_quantize.  The quantiser's scratch
+ * (the two amax words and the device status word, 12 bytes for any tensor
+ * size) lives in a 256-byte array compiled into the library; every GPU that
+ * loads the library keeps that array until the process exits.  The call
+ * allocates nothing and calls no allocating routine.
+ *  - Maximum: the scratch a call needs (nvfp4_quantize_workspace_size) must fit
+ *    in the 256-byte array, otherwise NVFP4_ERR_WORKSPACE and nothing is
+ *    launched.  Today's quantiser needs 256 bytes for every accepted shape.
+ *  - The first call on each device looks up the array's device address (with
+ *    that device current); make that first call before any stream capture.
+ *  - All calls share the one array, and each clears it before use: calls that
+ *    may overlap on the GPU (different streams, or concurrent host threads)
+ *    race on it and must be serialised by the caller.  Device-side errors land
+ *    in the array's status word, which the caller cannot read through
+ *    nvfp4_workspace_status.
+ */
+nvfp4_status nvfp4_quantize_noalloc(const void* x_bf16, int64_t rows, int64_t cols, int64_t ld,
+                                    const nvfp4_quant_params* p, uint8_t* q_row, uint8_t* sf_row,
+                                    float* g_row, uint8_t* q_col, uint8_t* sf_col, float* g_col,
+                                    void* stream);
+
+/*
  * mxfp8_quantize -- MXFP8 (iitak, "How it works" and "But"): per 32-element
  * block e = clamp(floor(log2 amax) - 8, -127, 127) (OCP MX v1.0 rule),
  * E8M0 byte e + 127 (amax 0 -> byte 0), element = E4M3 of x * 2^-e, RNE

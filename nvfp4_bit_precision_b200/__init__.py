@@ -45,7 +45,7 @@ EXPORTED = [
     "nvfp4_quantize", "nvfp4_dequantize", "mxfp8_quantize", "nvfp4_gemm", "nvfp4_grouped_gemm",
     "nvfp4_quantize_workspace_size", "nvfp4_gemm_workspace_size", "nvfp4_sf_mma_bytes",
     "nvfp4_sf_mma_grouped_bytes", "nvfp4_workspace_status", "nvfp4_status_string",
-    "nvfp4_version",
+    "nvfp4_version", "nvfp4_quantize_noalloc",
 ]
 
 
@@ -67,6 +67,8 @@ class QuantParams(ctypes.Structure):
 _P, _I64, _SZ = ctypes.c_void_p, ctypes.c_int64, ctypes.c_size_t
 _lib.nvfp4_quantize.argtypes = [_P, _I64, _I64, _I64, ctypes.POINTER(QuantParams), _P, _P, _P,
                                 _P, _P, _P, _P, _SZ, _P]
+_lib.nvfp4_quantize_noalloc.argtypes = [_P, _I64, _I64, _I64, ctypes.POINTER(QuantParams), _P,
+                                        _P, _P, _P, _P, _P, _P]
 _lib.mxfp8_quantize.argtypes = [_P, _I64, _I64, _I64, ctypes.c_int, ctypes.c_int,
                                 ctypes.c_uint64, ctypes.c_uint32, _P, _P, _P, _P, _P]
 _lib.nvfp4_dequantize.argtypes = [_P, _P, _P, _I64, _I64, ctypes.c_int, ctypes.c_int, _P, _P]
@@ -86,7 +88,7 @@ _lib.nvfp4_workspace_status.argtypes = [_P, _P]
 _lib.nvfp4_status_string.argtypes = [ctypes.c_int]
 _lib.nvfp4_status_string.restype = ctypes.c_char_p
 _lib.nvfp4_version.restype = ctypes.c_int
-for _n in ("nvfp4_quantize", "mxfp8_quantize", "nvfp4_dequantize", "nvfp4_gemm",
+for _n in ("nvfp4_quantize", "nvfp4_quantize_noalloc", "mxfp8_quantize", "nvfp4_dequantize", "nvfp4_gemm",
            "nvfp4_grouped_gemm", "nvfp4_workspace_status"):
     getattr(_lib, _n).restype = ctypes.c_int
 
@@ -129,6 +131,15 @@ def nvfp4_quantize(x, rows, cols, ld, params: QuantParams, q_row, sf_row, g_row,
     _check(_lib.nvfp4_quantize(_ptr(x), rows, cols, ld, ctypes.byref(params), _ptr(q_row),
                                _ptr(sf_row), _ptr(g_row), _ptr(q_col), _ptr(sf_col), _ptr(g_col),
                                _ptr(workspace), ws_bytes, _stream(stream)), "nvfp4_quantize")
+
+
+def nvfp4_quantize_noalloc(x, rows, cols, ld, params: QuantParams, q_row, sf_row, g_row, q_col,
+                           sf_col, g_col, stream=None) -> None:
+    """nvfp4_quantize without a workspace, for callers that cannot allocate device
+    memory; its scratch lives in an array inside the library (see include/nvfp4.h)."""
+    _check(_lib.nvfp4_quantize_noalloc(_ptr(x), rows, cols, ld, ctypes.byref(params), _ptr(q_row),
+                                       _ptr(sf_row), _ptr(g_row), _ptr(q_col), _ptr(sf_col),
+                                       _ptr(g_col), _stream(stream)), "nvfp4_quantize_noalloc")
 
 
 def mxfp8_quantize(x, rows, cols, ld, directions, rounding, seed, offset, q_row, e8_row, q_col,

@@ -758,6 +758,51 @@ extern "C" nvfp4_status nvfp4_quantize(const void* x_bf16, int64_t rows, int64_t
     return launch_quant(a, need_amax, workspace, static_cast<cudaStream_t>(stream));
 }
 
+// --------------------------------------------------------------------------
+// Allocation-free quantisation.
+//
+// Some callers cannot hand the library a workspace: code running under a host
+// framework whose device memory is fully reserved by its own caching
+// allocator, or latency-critical paths that must never reach cudaMalloc
+// (which can synchronise the whole device).  For them nvfp4_quantize_noalloc
+// keeps the quantiser's scratch (two amax words and the status word) in the
+// file-scope array below instead of a caller buffer.  Every GPU that loads
+// this library holds the array until the process exits.
+// --------------------------------------------------------------------------
+constexpr size_t kNoAllocScratchBytes = 256;
+static __device__ __align__(256) uint8_t g_noalloc_scratch[kNoAllocScratchBytes];
+
+// Device address of the array on device `dev`, looked up once per device with
+// that device current (host code only sees a stand-in symbol, never the
+// device address).
+static void* noalloc_scratch(int dev)
+{
+    static void* ptrs[64];
+    static cudaError_t errs[64];
+    static std::once_flag flags[64];
+    std::call_once(flags[dev], [dev]() {
+        errs[dev] = cudaGetSymbolAddress(&ptrs[dev], g_noalloc_scratch);
+    });
+    return errs[dev] == cudaSuccess ? ptrs[dev] : nullptr;
+}
+
+extern "C" nvfp4_status nvfp4_quantize_noalloc(const void* x_bf16, int64_t rows, int64_t cols,
+                                               int64_t ld, const nvfp4_quant_params* p,
+                                               uint8_t* q_row, uint8_t* sf_row, float* g_row,
+                                               uint8_t* q_col, uint8_t* sf_col, float* g_col,
+                                               void* stream)
+{
+    if (nvfp4_quantize_workspace_size(rows, cols, p) > kNoAllocScratchBytes)
+        return NVFP4_ERR_WORKSPACE;
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return NVFP4_ERR_CUDA;
+    if (dev < 0 || dev >= 64) return NVFP4_ERR_UNSUPPORTED;
+    void* scratch = noalloc_scratch(dev);
+    if (!scratch) return NVFP4_ERR_CUDA;
+    return nvfp4_quantize(x_bf16, rows, cols, ld, p, q_row, sf_row, g_row, q_col, sf_col, g_col,
+                          scratch, kNoAllocScratchBytes, stream);
+}
+
 extern "C" nvfp4_status mxfp8_quantize(const void* x_bf16, int64_t rows, int64_t cols, int64_t ld,
                                        int directions, int rounding, uint64_t seed,
                                        uint32_t offset, uint8_t* q_row, uint8_t* e8_row,
