@@ -8,7 +8,7 @@
 // Machines uskorila obuchenie Inkling 2 Small 4-bitnymi chislami", section
 // "Details": NVFP4 in the expert layers -> the grouped form).
 //
-// Structure (one persistent CTA per SM, 192 threads):
+// Structure (one persistent CTA per SM, 320 threads):
 //   warp 0      TMA producer: A/B tiles (128-byte swizzled, 4-bit codes packed
 //               two per byte) by cp.async.bulk.tensor, scale atoms by
 //               cp.async.bulk, into a 4-stage ring guarded by mbarriers.
@@ -16,8 +16,9 @@
 //               memory (tcgen05.cp 32x128b.warpx4) and issues 4 MMAs of
 //               128x256x64, then commits the stage back to the producer and,
 //               after the last K stage, the accumulator to the epilogue.
-//   warps 2..5  epilogue: tcgen05.ld of the 128x256 FP32 accumulator, times
-//               ga*gb, converted and stored to global memory.
+//   warps 2..9  epilogue: tcgen05.ld of the 128x256 FP32 accumulator (two
+//               warps per lane quadrant), release of the accumulator, then
+//               times ga*gb, conversion and stores to global memory.
 // Every mbarrier wait is bounded (2 s); a timeout sets the workspace status
 // word and the kernel winds down instead of hanging.
 #include <cudaTypedefs.h>
@@ -38,10 +39,13 @@ constexpr int kB_Bytes = BN * BK / 2;      // 32 KB
 constexpr int kSFA_Bytes = BM * BK / 16;   // 2 KB: 4 atoms of 512 B
 constexpr int kSFB_Bytes = BN * BK / 16;   // 4 KB: 2 row blocks x 4 atoms
 constexpr int kStageBytes = kA_Bytes + kB_Bytes + kSFA_Bytes + kSFB_Bytes;
-constexpr int kGemmThreads = 192;
-constexpr int kTmemCols = 512;             // accumulator 256 + SFA 16 + SFB 32, rounded up
-constexpr int kTmemSFA = 256;
-constexpr int kTmemSFB = 256 + 16;
+constexpr int kGemmThreads = 320;  // producer, MMA, 8 epilogue warps
+// Tensor memory: the 128x256 FP32 accumulator in columns 0..255, then one
+// 48-column scale region per pipeline stage (SFA 4 x 4 columns, SFB 4 x 8).
+constexpr int kTmemCols = 512;
+constexpr int kTmemSF = 256;
+constexpr int kTmemSFStage = 48;
+static_assert(kTmemSF + kGemmStages * kTmemSFStage <= kTmemCols, "tensor memory overflow");
 constexpr int kMaxGemmGroups = 256;
 
 struct GemmArgs {
@@ -226,7 +230,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
             mbar_init(&sh->empty[s], 1);
         }
         mbar_init(&sh->acc_full, 1);
-        mbar_init(&sh->acc_empty, 4);
+        mbar_init(&sh->acc_empty, 8);
         fence_barrier_init();
         // tile table
         const int64_t tiles_n = (a.N + BN - 1) / BN;
@@ -321,19 +325,22 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
                     uint8_t* st = smem + s * kStageBytes;
                     const uint8_t* sfa_s = st + kA_Bytes + kB_Bytes;
                     const uint8_t* sfb_s = sfa_s + kSFA_Bytes;
+                    // this stage's own scale columns: no overwrite of scales that
+                    // the previous stages' MMAs may still be reading
+                    const uint32_t t_sfa = tmem + kTmemSF + (uint32_t)s * kTmemSFStage;
+                    const uint32_t t_sfb = t_sfa + 16;
 #pragma unroll
                     for (int j = 0; j < 4; ++j) {
-                        tc_cp_sf(tmem + kTmemSFA + 4 * j, desc_sf_atom(sfa_s + j * 512));
-                        tc_cp_sf(tmem + kTmemSFB + 8 * j, desc_sf_atom(sfb_s + j * 512));
-                        tc_cp_sf(tmem + kTmemSFB + 8 * j + 4,
-                                 desc_sf_atom(sfb_s + kSFB_Bytes / 2 + j * 512));
+                        tc_cp_sf(t_sfa + 4 * j, desc_sf_atom(sfa_s + j * 512));
+                        tc_cp_sf(t_sfb + 8 * j, desc_sf_atom(sfb_s + j * 512));
+                        tc_cp_sf(t_sfb + 8 * j + 4, desc_sf_atom(sfb_s + kSFB_Bytes / 2 + j * 512));
                     }
                     const uint64_t ad = desc_sw128(st), bd = desc_sw128(st + kA_Bytes);
 #pragma unroll
                     for (int j = 0; j < 4; ++j) {
                         // +32 bytes (64 four-bit elements) along K inside the swizzled row
-                        tc_mma(tmem, ad + 2 * j, bd + 2 * j, idesc, tmem + kTmemSFA + 4 * j,
-                               tmem + kTmemSFB + 8 * j, (ks > 0 || j > 0) ? 1u : 0u);
+                        tc_mma(tmem, ad + 2 * j, bd + 2 * j, idesc, t_sfa + 4 * j, t_sfb + 8 * j,
+                               (ks > 0 || j > 0) ? 1u : 0u);
                     }
                     tc_commit(&sh->empty[s]);  // stage free once these MMAs completed
                 }
@@ -342,8 +349,13 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
             }
         }
     } else {
-        // ------------------------------------------------ epilogue (warps 2..5)
-        const int quad = warp & 3;  // TMEM lanes 32*quad .. 32*quad+31
+        // ------------------------------------------------ epilogue (warps 2..9)
+        // Two warps per TMEM lane quadrant, 128 accumulator columns each.  All
+        // of a warp's tcgen05.ld are issued before one wait, and the accumulator
+        // is handed back to the MMA thread before the conversion and stores, so
+        // the next tile's MMAs overlap this tile's stores.
+        const int quad = warp & 3;                   // TMEM lanes 32*quad .. 32*quad+31
+        const int col0 = ((warp - 2) >> 2) * (BN / 2);  // 0 or 128
         uint32_t tcount = 0;
         for (int t = blockIdx.x; t < total; t += gridDim.x, ++tcount) {
             const TileCoord c = tile_coord(a, sh, t);
@@ -353,63 +365,54 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
                 break;
             }
             tc_fence_after();
+            const uint32_t tbase = tmem + ((uint32_t)(32 * quad) << 16) + (uint32_t)col0;
+            uint32_t r[4][32];
+            TMEM_LD_32(tbase + 0, r[0]);
+            TMEM_LD_32(tbase + 32, r[1]);
+            TMEM_LD_32(tbase + 64, r[2]);
+            TMEM_LD_32(tbase + 96, r[3]);
+            tmem_ld_wait();
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&sh->acc_empty);  // accumulator drained
+
             const float alpha = __fmul_rn(a.ga[0], a.gb[c.group]);
             const int64_t row = c.row0 + 32 * quad + lane;
-            const bool row_ok = row < c.row_end;
-            const uint32_t tbase = tmem + ((uint32_t)(32 * quad) << 16);
+            if (row >= c.row_end) continue;
+            const int64_t cbase = c.n0 + col0;
             if (a.bf16_out) {
-                uint32_t packed[BN / 2];
+                uint16_t* drow = static_cast<uint16_t*>(a.D) + row * a.ldd + cbase;
 #pragma unroll
-                for (int ch = 0; ch < BN / 32; ++ch) {
-                    uint32_t r[32];
-                    TMEM_LD_32(tbase + 32 * ch, r);
-                    tmem_ld_wait();
+                for (int ch = 0; ch < 4; ++ch) {
 #pragma unroll
-                    for (int i = 0; i < 16; ++i) {
-                        const __nv_bfloat162 p = __floats2bfloat162_rn(
-                            __fmul_rn(__uint_as_float(r[2 * i]), alpha),
-                            __fmul_rn(__uint_as_float(r[2 * i + 1]), alpha));
-                        packed[16 * ch + i] = *reinterpret_cast<const uint32_t*>(&p);
-                    }
-                }
-                // accumulator drained: the next tile's MMAs may start
-                tc_fence_before();
-                __syncwarp();
-                if (lane == 0) mbar_arrive(&sh->acc_empty);
-                if (row_ok) {
-                    uint16_t* drow = static_cast<uint16_t*>(a.D) + row * a.ldd;
+                    for (int v = 0; v < 4; ++v) {
+                        uint32_t w[4];
 #pragma unroll
-                    for (int v = 0; v < BN / 8; ++v) {
-                        const int64_t col = c.n0 + 8 * v;
-                        if (col < a.N)
-                            *reinterpret_cast<uint4*>(drow + col) =
-                                make_uint4(packed[4 * v], packed[4 * v + 1], packed[4 * v + 2],
-                                           packed[4 * v + 3]);
+                        for (int i = 0; i < 4; ++i) {
+                            const __nv_bfloat162 p = __floats2bfloat162_rn(
+                                __fmul_rn(__uint_as_float(r[ch][8 * v + 2 * i]), alpha),
+                                __fmul_rn(__uint_as_float(r[ch][8 * v + 2 * i + 1]), alpha));
+                            w[i] = *reinterpret_cast<const uint32_t*>(&p);
+                        }
+                        if (cbase + 32 * ch + 8 * v < a.N)
+                            *reinterpret_cast<uint4*>(drow + 32 * ch + 8 * v) =
+                                make_uint4(w[0], w[1], w[2], w[3]);
                     }
                 }
             } else {
-#pragma unroll 1
-                for (int ch = 0; ch < BN / 32; ++ch) {
-                    uint32_t r[32];
-                    TMEM_LD_32(tbase + 32 * ch, r);
-                    tmem_ld_wait();
-                    if (row_ok) {
-                        float* drow = static_cast<float*>(a.D) + row * a.ldd;
+                float* drow = static_cast<float*>(a.D) + row * a.ldd + cbase;
 #pragma unroll
-                        for (int v = 0; v < 8; ++v) {
-                            const int64_t col = c.n0 + 32 * ch + 4 * v;
-                            if (col < a.N)
-                                *reinterpret_cast<float4*>(drow + col) =
-                                    make_float4(__fmul_rn(__uint_as_float(r[4 * v]), alpha),
-                                                __fmul_rn(__uint_as_float(r[4 * v + 1]), alpha),
-                                                __fmul_rn(__uint_as_float(r[4 * v + 2]), alpha),
-                                                __fmul_rn(__uint_as_float(r[4 * v + 3]), alpha));
-                        }
+                for (int ch = 0; ch < 4; ++ch) {
+#pragma unroll
+                    for (int v = 0; v < 8; ++v) {
+                        if (cbase + 32 * ch + 4 * v < a.N)
+                            *reinterpret_cast<float4*>(drow + 32 * ch + 4 * v) =
+                                make_float4(__fmul_rn(__uint_as_float(r[ch][4 * v]), alpha),
+                                            __fmul_rn(__uint_as_float(r[ch][4 * v + 1]), alpha),
+                                            __fmul_rn(__uint_as_float(r[ch][4 * v + 2]), alpha),
+                                            __fmul_rn(__uint_as_float(r[ch][4 * v + 3]), alpha));
                     }
                 }
-                tc_fence_before();
-                __syncwarp();
-                if (lane == 0) mbar_arrive(&sh->acc_empty);
             }
         }
     }

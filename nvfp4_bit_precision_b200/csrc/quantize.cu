@@ -133,7 +133,7 @@ __global__ void __launch_bounds__(256) amax_kernel(QArgs a, uint32_t* amax_out)
                 mr = fmaxf(mr, fabsf(v[i]));
             }
             if (a.rht) {
-                rht16(v, signs);
+                rht16_times4(v, signs);  // 4x the transform; the 1/4 is applied once below
 #pragma unroll
                 for (int i = 0; i < 16; ++i) mc = fmaxf(mc, fabsf(v[i]));
             }
@@ -156,6 +156,7 @@ __global__ void __launch_bounds__(256) amax_kernel(QArgs a, uint32_t* amax_out)
             mr = fmaxf(mr, red[0][w]);
             mc = fmaxf(mc, red[1][w]);
         }
+        mc = __fmul_rn(mc, 0.25f);  // the transform's factor 1/4 (exact)
         // non-negative floats order like their bit patterns
         atomicMax(&amax_out[0], __float_as_uint(mr));
         atomicMax(&amax_out[1], __float_as_uint(mc));
@@ -214,28 +215,39 @@ __device__ __forceinline__ void unpack8(const uint4& p, float* v)
 }
 
 // Quantise one 16-value block given its (possibly 2D-reduced) amax.
-// Returns the scale byte; writes 8 code bytes to c0/c1.
+// Returns the scale byte; writes 8 code bytes to c0/c1.  times4: v and amax_b
+// hold 4x the values (Hadamard path without its factor 1/4); the factor is
+// applied here exactly: amax_b/4 never rounds, and v*(r/4) == (v/4)*r whenever
+// r/4 is a normal float (otherwise the division is done per element).
 __device__ __forceinline__ uint32_t quant_block16(float (&v)[16], float amax_b, float S,
-                                                  bool sr, uint64_t seed, uint32_t offset,
-                                                  uint32_t stream, uint64_t idx, uint32_t& c0,
-                                                  uint32_t& c1)
+                                                  bool times4, bool sr, uint64_t seed,
+                                                  uint32_t offset, uint32_t stream, uint64_t idx,
+                                                  uint32_t& c0, uint32_t& c1)
 {
+    if (times4) amax_b = __fmul_rn(amax_b, 0.25f);
     const float s = __fmul_rn(__fdiv_rn(amax_b, 6.0f), S);
     const uint32_t byte = e4m3_rne_sat(s);
     const float d = e4m3_value(byte);
-    const float r = (d != 0.0f) ? __fdiv_rn(S, d) : 0.0f;  // d = 0: every y is +-0
+    float r = (d != 0.0f) ? __fdiv_rn(S, d) : 0.0f;  // d = 0: every y is +-0
+    if (times4) {
+        if (r >= 7.52316384526264005100e-37f) {  // 2^-120: r/4 stays normal
+            r = __fmul_rn(r, 0.25f);
+        } else {
+#pragma unroll
+            for (int i = 0; i < 16; ++i) v[i] = __fmul_rn(v[i], 0.25f);
+        }
+    }
 #pragma unroll
     for (int i = 0; i < 16; ++i) v[i] = __fmul_rn(v[i], r);
     if (sr) {
-        const U4 w0 = sr_block8(seed, offset, stream, idx >> 3);
-        const U4 w1 = sr_block8(seed, offset, stream, (idx >> 3) + 1);
-#pragma unroll
-        for (int i = 0; i < 8; ++i) v[i] = e2m1_sr_value(v[i], u16_of(w0, i));
-#pragma unroll
-        for (int i = 0; i < 8; ++i) v[8 + i] = e2m1_sr_value(v[8 + i], u16_of(w1, i));
+        // one Philox call per 16-element block: word q drives elements 4q..4q+3
+        const U4 w = sr_block16(seed, offset, stream, idx >> 4);
+        c0 = e2m1x4_sr(v + 0, w.x) | (e2m1x4_sr(v + 4, w.y) << 16);
+        c1 = e2m1x4_sr(v + 8, w.z) | (e2m1x4_sr(v + 12, w.w) << 16);
+    } else {
+        c0 = e2m1x8_rne(v);
+        c1 = e2m1x8_rne(v + 8);
     }
-    c0 = e2m1x8_rne(v);
-    c1 = e2m1x8_rne(v + 8);
     return byte;
 }
 
@@ -398,7 +410,7 @@ __global__ void __launch_bounds__(kQuantThreads) quant_kernel(QArgs a)
                     for (int i = 0; i < 16; ++i) am = fmaxf(am, fabsf(v[i]));
                     if (two_d) am = warp_max16(am);
                     uint32_t cw0, cw1;
-                    const uint32_t byte = quant_block16(v, am, S_row, sr && valid, a.seed,
+                    const uint32_t byte = quant_block16(v, am, S_row, false, sr && valid, a.seed,
                                                         a.offset, 0u,
                                                         (uint64_t)(rg * a.cols + cg), cw0, cw1);
                     codes[2 * blk] = cw0;
@@ -486,14 +498,14 @@ __global__ void __launch_bounds__(kQuantThreads) quant_kernel(QArgs a)
                         float v[16];
 #pragma unroll
                         for (int i = 0; i < 16; ++i) v[i] = x[16 * sub + i];
-                        if (a.rht) rht16(v, signs);
+                        if (a.rht) rht16_times4(v, signs);
                         float am = 0.0f;
 #pragma unroll
                         for (int i = 0; i < 16; ++i) am = fmaxf(am, fabsf(v[i]));
                         if (two_d) am = warp_max16(am);
                         uint32_t cw0, cw1;
                         const uint32_t byte =
-                            quant_block16(v, am, S_col, sr && valid, a.seed, a.offset, 1u,
+                            quant_block16(v, am, S_col, a.rht != 0, sr && valid, a.seed, a.offset, 1u,
                                           (uint64_t)(cgl * a.rows + rg), cw0, cw1);
                         const int blk = 2 * part + sub;
                         codes[2 * blk] = cw0;

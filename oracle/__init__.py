@@ -50,6 +50,8 @@ def lib():
         L.orc_philox4x32_10.argtypes = [P, P, P]
         L.orc_sr_bits.argtypes = [u64, u32, u32, u64]
         L.orc_sr_bits.restype = u16
+        L.orc_sr_bits_nvfp4.argtypes = [u64, u32, u32, u64]
+        L.orc_sr_bits_nvfp4.restype = u16
         L.orc_e2m1_decode.argtypes = [u8]
         L.orc_e2m1_decode.restype = ctypes.c_double
         L.orc_e2m1_rne.argtypes = [ctypes.c_float]
@@ -101,6 +103,10 @@ def philox4x32_10(ctr: Sequence[int], key: Sequence[int]) -> Tuple[int, int, int
 
 def sr_bits(seed: int, offset: int, stream: int, idx: int) -> int:
     return int(lib().orc_sr_bits(seed, offset, stream, idx))
+
+
+def sr_bits_nvfp4(seed: int, offset: int, stream: int, idx: int) -> int:
+    return int(lib().orc_sr_bits_nvfp4(seed, offset, stream, idx))
 
 
 def e2m1_decode(code: int) -> float:

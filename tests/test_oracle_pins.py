@@ -299,14 +299,34 @@ def test_philox_known_answers(orc):
 
 
 def test_sr_bits_mapping(orc):
-    # idx -> counter idx/8, word (idx%8)/2, half idx%2
+    # MXFP8 stream: idx -> counter idx/8, word (idx%8)/2, half idx%2
     seed, off = 0x1234_5678_9ABC_DEF0, 77
     for idx in [0, 1, 7, 8, 9, 1000003, 2 ** 40 + 5]:
         j = idx >> 3
-        w = orc.philox4x32_10([j & 0xFFFFFFFF, j >> 32, 1, off], [seed & 0xFFFFFFFF, seed >> 32])
+        w = orc.philox4x32_10([j & 0xFFFFFFFF, j >> 32, 2, off], [seed & 0xFFFFFFFF, seed >> 32])
         word = w[(idx & 7) >> 1]
         expect = (word >> 16) if idx & 1 else word & 0xFFFF
-        assert orc.sr_bits(seed, off, 1, idx) == expect
+        assert orc.sr_bits(seed, off, 2, idx) == expect
+
+
+def test_sr_bits_nvfp4_mapping(orc):
+    """NVFP4 streams: one 32-bit word per 4 elements (word (idx/4)%4 of the Philox call
+    for idx/16); element k takes v = (hi byte, lo byte) = (B2,B0), (rev B0, rev B2),
+    (B3,B1), (rev B1, rev B3) and u = 65535 - v."""
+    rev = lambda b: int(f"{b:08b}"[::-1], 2)
+    seed, off = 0xDEADBEEF_0BADF00D, 3
+    for idx in [0, 1, 2, 3, 4, 15, 16, 17, 999999, 2 ** 36 + 13]:
+        j = idx >> 4
+        w = orc.philox4x32_10([j & 0xFFFFFFFF, j >> 32, 0, off], [seed & 0xFFFFFFFF, seed >> 32])
+        word = w[(idx >> 2) & 3]
+        B = [(word >> (8 * i)) & 0xFF for i in range(4)]
+        hi, lo = [(B[2], B[0]), (rev(B[0]), rev(B[2])), (B[3], B[1]), (rev(B[1]), rev(B[3]))][idx & 3]
+        assert orc.sr_bits_nvfp4(seed, off, 0, idx) == 65535 - ((hi << 8) | lo)
+    # every element's draw is uniform: over many groups each bit is set about half the time
+    us = np.array([orc.sr_bits_nvfp4(7, 0, 1, i) for i in range(40000)])
+    for k in range(4):
+        bits = (us[k::4][:, None] >> np.arange(16)) & 1
+        assert np.all(np.abs(bits.mean(axis=0) - 0.5) < 0.03)
 
 
 # ------------------------------------------------------------------ global scale
