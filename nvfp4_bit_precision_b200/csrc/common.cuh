@@ -184,26 +184,81 @@ __device__ __forceinline__ uint32_t rht_sign_bits(uint64_t seed)
         .x;
 }
 
-// 16-point random-sign Hadamard in registers, fixed order: sign flip, then
-// butterfly stages h = 1, 2, 4, 8 with IEEE add/sub.  The transform's factor
-// 1/4 is NOT applied here: callers fold it into the scale arithmetic.  That is
-// exact -- every value the butterflies produce is a multiple of 2^-133 (sums
-// of bf16 values) or a normal float, so dividing it by 4 never rounds.
-__device__ __forceinline__ void rht16_times4(float (&v)[16], uint32_t signs)
+// --------------------------------------------------------------------------
+// Packed FP32 pairs: sm_100a's add/sub/mul .f32x2 perform two IEEE binary32
+// operations (round to nearest even) per instruction, lane by lane.
+// --------------------------------------------------------------------------
+__device__ __forceinline__ void add2(float& d0, float& d1, float a0, float a1, float b0, float b1)
+{
+    asm("{\n\t.reg .b64 a, b, d;\n\tmov.b64 a, {%2, %3};\n\tmov.b64 b, {%4, %5};\n\t"
+        "add.rn.f32x2 d, a, b;\n\tmov.b64 {%0, %1}, d;\n\t}"
+        : "=f"(d0), "=f"(d1)
+        : "f"(a0), "f"(a1), "f"(b0), "f"(b1));
+}
+
+__device__ __forceinline__ void sub2(float& d0, float& d1, float a0, float a1, float b0, float b1)
+{
+    asm("{\n\t.reg .b64 a, b, d;\n\tmov.b64 a, {%2, %3};\n\tmov.b64 b, {%4, %5};\n\t"
+        "sub.rn.f32x2 d, a, b;\n\tmov.b64 {%0, %1}, d;\n\t}"
+        : "=f"(d0), "=f"(d1)
+        : "f"(a0), "f"(a1), "f"(b0), "f"(b1));
+}
+
+__device__ __forceinline__ void mul2(float& d0, float& d1, float a0, float a1, float b0, float b1)
+{
+    asm("{\n\t.reg .b64 a, b, d;\n\tmov.b64 a, {%2, %3};\n\tmov.b64 b, {%4, %5};\n\t"
+        "mul.rn.f32x2 d, a, b;\n\tmov.b64 {%0, %1}, d;\n\t}"
+        : "=f"(d0), "=f"(d1)
+        : "f"(a0), "f"(a1), "f"(b0), "f"(b1));
+}
+
+// max(|a|, |b|, |c|) in one instruction (exact).
+__device__ __forceinline__ float absmax3(float a, float b, float c)
+{
+    float d;
+    asm("max.abs.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
+    return d;
+}
+
+// max |v_i| over 16 values, starting from m (m >= 0).
+__device__ __forceinline__ float absmax16(const float* v, float m)
 {
 #pragma unroll
-    for (int i = 0; i < 16; ++i)
-        v[i] = __uint_as_float(__float_as_uint(v[i]) ^ (((signs >> i) & 1u) << 31));
+    for (int i = 0; i < 16; i += 2) m = absmax3(m, v[i], v[i + 1]);
+    return m;
+}
+
+// Butterfly stages h = 1, 2, 4, 8 of the 16-point Hadamard (IEEE add/sub in a
+// fixed order) on two vectors at once, one per lane of the packed pairs.  The
+// random sign flip is applied by the caller when it unpacks the inputs, and
+// the transform's factor 1/4 is NOT applied: callers fold it into the scale
+// arithmetic, which is exact -- every value the butterflies produce is a
+// multiple of 2^-133 (sums of bf16 values) or a normal float, so dividing it by
+// 4 never rounds.
+__device__ __forceinline__ void hadamard16x2_times4(float (&a)[16], float (&b)[16])
+{
 #pragma unroll
     for (int h = 1; h < 16; h <<= 1) {
 #pragma unroll
         for (int i = 0; i < 16; ++i) {
             if (i & h) continue;
-            const float a = v[i], b = v[i + h];
-            v[i] = __fadd_rn(a, b);
-            v[i + h] = __fsub_rn(a, b);
+            float s0, s1, d0, d1;
+            add2(s0, s1, a[i], b[i], a[i + h], b[i + h]);
+            sub2(d0, d1, a[i], b[i], a[i + h], b[i + h]);
+            a[i] = s0;
+            b[i] = s1;
+            a[i + h] = d0;
+            b[i + h] = d1;
         }
     }
+}
+
+// bf16 pair (element 0 in the low half) -> two floats with the sign bit
+// flipped by `flip` (0 or 0x80000000).
+__device__ __forceinline__ void unpack_bf16x2(uint32_t w, uint32_t flip, float& lo, float& hi)
+{
+    lo = __uint_as_float(w * 65536u + flip);  // low bf16 into the high half; + flip == xor bit 31
+    hi = __uint_as_float((w & 0xFFFF0000u) ^ flip);
 }
 
 // --------------------------------------------------------------------------

@@ -66,6 +66,13 @@ __device__ __forceinline__ uint4 ld_global_v4(const void* p)
     return r;
 }
 
+__device__ __forceinline__ uint2 ld_global_v2(const void* p)
+{
+    uint2 r;
+    asm volatile("ld.global.nc.v2.u32 {%0,%1}, [%2];" : "=r"(r.x), "=r"(r.y) : "l"(p));
+    return r;
+}
+
 __device__ __forceinline__ uint4 ld_shared_v4(const void* p)
 {
     uint4 r;
@@ -75,10 +82,10 @@ __device__ __forceinline__ uint4 ld_shared_v4(const void* p)
     return r;
 }
 
-__device__ __forceinline__ uint32_t ld_shared_u16(const void* p)
+__device__ __forceinline__ uint32_t ld_shared_u32(const void* p)
 {
-    uint16_t r;
-    asm volatile("ld.shared.u16 %0, [%1];" : "=h"(r) : "r"(smem_addr(p)));
+    uint32_t r;
+    asm volatile("ld.shared.u32 %0, [%1];" : "=r"(r) : "r"(smem_addr(p)));
     return r;
 }
 
@@ -105,37 +112,40 @@ __device__ __forceinline__ float warp_max16(float v)
 // --------------------------------------------------------------------------
 // Pass 1: global amax.
 // --------------------------------------------------------------------------
-__global__ void __launch_bounds__(256) amax_kernel(QArgs a, uint32_t* amax_out)
+__global__ void __launch_bounds__(256, 2) amax_kernel(QArgs a, uint32_t* amax_out)
 {
     const uint32_t signs = a.rht ? rht_sign_bits(a.seed) : 0u;
     float mr = 0.0f, mc = 0.0f;
-    const int64_t ncg = a.cols / 8;
+    // unit = 16 rows x 4 columns (8-byte loads, 16 in flight per thread)
+    const int64_t ncg = a.cols / 4;
     const int64_t units = (a.rows / 16) * ncg;
     for (int64_t u = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; u < units;
          u += (int64_t)gridDim.x * blockDim.x) {
         const int64_t rb = u / ncg, cg = u - rb * ncg;
-        uint4 raw[16];
+        uint2 raw[16];
+        if (a.row_index) {
 #pragma unroll
-        for (int i = 0; i < 16; ++i) {
-            const int64_t sr = source_row(a, rb * 16 + i);
-            raw[i] = ld_global_v4(a.x + sr * a.ld + cg * 8);
+            for (int i = 0; i < 16; ++i)
+                raw[i] = ld_global_v2(a.x + source_row(a, rb * 16 + i) * a.ld + cg * 4);
+        } else {
+            const uint16_t* p = a.x + (rb * 16) * a.ld + cg * 4;
+#pragma unroll
+            for (int i = 0; i < 16; ++i) raw[i] = ld_global_v2(p + i * a.ld);
         }
+        // columns 2p and 2p+1 form one packed pair; the sign flip of row i
+        // (the Hadamard's D) is applied while unpacking -- |x| is unaffected
 #pragma unroll
-        for (int j = 0; j < 8; ++j) {
-            float v[16];
+        for (int p = 0; p < 2; ++p) {
+            float va[16], vb[16];
 #pragma unroll
             for (int i = 0; i < 16; ++i) {
-                const uint32_t w = (j >> 1) == 0 ? raw[i].x
-                                   : (j >> 1) == 1 ? raw[i].y
-                                   : (j >> 1) == 2 ? raw[i].z
-                                                   : raw[i].w;
-                v[i] = (j & 1) ? bf16_hi(w) : bf16_lo(w);
-                mr = fmaxf(mr, fabsf(v[i]));
+                const uint32_t w = p == 0 ? raw[i].x : raw[i].y;
+                unpack_bf16x2(w, ((signs >> i) & 1u) << 31, va[i], vb[i]);
             }
+            mr = absmax16(vb, absmax16(va, mr));
             if (a.rht) {
-                rht16_times4(v, signs);  // 4x the transform; the 1/4 is applied once below
-#pragma unroll
-                for (int i = 0; i < 16; ++i) mc = fmaxf(mc, fabsf(v[i]));
+                hadamard16x2_times4(va, vb);  // 4x the transform; the 1/4 is applied once below
+                mc = absmax16(vb, absmax16(va, mc));
             }
         }
     }
@@ -238,7 +248,7 @@ __device__ __forceinline__ uint32_t quant_block16(float (&v)[16], float amax_b, 
         }
     }
 #pragma unroll
-    for (int i = 0; i < 16; ++i) v[i] = __fmul_rn(v[i], r);
+    for (int i = 0; i < 16; i += 2) mul2(v[i], v[i + 1], v[i], v[i + 1], r, r);
     if (sr) {
         // one Philox call per 16-element block: word q drives elements 4q..4q+3
         const U4 w = sr_block16(seed, offset, stream, idx >> 4);
@@ -255,29 +265,32 @@ __device__ __forceinline__ uint32_t quant_block16(float (&v)[16], float amax_b, 
 __device__ __forceinline__ uint32_t mx_block32(const float* v, bool sr, uint64_t seed,
                                                uint32_t offset, uint64_t idx, uint32_t* out)
 {
-    float am = 0.0f;
-#pragma unroll
-    for (int i = 0; i < 32; ++i) am = fmaxf(am, fabsf(v[i]));
+    const float am = absmax16(v + 16, absmax16(v, 0.0f));
     // floor(log2 amax) - 8 from the exponent field; subnormal or zero amax -> -127
     const int ef = (int)((__float_as_uint(am) >> 23) & 0xFFu);
     const int e = max(ef - 127 - 8, -127);
     const float scale = __uint_as_float((uint32_t)(127 - e) << 23);  // 2^-e, exact
-    U4 w[4];
     if (sr) {
+        U4 w[4];
 #pragma unroll
         for (int q = 0; q < 4; ++q) w[q] = sr_block8(seed, offset, 2u, (idx >> 3) + q);
-    }
 #pragma unroll
-    for (int k = 0; k < 8; ++k) {
-        float y[4];
+        for (int k = 0; k < 8; ++k) {
+            float y[4];
 #pragma unroll
-        for (int i = 0; i < 4; ++i) {
-            y[i] = __fmul_rn(v[4 * k + i], scale);
-            if (sr) y[i] = e4m3_sr_value(y[i], u16_of(w[(4 * k + i) >> 3], (4 * k + i) & 7));
+            for (int i = 0; i < 4; ++i)
+                y[i] = e4m3_sr_value(__fmul_rn(v[4 * k + i], scale),
+                                     u16_of(w[(4 * k + i) >> 3], (4 * k + i) & 7));
+            out[k] = e4m3x2_rne_sat(y[1], y[0]) | (e4m3x2_rne_sat(y[3], y[2]) << 16);
         }
-        const uint32_t lo = e4m3x2_rne_sat(y[1], y[0]);
-        const uint32_t hi = e4m3x2_rne_sat(y[3], y[2]);
-        out[k] = lo | (hi << 16);
+    } else {
+#pragma unroll
+        for (int k = 0; k < 8; ++k) {
+            float y[4];
+            mul2(y[0], y[1], v[4 * k], v[4 * k + 1], scale, scale);
+            mul2(y[2], y[3], v[4 * k + 2], v[4 * k + 3], scale, scale);
+            out[k] = e4m3x2_rne_sat(y[1], y[0]) | (e4m3x2_rne_sat(y[3], y[2]) << 16);
+        }
     }
     return (uint32_t)(e + 127);
 }
@@ -294,7 +307,7 @@ __device__ __forceinline__ void store_codes32(uint8_t* dst, const uint32_t (&c)[
     }
 }
 
-__global__ void __launch_bounds__(kQuantThreads) quant_kernel(QArgs a)
+__global__ void __launch_bounds__(kQuantThreads, 2) quant_kernel(QArgs a)
 {
     extern __shared__ __align__(128) uint8_t smem[];
     uint8_t* tiles = smem;
@@ -361,7 +374,7 @@ __global__ void __launch_bounds__(kQuantThreads) quant_kernel(QArgs a)
     const bool q_row_vec = (a.cols % 32) == 0;
     const bool q_col_vec = (a.rows % 32) == 0;
     const bool sf_row_vec = mma_sf || (a.cols % 64) == 0;
-    const bool sf_col_vec = mma_sf || (a.rows % 64) == 0;
+    const bool sf_col_vec = mma_sf || (a.rows % 32) == 0;  // 2 scale bytes per column store
 
     int64_t k = 0;
     for (; k < my_count; ++k) {
@@ -405,9 +418,7 @@ __global__ void __launch_bounds__(kQuantThreads) quant_kernel(QArgs a)
 #pragma unroll
                         for (int i = 0; i < 16; ++i) v[i] = 0.0f;
                     }
-                    float am = 0.0f;
-#pragma unroll
-                    for (int i = 0; i < 16; ++i) am = fmaxf(am, fabsf(v[i]));
+                    float am = absmax16(v, 0.0f);
                     if (two_d) am = warp_max16(am);
                     uint32_t cw0, cw1;
                     const uint32_t byte = quant_block16(v, am, S_row, false, sr && valid, a.seed,
@@ -460,82 +471,106 @@ __global__ void __launch_bounds__(kQuantThreads) quant_kernel(QArgs a)
             }
         }
 
-        // ---------------- columnwise: thread = (column, 64-row half) --------
+        // ---------------- columnwise: thread = (column pair, 32-row group) --
+        // One 32-bit shared load per row gives both columns of the pair; the
+        // pair's two Hadamard transforms run in the two lanes of f32x2.
         if (nv_col || mx_col) {
-            const int cl = 32 * (warp & 3) + lane;
-            const int hh = warp >> 2;
-            const int64_t cgl = c0 + cl;
-            const bool cvalid = cgl < a.cols;
-            const int64_t rbase = r0 + 64 * hh;
-            const uint8_t* colp = T + (64 * hh) * kPitch + cl * 2;
-            uint32_t codes[8];
-            uint32_t sfw = 0;
-            bool all_valid = true;
+            const int cp = 32 * (warp & 1) + lane;  // column pair 0..63
+            const int rgrp = warp >> 1;              // 32-row group 0..3
+            const int64_t cg0 = c0 + 2 * cp;         // columns cg0, cg0 + 1
+            const bool cvalid = cg0 < a.cols;        // cols is even: the pair is whole
+            const int64_t rbase = r0 + 32 * rgrp;
+            const uint8_t* colp = T + (32 * rgrp) * kPitch + cp * 4;
+            if (mx_col && cvalid && rbase + 32 <= a.rows) {
 #pragma unroll 1
-            for (int part = 0; part < 2; ++part) {
-                const int64_t rg0 = rbase + 32 * part;
-                float x[32];
+                for (int half = 0; half < 2; ++half) {
+                    float x[32];
 #pragma unroll
-                for (int i = 0; i < 32; ++i) {
-                    const bool ok = cvalid && (rg0 + i) < a.rows;
-                    x[i] = ok ? bf16_lo(ld_shared_u16(colp + (32 * part + i) * kPitch)) : 0.0f;
-                }
-                if (mx_col && cvalid && rg0 + 32 <= a.rows) {
+                    for (int i = 0; i < 32; ++i) {
+                        const uint32_t wi = ld_shared_u32(colp + i * kPitch);
+                        x[i] = half ? bf16_hi(wi) : bf16_lo(wi);
+                    }
+                    const int64_t cg = cg0 + half;
                     uint32_t out[8];
                     const uint32_t e8 = mx_block32(x, mx_sr, a.seed, a.offset,
-                                                   (uint64_t)(cgl * a.rows + rg0), out);
-                    uint4* dst = reinterpret_cast<uint4*>(a.mx_q_col + cgl * a.rows + rg0);
+                                                   (uint64_t)(cg * a.rows + rbase), out);
+                    uint4* dst = reinterpret_cast<uint4*>(a.mx_q_col + cg * a.rows + rbase);
                     dst[0] = make_uint4(out[0], out[1], out[2], out[3]);
                     dst[1] = make_uint4(out[4], out[5], out[6], out[7]);
-                    a.mx_sf_col[cgl * (a.rows / 32) + rg0 / 32] = (uint8_t)e8;
-                }
-                if (nv_col) {
-#pragma unroll
-                    for (int sub = 0; sub < 2; ++sub) {
-                        const int64_t rg = rg0 + 16 * sub;
-                        const bool valid = cvalid && rg < a.rows;
-                        all_valid &= valid;
-                        float v[16];
-#pragma unroll
-                        for (int i = 0; i < 16; ++i) v[i] = x[16 * sub + i];
-                        if (a.rht) rht16_times4(v, signs);
-                        float am = 0.0f;
-#pragma unroll
-                        for (int i = 0; i < 16; ++i) am = fmaxf(am, fabsf(v[i]));
-                        if (two_d) am = warp_max16(am);
-                        uint32_t cw0, cw1;
-                        const uint32_t byte =
-                            quant_block16(v, am, S_col, a.rht != 0, sr && valid, a.seed, a.offset, 1u,
-                                          (uint64_t)(cgl * a.rows + rg), cw0, cw1);
-                        const int blk = 2 * part + sub;
-                        codes[2 * blk] = cw0;
-                        codes[2 * blk + 1] = cw1;
-                        sfw |= byte << (8 * blk);
-                    }
+                    a.mx_sf_col[cg * (a.rows / 32) + rbase / 32] = (uint8_t)e8;
                 }
             }
             if (nv_col) {
-                if (all_valid) {
-                    store_codes32(a.q_col + cgl * (a.rows / 2) + rbase / 2, codes, q_col_vec);
-                    const int64_t b0 = rbase / 16;
-                    const int64_t off = mma_sf ? sf_mma_offset(cgl, b0, a.rows / 16)
-                                               : cgl * (a.rows / 16) + b0;
-                    if (sf_col_vec) {
-                        *reinterpret_cast<uint32_t*>(a.sf_col + off) = sfw;
-                    } else {
+                uint32_t codes[2][4];
+                uint32_t sfw[2] = {0u, 0u};
+                bool all_valid = true;
 #pragma unroll
-                        for (int blk = 0; blk < 4; ++blk) a.sf_col[off + blk] = (sfw >> (8 * blk)) & 0xFFu;
+                for (int sub = 0; sub < 2; ++sub) {
+                    const int64_t rg = rbase + 16 * sub;
+                    const bool valid = cvalid && rg < a.rows;
+                    all_valid &= valid;
+                    float va[16], vb[16];
+#pragma unroll
+                    for (int i = 0; i < 16; ++i) {
+                        const uint32_t wi = valid ? ld_shared_u32(colp + (16 * sub + i) * kPitch) : 0u;
+                        unpack_bf16x2(wi, a.rht ? ((signs >> i) & 1u) << 31 : 0u, va[i], vb[i]);
+                    }
+                    if (a.rht) hadamard16x2_times4(va, vb);
+                    float ama = absmax16(va, 0.0f), amb = absmax16(vb, 0.0f);
+                    if (two_d) {  // 16x16 tile = 8 column pairs (lanes) x 16 rows
+                        float m = fmaxf(ama, amb);
+#pragma unroll
+                        for (int o = 1; o < 8; o <<= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+                        ama = amb = m;
+                    }
+                    uint32_t c0w, c1w;
+                    uint32_t byte = quant_block16(va, ama, S_col, a.rht != 0, sr && valid, a.seed,
+                                                  a.offset, 1u, (uint64_t)(cg0 * a.rows + rg), c0w, c1w);
+                    codes[0][2 * sub] = c0w;
+                    codes[0][2 * sub + 1] = c1w;
+                    sfw[0] |= byte << (8 * sub);
+                    byte = quant_block16(vb, amb, S_col, a.rht != 0, sr && valid, a.seed, a.offset, 1u,
+                                         (uint64_t)((cg0 + 1) * a.rows + rg), c0w, c1w);
+                    codes[1][2 * sub] = c0w;
+                    codes[1][2 * sub + 1] = c1w;
+                    sfw[1] |= byte << (8 * sub);
+                }
+                const int64_t b0 = rbase / 16;
+                if (all_valid) {
+#pragma unroll
+                    for (int half = 0; half < 2; ++half) {
+                        const int64_t cg = cg0 + half;
+                        uint8_t* dst = a.q_col + cg * (a.rows / 2) + rbase / 2;
+                        if (q_col_vec)
+                            *reinterpret_cast<uint4*>(dst) = make_uint4(codes[half][0], codes[half][1],
+                                                                        codes[half][2], codes[half][3]);
+                        else {
+                            reinterpret_cast<uint2*>(dst)[0] = make_uint2(codes[half][0], codes[half][1]);
+                            reinterpret_cast<uint2*>(dst)[1] = make_uint2(codes[half][2], codes[half][3]);
+                        }
+                        const int64_t off = mma_sf ? sf_mma_offset(cg, b0, a.rows / 16)
+                                                   : cg * (a.rows / 16) + b0;
+                        if (sf_col_vec)
+                            *reinterpret_cast<uint16_t*>(a.sf_col + off) = (uint16_t)sfw[half];
+                        else {
+                            a.sf_col[off] = sfw[half] & 0xFFu;
+                            a.sf_col[off + 1] = (sfw[half] >> 8) & 0xFFu;
+                        }
                     }
                 } else if (cvalid) {
 #pragma unroll
-                    for (int blk = 0; blk < 4; ++blk) {
-                        const int64_t rg = rbase + 16 * blk;
-                        if (rg >= a.rows) continue;
-                        *reinterpret_cast<uint2*>(a.q_col + cgl * (a.rows / 2) + rg / 2) =
-                            make_uint2(codes[2 * blk], codes[2 * blk + 1]);
-                        const int64_t off = mma_sf ? sf_mma_offset(cgl, rg / 16, a.rows / 16)
-                                                   : cgl * (a.rows / 16) + rg / 16;
-                        a.sf_col[off] = (sfw >> (8 * blk)) & 0xFFu;
+                    for (int half = 0; half < 2; ++half) {
+                        const int64_t cg = cg0 + half;
+#pragma unroll
+                        for (int sub = 0; sub < 2; ++sub) {
+                            const int64_t rg = rbase + 16 * sub;
+                            if (rg >= a.rows) continue;
+                            *reinterpret_cast<uint2*>(a.q_col + cg * (a.rows / 2) + rg / 2) =
+                                make_uint2(codes[half][2 * sub], codes[half][2 * sub + 1]);
+                            const int64_t off = mma_sf ? sf_mma_offset(cg, rg / 16, a.rows / 16)
+                                                       : cg * (a.rows / 16) + rg / 16;
+                            a.sf_col[off] = (sfw[half] >> (8 * sub)) & 0xFFu;
+                        }
                     }
                 }
             }
@@ -681,7 +716,7 @@ static nvfp4_status launch_quant(QArgs& a, bool need_amax, void* workspace, cuda
     if (need_amax) {
         uint32_t* amax = static_cast<uint32_t*>(workspace);
         a.amax_ws = amax;
-        const int64_t units = (a.rows / 16) * (a.cols / 8);
+        const int64_t units = (a.rows / 16) * (a.cols / 4);  // 16 rows x 4 columns each
         const int64_t want = (units + 255) / 256;
         const int blocks = (int)std::max<int64_t>(1, std::min<int64_t>(want, (int64_t)info.sms * 8));
         amax_kernel<<<blocks, 256, 0, st>>>(a, amax);
