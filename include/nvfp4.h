@@ -103,7 +103,7 @@ typedef struct {
     const int32_t* row_index;
     int64_t src_rows;
     /* MoE scale layout: device offsets [num_groups+1] of output rows; only with
-     * NVFP4_SF_MMA and the rowwise output.  NULL = dense. */
+     * NVFP4_SF_MMA and the rowwise output; 1 <= num_groups <= 256.  NULL = dense. */
     const int32_t* group_offsets;
     int num_groups;
     /* Optional MXFP8 copy produced in the same pass (E4M3 codes [rows, cols] /
@@ -233,7 +233,7 @@ nvfp4_status nvfp4_gemm(const uint8_t* qa, const uint8_t* sfa, const float* ga,
  * expert layers): rows [off[e], off[e+1]) of the stacked A [total_rows, K]
  * are multiplied by expert e's B_e [N, K]:
  *   D[i][j] = ga * gb[e] * sum_k a_hat_ik b_hat_e,jk.
- * group_offsets: device int32 [G+1], non-decreasing, off[0] = 0,
+ * 1 <= G <= 256.  group_offsets: device int32 [G+1], non-decreasing, off[0] = 0,
  * off[G] = total_rows.  sfa in the grouped NVFP4_SF_MMA layout (see above);
  * qb [G, N, K/2], sfb [G] consecutive NVFP4_SF_MMA blocks of N rows each,
  * gb device [G].  D [total_rows, N] row-major.  The tile schedule is computed

@@ -5,6 +5,7 @@
 // after a wall-clock limit instead of hanging the GPU.
 #pragma once
 
+#include <cudaTypedefs.h>
 #include <cuda_bf16.h>
 #include <cuda_fp16.h>
 #include <cuda_runtime.h>
@@ -104,6 +105,36 @@ __device__ __forceinline__ void bulk_copy_g2s(void* dst, const void* src, uint32
         : "memory");
 }
 
+// Two-dimensional TMA tile load (box given by the tensor map) completing on
+// `bar`.  x is the innermost coordinate in elements; x * element size must be
+// a multiple of 16 bytes.
+__device__ __forceinline__ void tma_load_2d(void* dst, const CUtensorMap* map, int32_t x, int32_t y,
+                                            uint64_t* bar)
+{
+    asm volatile(
+        "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes [%0], "
+        "[%1, {%2, %3}], [%4];" ::"r"(smem_addr(dst)),
+        "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(smem_addr(bar))
+        : "memory");
+}
+
+// cuTensorMapEncodeTiled through the runtime's driver entry point (host).
+inline PFN_cuTensorMapEncodeTiled_v12000 encode_tiled_fn()
+{
+    static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+    static bool looked = false;
+    if (!looked) {
+        void* p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) ==
+                cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+        looked = true;
+    }
+    return fn;
+}
+
 __device__ __forceinline__ void record_status(uint32_t* status, uint32_t code)
 {
     if (status) atomicCAS(status, 0u, code);
@@ -122,14 +153,15 @@ __device__ __forceinline__ U4 philox4x32_10(uint32_t c0, uint32_t c1, uint32_t c
 {
 #pragma unroll
     for (int r = 0; r < 10; ++r) {
-        const uint32_t lo0 = 0xD2511F53u * c0, hi0 = __umulhi(0xD2511F53u, c0);
-        const uint32_t lo1 = 0xCD9E8D57u * c2, hi1 = __umulhi(0xCD9E8D57u, c2);
-        const uint32_t n0 = hi1 ^ c1 ^ k0;
-        const uint32_t n2 = hi0 ^ c3 ^ k1;
+        // one 32x32 -> 64-bit product gives both halves
+        const uint64_t p0 = static_cast<uint64_t>(c0) * 0xD2511F53u;
+        const uint64_t p1 = static_cast<uint64_t>(c2) * 0xCD9E8D57u;
+        const uint32_t n0 = static_cast<uint32_t>(p1 >> 32) ^ c1 ^ k0;
+        const uint32_t n2 = static_cast<uint32_t>(p0 >> 32) ^ c3 ^ k1;
         c0 = n0;
-        c1 = lo1;
+        c1 = static_cast<uint32_t>(p1);
         c2 = n2;
-        c3 = lo0;
+        c3 = static_cast<uint32_t>(p0);
         k0 += 0x9E3779B9u;
         k1 += 0xBB67AE85u;
     }

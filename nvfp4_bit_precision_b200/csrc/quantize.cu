@@ -31,9 +31,9 @@ constexpr int kTileRows = 128;
 constexpr int kTileCols = 128;
 constexpr int kPitch = kTileCols * 2 + 16;  // bytes per staged row (+16 breaks bank aliasing)
 constexpr int kTileBytes = kTileRows * kPitch;
-constexpr int kStages = 2;
+constexpr int kStages = 3;
 constexpr int kQuantThreads = 256;
-constexpr int kMaxGroups = 1024;
+constexpr int kMaxGroups = 256;  // MoE groups per call (the grouped GEMM's limit too)
 
 struct QArgs {
     const uint16_t* x;
@@ -197,11 +197,36 @@ __device__ __forceinline__ int64_t padded_row(const QShared* sh, const QArgs& a,
     return r - sh->group_start[lo] + sh->group_padded[lo];
 }
 
-__device__ __forceinline__ void issue_tile(const QArgs& a, int64_t tile, uint8_t* buf,
-                                           uint64_t* bar, int lane)
+// Staged tile layouts.
+//  kTma (dense input): two TMA boxes of 128 rows x 64 columns (128 bytes per
+//    row) with the 128-byte swizzle -- 16-byte chunk q of a row sits at chunk
+//    q ^ (row & 7) -- so both the rowwise 16-byte reads (8 rows per quarter
+//    warp) and the columnwise 4-byte reads are bank-conflict free.
+//  rows (gather): one bulk copy per row, rows kPitch bytes apart.
+// Address of the 16-byte chunk holding columns 8q .. 8q+7 of tile row r.
+template <bool kTma>
+__device__ __forceinline__ const uint8_t* chunk_addr(const uint8_t* T, int r, int q)
+{
+    if (kTma) return T + (q >> 3) * (kTileRows * 128) + r * 128 + (((q & 7) ^ (r & 7)) << 4);
+    return T + r * kPitch + q * 16;
+}
+
+template <bool kTma>
+__device__ __forceinline__ void issue_tile(const QArgs& a, const CUtensorMap* map, int64_t tile,
+                                           uint8_t* buf, uint64_t* bar, int lane)
 {
     const int64_t tr = tile / a.tiles_c, tc = tile - tr * a.tiles_c;
     const int64_t r0 = tr * kTileRows, c0 = tc * kTileCols;
+    if (kTma) {
+        // one box per 64-column panel; rows and columns past the tensor read as 0
+        if (lane == 0) {
+            const bool second = c0 + 64 < a.cols;
+            mbar_arrive_expect_tx(bar, (second ? 2u : 1u) * kTileRows * 128u);
+            tma_load_2d(buf, map, (int32_t)c0, (int32_t)r0, bar);
+            if (second) tma_load_2d(buf + kTileRows * 128, map, (int32_t)(c0 + 64), (int32_t)r0, bar);
+        }
+        return;
+    }
     const int nrows = (int)(a.rows - r0 < kTileRows ? a.rows - r0 : kTileRows);
     const uint32_t row_bytes = (uint32_t)(a.cols - c0 < kTileCols ? a.cols - c0 : kTileCols) * 2u;
     if (lane == 0) mbar_arrive_expect_tx(bar, (uint32_t)nrows * row_bytes);
@@ -307,16 +332,24 @@ __device__ __forceinline__ void store_codes32(uint8_t* dst, const uint32_t (&c)[
     }
 }
 
-__global__ void __launch_bounds__(kQuantThreads, 2) quant_kernel(QArgs a)
+template <bool kTma>
+__global__ void __launch_bounds__(kQuantThreads, 2)
+    quant_kernel(const __grid_constant__ CUtensorMap map_x, QArgs a)
 {
-    extern __shared__ __align__(128) uint8_t smem[];
+    extern __shared__ uint8_t smem_raw[];
+    // the swizzled TMA boxes need 1024-byte alignment
+    uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                               ~uintptr_t(1023));
     uint8_t* tiles = smem;
     uint64_t* bars = reinterpret_cast<uint64_t*>(smem + kStages * kTileBytes);
     QShared* sh = reinterpret_cast<QShared*>(smem + kStages * kTileBytes + 64);
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     if (threadIdx.x == 0) {
-        for (int s = 0; s < kStages; ++s) mbar_init(&bars[s], 1);
+        for (int s = 0; s < kStages; ++s) {
+            mbar_init(&bars[s], 1);                              // full: producer + tx bytes
+            mbar_init(&bars[kStages + s], kQuantThreads / 32);  // empty: one arrival per warp
+        }
         fence_barrier_init();
     }
     if (a.group_offsets) {
@@ -369,7 +402,17 @@ __global__ void __launch_bounds__(kQuantThreads, 2) quant_kernel(QArgs a)
         first < a.n_tiles ? (a.n_tiles - first + gridDim.x - 1) / gridDim.x : 0;
     auto tile_of = [&](int64_t k) { return a.n_tiles - 1 - (first + k * (int64_t)gridDim.x); };
 
-    if (warp == 0 && my_count > 0) issue_tile(a, tile_of(0), tiles, &bars[0], lane);
+    // Stage ring: full[s] completes when tile data landed, empty[s] when all 8
+    // warps are done with it.  Warp 0 keeps two tiles in flight ahead of the
+    // tile it computes; no CTA-wide barrier, so warps drift apart freely.
+    uint64_t* full = bars;
+    uint64_t* empty = bars + kStages;
+    int64_t issued = 0;  // tiles whose copies warp 0 has issued
+    if (warp == 0) {
+        for (; issued < my_count && issued < kStages - 1; ++issued)
+            issue_tile<kTma>(a, &map_x, tile_of(issued), tiles + (issued % kStages) * kTileBytes,
+                             &full[issued % kStages], lane);
+    }
 
     const bool q_row_vec = (a.cols % 32) == 0;
     const bool q_col_vec = (a.rows % 32) == 0;
@@ -378,14 +421,22 @@ __global__ void __launch_bounds__(kQuantThreads, 2) quant_kernel(QArgs a)
 
     int64_t k = 0;
     for (; k < my_count; ++k) {
-        const int stage = (int)(k & 1);
-        const uint32_t parity = (uint32_t)((k >> 1) & 1);
-        if (warp == 0 && k + 1 < my_count)
-            issue_tile(a, tile_of(k + 1), tiles + (stage ^ 1) * kTileBytes, &bars[stage ^ 1],
-                       lane);
-        const bool ok = mbar_wait(&bars[stage], parity);
-        if (__syncthreads_or(!ok)) {
-            if (threadIdx.x == 0) record_status(a.status, NVFP4_ERR_TIMEOUT);
+        const int stage = (int)(k % kStages);
+        if (warp == 0 && issued < my_count) {
+            // refill the stage tile `issued - kStages` used, once every warp released it
+            const int s = (int)(issued % kStages);
+            bool ok = true;
+            if (issued >= kStages)
+                ok = mbar_wait(&empty[s], (uint32_t)((issued / kStages - 1) & 1));
+            if (!ok) {
+                if (lane == 0) record_status(a.status, NVFP4_ERR_TIMEOUT);
+                break;
+            }
+            issue_tile<kTma>(a, &map_x, tile_of(issued), tiles + s * kTileBytes, &full[s], lane);
+            ++issued;
+        }
+        if (!mbar_wait(&full[stage], (uint32_t)((k / kStages) & 1))) {
+            if (lane == 0) record_status(a.status, NVFP4_ERR_TIMEOUT);
             break;
         }
         const uint8_t* T = tiles + stage * kTileBytes;
@@ -399,8 +450,11 @@ __global__ void __launch_bounds__(kQuantThreads, 2) quant_kernel(QArgs a)
             const int h = lane >> 4;
             const int64_t rg = r0 + rl;
             const bool rvalid = rg < a.rows;
-            const uint8_t* rowp = T + rl * kPitch + h * 128;
             const int64_t cbase = c0 + 64 * h;
+            // Shared-memory reads are unconditional: positions past the tensor
+            // hold zeros (TMA) or stale bytes (gather), and blocks made of them
+            // are never stored; 1D blocks and 16x16 tiles never mix valid and
+            // invalid elements because rows and cols are multiples of 16.
             if (nv_row) {
                 uint32_t codes[8];
                 uint32_t sfw = 0;
@@ -411,13 +465,8 @@ __global__ void __launch_bounds__(kQuantThreads, 2) quant_kernel(QArgs a)
                     const bool valid = rvalid && cg < a.cols;
                     all_valid &= valid;
                     float v[16];
-                    if (valid) {
-                        unpack8(ld_shared_v4(rowp + blk * 32), v);
-                        unpack8(ld_shared_v4(rowp + blk * 32 + 16), v + 8);
-                    } else {
-#pragma unroll
-                        for (int i = 0; i < 16; ++i) v[i] = 0.0f;
-                    }
+                    unpack8(ld_shared_v4(chunk_addr<kTma>(T, rl, 8 * h + 2 * blk)), v);
+                    unpack8(ld_shared_v4(chunk_addr<kTma>(T, rl, 8 * h + 2 * blk + 1)), v + 8);
                     float am = absmax16(v, 0.0f);
                     if (two_d) am = warp_max16(am);
                     uint32_t cw0, cw1;
@@ -459,7 +508,8 @@ __global__ void __launch_bounds__(kQuantThreads, 2) quant_kernel(QArgs a)
                     if (cg >= a.cols) continue;
                     float v[32];
 #pragma unroll
-                    for (int q = 0; q < 4; ++q) unpack8(ld_shared_v4(rowp + part * 64 + q * 16), v + 8 * q);
+                    for (int q = 0; q < 4; ++q)
+                        unpack8(ld_shared_v4(chunk_addr<kTma>(T, rl, 8 * h + 4 * part + q)), v + 8 * q);
                     uint32_t out[8];
                     const uint32_t e8 = mx_block32(v, mx_sr, a.seed, a.offset,
                                                    (uint64_t)(rg * a.cols + cg), out);
@@ -480,14 +530,17 @@ __global__ void __launch_bounds__(kQuantThreads, 2) quant_kernel(QArgs a)
             const int64_t cg0 = c0 + 2 * cp;         // columns cg0, cg0 + 1
             const bool cvalid = cg0 < a.cols;        // cols is even: the pair is whole
             const int64_t rbase = r0 + 32 * rgrp;
-            const uint8_t* colp = T + (32 * rgrp) * kPitch + cp * 4;
+            // the pair's 4 bytes: chunk cp/4 of each row, byte 4*(cp%4) within it
+            auto pair_word = [&](int i) -> uint32_t {
+                return ld_shared_u32(chunk_addr<kTma>(T, 32 * rgrp + i, cp >> 2) + 4 * (cp & 3));
+            };
             if (mx_col && cvalid && rbase + 32 <= a.rows) {
 #pragma unroll 1
                 for (int half = 0; half < 2; ++half) {
                     float x[32];
 #pragma unroll
                     for (int i = 0; i < 32; ++i) {
-                        const uint32_t wi = ld_shared_u32(colp + i * kPitch);
+                        const uint32_t wi = pair_word(i);
                         x[i] = half ? bf16_hi(wi) : bf16_lo(wi);
                     }
                     const int64_t cg = cg0 + half;
@@ -511,10 +564,9 @@ __global__ void __launch_bounds__(kQuantThreads, 2) quant_kernel(QArgs a)
                     all_valid &= valid;
                     float va[16], vb[16];
 #pragma unroll
-                    for (int i = 0; i < 16; ++i) {
-                        const uint32_t wi = valid ? ld_shared_u32(colp + (16 * sub + i) * kPitch) : 0u;
-                        unpack_bf16x2(wi, a.rht ? ((signs >> i) & 1u) << 31 : 0u, va[i], vb[i]);
-                    }
+                    for (int i = 0; i < 16; ++i)
+                        unpack_bf16x2(pair_word(16 * sub + i), a.rht ? ((signs >> i) & 1u) << 31 : 0u,
+                                      va[i], vb[i]);
                     if (a.rht) hadamard16x2_times4(va, vb);
                     float ama = absmax16(va, 0.0f), amb = absmax16(vb, 0.0f);
                     if (two_d) {  // 16x16 tile = 8 column pairs (lanes) x 16 rows
@@ -575,13 +627,14 @@ __global__ void __launch_bounds__(kQuantThreads, 2) quant_kernel(QArgs a)
                 }
             }
         }
-        __syncthreads();  // the stage may be refilled next iteration
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&empty[stage]);  // this warp is done with the stage
     }
-    // A copy issued for a tile this CTA did not consume (only after a timeout)
+    // Copies issued for tiles this CTA did not consume (only after a timeout)
     // must land before the CTA's shared memory goes away.
-    if (k < my_count && k + 1 < my_count && warp == 0) {
-        const int stage = (int)((k + 1) & 1);
-        (void)mbar_wait(&bars[stage], (uint32_t)(((k + 1) >> 1) & 1));
+    if (warp == 0) {
+        for (int64_t j = k + 1; j < issued; ++j)
+            (void)mbar_wait(&full[j % kStages], (uint32_t)((j / kStages) & 1));
     }
 }
 
@@ -647,7 +700,25 @@ struct DeviceInfo {
     bool ok = false;
 };
 
-static size_t quant_smem_bytes() { return (size_t)kStages * kTileBytes + 64 + sizeof(QShared); }
+static size_t quant_smem_bytes()
+{
+    return (size_t)kStages * kTileBytes + 64 + sizeof(QShared) + 1024;  // + alignment slack
+}
+
+// Tensor map of the bf16 input for the TMA tile path: boxes of 128 rows x 64
+// columns (128 bytes) with the 128-byte swizzle.
+static bool make_input_map(CUtensorMap* m, const void* x, int64_t rows, int64_t cols, int64_t ld)
+{
+    auto fn = encode_tiled_fn();
+    if (!fn) return false;
+    cuuint64_t dims[2] = {(cuuint64_t)cols, (cuuint64_t)rows};
+    cuuint64_t strides[1] = {(cuuint64_t)(ld * 2)};
+    cuuint32_t box[2] = {64u, (cuuint32_t)kTileRows};
+    cuuint32_t estr[2] = {1u, 1u};
+    return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(x), dims, strides, box, estr,
+              CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+              CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
 
 static DeviceInfo& device_info(int dev)
 {
@@ -659,15 +730,19 @@ static DeviceInfo& device_info(int dev)
         if (cudaGetDeviceProperties(&prop, dev) != cudaSuccess) return;
         if (prop.major != 10) return;
         d.sms = prop.multiProcessorCount;
-        if (cudaFuncSetAttribute(quant_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+        if (cudaFuncSetAttribute(quant_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 (int)quant_smem_bytes()) != cudaSuccess ||
+            cudaFuncSetAttribute(quant_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                  (int)quant_smem_bytes()) != cudaSuccess)
             return;
-        int nb = 0;
-        if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&nb, quant_kernel, kQuantThreads,
+        int nb = 0, nb2 = 0;
+        if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&nb, quant_kernel<true>, kQuantThreads,
                                                           quant_smem_bytes()) != cudaSuccess ||
-            nb < 1)
+            cudaOccupancyMaxActiveBlocksPerMultiprocessor(&nb2, quant_kernel<false>, kQuantThreads,
+                                                          quant_smem_bytes()) != cudaSuccess ||
+            std::min(nb, nb2) < 1)
             return;
-        d.quant_blocks_per_sm = nb;
+        d.quant_blocks_per_sm = std::min(nb, nb2);
         d.ok = true;
     });
     return infos[dev & 63];
@@ -723,7 +798,14 @@ static nvfp4_status launch_quant(QArgs& a, bool need_amax, void* workspace, cuda
         if (cudaGetLastError() != cudaSuccess) return NVFP4_ERR_CUDA;
     }
     const int64_t grid = std::min<int64_t>(a.n_tiles, (int64_t)info.sms * info.quant_blocks_per_sm);
-    quant_kernel<<<(int)grid, kQuantThreads, quant_smem_bytes(), st>>>(a);
+    CUtensorMap map;
+    memset(&map, 0, sizeof(map));
+    if (!a.row_index) {  // dense input: TMA tiles; the gather reads rows one by one
+        if (!make_input_map(&map, a.x, a.rows, a.cols, a.ld)) return NVFP4_ERR_CUDA;
+        quant_kernel<true><<<(int)grid, kQuantThreads, quant_smem_bytes(), st>>>(map, a);
+    } else {
+        quant_kernel<false><<<(int)grid, kQuantThreads, quant_smem_bytes(), st>>>(map, a);
+    }
     if (cudaGetLastError() != cudaSuccess) return NVFP4_ERR_CUDA;
     return NVFP4_OK;
 }
