@@ -7,8 +7,9 @@ One step = one pass of every hot-path operation over one batch of synthetic inpu
     forward GEMM Y = X W^T, quantise dY (rowwise SR, columnwise Hadamard + SR, MXFP8
     columnwise), dgrad dX = dY W, wgrad dW = dY^T X;
   MoE expert forward (64 experts, hidden 4096, FFN 1536, 16384 tokens, top-4 routing with
-    Zipf(1.1)-skewed counts): gather + activation quantise into the grouped layout,
-    grouped GEMM up, requantise the up output, grouped GEMM down.
+    Zipf(1.1)-skewed counts): quantise the tokens once, dispatch the quantised rows into
+    the grouped layout, grouped GEMM up (its epilogue also returns max |H|), requantise
+    the up output with that amax, grouped GEMM down.
 
 value = GEMM FLOP of the step / device time of the step (TFLOP/s), over all ranks.
 Multi-GPU: independent replicas (weak scaling); the only collectives are the barrier
@@ -22,7 +23,6 @@ import argparse
 import json
 import os
 import statistics
-import subprocess
 import sys
 import time
 
@@ -69,14 +69,16 @@ class Step:
         bf = dict(dtype=torch.bfloat16, device=dev)
         T, H, F = TOKENS, HIDDEN, FFN
         # inputs (device copies; the e2e loop refreshes them from pinned host memory)
-        self.x = torch.empty((T, H), **bf)
-        self.w = torch.empty((F, H), **bf)
-        self.dy = torch.empty((T, F), **bf)
-        self.tok = torch.empty((MOE_TOKENS, MOE_HIDDEN), **bf)
+        # Two input slots, so the end-to-end loop can copy step i+1's inputs
+        # while step i computes; the device-timed loop uses slot 0 only.
+        self.inputs = [dict(x=torch.empty((T, H), **bf), w=torch.empty((F, H), **bf),
+                            dy=torch.empty((T, F), **bf),
+                            tok=torch.empty((MOE_TOKENS, MOE_HIDDEN), **bf)) for _ in range(2)]
         self.row_token = torch.from_numpy(h["row_token"].astype(np.int32)).to(dev)
         self.offsets = torch.from_numpy(h["offsets"].astype(np.int32)).to(dev)
         self.routed = int(h["offsets"][-1])
-        self.upload_inputs()
+        self.upload_inputs(0)
+        self.upload_inputs(1)
         sfm = nv.nvfp4_sf_mma_bytes
         mk = lambda r, k: nv.NVFP4Tensor(torch.empty((r, k // 2), **u8),
                                          torch.zeros(sfm(r, k), **u8), torch.empty(1, **f32),
@@ -93,9 +95,12 @@ class Step:
         # MoE: expert weights are quantised once (outside the step), activations every step
         R = self.routed
         gsf = nv.nvfp4_sf_mma_grouped_bytes
+        self.Tq = mk(MOE_TOKENS, MOE_HIDDEN)  # tokens, quantised once before dispatch
+        # the dispatched rows share the tokens' global scale
         self.A_up = nv.NVFP4Tensor(torch.empty((R, MOE_HIDDEN // 2), **u8),
                                    torch.zeros(gsf(R, EXPERTS, MOE_HIDDEN), **u8),
-                                   torch.empty(1, **f32), R, MOE_HIDDEN, nv.NVFP4_SF_MMA)
+                                   self.Tq.g, R, MOE_HIDDEN, nv.NVFP4_SF_MMA)
+        self.h_amax = torch.zeros(2, **f32)  # [0] = max |H| from the up GEMM's epilogue
         self.Hup = torch.empty((R, MOE_FFN), **bf)
         self.A_dn = nv.NVFP4Tensor(torch.empty((R, MOE_FFN // 2), **u8),
                                    torch.zeros(gsf(R, EXPERTS, MOE_FFN), **u8),
@@ -119,18 +124,18 @@ class Step:
                               None, None, None, self.ws[0], 256)
         return q, sf, g
 
-    def upload_inputs(self, non_blocking=False):
+    def upload_inputs(self, slot, non_blocking=False):
         torch = self.torch
-        for name, dst in (("x", self.x), ("w", self.w), ("dy", self.dy), ("tok", self.tok)):
+        for name, dst in self.inputs[slot].items():
             src = self.h["pinned"][name] if "pinned" in self.h else torch.from_numpy(
                 self.h[name].view(np.int16))
             dst.view(torch.int16).copy_(src, non_blocking=non_blocking)
 
     def h2d_bytes(self):
-        return sum(t.numel() * t.element_size() for t in (self.x, self.w, self.dy, self.tok))
+        return sum(t.numel() * t.element_size() for t in self.inputs[0].values())
 
     def _q(self, x, rows, cols, ld, out_row, out_col, ws, rounding=0, scaling=0, rht=0,
-           mx_col=None, row_index=None, src_rows=0, groups=False):
+           mx_col=None, row_index=None, src_rows=0, groups=False, amax=None):
         nv = self.nv
         p = nv.QuantParams()
         p.rounding, p.scaling, p.rht_colwise, p.sf_layout = rounding, scaling, rht, nv.NVFP4_SF_MMA
@@ -144,6 +149,8 @@ class Step:
             p.row_index, p.src_rows = row_index.data_ptr(), src_rows
         if groups:
             p.group_offsets, p.num_groups = self.offsets.data_ptr(), EXPERTS
+        if amax is not None:
+            p.amax_in = amax.data_ptr()
         r, c = out_row, out_col
         nv.nvfp4_quantize(x, rows, cols, ld, p, r.q if r else None, r.sf if r else None,
                           r.g if r else None, c.q if c else None, c.sf if c else None,
@@ -152,10 +159,11 @@ class Step:
     def _g(self, A, B, D, ws):
         nv = self.nv
         nv.nvfp4_gemm(A.q, A.sf, A.g, B.q, B.sf, B.g, A.rows, B.rows, A.k, nv.NVFP4_OUT_BF16, D,
-                      D.stride(0), ws, 256)
+                      D.stride(0), None, ws, 256)
 
-    def run(self, ev=None):
-        """Enqueue one step.  ev: optional dict name -> list of (start, end) event pairs."""
+    def run(self, ev=None, slot=0):
+        """Enqueue one step on the inputs of `slot`.  ev: optional dict name -> list of
+        (start, end) event pairs."""
         nv, torch = self.nv, self.torch
         T, H, F = TOKENS, HIDDEN, FFN
 
@@ -170,38 +178,49 @@ class Step:
             ev.setdefault(name, []).append((s, e))
 
         ws = self.ws
-        timed("quant_x", lambda: self._q(self.x, T, H, H, self.Xr, self.Xc, ws[0], rht=1))
-        timed("quant_w", lambda: self._q(self.w, F, H, H, self.Wr, self.Wc, ws[1], scaling=1))
+        inp = self.inputs[slot]
+        timed("quant_x", lambda: self._q(inp["x"], T, H, H, self.Xr, self.Xc, ws[0], rht=1))
+        timed("quant_w", lambda: self._q(inp["w"], F, H, H, self.Wr, self.Wc, ws[1], scaling=1))
         timed("gemm_dense", lambda: self._g(self.Xr, self.Wr, self.Y, ws[2]))
-        timed("quant_dy", lambda: self._q(self.dy, T, F, F, self.Dr, self.Dc, ws[3], rounding=1,
+        timed("quant_dy", lambda: self._q(inp["dy"], T, F, F, self.Dr, self.Dc, ws[3], rounding=1,
                                           rht=1, mx_col=(self.mx_q, self.mx_e)))
         timed("gemm_dense", lambda: self._g(self.Dr, self.Wc, self.dX, ws[4]))
         timed("gemm_dense", lambda: self._g(self.Dc, self.Xc, self.dW, ws[5]))
         # MoE expert forward
         R = self.routed
-        timed("quant_act", lambda: self._q(self.tok, R, MOE_HIDDEN, MOE_HIDDEN, self.A_up, None,
-                                           ws[6], row_index=self.row_token, src_rows=MOE_TOKENS,
-                                           groups=True))
+        timed("quant_tok", lambda: self._q(inp["tok"], MOE_TOKENS, MOE_HIDDEN, MOE_HIDDEN, self.Tq,
+                                           None, ws[6]))
+        timed("dispatch", lambda: nv.nvfp4_gather_rows(
+            self.Tq.q, self.Tq.sf, MOE_TOKENS, MOE_HIDDEN, self.row_token, R, self.offsets,
+            EXPERTS, self.A_up.q, self.A_up.sf, ws[6], 256))
         qu, su, gu = self.wup
         timed("gemm_grouped", lambda: nv.nvfp4_grouped_gemm(
             EXPERTS, self.offsets, R, self.A_up.q, self.A_up.sf, self.A_up.g, qu, su, gu,
-            MOE_FFN, MOE_HIDDEN, nv.NVFP4_OUT_BF16, self.Hup, ws[7], 256))
-        timed("quant_act", lambda: self._q(self.Hup, R, MOE_FFN, MOE_FFN, self.A_dn, None,
-                                           ws[6], groups=True))
+            MOE_FFN, MOE_HIDDEN, nv.NVFP4_OUT_BF16, self.Hup, self.h_amax, ws[7], 256))
+        timed("quant_h", lambda: self._q(self.Hup, R, MOE_FFN, MOE_FFN, self.A_dn, None,
+                                         ws[6], groups=True, amax=self.h_amax))
         qd, sd, gd = self.wdn
         timed("gemm_grouped", lambda: nv.nvfp4_grouped_gemm(
             EXPERTS, self.offsets, R, self.A_dn.q, self.A_dn.sf, self.A_dn.g, qd, sd, gd,
-            MOE_HIDDEN, MOE_FFN, nv.NVFP4_OUT_BF16, self.Out, ws[7], 256))
+            MOE_HIDDEN, MOE_FFN, nv.NVFP4_OUT_BF16, self.Out, None, ws[7], 256))
 
-    LAUNCHES_PER_STEP = 15  # 5 quantise calls x (amax + fused pass) + 3 dense + 2 grouped GEMMs
+    # dense: 3 quantise calls x (amax + fused pass) + 3 GEMMs; MoE: token quantise (amax +
+    # fused pass), dispatch, 2 grouped GEMMs, H quantise (fused pass only: amax from the GEMM)
+    LAUNCHES_PER_STEP = 15
 
     def flops(self):
         return DENSE_FLOP + 2 * 2 * self.routed * MOE_FFN * MOE_HIDDEN
 
-    def results_d2h(self):
-        """Read a slice of every output back (the step's result)."""
+    def results_d2h(self, host_bufs):
+        """Copy a slice of every output (the step's result) into pinned host buffers,
+        asynchronously on the current stream; returns the bytes copied."""
         outs = [self.Y[0, :2048], self.dX[0, :2048], self.dW[0, :2048], self.Out[0, :2048]]
-        return [o.cpu() for o in outs], sum(o.numel() * o.element_size() for o in outs)
+        for h, o in zip(host_bufs, outs):
+            h.copy_(o, non_blocking=True)
+        return sum(o.numel() * o.element_size() for o in outs)
+
+    def result_host_buffers(self):
+        return [self.torch.empty(2048, dtype=self.torch.bfloat16).pin_memory() for _ in range(4)]
 
     def check_status(self):
         for w in self.ws:
@@ -230,55 +249,82 @@ def host_inputs(seed_dense=4, seed_moe=3):
 
 # ----------------------------------------------------------------------------- clocks
 class ClockSampler:
-    def __init__(self, index):
-        self.proc = None
-        self.index = index
-        self.path = os.path.join(ROOT, "gpurun_out", f"clocks_bench_{os.getpid()}.csv")
+    """SM clock and clock-event reasons sampled every 5 ms by NVML (read-only queries)
+    on a host thread while the timed region runs; `nvidia-smi` starts too slowly for a
+    region of a few hundred milliseconds."""
+    REASONS = (("hw_slowdown", "nvmlClocksEventReasonHwSlowdown", 0x8),
+               ("hw_thermal_slowdown", "nvmlClocksEventReasonHwThermalSlowdown", 0x40),
+               ("sw_thermal_slowdown", "nvmlClocksEventReasonSwThermalSlowdown", 0x20),
+               ("sw_power_cap", "nvmlClocksEventReasonSwPowerCap", 0x4))
+
+    def __init__(self, device):
+        self.device = device
+        self.samples = []
+        self.max_mhz = None
+        self.handle = None
+        self.nvml = None
+        self.thread = None
+        self.stop = None
+
+    def _open(self):
+        import pynvml as N
+        N.nvmlInit()
+        self.nvml = N
+        try:
+            import torch
+            p = torch.cuda.get_device_properties(self.device)
+            bus = f"{p.pci_domain_id:08X}:{p.pci_bus_id:02X}:{p.pci_device_id:02X}.0"
+            self.handle = N.nvmlDeviceGetHandleByPciBusId(bus)
+        except Exception:
+            self.handle = N.nvmlDeviceGetHandleByIndex(int(getattr(self.device, "index", 0) or 0))
+        self.max_mhz = N.nvmlDeviceGetMaxClockInfo(self.handle, N.NVML_CLOCK_SM)
+
+    def _run(self):
+        N = self.nvml
+        get_reasons = getattr(N, "nvmlDeviceGetCurrentClocksEventReasons",
+                              getattr(N, "nvmlDeviceGetCurrentClocksThrottleReasons", None))
+        while not self.stop.is_set():
+            try:
+                mhz = N.nvmlDeviceGetClockInfo(self.handle, N.NVML_CLOCK_SM)
+                bits = get_reasons(self.handle) if get_reasons else 0
+                self.samples.append((mhz, bits))
+            except Exception:
+                pass
+            self.stop.wait(0.005)
 
     def __enter__(self):
-        os.makedirs(os.path.dirname(self.path), exist_ok=True)
+        import threading
         try:
-            self.f = open(self.path, "w")
-            self.proc = subprocess.Popen(
-                ["nvidia-smi", "-i", str(self.index), "--query-gpu=index,clocks.sm,clocks.max.sm,"
-                 "power.draw,clocks_event_reasons.active,clocks_event_reasons.hw_slowdown,"
-                 "clocks_event_reasons.hw_thermal_slowdown,clocks_event_reasons.sw_thermal_slowdown,"
-                 "clocks_event_reasons.sw_power_cap", "--format=csv,noheader,nounits", "-lms", "50"],
-                stdout=self.f, stderr=subprocess.DEVNULL)
+            self._open()
         except Exception:
-            self.proc = None
+            self.handle = None
+            return self
+        self.stop = threading.Event()
+        self.thread = threading.Thread(target=self._run, daemon=True)
+        self.thread.start()
         return self
 
     def __exit__(self, *a):
-        if self.proc is not None:
-            self.proc.terminate()
+        if self.thread is not None:
+            self.stop.set()
+            self.thread.join(timeout=5)
+        if self.nvml is not None:
             try:
-                self.proc.wait(timeout=5)
+                self.nvml.nvmlShutdown()
             except Exception:
-                self.proc.kill()
-            self.f.close()
+                pass
 
     def summary(self):
-        if self.proc is None or not os.path.exists(self.path):
-            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unsampled"]}
-        sm, mx, reasons = [], [], set()
-        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
-        for line in open(self.path):
-            parts = [p.strip() for p in line.split(",")]
-            if len(parts) < 9:
-                continue
-            try:
-                sm.append(float(parts[1]))
-                mx.append(float(parts[2]))
-            except ValueError:
-                continue
-            for n, v in zip(names, parts[5:9]):
-                if v.lower().startswith("active"):
-                    reasons.add(n)
-        if not sm:
-            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unsampled"]}
-        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": max(mx), "reasons": sorted(reasons),
-                "samples": len(sm)}
+        if not self.samples:
+            return {"sm_mhz": None, "sm_max_mhz": self.max_mhz, "reasons": ["unsampled"]}
+        reasons = set()
+        for _, bits in self.samples:
+            for name, attr, default in self.REASONS:
+                if bits & getattr(self.nvml, attr, default):
+                    reasons.add(name)
+        return {"sm_mhz": statistics.median(m for m, _ in self.samples),
+                "sm_max_mhz": self.max_mhz, "reasons": sorted(reasons),
+                "samples": len(self.samples), "source": "nvml, 5 ms"}
 
 
 # ----------------------------------------------------------------------------- CPU oracle
@@ -319,7 +365,8 @@ def oracle_sample(budget_s=12.0):
        3 * TOKENS / 2)
     routed = MOE_TOKENS * TOPK
     acts = W.f32_to_bf16_bits(W.normal(rng, (32, MOE_HIDDEN)))
-    tq(0, 0, 0, lambda: orc.nvfp4_quantize(acts, 0, amax=am), routed / 32)
+    # the tokens are quantised once, then dispatched
+    tq(0, 0, 0, lambda: orc.nvfp4_quantize(acts, 0, amax=am), MOE_TOKENS / 32)
     tq(0, 0, 0, lambda: orc.nvfp4_quantize(
         W.f32_to_bf16_bits(W.normal(rng, (32, MOE_FFN))), 0, amax=am), routed / 32)
     # grouped GEMMs: per routed row the work equals one dense row of N x K
@@ -420,7 +467,7 @@ def main():
     ev = {}
     barrier()
     torch.cuda.synchronize()
-    with ClockSampler(local) as clk:
+    with ClockSampler(dev) as clk:
         t0 = torch.cuda.Event(enable_timing=True)
         t1 = torch.cuda.Event(enable_timing=True)
         t0.record(stream)
@@ -437,14 +484,33 @@ def main():
     # ---------------- end to end: pinned host inputs -> device, results -> host
     barrier()
     torch.cuda.synchronize()
+    # Step i+1's inputs are copied (from pinned host memory, on a copy stream) while
+    # step i computes; every step copies its own inputs and reads its results back.
     e0 = torch.cuda.Event(enable_timing=True)
     e1 = torch.cuda.Event(enable_timing=True)
+    copy_stream = torch.cuda.Stream(device=dev)
+    landed = [torch.cuda.Event(), torch.cuda.Event()]   # slot's inputs copied
+    consumed = [torch.cuda.Event(), torch.cuda.Event()]  # slot's step done with its inputs
+    host_out = [step.result_host_buffers() for _ in range(2)]
     e0.record(stream)
+    copy_stream.wait_event(e0)
+    with torch.cuda.stream(copy_stream):
+        step.upload_inputs(0, non_blocking=True)
+    landed[0].record(copy_stream)
     d2h = 0
-    for _ in range(args.steps):
-        step.upload_inputs(non_blocking=True)
-        step.run()
-        _, d2h = step.results_d2h()
+    for i in range(args.steps):
+        slot = i % 2
+        if i + 1 < args.steps:
+            nxt = 1 - slot
+            if i >= 1:
+                copy_stream.wait_event(consumed[nxt])
+            with torch.cuda.stream(copy_stream):
+                step.upload_inputs(nxt, non_blocking=True)
+            landed[nxt].record(copy_stream)
+        stream.wait_event(landed[slot])
+        step.run(slot=slot)
+        consumed[slot].record(stream)
+        d2h = step.results_d2h(host_out[slot])
     e1.record(stream)
     torch.cuda.synchronize()
     barrier()

@@ -201,6 +201,24 @@ nvfp4_status mxfp8_quantize(const void* x_bf16, int64_t rows, int64_t cols, int6
                             void* stream);
 
 /*
+ * nvfp4_gather_rows -- MoE dispatch of quantised rows (iitak, "Details" and
+ * "But": tokens travel to the expert layers, where NVFP4 is used).  Output row
+ * i is source row row_index[i]: its codes [k/2 bytes] and its scale bytes,
+ * moved from the dense NVFP4_SF_MMA layout of a [src_rows, k] operand into the
+ * grouped NVFP4_SF_MMA layout of group_offsets (device [num_groups+1],
+ * 1 <= num_groups <= 256), or into the dense layout when group_offsets is NULL.
+ * Quantising the tokens once and gathering gives the same bytes as quantising
+ * the gathered rows whenever every token is routed at least once (the global
+ * scale then comes from the same amax).  k a multiple of 64; q_src, q_dst
+ * 16-byte aligned, scale pointers 4-byte aligned.  Out-of-range indices are
+ * reported in the workspace status word (optional workspace).
+ */
+nvfp4_status nvfp4_gather_rows(const uint8_t* q_src, const uint8_t* sf_src, int64_t src_rows,
+                               int64_t k, const int32_t* row_index, int64_t rows,
+                               const int32_t* group_offsets, int num_groups, uint8_t* q_dst,
+                               uint8_t* sf_dst, void* workspace, size_t ws_bytes, void* stream);
+
+/*
  * nvfp4_dequantize -- x_hat = (e2m1(code) * d) * g, the first product exact,
  * one FP32 rounding, then (for NVFP4_OUT_BF16) RNE to bf16.
  * q [rows, cols/2], sf in sf_layout, g device [1]; out [rows, cols].
@@ -220,13 +238,16 @@ size_t nvfp4_gemm_workspace_size(int64_t M, int64_t N, int64_t K);
  * with FP32 accumulation.  "TN": A [M, K] and B [N, K] are both K-contiguous
  * codes (qa [M, K/2], qb [N, K/2]); scales sfa / sfb in NVFP4_SF_MMA layout;
  * ga, gb device FP32 [1].  D [M, ldd] FP32 or bf16 (RNE), row-major.
+ * amax_out: optional device FP32 [1]; the call sets it to max |D| over the
+ * stored values (after rounding to the output type), so the next NVFP4
+ * quantisation of D can take it as amax_in and skip its amax pass.
  * Shapes: K a multiple of 256 (one pipeline stage), M and N multiples of 16;
  * ldd >= N with ldd * element size a multiple of 16 bytes.
  */
 nvfp4_status nvfp4_gemm(const uint8_t* qa, const uint8_t* sfa, const float* ga,
                         const uint8_t* qb, const uint8_t* sfb, const float* gb, int64_t M,
                         int64_t N, int64_t K, int out_dtype, void* D, int64_t ldd,
-                        void* workspace, size_t ws_bytes, void* stream);
+                        float* amax_out, void* workspace, size_t ws_bytes, void* stream);
 
 /*
  * nvfp4_grouped_gemm -- MoE grouped form (iitak, "Details": NVFP4 in the
@@ -236,14 +257,15 @@ nvfp4_status nvfp4_gemm(const uint8_t* qa, const uint8_t* sfa, const float* ga,
  * 1 <= G <= 256.  group_offsets: device int32 [G+1], non-decreasing, off[0] = 0,
  * off[G] = total_rows.  sfa in the grouped NVFP4_SF_MMA layout (see above);
  * qb [G, N, K/2], sfb [G] consecutive NVFP4_SF_MMA blocks of N rows each,
- * gb device [G].  D [total_rows, N] row-major.  The tile schedule is computed
- * on the device from group_offsets: the host never reads the offsets.
+ * gb device [G].  D [total_rows, N] row-major; amax_out as for nvfp4_gemm.
+ * The tile schedule is computed on the device from group_offsets: the host
+ * never reads the offsets.
  */
 nvfp4_status nvfp4_grouped_gemm(int G, const int32_t* group_offsets, int64_t total_rows,
                                 const uint8_t* qa, const uint8_t* sfa, const float* ga,
                                 const uint8_t* qb, const uint8_t* sfb, const float* gb,
-                                int64_t N, int64_t K, int out_dtype, void* D, void* workspace,
-                                size_t ws_bytes, void* stream);
+                                int64_t N, int64_t K, int out_dtype, void* D, float* amax_out,
+                                void* workspace, size_t ws_bytes, void* stream);
 
 /* Synchronise `stream` and return the device status word of a workspace
  * (NVFP4_OK, NVFP4_ERR_TIMEOUT or NVFP4_ERR_INDEX); clears it. */

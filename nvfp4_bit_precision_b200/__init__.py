@@ -45,7 +45,7 @@ EXPORTED = [
     "nvfp4_quantize", "nvfp4_dequantize", "mxfp8_quantize", "nvfp4_gemm", "nvfp4_grouped_gemm",
     "nvfp4_quantize_workspace_size", "nvfp4_gemm_workspace_size", "nvfp4_sf_mma_bytes",
     "nvfp4_sf_mma_grouped_bytes", "nvfp4_workspace_status", "nvfp4_status_string",
-    "nvfp4_version", "nvfp4_quantize_noalloc",
+    "nvfp4_version", "nvfp4_quantize_noalloc", "nvfp4_gather_rows",
 ]
 
 
@@ -73,9 +73,11 @@ _lib.mxfp8_quantize.argtypes = [_P, _I64, _I64, _I64, ctypes.c_int, ctypes.c_int
                                 ctypes.c_uint64, ctypes.c_uint32, _P, _P, _P, _P, _P]
 _lib.nvfp4_dequantize.argtypes = [_P, _P, _P, _I64, _I64, ctypes.c_int, ctypes.c_int, _P, _P]
 _lib.nvfp4_gemm.argtypes = [_P, _P, _P, _P, _P, _P, _I64, _I64, _I64, ctypes.c_int, _P, _I64, _P,
-                            _SZ, _P]
+                            _P, _SZ, _P]
 _lib.nvfp4_grouped_gemm.argtypes = [ctypes.c_int, _P, _I64, _P, _P, _P, _P, _P, _P, _I64, _I64,
-                                    ctypes.c_int, _P, _P, _SZ, _P]
+                                    ctypes.c_int, _P, _P, _P, _SZ, _P]
+_lib.nvfp4_gather_rows.argtypes = [_P, _P, _I64, _I64, _P, _I64, _P, ctypes.c_int, _P, _P, _P,
+                                   _SZ, _P]
 _lib.nvfp4_quantize_workspace_size.argtypes = [_I64, _I64, ctypes.POINTER(QuantParams)]
 _lib.nvfp4_quantize_workspace_size.restype = _SZ
 _lib.nvfp4_gemm_workspace_size.argtypes = [_I64, _I64, _I64]
@@ -89,7 +91,7 @@ _lib.nvfp4_status_string.argtypes = [ctypes.c_int]
 _lib.nvfp4_status_string.restype = ctypes.c_char_p
 _lib.nvfp4_version.restype = ctypes.c_int
 for _n in ("nvfp4_quantize", "nvfp4_quantize_noalloc", "mxfp8_quantize", "nvfp4_dequantize", "nvfp4_gemm",
-           "nvfp4_grouped_gemm", "nvfp4_workspace_status"):
+           "nvfp4_grouped_gemm", "nvfp4_gather_rows", "nvfp4_workspace_status"):
     getattr(_lib, _n).restype = ctypes.c_int
 
 
@@ -154,19 +156,29 @@ def nvfp4_dequantize(q, sf, g, rows, cols, sf_layout, out_dtype, out, stream=Non
                                  _ptr(out), _stream(stream)), "nvfp4_dequantize")
 
 
-def nvfp4_gemm(qa, sfa, ga, qb, sfb, gb, M, N, K, out_dtype, D, ldd, workspace, ws_bytes,
-               stream=None) -> None:
+def nvfp4_gemm(qa, sfa, ga, qb, sfb, gb, M, N, K, out_dtype, D, ldd, amax_out, workspace,
+               ws_bytes, stream=None) -> None:
     _check(_lib.nvfp4_gemm(_ptr(qa), _ptr(sfa), _ptr(ga), _ptr(qb), _ptr(sfb), _ptr(gb), M, N, K,
-                           out_dtype, _ptr(D), ldd, _ptr(workspace), ws_bytes, _stream(stream)),
+                           out_dtype, _ptr(D), ldd, _ptr(amax_out), _ptr(workspace), ws_bytes,
+                           _stream(stream)),
            "nvfp4_gemm")
 
 
 def nvfp4_grouped_gemm(G, group_offsets, total_rows, qa, sfa, ga, qb, sfb, gb, N, K, out_dtype, D,
-                       workspace, ws_bytes, stream=None) -> None:
+                       amax_out, workspace, ws_bytes, stream=None) -> None:
     _check(_lib.nvfp4_grouped_gemm(G, _ptr(group_offsets), total_rows, _ptr(qa), _ptr(sfa),
                                    _ptr(ga), _ptr(qb), _ptr(sfb), _ptr(gb), N, K, out_dtype,
-                                   _ptr(D), _ptr(workspace), ws_bytes, _stream(stream)),
+                                   _ptr(D), _ptr(amax_out), _ptr(workspace), ws_bytes,
+                                   _stream(stream)),
            "nvfp4_grouped_gemm")
+
+
+def nvfp4_gather_rows(q_src, sf_src, src_rows, k, row_index, rows, group_offsets, num_groups,
+                      q_dst, sf_dst, workspace, ws_bytes, stream=None) -> None:
+    _check(_lib.nvfp4_gather_rows(_ptr(q_src), _ptr(sf_src), src_rows, k, _ptr(row_index), rows,
+                                  _ptr(group_offsets), num_groups, _ptr(q_dst), _ptr(sf_dst),
+                                  _ptr(workspace), ws_bytes, _stream(stream)),
+           "nvfp4_gather_rows")
 
 
 def nvfp4_workspace_status(workspace, stream=None) -> int:
@@ -297,8 +309,9 @@ def dequantize(t: NVFP4Tensor, out_dtype: int = NVFP4_OUT_F32, stream=None):
 
 
 def gemm(a: NVFP4Tensor, b: NVFP4Tensor, out_dtype: int = NVFP4_OUT_BF16, out=None,
-         workspace=None, stream=None):
-    """D = A B^T for NVFP4 operands A [M, K] and B [N, K] (tiled scale layout)."""
+         amax_out=None, workspace=None, stream=None):
+    """D = A B^T for NVFP4 operands A [M, K] and B [N, K] (tiled scale layout).
+    ``amax_out`` (optional device f32 [1]) receives max |D| as stored."""
     import torch
     assert a.k == b.k and a.sf_layout == NVFP4_SF_MMA and b.sf_layout == NVFP4_SF_MMA
     M, N, K = a.rows, b.rows, a.k
@@ -306,13 +319,13 @@ def gemm(a: NVFP4Tensor, b: NVFP4Tensor, out_dtype: int = NVFP4_OUT_BF16, out=No
     if out is None:
         out = torch.empty((M, N), dtype=dt, device=a.q.device)
     ws = workspace if workspace is not None else _workspace(a.q.device)
-    nvfp4_gemm(a.q, a.sf, a.g, b.q, b.sf, b.g, M, N, K, out_dtype, out, out.stride(0), ws,
-               ws.numel(), stream)
+    nvfp4_gemm(a.q, a.sf, a.g, b.q, b.sf, b.g, M, N, K, out_dtype, out, out.stride(0), amax_out,
+               ws, ws.numel(), stream)
     return out
 
 
 def grouped_gemm(group_offsets, a: NVFP4Tensor, qb, sfb, gb, N: int, out_dtype: int = NVFP4_OUT_BF16,
-                 out=None, workspace=None, stream=None):
+                 out=None, amax_out=None, workspace=None, stream=None):
     """MoE grouped D = A_e B_e^T; qb [G, N, K/2], sfb tiled per expert, gb [G]."""
     import torch
     G = group_offsets.numel() - 1
@@ -321,5 +334,23 @@ def grouped_gemm(group_offsets, a: NVFP4Tensor, qb, sfb, gb, N: int, out_dtype: 
         out = torch.empty((a.rows, N), dtype=dt, device=a.q.device)
     ws = workspace if workspace is not None else _workspace(a.q.device)
     nvfp4_grouped_gemm(G, group_offsets, a.rows, a.q, a.sf, a.g, qb, sfb, gb, N, a.k, out_dtype,
-                       out, ws, ws.numel(), stream)
+                       out, amax_out, ws, ws.numel(), stream)
     return out
+
+
+def gather_rows(t: NVFP4Tensor, row_index, group_offsets=None, workspace=None, stream=None):
+    """MoE dispatch of an already quantised operand: row i of the result is row
+    ``row_index[i]`` of ``t`` (codes and tiled scales), laid out per expert
+    group when ``group_offsets`` (device int32 [G+1]) is given."""
+    import torch
+    assert t.sf_layout == NVFP4_SF_MMA
+    rows = row_index.numel()
+    G = 0 if group_offsets is None else group_offsets.numel() - 1
+    u8 = dict(dtype=torch.uint8, device=t.q.device)
+    q = torch.empty((rows, t.k // 2), **u8)
+    n = nvfp4_sf_mma_grouped_bytes(rows, G, t.k) if G else nvfp4_sf_mma_bytes(rows, t.k)
+    sf = torch.zeros(n, **u8)
+    ws = workspace if workspace is not None else _workspace(t.q.device)
+    nvfp4_gather_rows(t.q, t.sf, t.rows, t.k, row_index, rows, group_offsets, G, q, sf, ws,
+                      ws.numel(), stream)
+    return NVFP4Tensor(q, sf, t.g, rows, t.k, NVFP4_SF_MMA)

@@ -62,6 +62,7 @@ struct GemmArgs {
     const int32_t* group_offsets;
     int64_t total_rows;
     uint32_t* status;
+    float* amax_out;  // optional: max |D| (as stored), atomically accumulated
 };
 
 struct GemmShared {
@@ -346,6 +347,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         // the next tile's MMAs overlap this tile's stores.
         const int quad = warp & 3;                   // TMEM lanes 32*quad .. 32*quad+31
         const int col0 = ((warp - 2) >> 2) * (BN / 2);  // 0 or 128
+        float out_max = 0.0f;                            // max |D| stored by this thread
         uint32_t tcount = 0;
         for (int t = blockIdx.x; t < total; t += gridDim.x, ++tcount) {
             const TileCoord c = tile_coord(a, sh, t);
@@ -377,16 +379,20 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
 #pragma unroll
                     for (int v = 0; v < 4; ++v) {
                         uint32_t w[4];
+                        float vm = 0.0f;
 #pragma unroll
                         for (int i = 0; i < 4; ++i) {
-                            const __nv_bfloat162 p = __floats2bfloat162_rn(
-                                __fmul_rn(__uint_as_float(r[ch][8 * v + 2 * i]), alpha),
-                                __fmul_rn(__uint_as_float(r[ch][8 * v + 2 * i + 1]), alpha));
+                            const float x0 = __fmul_rn(__uint_as_float(r[ch][8 * v + 2 * i]), alpha);
+                            const float x1 = __fmul_rn(__uint_as_float(r[ch][8 * v + 2 * i + 1]), alpha);
+                            vm = absmax3(vm, x0, x1);
+                            const __nv_bfloat162 p = __floats2bfloat162_rn(x0, x1);
                             w[i] = *reinterpret_cast<const uint32_t*>(&p);
                         }
-                        if (cbase + 32 * ch + 8 * v < a.N)
+                        if (cbase + 32 * ch + 8 * v < a.N) {
                             *reinterpret_cast<uint4*>(drow + 32 * ch + 8 * v) =
                                 make_uint4(w[0], w[1], w[2], w[3]);
+                            out_max = fmaxf(out_max, vm);
+                        }
                     }
                 }
             } else {
@@ -395,15 +401,27 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
                 for (int ch = 0; ch < 4; ++ch) {
 #pragma unroll
                     for (int v = 0; v < 8; ++v) {
-                        if (cbase + 32 * ch + 4 * v < a.N)
+                        const float x0 = __fmul_rn(__uint_as_float(r[ch][4 * v]), alpha);
+                        const float x1 = __fmul_rn(__uint_as_float(r[ch][4 * v + 1]), alpha);
+                        const float x2 = __fmul_rn(__uint_as_float(r[ch][4 * v + 2]), alpha);
+                        const float x3 = __fmul_rn(__uint_as_float(r[ch][4 * v + 3]), alpha);
+                        if (cbase + 32 * ch + 4 * v < a.N) {
                             *reinterpret_cast<float4*>(drow + 32 * ch + 4 * v) =
-                                make_float4(__fmul_rn(__uint_as_float(r[ch][4 * v]), alpha),
-                                            __fmul_rn(__uint_as_float(r[ch][4 * v + 1]), alpha),
-                                            __fmul_rn(__uint_as_float(r[ch][4 * v + 2]), alpha),
-                                            __fmul_rn(__uint_as_float(r[ch][4 * v + 3]), alpha));
+                                make_float4(x0, x1, x2, x3);
+                            out_max = absmax3(out_max, absmax3(x0, x1, x2), x3);
+                        }
                     }
                 }
             }
+        }
+        // max |D| over this thread's stored values -> one atomic per warp.  For
+        // bf16 output the max is rounded like the values were: rounding is
+        // monotonic, so that is the max of the stored values.
+        if (a.amax_out) {
+#pragma unroll
+            for (int o = 16; o > 0; o >>= 1) out_max = fmaxf(out_max, __shfl_xor_sync(0xffffffffu, out_max, o));
+            if (a.bf16_out) out_max = __bfloat162float(__float2bfloat16_rn(out_max));
+            if (lane == 0) atomicMax(reinterpret_cast<uint32_t*>(a.amax_out), __float_as_uint(out_max));
         }
     }
 
@@ -484,8 +502,9 @@ static nvfp4_status launch_gemm(const CUtensorMap& ma, const CUtensorMap& mb, Ge
     if (cudaGetDevice(&dev) != cudaSuccess) return NVFP4_ERR_CUDA;
     GemmDevice& info = gemm_device(dev);
     if (!info.ok) return NVFP4_ERR_UNSUPPORTED;
-    // the status word reports this call only
+    // the status word reports this call only; the output amax starts at 0
     if (cudaMemsetAsync(a.status, 0, 4, st) != cudaSuccess) return NVFP4_ERR_CUDA;
+    if (a.amax_out && cudaMemsetAsync(a.amax_out, 0, 4, st) != cudaSuccess) return NVFP4_ERR_CUDA;
     const int grid = (int)std::max<int64_t>(1, std::min<int64_t>(max_tiles, info.sms));
     gemm_kernel<<<grid, kGemmThreads, gemm_smem_bytes(), st>>>(ma, mb, a);
     return cudaGetLastError() == cudaSuccess ? NVFP4_OK : NVFP4_ERR_CUDA;
@@ -494,14 +513,16 @@ static nvfp4_status launch_gemm(const CUtensorMap& ma, const CUtensorMap& mb, Ge
 extern "C" nvfp4_status nvfp4_gemm(const uint8_t* qa, const uint8_t* sfa, const float* ga,
                                    const uint8_t* qb, const uint8_t* sfb, const float* gb,
                                    int64_t M, int64_t N, int64_t K, int out_dtype, void* D,
-                                   int64_t ldd, void* workspace, size_t ws_bytes, void* stream)
+                                   int64_t ldd, float* amax_out, void* workspace, size_t ws_bytes,
+                                   void* stream)
 {
     if (!qa || !sfa || !ga || !qb || !sfb || !gb || !D) return NVFP4_ERR_INVALID_ARG;
     if (out_dtype != NVFP4_OUT_F32 && out_dtype != NVFP4_OUT_BF16) return NVFP4_ERR_INVALID_ARG;
     if (M <= 0 || N <= 0 || K <= 0 || M % 16 || N % 16 || K % BK || ldd < N) return NVFP4_ERR_SHAPE;
     if (M > (int64_t)1 << 31 || N > (int64_t)1 << 31) return NVFP4_ERR_SHAPE;
     const int esz = out_dtype == NVFP4_OUT_BF16 ? 2 : 4;
-    if (!al16(qa) || !al16(qb) || !al16(sfa) || !al16(sfb) || !al16(D) || (ldd * esz) % 16)
+    if (!al16(qa) || !al16(qb) || !al16(sfa) || !al16(sfb) || !al16(D) || (ldd * esz) % 16 ||
+        (reinterpret_cast<uintptr_t>(amax_out) & 3u))
         return NVFP4_ERR_ALIGN;
     if (!workspace || ws_bytes < kGemmWorkspace) return NVFP4_ERR_WORKSPACE;
     if (!al16(workspace)) return NVFP4_ERR_ALIGN;
@@ -521,6 +542,7 @@ extern "C" nvfp4_status nvfp4_gemm(const uint8_t* qa, const uint8_t* sfa, const 
     a.grouped = 0;
     a.G = 1;
     a.status = static_cast<uint32_t*>(workspace) + 2;
+    a.amax_out = amax_out;
     const int64_t tiles = ((M + BM - 1) / BM) * ((N + BN - 1) / BN);
     return launch_gemm(ma, mb, a, tiles, static_cast<cudaStream_t>(stream));
 }
@@ -529,7 +551,8 @@ extern "C" nvfp4_status nvfp4_grouped_gemm(int G, const int32_t* group_offsets, 
                                            const uint8_t* qa, const uint8_t* sfa, const float* ga,
                                            const uint8_t* qb, const uint8_t* sfb, const float* gb,
                                            int64_t N, int64_t K, int out_dtype, void* D,
-                                           void* workspace, size_t ws_bytes, void* stream)
+                                           float* amax_out, void* workspace, size_t ws_bytes,
+                                           void* stream)
 {
     if (G < 1 || G > kMaxGemmGroups || !group_offsets || !qa || !sfa || !ga || !qb || !sfb ||
         !gb || !D)
@@ -537,7 +560,9 @@ extern "C" nvfp4_status nvfp4_grouped_gemm(int G, const int32_t* group_offsets, 
     if (out_dtype != NVFP4_OUT_F32 && out_dtype != NVFP4_OUT_BF16) return NVFP4_ERR_INVALID_ARG;
     if (total_rows <= 0 || N <= 0 || K <= 0 || N % 128 || K % BK) return NVFP4_ERR_SHAPE;
     if (total_rows > (int64_t)1 << 31 || (int64_t)G * N > (int64_t)1 << 31) return NVFP4_ERR_SHAPE;
-    if (!al16(qa) || !al16(qb) || !al16(sfa) || !al16(sfb) || !al16(D)) return NVFP4_ERR_ALIGN;
+    if (!al16(qa) || !al16(qb) || !al16(sfa) || !al16(sfb) || !al16(D) ||
+        (reinterpret_cast<uintptr_t>(amax_out) & 3u))
+        return NVFP4_ERR_ALIGN;
     if (!workspace || ws_bytes < kGemmWorkspace) return NVFP4_ERR_WORKSPACE;
     if (!al16(workspace)) return NVFP4_ERR_ALIGN;
     CUtensorMap ma, mb;
@@ -559,6 +584,7 @@ extern "C" nvfp4_status nvfp4_grouped_gemm(int G, const int32_t* group_offsets, 
     a.group_offsets = group_offsets;
     a.total_rows = total_rows;
     a.status = static_cast<uint32_t*>(workspace) + 2;
+    a.amax_out = amax_out;
     // upper bound on tiles: every group may add one partial M tile
     const int64_t tiles = ((total_rows + BM - 1) / BM + G) * (N / BN + 1);
     return launch_gemm(ma, mb, a, tiles, static_cast<cudaStream_t>(stream));

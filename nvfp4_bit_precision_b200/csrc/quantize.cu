@@ -1,13 +1,14 @@
 // quantize.cu -- NVFP4 / MXFP8 quantisation and NVFP4 dequantisation on sm_100a.
 //
-// Two HBM-bound passes:
-//   1. amax_kernel: one read of the tensor, warp-shuffle max of |x| and, when
-//      the columnwise Hadamard is on, of |RHT(x)| over the columnwise
-//      16-vectors; one atomicMax per CTA on the float bit pattern.
-//   2. quant_kernel: a persistent grid walks 128x128 tiles in the reverse
-//      order of pass 1 (so the tail pass 1 left in L2 is read first).  One warp
-//      stages each tile into shared memory with mbarrier-tracked bulk copies
-//      (double-buffered); all eight warps then produce, from that one copy,
+// Two HBM-bound passes over 128x128 bf16 tiles, each a persistent grid whose
+// warp 0 keeps a 3-stage ring of tiles in flight (TMA boxes with the 128-byte
+// swizzle for dense input, per-row bulk copies for a gather) while all eight
+// warps compute from shared memory:
+//   1. amax_kernel: max |x| and, when the columnwise Hadamard is on, max
+//      |RHT(x)| over the columnwise 16-vectors; one atomicMax per CTA
+//      (amax_rows_kernel, with direct loads, when rows are gathered).
+//   2. quant_kernel: walks the tiles in the reverse order of pass 1 (the tail
+//      pass 1 left in L2 is read first) and produces, from one staged copy,
 //      the rowwise codes/scales, the columnwise (transposed, optionally
 //      Hadamard-rotated) codes/scales and the MXFP8 copies, with Philox
 //      stochastic rounding in registers and 8/16-byte vector stores.
@@ -110,71 +111,7 @@ __device__ __forceinline__ float warp_max16(float v)
 }
 
 // --------------------------------------------------------------------------
-// Pass 1: global amax.
-// --------------------------------------------------------------------------
-__global__ void __launch_bounds__(256, 2) amax_kernel(QArgs a, uint32_t* amax_out)
-{
-    const uint32_t signs = a.rht ? rht_sign_bits(a.seed) : 0u;
-    float mr = 0.0f, mc = 0.0f;
-    // unit = 16 rows x 4 columns (8-byte loads, 16 in flight per thread)
-    const int64_t ncg = a.cols / 4;
-    const int64_t units = (a.rows / 16) * ncg;
-    for (int64_t u = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; u < units;
-         u += (int64_t)gridDim.x * blockDim.x) {
-        const int64_t rb = u / ncg, cg = u - rb * ncg;
-        uint2 raw[16];
-        if (a.row_index) {
-#pragma unroll
-            for (int i = 0; i < 16; ++i)
-                raw[i] = ld_global_v2(a.x + source_row(a, rb * 16 + i) * a.ld + cg * 4);
-        } else {
-            const uint16_t* p = a.x + (rb * 16) * a.ld + cg * 4;
-#pragma unroll
-            for (int i = 0; i < 16; ++i) raw[i] = ld_global_v2(p + i * a.ld);
-        }
-        // columns 2p and 2p+1 form one packed pair; the sign flip of row i
-        // (the Hadamard's D) is applied while unpacking -- |x| is unaffected
-#pragma unroll
-        for (int p = 0; p < 2; ++p) {
-            float va[16], vb[16];
-#pragma unroll
-            for (int i = 0; i < 16; ++i) {
-                const uint32_t w = p == 0 ? raw[i].x : raw[i].y;
-                unpack_bf16x2(w, ((signs >> i) & 1u) << 31, va[i], vb[i]);
-            }
-            mr = absmax16(vb, absmax16(va, mr));
-            if (a.rht) {
-                hadamard16x2_times4(va, vb);  // 4x the transform; the 1/4 is applied once below
-                mc = absmax16(vb, absmax16(va, mc));
-            }
-        }
-    }
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) {
-        mr = fmaxf(mr, __shfl_xor_sync(0xffffffffu, mr, o));
-        mc = fmaxf(mc, __shfl_xor_sync(0xffffffffu, mc, o));
-    }
-    __shared__ float red[2][8];
-    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    if (lane == 0) {
-        red[0][warp] = mr;
-        red[1][warp] = mc;
-    }
-    __syncthreads();
-    if (threadIdx.x == 0) {
-        for (int w = 1; w < (int)(blockDim.x >> 5); ++w) {
-            mr = fmaxf(mr, red[0][w]);
-            mc = fmaxf(mc, red[1][w]);
-        }
-        mc = __fmul_rn(mc, 0.25f);  // the transform's factor 1/4 (exact)
-        // non-negative floats order like their bit patterns
-        atomicMax(&amax_out[0], __float_as_uint(mr));
-        atomicMax(&amax_out[1], __float_as_uint(mc));
-    }
-}
-
-// --------------------------------------------------------------------------
-// Pass 2: fused quantisation of 128x128 tiles.
+// Tile staging and block quantisation, shared by the passes.
 // --------------------------------------------------------------------------
 struct QShared {
     int32_t n_groups;
@@ -183,9 +120,9 @@ struct QShared {
 };
 
 // Padded scale row of output row r (MoE layout); identity when dense.
-__device__ __forceinline__ int64_t padded_row(const QShared* sh, const QArgs& a, int64_t r)
+__device__ __forceinline__ int64_t padded_row(const QShared* sh, bool grouped, int64_t r)
 {
-    if (!a.group_offsets) return r;
+    if (!grouped) return r;
     int lo = 0, hi = sh->n_groups - 1;  // find e with start[e] <= r < start[e+1]
     while (lo < hi) {
         const int mid = (lo + hi + 1) >> 1;
@@ -320,6 +257,33 @@ __device__ __forceinline__ uint32_t mx_block32(const float* v, bool sr, uint64_t
     return (uint32_t)(e + 127);
 }
 
+// E8M0 exponent of an MXFP8 block with absolute maximum am (OCP rule:
+// floor(log2 am) - 8, clamped to -127; subnormal or zero am -> -127) and the
+// exact scale 2^-e the elements are multiplied by.
+__device__ __forceinline__ int mx_exponent(float am, float& scale)
+{
+    const int ef = (int)((__float_as_uint(am) >> 23) & 0xFFu);
+    const int e = max(ef - 127 - 8, -127);
+    scale = __uint_as_float((uint32_t)(127 - e) << 23);
+    return e;
+}
+
+// 8 consecutive elements of one MXFP8 block -> 8 E4M3 bytes (element 0 in the
+// low byte).  SR: 16-bit uniforms from the Philox block w of these 8 elements.
+__device__ __forceinline__ uint2 mx_convert8(const float (&v)[8], float scale, bool sr, const U4& w)
+{
+    float y[8];
+    if (sr) {
+#pragma unroll
+        for (int i = 0; i < 8; ++i) y[i] = e4m3_sr_value(__fmul_rn(v[i], scale), u16_of(w, i));
+    } else {
+#pragma unroll
+        for (int i = 0; i < 8; i += 2) mul2(y[i], y[i + 1], v[i], v[i + 1], scale, scale);
+    }
+    return make_uint2(e4m3x2_rne_sat(y[1], y[0]) | (e4m3x2_rne_sat(y[3], y[2]) << 16),
+                      e4m3x2_rne_sat(y[5], y[4]) | (e4m3x2_rne_sat(y[7], y[6]) << 16));
+}
+
 __device__ __forceinline__ void store_codes32(uint8_t* dst, const uint32_t (&c)[8], bool vec16)
 {
     if (vec16) {
@@ -332,10 +296,209 @@ __device__ __forceinline__ void store_codes32(uint8_t* dst, const uint32_t (&c)[
     }
 }
 
-template <bool kTma>
+// --------------------------------------------------------------------------
+// Pass 1: global amax (dense input).  The same 128x128 TMA tiles and 3-stage
+// copy ring as pass 2, walked in the opposite order; each thread takes one column pair over 32
+// rows (two 16-row blocks): max |x| for the rowwise and 2D scales and, with the
+// Hadamard on, max |RHT(x)| over the columnwise 16-vectors.  One atomicMax per
+// CTA on the float bit pattern.
+// --------------------------------------------------------------------------
+__global__ void __launch_bounds__(kQuantThreads, 2)
+    amax_kernel(const __grid_constant__ CUtensorMap map_x, QArgs a, uint32_t* amax_out)
+{
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                               ~uintptr_t(1023));
+    uint8_t* tiles = smem;
+    uint64_t* full = reinterpret_cast<uint64_t*>(smem + kStages * kTileBytes);
+    uint64_t* empty = full + kStages;
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < kStages; ++s) {
+            mbar_init(&full[s], 1);
+            mbar_init(&empty[s], kQuantThreads / 32);
+        }
+        fence_barrier_init();
+    }
+    __syncthreads();
+    const bool rht = a.rht != 0;
+    const uint32_t signs = rht ? rht_sign_bits(a.seed) : 0u;
+    const int64_t first = blockIdx.x;
+    const int64_t my_count =
+        first < a.n_tiles ? (a.n_tiles - first + gridDim.x - 1) / gridDim.x : 0;
+    auto tile_of = [&](int64_t k) { return first + k * (int64_t)gridDim.x; };
+    int64_t issued = 0;
+    if (warp == 0) {
+        for (; issued < my_count && issued < kStages - 1; ++issued)
+            issue_tile<true>(a, &map_x, tile_of(issued), tiles + (issued % kStages) * kTileBytes,
+                             &full[issued % kStages], lane);
+    }
+    const int cp = 32 * (warp & 1) + lane;  // column pair 0..63
+    const int rgrp = warp >> 1;              // 32-row group 0..3
+    float mr = 0.0f, mc = 0.0f;
+    int64_t k = 0;
+    for (; k < my_count; ++k) {
+        const int stage = (int)(k % kStages);
+        if (warp == 0 && issued < my_count) {
+            const int s = (int)(issued % kStages);
+            bool ok = true;
+            if (issued >= kStages) ok = mbar_wait(&empty[s], (uint32_t)((issued / kStages - 1) & 1));
+            if (!ok) {
+                if (lane == 0) record_status(a.status, NVFP4_ERR_TIMEOUT);
+                break;
+            }
+            issue_tile<true>(a, &map_x, tile_of(issued), tiles + s * kTileBytes, &full[s], lane);
+            ++issued;
+        }
+        if (!mbar_wait(&full[stage], (uint32_t)((k / kStages) & 1))) {
+            if (lane == 0) record_status(a.status, NVFP4_ERR_TIMEOUT);
+            break;
+        }
+        const uint8_t* T = tiles + stage * kTileBytes;
+        const int64_t tile = tile_of(k);
+        const int64_t tr = tile / a.tiles_c, tc = tile - tr * a.tiles_c;
+        const int64_t cg0 = tc * kTileCols + 2 * cp;
+        const int64_t rbase = tr * kTileRows + 32 * rgrp;
+#pragma unroll
+        for (int sub = 0; sub < 2; ++sub) {
+            // positions past the tensor hold zeros (rows) or stale bytes (an
+            // uncopied second panel): skip them
+            if (cg0 >= a.cols || rbase + 16 * sub >= a.rows) continue;
+            float va[16], vb[16];
+#pragma unroll
+            for (int i = 0; i < 16; ++i) {
+                const uint32_t w =
+                    ld_shared_u32(chunk_addr<true>(T, 32 * rgrp + 16 * sub + i, cp >> 2) + 4 * (cp & 3));
+                unpack_bf16x2(w, ((signs >> i) & 1u) << 31, va[i], vb[i]);  // |x| unaffected
+            }
+            mr = absmax16(vb, absmax16(va, mr));
+            if (rht) {
+                hadamard16x2_times4(va, vb);  // 4x the transform; the 1/4 is applied once below
+                mc = absmax16(vb, absmax16(va, mc));
+            }
+        }
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&empty[stage]);
+    }
+    if (warp == 0) {
+        for (int64_t j = k + 1; j < issued; ++j)
+            (void)mbar_wait(&full[j % kStages], (uint32_t)((j / kStages) & 1));
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) {
+        mr = fmaxf(mr, __shfl_xor_sync(0xffffffffu, mr, o));
+        mc = fmaxf(mc, __shfl_xor_sync(0xffffffffu, mc, o));
+    }
+    __shared__ float red[2][kQuantThreads / 32];
+    if (lane == 0) {
+        red[0][warp] = mr;
+        red[1][warp] = mc;
+    }
+    __syncthreads();
+    if (threadIdx.x == 0) {
+        for (int w = 1; w < kQuantThreads / 32; ++w) {
+            mr = fmaxf(mr, red[0][w]);
+            mc = fmaxf(mc, red[1][w]);
+        }
+        mc = __fmul_rn(mc, 0.25f);  // the transform's factor 1/4 (exact)
+        // non-negative floats order like their bit patterns
+        atomicMax(&amax_out[0], __float_as_uint(mr));
+        atomicMax(&amax_out[1], __float_as_uint(mc));
+    }
+}
+
+// Pass 1 for a gather: rows come from row_index, so tiles would be staged by
+// one small copy per row; direct loads of 16 rows x 4 columns per thread (16
+// in flight) serve it better.
+__global__ void __launch_bounds__(256, 2) amax_rows_kernel(QArgs a, uint32_t* amax_out)
+{
+    const bool rht = a.rht != 0;
+    const uint32_t signs = rht ? rht_sign_bits(a.seed) : 0u;
+    float mr = 0.0f, mc = 0.0f;
+    const int64_t ncg = a.cols / 4;
+    const int64_t units = (a.rows / 16) * ncg;
+    for (int64_t u = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; u < units;
+         u += (int64_t)gridDim.x * blockDim.x) {
+        const int64_t rb = u / ncg, cg = u - rb * ncg;
+        uint2 raw[16];
+#pragma unroll
+        for (int i = 0; i < 16; ++i)
+            raw[i] = ld_global_v2(a.x + source_row(a, rb * 16 + i) * a.ld + cg * 4);
+        // columns 2p and 2p+1 form one packed pair; row i's sign flip (the
+        // Hadamard's D) is applied while unpacking -- |x| is unaffected
+#pragma unroll
+        for (int p = 0; p < 2; ++p) {
+            float va[16], vb[16];
+#pragma unroll
+            for (int i = 0; i < 16; ++i)
+                unpack_bf16x2(p == 0 ? raw[i].x : raw[i].y, ((signs >> i) & 1u) << 31, va[i], vb[i]);
+            mr = absmax16(vb, absmax16(va, mr));
+            if (rht) {
+                hadamard16x2_times4(va, vb);
+                mc = absmax16(vb, absmax16(va, mc));
+            }
+        }
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) {
+        mr = fmaxf(mr, __shfl_xor_sync(0xffffffffu, mr, o));
+        mc = fmaxf(mc, __shfl_xor_sync(0xffffffffu, mc, o));
+    }
+    __shared__ float red[2][8];
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    if (lane == 0) {
+        red[0][warp] = mr;
+        red[1][warp] = mc;
+    }
+    __syncthreads();
+    if (threadIdx.x == 0) {
+        for (int w = 1; w < 8; ++w) {
+            mr = fmaxf(mr, red[0][w]);
+            mc = fmaxf(mc, red[1][w]);
+        }
+        mc = __fmul_rn(mc, 0.25f);  // the transform's factor 1/4 (exact)
+        atomicMax(&amax_out[0], __float_as_uint(mr));
+        atomicMax(&amax_out[1], __float_as_uint(mc));
+    }
+}
+
+// --------------------------------------------------------------------------
+// Pass 2: fused quantisation.
+// --------------------------------------------------------------------------
+// Compile-time variants of the fused pass.  Each switch is off, on, or read
+// from the call's arguments (run time).  Variant 0 reads every switch at run
+// time; the others fix the switches for the tensor roles of the training
+// recipe (asector.ru, "Experiments and comparison with FP8": 2D weight scales
+// and random Hadamard transforms for outlier gradients; iitak.ru, "How it
+// works": 16x16 weight squares, random re-rounding and the MXFP8 backward):
+//   1 gradients:   rowwise SR, columnwise Hadamard + SR, MXFP8 columnwise RNE
+//   2 activations: rowwise RNE, columnwise Hadamard RNE
+//   3 weights:     16x16 2D scales, both directions, RNE
+//   4 MoE rows:    rowwise RNE only (gather and groups at run time)
+// Fixed switches let the compiler drop the unused branches and the registers
+// they hold; results are identical to variant 0.
+enum : int8_t { kOff = 0, kOn = 1, kRt = 2 };
+struct QSpec {
+    int8_t nv_row, nv_col, mx_row, mx_col, sr, mx_sr, rht, two_d, groups;
+};
+constexpr int kNumSpecs = 5;
+constexpr QSpec kSpecs[kNumSpecs] = {
+    {kRt, kRt, kRt, kRt, kRt, kRt, kRt, kRt, kRt},
+    {kOn, kOn, kOff, kOn, kOn, kOff, kOn, kOff, kOff},
+    {kOn, kOn, kOff, kOff, kOff, kRt, kOn, kOff, kOff},
+    {kOn, kOn, kOff, kOff, kOff, kRt, kOff, kOn, kOff},
+    {kOn, kOff, kOff, kOff, kOff, kRt, kRt, kOff, kRt},
+};
+__host__ __device__ constexpr bool spec_pick(int8_t s, bool run_time)
+{
+    return s == kRt ? run_time : s == kOn;
+}
+
+template <bool kTma, int kSpec>
 __global__ void __launch_bounds__(kQuantThreads, 2)
     quant_kernel(const __grid_constant__ CUtensorMap map_x, QArgs a)
 {
+    constexpr QSpec sp = kSpecs[kSpec];
     extern __shared__ uint8_t smem_raw[];
     // the swizzled TMA boxes need 1024-byte alignment
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
@@ -352,7 +515,8 @@ __global__ void __launch_bounds__(kQuantThreads, 2)
         }
         fence_barrier_init();
     }
-    if (a.group_offsets) {
+    const bool grouped = spec_pick(sp.groups, a.group_offsets != nullptr);
+    if (grouped) {
         if (threadIdx.x == 0) {
             sh->n_groups = a.num_groups;
             int32_t pad = 0;
@@ -369,13 +533,14 @@ __global__ void __launch_bounds__(kQuantThreads, 2)
     }
     __syncthreads();
 
-    const bool nv_row = (a.outputs & NVFP4_ROWWISE) != 0;
-    const bool nv_col = (a.outputs & NVFP4_COLWISE) != 0;
-    const bool mx_row = (a.mx_outputs & NVFP4_ROWWISE) != 0;
-    const bool mx_col = (a.mx_outputs & NVFP4_COLWISE) != 0;
-    const bool sr = a.rounding == NVFP4_SR;
-    const bool mx_sr = a.mx_rounding == NVFP4_SR;
-    const bool two_d = a.scaling == NVFP4_2D16x16;
+    const bool nv_row = spec_pick(sp.nv_row, (a.outputs & NVFP4_ROWWISE) != 0);
+    const bool nv_col = spec_pick(sp.nv_col, (a.outputs & NVFP4_COLWISE) != 0);
+    const bool mx_row = spec_pick(sp.mx_row, (a.mx_outputs & NVFP4_ROWWISE) != 0);
+    const bool mx_col = spec_pick(sp.mx_col, (a.mx_outputs & NVFP4_COLWISE) != 0);
+    const bool sr = spec_pick(sp.sr, a.rounding == NVFP4_SR);
+    const bool mx_sr = spec_pick(sp.mx_sr, a.mx_rounding == NVFP4_SR);
+    const bool two_d = spec_pick(sp.two_d, a.scaling == NVFP4_2D16x16);
+    const bool rht = spec_pick(sp.rht, a.rht != 0);
     const bool mma_sf = a.sf_layout == NVFP4_SF_MMA;
 
     float S_row = 1.0f, g_row = 1.0f, S_col = 1.0f, g_col = 1.0f;
@@ -386,7 +551,7 @@ __global__ void __launch_bounds__(kQuantThreads, 2)
             amax_c = a.amax_in[1];
         } else {
             amax_r = __uint_as_float(a.amax_ws[0]);
-            amax_c = a.rht ? __uint_as_float(a.amax_ws[1]) : amax_r;
+            amax_c = rht ? __uint_as_float(a.amax_ws[1]) : amax_r;
         }
         global_scales(amax_r, S_row, g_row);
         global_scales(amax_c, S_col, g_col);
@@ -395,7 +560,7 @@ __global__ void __launch_bounds__(kQuantThreads, 2)
             if (nv_col) *a.g_col = g_col;
         }
     }
-    const uint32_t signs = (nv_col && a.rht) ? rht_sign_bits(a.seed) : 0u;
+    const uint32_t signs = (nv_col && rht) ? rht_sign_bits(a.seed) : 0u;
 
     const int64_t first = blockIdx.x;
     const int64_t my_count =
@@ -480,7 +645,7 @@ __global__ void __launch_bounds__(kQuantThreads, 2)
                 if (all_valid) {
                     store_codes32(a.q_row + rg * (a.cols / 2) + cbase / 2, codes, q_row_vec);
                     const int64_t b0 = cbase / 16;
-                    const int64_t off = mma_sf ? sf_mma_offset(padded_row(sh, a, rg), b0, a.cols / 16)
+                    const int64_t off = mma_sf ? sf_mma_offset(padded_row(sh, grouped, rg), b0, a.cols / 16)
                                                : rg * (a.cols / 16) + b0;
                     if (sf_row_vec) {
                         *reinterpret_cast<uint32_t*>(a.sf_row + off) = sfw;
@@ -495,7 +660,7 @@ __global__ void __launch_bounds__(kQuantThreads, 2)
                         if (cg >= a.cols) continue;
                         *reinterpret_cast<uint2*>(a.q_row + rg * (a.cols / 2) + cg / 2) =
                             make_uint2(codes[2 * blk], codes[2 * blk + 1]);
-                        const int64_t off = mma_sf ? sf_mma_offset(padded_row(sh, a, rg), cg / 16, a.cols / 16)
+                        const int64_t off = mma_sf ? sf_mma_offset(padded_row(sh, grouped, rg), cg / 16, a.cols / 16)
                                                    : rg * (a.cols / 16) + cg / 16;
                         a.sf_row[off] = (sfw >> (8 * blk)) & 0xFFu;
                     }
@@ -534,40 +699,33 @@ __global__ void __launch_bounds__(kQuantThreads, 2)
             auto pair_word = [&](int i) -> uint32_t {
                 return ld_shared_u32(chunk_addr<kTma>(T, 32 * rgrp + i, cp >> 2) + 4 * (cp & 3));
             };
-            if (mx_col && cvalid && rbase + 32 <= a.rows) {
-#pragma unroll 1
-                for (int half = 0; half < 2; ++half) {
-                    float x[32];
-#pragma unroll
-                    for (int i = 0; i < 32; ++i) {
-                        const uint32_t wi = pair_word(i);
-                        x[i] = half ? bf16_hi(wi) : bf16_lo(wi);
-                    }
-                    const int64_t cg = cg0 + half;
-                    uint32_t out[8];
-                    const uint32_t e8 = mx_block32(x, mx_sr, a.seed, a.offset,
-                                                   (uint64_t)(cg * a.rows + rbase), out);
-                    uint4* dst = reinterpret_cast<uint4*>(a.mx_q_col + cg * a.rows + rbase);
-                    dst[0] = make_uint4(out[0], out[1], out[2], out[3]);
-                    dst[1] = make_uint4(out[4], out[5], out[6], out[7]);
-                    a.mx_sf_col[cg * (a.rows / 32) + rbase / 32] = (uint8_t)e8;
-                }
-            }
-            if (nv_col) {
-                uint32_t codes[2][4];
-                uint32_t sfw[2] = {0u, 0u};
-                bool all_valid = true;
+            // MXFP8 columnwise: the 32-row block's amax of each column is
+            // gathered while the NVFP4 pass below unpacks the rows (the
+            // Hadamard's sign flips leave |x| alone); the conversion then
+            // re-reads the rows 8 at a time.  rows is a multiple of 32 here.
+            float mxa = 0.0f, mxb = 0.0f;
+            if (rbase < a.rows) {
+                // rows is a multiple of 16: both 16-row blocks exist, or (at the
+                // bottom edge) only the first.  The first block's codes wait in
+                // registers so each column gets one 16-byte store.
+                const bool two = rbase + 32 <= a.rows;
+                const int64_t b0 = rbase / 16;
+                uint32_t keep0 = 0, keep1 = 0, keep2 = 0, keep3 = 0, keep_sf = 0;
 #pragma unroll
                 for (int sub = 0; sub < 2; ++sub) {
+                    if (sub == 1 && !two) break;
                     const int64_t rg = rbase + 16 * sub;
-                    const bool valid = cvalid && rg < a.rows;
-                    all_valid &= valid;
                     float va[16], vb[16];
 #pragma unroll
                     for (int i = 0; i < 16; ++i)
-                        unpack_bf16x2(pair_word(16 * sub + i), a.rht ? ((signs >> i) & 1u) << 31 : 0u,
+                        unpack_bf16x2(pair_word(16 * sub + i), rht ? ((signs >> i) & 1u) << 31 : 0u,
                                       va[i], vb[i]);
-                    if (a.rht) hadamard16x2_times4(va, vb);
+                    if (mx_col) {
+                        mxa = absmax16(va, mxa);
+                        mxb = absmax16(vb, mxb);
+                    }
+                    if (!nv_col) continue;
+                    if (rht) hadamard16x2_times4(va, vb);
                     float ama = absmax16(va, 0.0f), amb = absmax16(vb, 0.0f);
                     if (two_d) {  // 16x16 tile = 8 column pairs (lanes) x 16 rows
                         float m = fmaxf(ama, amb);
@@ -575,56 +733,79 @@ __global__ void __launch_bounds__(kQuantThreads, 2)
                         for (int o = 1; o < 8; o <<= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
                         ama = amb = m;
                     }
-                    uint32_t c0w, c1w;
-                    uint32_t byte = quant_block16(va, ama, S_col, a.rht != 0, sr && valid, a.seed,
-                                                  a.offset, 1u, (uint64_t)(cg0 * a.rows + rg), c0w, c1w);
-                    codes[0][2 * sub] = c0w;
-                    codes[0][2 * sub + 1] = c1w;
-                    sfw[0] |= byte << (8 * sub);
-                    byte = quant_block16(vb, amb, S_col, a.rht != 0, sr && valid, a.seed, a.offset, 1u,
-                                         (uint64_t)((cg0 + 1) * a.rows + rg), c0w, c1w);
-                    codes[1][2 * sub] = c0w;
-                    codes[1][2 * sub + 1] = c1w;
-                    sfw[1] |= byte << (8 * sub);
-                }
-                const int64_t b0 = rbase / 16;
-                if (all_valid) {
-#pragma unroll
-                    for (int half = 0; half < 2; ++half) {
-                        const int64_t cg = cg0 + half;
-                        uint8_t* dst = a.q_col + cg * (a.rows / 2) + rbase / 2;
-                        if (q_col_vec)
-                            *reinterpret_cast<uint4*>(dst) = make_uint4(codes[half][0], codes[half][1],
-                                                                        codes[half][2], codes[half][3]);
-                        else {
-                            reinterpret_cast<uint2*>(dst)[0] = make_uint2(codes[half][0], codes[half][1]);
-                            reinterpret_cast<uint2*>(dst)[1] = make_uint2(codes[half][2], codes[half][3]);
-                        }
-                        const int64_t off = mma_sf ? sf_mma_offset(cg, b0, a.rows / 16)
-                                                   : cg * (a.rows / 16) + b0;
-                        if (sf_col_vec)
-                            *reinterpret_cast<uint16_t*>(a.sf_col + off) = (uint16_t)sfw[half];
-                        else {
-                            a.sf_col[off] = sfw[half] & 0xFFu;
-                            a.sf_col[off + 1] = (sfw[half] >> 8) & 0xFFu;
-                        }
+                    uint32_t ca0, ca1, cb0, cb1;
+                    const uint32_t ba = quant_block16(va, ama, S_col, rht, sr && cvalid, a.seed,
+                                                      a.offset, 1u, (uint64_t)(cg0 * a.rows + rg),
+                                                      ca0, ca1);
+                    const uint32_t bb = quant_block16(vb, amb, S_col, rht, sr && cvalid, a.seed,
+                                                      a.offset, 1u,
+                                                      (uint64_t)((cg0 + 1) * a.rows + rg), cb0, cb1);
+                    if (!cvalid) continue;
+                    if (two && sub == 0) {
+                        keep0 = ca0, keep1 = ca1, keep2 = cb0, keep3 = cb1;
+                        keep_sf = ba | (bb << 8);
+                        continue;
                     }
-                } else if (cvalid) {
-#pragma unroll
-                    for (int half = 0; half < 2; ++half) {
-                        const int64_t cg = cg0 + half;
-#pragma unroll
-                        for (int sub = 0; sub < 2; ++sub) {
-                            const int64_t rg = rbase + 16 * sub;
-                            if (rg >= a.rows) continue;
-                            *reinterpret_cast<uint2*>(a.q_col + cg * (a.rows / 2) + rg / 2) =
-                                make_uint2(codes[half][2 * sub], codes[half][2 * sub + 1]);
-                            const int64_t off = mma_sf ? sf_mma_offset(cg, rg / 16, a.rows / 16)
-                                                       : cg * (a.rows / 16) + rg / 16;
-                            a.sf_col[off] = (sfw[half] >> (8 * sub)) & 0xFFu;
+                    uint8_t* da = a.q_col + cg0 * (a.rows / 2) + rbase / 2;
+                    uint8_t* db = da + a.rows / 2;
+                    const int64_t offa = mma_sf ? sf_mma_offset(cg0, b0, a.rows / 16)
+                                                : cg0 * (a.rows / 16) + b0;
+                    const int64_t offb = mma_sf ? sf_mma_offset(cg0 + 1, b0, a.rows / 16)
+                                                : offa + a.rows / 16;
+                    if (!two) {  // a lone 16-row block: 8 code bytes and one scale per column
+                        *reinterpret_cast<uint2*>(da) = make_uint2(ca0, ca1);
+                        *reinterpret_cast<uint2*>(db) = make_uint2(cb0, cb1);
+                        a.sf_col[offa] = (uint8_t)ba;
+                        a.sf_col[offb] = (uint8_t)bb;
+                    } else {
+                        if (q_col_vec) {
+                            *reinterpret_cast<uint4*>(da) = make_uint4(keep0, keep1, ca0, ca1);
+                            *reinterpret_cast<uint4*>(db) = make_uint4(keep2, keep3, cb0, cb1);
+                        } else {
+                            reinterpret_cast<uint2*>(da)[0] = make_uint2(keep0, keep1);
+                            reinterpret_cast<uint2*>(da)[1] = make_uint2(ca0, ca1);
+                            reinterpret_cast<uint2*>(db)[0] = make_uint2(keep2, keep3);
+                            reinterpret_cast<uint2*>(db)[1] = make_uint2(cb0, cb1);
+                        }
+                        const uint32_t sfa = (keep_sf & 0xFFu) | (ba << 8);
+                        const uint32_t sfb = (keep_sf >> 8) | (bb << 8);
+                        if (sf_col_vec) {
+                            *reinterpret_cast<uint16_t*>(a.sf_col + offa) = (uint16_t)sfa;
+                            *reinterpret_cast<uint16_t*>(a.sf_col + offb) = (uint16_t)sfb;
+                        } else {
+                            a.sf_col[offa] = (uint8_t)sfa;
+                            a.sf_col[offa + 1] = (uint8_t)(sfa >> 8);
+                            a.sf_col[offb] = (uint8_t)sfb;
+                            a.sf_col[offb + 1] = (uint8_t)(sfb >> 8);
                         }
                     }
                 }
+            }
+            if (mx_col && cvalid && rbase < a.rows) {
+                float sa, sb;
+                const int ea = mx_exponent(mxa, sa), eb = mx_exponent(mxb, sb);
+                const int64_t ia = cg0 * a.rows + rbase, ib = ia + a.rows;  // element indices
+                uint8_t* qa = a.mx_q_col + ia;
+                uint8_t* qb = a.mx_q_col + ib;
+#pragma unroll 2
+                for (int g = 0; g < 4; ++g) {
+                    float va[8], vb[8];
+#pragma unroll
+                    for (int i = 0; i < 8; ++i) {
+                        const uint32_t w = pair_word(8 * g + i);
+                        va[i] = bf16_lo(w);
+                        vb[i] = bf16_hi(w);
+                    }
+                    U4 wa{}, wb{};
+                    if (mx_sr) {
+                        wa = sr_block8(a.seed, a.offset, 2u, (uint64_t)(ia >> 3) + g);
+                        wb = sr_block8(a.seed, a.offset, 2u, (uint64_t)(ib >> 3) + g);
+                    }
+                    *reinterpret_cast<uint2*>(qa + 8 * g) = mx_convert8(va, sa, mx_sr, wa);
+                    *reinterpret_cast<uint2*>(qb + 8 * g) = mx_convert8(vb, sb, mx_sr, wb);
+                }
+                a.mx_sf_col[cg0 * (a.rows / 32) + rbase / 32] = (uint8_t)(ea + 127);
+                a.mx_sf_col[(cg0 + 1) * (a.rows / 32) + rbase / 32] = (uint8_t)(eb + 127);
             }
         }
         __syncwarp();
@@ -635,6 +816,78 @@ __global__ void __launch_bounds__(kQuantThreads, 2)
     if (warp == 0) {
         for (int64_t j = k + 1; j < issued; ++j)
             (void)mbar_wait(&full[j % kStages], (uint32_t)((j / kStages) & 1));
+    }
+}
+
+// --------------------------------------------------------------------------
+// MoE dispatch of quantised rows: output row i = source row row_index[i]
+// (codes and scale bytes), scales rewritten from the dense tiled layout into
+// the grouped tiled layout.  One CTA per (group, 128-row block), the blocks the
+// grouped GEMM tiles over, so each CTA writes whole 512-byte scale atoms.
+// --------------------------------------------------------------------------
+__global__ void __launch_bounds__(256) gather_rows_kernel(
+    const uint8_t* q_src, const uint8_t* sf_src, int64_t src_rows, int64_t k,
+    const int32_t* row_index, int64_t rows, const int32_t* group_offsets, int G, uint8_t* q_dst,
+    uint8_t* sf_dst, uint32_t* status)
+{
+    // locate this CTA's (group, block): group e has ceil(count/128) blocks
+    __shared__ int s_e, s_t, s_pad_blk;
+    if (threadIdx.x == 0) {
+        int64_t b = blockIdx.x, pad_blk = 0;
+        int e = -1, t = 0;
+        if (!group_offsets) {
+            if (b * 128 < rows) e = 0, t = (int)b, pad_blk = 0;
+        } else {
+            for (int g = 0; g < G; ++g) {
+                const int64_t cnt = group_offsets[g + 1] - group_offsets[g];
+                const int64_t nb = (cnt + 127) / 128;
+                if (b < nb) {
+                    e = g;
+                    t = (int)b;
+                    break;
+                }
+                b -= nb;
+                pad_blk += nb;
+            }
+        }
+        s_e = e;
+        s_t = t;
+        s_pad_blk = (int)pad_blk;
+    }
+    __syncthreads();
+    const int e = s_e;
+    if (e < 0) return;
+    const int64_t g0 = group_offsets ? group_offsets[e] : 0;
+    const int64_t g1 = group_offsets ? group_offsets[e + 1] : rows;
+    const int64_t r0 = g0 + 128 * (int64_t)s_t;
+    const int nr = (int)(g1 - r0 < 128 ? g1 - r0 : 128);
+    const int64_t dst_blk = s_pad_blk + s_t;  // padded 128-row scale block
+    const int64_t k16 = k / 16, k64 = k / 64, chunks = k / 32;  // 16-byte code chunks per row
+
+    __shared__ int64_t s_src[128];
+    for (int i = threadIdx.x; i < nr; i += blockDim.x) {
+        int64_t s = row_index[r0 + i];
+        if (s < 0 || s >= src_rows) {
+            record_status(status, NVFP4_ERR_INDEX);
+            s = 0;
+        }
+        s_src[i] = s;
+    }
+    __syncthreads();
+    // codes: 16-byte vectors, one row after another
+    for (int64_t idx = threadIdx.x; idx < (int64_t)nr * chunks; idx += blockDim.x) {
+        const int i = (int)(idx / chunks);
+        const int64_t c = idx - (int64_t)i * chunks;
+        const uint4 v = *reinterpret_cast<const uint4*>(q_src + s_src[i] * (k / 2) + c * 16);
+        *reinterpret_cast<uint4*>(q_dst + (r0 + i) * (k / 2) + c * 16) = v;
+    }
+    // scales: 4 bytes (one row's four 16-blocks of a 64-column group) at a time
+    for (int64_t idx = threadIdx.x; idx < (int64_t)nr * k64; idx += blockDim.x) {
+        const int64_t j = idx / nr;
+        const int i = (int)(idx - j * nr);
+        const int64_t s = s_src[i];
+        const uint32_t v = *reinterpret_cast<const uint32_t*>(sf_src + sf_mma_offset(s, 4 * j, k16));
+        *reinterpret_cast<uint32_t*>(sf_dst + sf_mma_offset(dst_blk * 128 + i, 4 * j, k16)) = v;
     }
 }
 
@@ -720,6 +973,41 @@ static bool make_input_map(CUtensorMap* m, const void* x, int64_t rows, int64_t 
               CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+using QuantKernel = void (*)(const CUtensorMap, QArgs);
+
+// The compiled variants: TMA tiles for dense input, row copies for the gather
+// (which only variants 0 and 4 serve).  nullptr where none is built.
+static QuantKernel quant_variant(bool tma, int spec)
+{
+    switch (spec) {
+    case 0: return tma ? quant_kernel<true, 0> : quant_kernel<false, 0>;
+    case 1: return tma ? quant_kernel<true, 1> : nullptr;
+    case 2: return tma ? quant_kernel<true, 2> : nullptr;
+    case 3: return tma ? quant_kernel<true, 3> : nullptr;
+    case 4: return tma ? quant_kernel<true, 4> : quant_kernel<false, 4>;
+    }
+    return nullptr;
+}
+
+// First compiled variant whose fixed switches agree with the call (variant 0
+// agrees with every call).
+static int pick_variant(const QArgs& a, bool tma)
+{
+    auto agrees = [](int8_t s, bool v) { return s == kRt || (s == kOn) == v; };
+    for (int v = 1; v < kNumSpecs; ++v) {
+        const QSpec& q = kSpecs[v];
+        if (quant_variant(tma, v) && agrees(q.nv_row, (a.outputs & NVFP4_ROWWISE) != 0) &&
+            agrees(q.nv_col, (a.outputs & NVFP4_COLWISE) != 0) &&
+            agrees(q.mx_row, (a.mx_outputs & NVFP4_ROWWISE) != 0) &&
+            agrees(q.mx_col, (a.mx_outputs & NVFP4_COLWISE) != 0) &&
+            agrees(q.sr, a.rounding == NVFP4_SR) && agrees(q.mx_sr, a.mx_rounding == NVFP4_SR) &&
+            agrees(q.rht, a.rht != 0) && agrees(q.two_d, a.scaling == NVFP4_2D16x16) &&
+            agrees(q.groups, a.group_offsets != nullptr))
+            return v;
+    }
+    return 0;
+}
+
 static DeviceInfo& device_info(int dev)
 {
     static DeviceInfo infos[64];
@@ -730,19 +1018,33 @@ static DeviceInfo& device_info(int dev)
         if (cudaGetDeviceProperties(&prop, dev) != cudaSuccess) return;
         if (prop.major != 10) return;
         d.sms = prop.multiProcessorCount;
-        if (cudaFuncSetAttribute(quant_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                 (int)quant_smem_bytes()) != cudaSuccess ||
-            cudaFuncSetAttribute(quant_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                 (int)quant_smem_bytes()) != cudaSuccess)
-            return;
-        int nb = 0, nb2 = 0;
-        if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&nb, quant_kernel<true>, kQuantThreads,
-                                                          quant_smem_bytes()) != cudaSuccess ||
-            cudaOccupancyMaxActiveBlocksPerMultiprocessor(&nb2, quant_kernel<false>, kQuantThreads,
-                                                          quant_smem_bytes()) != cudaSuccess ||
-            std::min(nb, nb2) < 1)
-            return;
-        d.quant_blocks_per_sm = std::min(nb, nb2);
+        int blocks = 1 << 30;
+        for (int tma = 0; tma < 2; ++tma) {
+            for (int v = 0; v < kNumSpecs; ++v) {
+                const QuantKernel fn = quant_variant(tma != 0, v);
+                if (!fn) continue;
+                int nb = 0;
+                if (cudaFuncSetAttribute(reinterpret_cast<const void*>(fn),
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         (int)quant_smem_bytes()) != cudaSuccess ||
+                    cudaOccupancyMaxActiveBlocksPerMultiprocessor(&nb, fn, kQuantThreads,
+                                                                  quant_smem_bytes()) != cudaSuccess ||
+                    nb < 1)
+                    return;
+                blocks = std::min(blocks, nb);
+            }
+        }
+        for (const void* fn : {reinterpret_cast<const void*>(amax_kernel)}) {
+            int nb = 0;
+            if (cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                     (int)quant_smem_bytes()) != cudaSuccess ||
+                cudaOccupancyMaxActiveBlocksPerMultiprocessor(&nb, fn, kQuantThreads,
+                                                              quant_smem_bytes()) != cudaSuccess ||
+                nb < 1)
+                return;
+            blocks = std::min(blocks, nb);
+        }
+        d.quant_blocks_per_sm = blocks;
         d.ok = true;
     });
     return infos[dev & 63];
@@ -788,25 +1090,29 @@ static nvfp4_status launch_quant(QArgs& a, bool need_amax, void* workspace, cuda
         if (cudaMemsetAsync(need_amax ? ws : ws + 2, 0, need_amax ? 12 : 4, st) != cudaSuccess)
             return NVFP4_ERR_CUDA;
     }
-    if (need_amax) {
-        uint32_t* amax = static_cast<uint32_t*>(workspace);
-        a.amax_ws = amax;
-        const int64_t units = (a.rows / 16) * (a.cols / 4);  // 16 rows x 4 columns each
-        const int64_t want = (units + 255) / 256;
-        const int blocks = (int)std::max<int64_t>(1, std::min<int64_t>(want, (int64_t)info.sms * 8));
-        amax_kernel<<<blocks, 256, 0, st>>>(a, amax);
-        if (cudaGetLastError() != cudaSuccess) return NVFP4_ERR_CUDA;
-    }
     const int64_t grid = std::min<int64_t>(a.n_tiles, (int64_t)info.sms * info.quant_blocks_per_sm);
     CUtensorMap map;
     memset(&map, 0, sizeof(map));
-    if (!a.row_index) {  // dense input: TMA tiles; the gather reads rows one by one
-        if (!make_input_map(&map, a.x, a.rows, a.cols, a.ld)) return NVFP4_ERR_CUDA;
-        quant_kernel<true><<<(int)grid, kQuantThreads, quant_smem_bytes(), st>>>(map, a);
-    } else {
-        quant_kernel<false><<<(int)grid, kQuantThreads, quant_smem_bytes(), st>>>(map, a);
+    const bool tma = !a.row_index;  // dense input: TMA tiles; the gather reads rows one by one
+    if (tma && !make_input_map(&map, a.x, a.rows, a.cols, a.ld)) return NVFP4_ERR_CUDA;
+    if (need_amax) {
+        uint32_t* amax = static_cast<uint32_t*>(workspace);
+        a.amax_ws = amax;
+        if (tma) {
+            amax_kernel<<<(int)grid, kQuantThreads, quant_smem_bytes(), st>>>(map, a, amax);
+        } else {
+            const int64_t units = (a.rows / 16) * (a.cols / 4);  // 16 rows x 4 columns each
+            const int blocks = (int)std::max<int64_t>(
+                1, std::min<int64_t>((units + 255) / 256, (int64_t)info.sms * 8));
+            amax_rows_kernel<<<blocks, 256, 0, st>>>(a, amax);
+        }
+        if (cudaGetLastError() != cudaSuccess) return NVFP4_ERR_CUDA;
     }
-    if (cudaGetLastError() != cudaSuccess) return NVFP4_ERR_CUDA;
+    const QuantKernel fn = quant_variant(tma, pick_variant(a, tma));
+    void* args[] = {&map, &a};
+    if (cudaLaunchKernel(reinterpret_cast<const void*>(fn), dim3((unsigned)grid), dim3(kQuantThreads),
+                         args, quant_smem_bytes(), st) != cudaSuccess)
+        return NVFP4_ERR_CUDA;
     return NVFP4_OK;
 }
 
@@ -950,6 +1256,32 @@ extern "C" nvfp4_status mxfp8_quantize(const void* x_bf16, int64_t rows, int64_t
     if (directions == 0 || (directions & ~3)) return NVFP4_ERR_INVALID_ARG;
     return nvfp4_quantize(x_bf16, rows, cols, ld, &p, nullptr, nullptr, nullptr, nullptr, nullptr,
                           nullptr, nullptr, 0, stream);
+}
+
+extern "C" nvfp4_status nvfp4_gather_rows(const uint8_t* q_src, const uint8_t* sf_src,
+                                          int64_t src_rows, int64_t k, const int32_t* row_index,
+                                          int64_t rows, const int32_t* group_offsets,
+                                          int num_groups, uint8_t* q_dst, uint8_t* sf_dst,
+                                          void* workspace, size_t ws_bytes, void* stream)
+{
+    if (!q_src || !sf_src || !row_index || !q_dst || !sf_dst) return NVFP4_ERR_INVALID_ARG;
+    if (src_rows <= 0 || rows <= 0 || k <= 0 || k % 64) return NVFP4_ERR_SHAPE;
+    if (group_offsets && (num_groups < 1 || num_groups > kMaxGroups)) return NVFP4_ERR_INVALID_ARG;
+    if (!aligned16(q_src) || !aligned16(q_dst) || (reinterpret_cast<uintptr_t>(sf_src) & 3) ||
+        (reinterpret_cast<uintptr_t>(sf_dst) & 3))
+        return NVFP4_ERR_ALIGN;
+    if (workspace && (ws_bytes < kQuantWorkspace || !aligned16(workspace))) return NVFP4_ERR_WORKSPACE;
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return NVFP4_ERR_CUDA;
+    if (!device_info(dev).ok) return NVFP4_ERR_UNSUPPORTED;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    uint32_t* status = workspace ? static_cast<uint32_t*>(workspace) + 2 : nullptr;
+    if (status && cudaMemsetAsync(status, 0, 4, st) != cudaSuccess) return NVFP4_ERR_CUDA;
+    const int64_t blocks = (rows + 127) / 128 + (group_offsets ? num_groups : 0);
+    gather_rows_kernel<<<(int)blocks, 256, 0, st>>>(q_src, sf_src, src_rows, k, row_index, rows,
+                                                    group_offsets, num_groups, q_dst, sf_dst,
+                                                    status);
+    return cudaGetLastError() == cudaSuccess ? NVFP4_OK : NVFP4_ERR_CUDA;
 }
 
 extern "C" nvfp4_status nvfp4_dequantize(const uint8_t* q, const uint8_t* sf, const float* g,

@@ -83,14 +83,31 @@ def test_quantize_argument_errors(nv):
 def test_gemm_argument_errors(nv):
     L = nv._lib
     args = (FAKE,) * 6
-    assert L.nvfp4_gemm(*args, 128, 128, 100, 0, FAKE, 128, FAKE, 256, None) == 2   # K % 256
-    assert L.nvfp4_gemm(*args, 100, 128, 256, 0, FAKE, 128, FAKE, 256, None) == 2   # M % 16
-    assert L.nvfp4_gemm(*args, 128, 128, 256, 0, FAKE, 120, FAKE, 256, None) == 2   # ldd < N
-    assert L.nvfp4_gemm(*args, 128, 128, 256, 1, FAKE, 132, FAKE, 256, None) == 3   # ldd align
-    assert L.nvfp4_gemm(*args, 128, 128, 256, 0, FAKE, 128, None, 0, None) == 7     # workspace
-    assert L.nvfp4_gemm(*args, 128, 128, 256, 5, FAKE, 128, FAKE, 256, None) == 1   # dtype
-    assert L.nvfp4_grouped_gemm(0, FAKE, 128, *args, 128, 256, 0, FAKE, FAKE, 256, None) == 1
-    assert L.nvfp4_grouped_gemm(4, FAKE, 128, *args, 100, 256, 0, FAKE, FAKE, 256, None) == 2
+    g = L.nvfp4_gemm
+    assert g(*args, 128, 128, 100, 0, FAKE, 128, None, FAKE, 256, None) == 2       # K % 256
+    assert g(*args, 100, 128, 256, 0, FAKE, 128, None, FAKE, 256, None) == 2       # M % 16
+    assert g(*args, 128, 128, 256, 0, FAKE, 120, None, FAKE, 256, None) == 2       # ldd < N
+    assert g(*args, 128, 128, 256, 1, FAKE, 132, None, FAKE, 256, None) == 3       # ldd align
+    assert g(*args, 128, 128, 256, 0, FAKE, 128, None, None, 0, None) == 7         # workspace
+    assert g(*args, 128, 128, 256, 5, FAKE, 128, None, FAKE, 256, None) == 1       # dtype
+    assert g(*args, 128, 128, 256, 0, FAKE, 128, FAKE + 2, FAKE, 256, None) == 3   # amax_out
+    gg = L.nvfp4_grouped_gemm
+    assert gg(0, FAKE, 128, *args, 128, 256, 0, FAKE, None, FAKE, 256, None) == 1
+    assert gg(257, FAKE, 128, *args, 256, 256, 0, FAKE, None, FAKE, 256, None) == 1  # G > 256
+    assert gg(4, FAKE, 128, *args, 100, 256, 0, FAKE, None, FAKE, 256, None) == 2
+    assert gg(4, FAKE, 128, *args, 256, 256, 0, FAKE, FAKE + 1, FAKE, 256, None) == 3
+
+
+def test_gather_rows_argument_errors(nv):
+    L = nv._lib.nvfp4_gather_rows
+    assert L(None, FAKE, 64, 64, FAKE, 64, None, 0, FAKE, FAKE, FAKE, 256, None) == 1
+    assert L(FAKE, FAKE, 64, 48, FAKE, 64, None, 0, FAKE, FAKE, FAKE, 256, None) == 2  # k % 64
+    assert L(FAKE, FAKE, 0, 64, FAKE, 64, None, 0, FAKE, FAKE, FAKE, 256, None) == 2   # no source
+    assert L(FAKE, FAKE, 64, 64, FAKE, 64, FAKE, 0, FAKE, FAKE, FAKE, 256, None) == 1  # 0 groups
+    assert L(FAKE, FAKE, 64, 64, FAKE, 64, FAKE, 300, FAKE, FAKE, FAKE, 256, None) == 1
+    assert L(FAKE + 4, FAKE, 64, 64, FAKE, 64, None, 0, FAKE, FAKE, FAKE, 256, None) == 3
+    assert L(FAKE, FAKE + 2, 64, 64, FAKE, 64, None, 0, FAKE, FAKE, FAKE, 256, None) == 3
+    assert L(FAKE, FAKE, 64, 64, FAKE, 64, None, 0, FAKE, FAKE, FAKE, 8, None) == 7   # workspace
 
 
 def test_mxfp8_and_dequant_argument_errors(nv):

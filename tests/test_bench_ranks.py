@@ -46,3 +46,24 @@ def test_job_throughput_counts_all_replicas():
     assert bench.job_tflops(1e12, 1, 10, 1000.0) == pytest.approx(10.0)
     assert bench.job_tflops(1e12, 4, 10, 1000.0) == pytest.approx(40.0)
     assert bench.max_over_ranks([3.0, 4.0], 1) == [3.0, 4.0]
+
+
+def test_clock_summary_decodes_reasons():
+    """The clock record: median SM clock under load and the reasons seen, decoded from
+    the NVML bit mask (a fake NVML module; nothing is queried)."""
+    import types
+
+    import bench
+    fake = types.SimpleNamespace(nvmlClocksEventReasonHwSlowdown=0x8,
+                                 nvmlClocksEventReasonHwThermalSlowdown=0x40,
+                                 nvmlClocksEventReasonSwThermalSlowdown=0x20,
+                                 nvmlClocksEventReasonSwPowerCap=0x4)
+    c = bench.ClockSampler("cpu")
+    assert c.summary()["reasons"] == ["unsampled"]
+    c.nvml, c.max_mhz = fake, 1965
+    c.samples = [(1900, 0), (1950, 0x4), (1800, 0x4 | 0x1), (1965, 0)]
+    s = c.summary()
+    assert s["sm_mhz"] == 1925 and s["sm_max_mhz"] == 1965
+    assert s["reasons"] == ["sw_power_cap"]
+    c.samples.append((1200, 0x40))
+    assert bench.ClockSampler.summary(c)["reasons"] == ["hw_thermal_slowdown", "sw_power_cap"]

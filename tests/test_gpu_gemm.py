@@ -62,7 +62,7 @@ def test_gemm_padded_ldd(nv, orc):
     (qa, sa, ga), (qb, sb, gb), A, B = _operands(orc, nv, x, w)
     out = torch.full((M, N + 64), 7.0, dtype=torch.float32, device="cuda")
     ws = torch.empty(256, dtype=torch.uint8, device="cuda")
-    nv.nvfp4_gemm(A.q, A.sf, A.g, B.q, B.sf, B.g, M, N, K, nv.NVFP4_OUT_F32, out, N + 64, ws, 256)
+    nv.nvfp4_gemm(A.q, A.sf, A.g, B.q, B.sf, B.g, M, N, K, nv.NVFP4_OUT_F32, out, N + 64, None, ws, 256)
     D = host(out)
     assert np.all(D[:, N:] == 7.0)
     Dr, Ar = orc.nvfp4_gemm_rows(qa, sa, ga, qb, sb, gb)
@@ -163,3 +163,51 @@ def test_grouped_gemm_moe_up_sampled(nv, orc):
             qa, sa, ga = orc.nvfp4_quantize(xr, 0, amax=am)
             Dr, Ar = orc.nvfp4_gemm_rows(qa, sa, ga, qb, sb, gb, rows_sel=[0])
             check_gemm(D[r:r + 1], Dr, Ar, True)
+
+
+@pytest.mark.parametrize("bf16_out", [False, True])
+def test_gemm_amax_out(nv, orc, bf16_out):
+    """amax_out holds max |D| over the stored output, exactly, and replaces a stale value."""
+    import torch
+    M, N, K = 272, 400, 512
+    rng = np.random.default_rng(11)
+    x = W.f32_to_bf16_bits(W.student_t(rng, (M, K), 3.0, 1.0))
+    w = W.f32_to_bf16_bits(rng.standard_normal((N, K)).astype(np.float32) * 0.02)
+    _, _, A, B = _operands(orc, nv, x, w)
+    am = torch.full((1,), 1e30, dtype=torch.float32, device="cuda")
+    D = host(nv.gemm(A, B, nv.NVFP4_OUT_BF16 if bf16_out else nv.NVFP4_OUT_F32, amax_out=am))
+    if bf16_out:
+        D = W.bf16_bits_to_f32(D.view(np.uint16))
+    assert host(am)[0] == np.max(np.abs(D)).astype(np.float32)
+
+
+def test_grouped_gemm_amax_out(nv, orc):
+    """Grouped: the max covers every group's rows and nothing from padding tiles."""
+    import torch
+    N, K = 256, 512
+    offsets, _, _, A, qb_d, sfb_d, gb_d, off_d = _grouped_case(orc, nv, [0, 150, 7, 0, 33, 130],
+                                                                N, K, seed=5)
+    am = torch.zeros(1, dtype=torch.float32, device="cuda")
+    D = host(nv.grouped_gemm(off_d, A, qb_d, sfb_d, gb_d, N, amax_out=am))
+    D = W.bf16_bits_to_f32(D.view(np.uint16))
+    assert host(am)[0] == np.max(np.abs(D)).astype(np.float32)
+
+
+def test_requantize_with_gemm_amax(nv, orc):
+    """Quantising the up projection's output with the GEMM's amax_out as amax_in gives the
+    same bytes as the quantiser's own amax pass (and the oracle's quantisation)."""
+    import torch
+    N, K = 256, 512
+    counts = [0, 150, 7, 0, 33, 130]
+    offsets, _, _, A, qb_d, sfb_d, gb_d, off_d = _grouped_case(orc, nv, counts, N, K, seed=9)
+    am = torch.zeros(2, dtype=torch.float32, device="cuda")
+    H = nv.grouped_gemm(off_d, A, qb_d, sfb_d, gb_d, N, amax_out=am)
+    kw = dict(group_offsets=off_d, num_groups=len(counts), sf_layout=nv.NVFP4_SF_MMA)
+    fused = nv.quantize(H, amax=am, **kw)["row"]
+    own = nv.quantize(H, **kw)["row"]
+    for f in ("q", "sf", "g"):
+        assert np.array_equal(host(getattr(fused, f)), host(getattr(own, f)))
+    q, sf, g = orc.nvfp4_quantize(host(H), 0)
+    assert np.array_equal(host(fused.q), q)
+    assert np.array_equal(sf_mma_to_rowmajor(host(fused.sf), int(offsets[-1]), N,
+                                             grouped_padded_rows(offsets)), sf)

@@ -210,3 +210,42 @@ def test_full_size_gradient_bitexact(nv, orc, rht):
         q8, e8 = orc.mxfp8_quantize(xs, 1, 0, 1)
         np.testing.assert_array_equal(mq[c0:c0 + 64], q8)
         np.testing.assert_array_equal(me[c0:c0 + 64], e8)
+
+
+@pytest.mark.parametrize("grouped", [False, True])
+def test_gather_rows_matches_oracle(nv, orc, grouped):
+    """Quantise 512 tokens once, dispatch 1008 routed rows (every token routed at least
+    once, so the source amax is the routed rows' amax): the dispatched codes and scales
+    equal the oracle's quantisation of the gathered rows, and the fused gather-quantize."""
+    import torch
+    rng = np.random.default_rng(21)
+    tokens, k, E = 512, 320, 5
+    x = W.f32_to_bf16_bits(W.student_t(rng, (tokens, k), 4.0, 1.0))
+    row_index = np.concatenate([rng.permutation(tokens), rng.integers(0, tokens, 496)]).astype(np.int32)
+    total = row_index.size
+    offsets = np.array([0, 300, 300, 717, 718, total], dtype=np.int32) if grouped else None
+    src = nv.quantize(to_dev(x), sf_layout=nv.NVFP4_SF_MMA)["row"]
+    idx_d = torch.from_numpy(row_index).cuda()
+    off_d = torch.from_numpy(offsets).cuda() if grouped else None
+    got = nv.gather_rows(src, idx_d, off_d)
+    xg = np.ascontiguousarray(x[row_index])
+    qo, so, go = orc.nvfp4_quantize(xg, 0, amax=(orc.amax(x, 0), 0.0))
+    assert np.array_equal(host(got.q), qo)
+    pr = grouped_padded_rows(offsets) if grouped else None
+    assert np.array_equal(sf_mma_to_rowmajor(host(got.sf), total, k, pr), so)
+    assert host(got.g)[0] == np.float32(go)
+    fused = nv.quantize(to_dev(x), rows=total, row_index=idx_d, src_rows=tokens,
+                        group_offsets=off_d, num_groups=E if grouped else 0,
+                        sf_layout=nv.NVFP4_SF_MMA)["row"]
+    assert np.array_equal(host(fused.q), host(got.q))
+    assert np.array_equal(host(fused.sf), host(got.sf))
+
+
+def test_gather_rows_bad_index_reports(nv):
+    import torch
+    x = torch.zeros((64, 64), dtype=torch.bfloat16, device="cuda")
+    src = nv.quantize(x, sf_layout=nv.NVFP4_SF_MMA)["row"]
+    idx = torch.tensor([0, 5, 64] + [1] * 13, dtype=torch.int32, device="cuda")
+    ws = torch.zeros(256, dtype=torch.uint8, device="cuda")
+    nv.gather_rows(src, idx, workspace=ws)
+    assert nv.nvfp4_workspace_status(ws) == 8
