@@ -1,0 +1,93 @@
+"""Single-case drivers for profiling one kernel launch under ncu.
+
+    python -m nvfp4_bit_precision_b200.profile_cases gemm M N K [--warm W]
+    python -m nvfp4_bit_precision_b200.profile_cases grouped-gemm N K [--warm W]
+    python -m nvfp4_bit_precision_b200.profile_cases quant-grad ROWS COLS [--warm W]
+
+Each runs W untimed launches of the case, then one more, on synthetic operands
+(codes and in-range scale bytes drawn on the device; bf16 inputs ~N(0, 1e-3)),
+and exits 0 when the device status word is clear.  Pair with `ncu -s W -c 1`.
+"""
+from __future__ import annotations
+
+import argparse
+import sys
+
+
+def _gemm(nv, torch, M, N, K, warm):
+    dev = torch.device("cuda")
+    g = torch.Generator(device=dev)
+    g.manual_seed(0)
+    u8 = dict(dtype=torch.uint8, device=dev)
+    qa = torch.randint(0, 256, (M, K // 2), generator=g, **u8)
+    qb = torch.randint(0, 256, (N, K // 2), generator=g, **u8)
+    sa = torch.randint(0x30, 0x40, (nv.nvfp4_sf_mma_bytes(M, K),), generator=g, **u8)
+    sb = torch.randint(0x30, 0x40, (nv.nvfp4_sf_mma_bytes(N, K),), generator=g, **u8)
+    one = torch.ones(1, dtype=torch.float32, device=dev)
+    D = torch.empty((M, N), dtype=torch.bfloat16, device=dev)
+    ws = torch.zeros(256, **u8)
+    for _ in range(warm + 1):
+        nv.nvfp4_gemm(qa, sa, one, qb, sb, one, M, N, K, nv.NVFP4_OUT_BF16, D, N, None, ws, 256)
+    return ws
+
+
+def _grouped(nv, torch, N, K, warm):
+    import numpy as np
+
+    import workloads as W
+    dev = torch.device("cuda")
+    rng = np.random.default_rng(3)
+    _, _, offsets = W.moe_routing(rng, 16384, 64, 4)
+    R, G = int(offsets[-1]), 64
+    u8 = dict(dtype=torch.uint8, device=dev)
+    qa = torch.randint(0, 256, (R, K // 2), **u8)
+    sa = torch.randint(0x30, 0x40, (nv.nvfp4_sf_mma_grouped_bytes(R, G, K),), **u8)
+    qb = torch.randint(0, 256, (G, N, K // 2), **u8)
+    sb = torch.randint(0x30, 0x40, (G * nv.nvfp4_sf_mma_bytes(N, K),), **u8)
+    ga = torch.ones(1, dtype=torch.float32, device=dev)
+    gb = torch.ones(G, dtype=torch.float32, device=dev)
+    off = torch.from_numpy(offsets.astype(np.int32)).to(dev)
+    D = torch.empty((R, N), dtype=torch.bfloat16, device=dev)
+    ws = torch.zeros(256, **u8)
+    for _ in range(warm + 1):
+        nv.nvfp4_grouped_gemm(G, off, R, qa, sa, ga, qb, sb, gb, N, K, nv.NVFP4_OUT_BF16, D, None,
+                              ws, 256)
+    return ws
+
+
+def _quant_grad(nv, torch, rows, cols, warm):
+    """The gradient recipe: rowwise SR, columnwise Hadamard + SR, MXFP8 columnwise."""
+    dev = torch.device("cuda")
+    g = torch.Generator(device=dev)
+    g.manual_seed(1)
+    x = (torch.randn((rows, cols), generator=g, device=dev) * 1e-3).to(torch.bfloat16)
+    ws = torch.zeros(256, dtype=torch.uint8, device=dev)
+    for _ in range(warm + 1):
+        nv.quantize(x, rowwise=True, colwise=True, rounding=nv.NVFP4_SR, rht=True, seed=5,
+                    mx_outputs=nv.NVFP4_COLWISE, sf_layout=nv.NVFP4_SF_MMA, workspace=ws)
+    return ws
+
+
+def main(argv=None) -> int:
+    ap = argparse.ArgumentParser()
+    ap.add_argument("case", choices=["gemm", "grouped-gemm", "quant-grad"])
+    ap.add_argument("dims", type=int, nargs="+")
+    ap.add_argument("--warm", type=int, default=3)
+    args = ap.parse_args(argv)
+    import torch
+
+    import nvfp4_bit_precision_b200 as nv
+    if args.case == "gemm":
+        ws = _gemm(nv, torch, *args.dims[:3], args.warm)
+    elif args.case == "grouped-gemm":
+        ws = _grouped(nv, torch, *args.dims[:2], args.warm)
+    else:
+        ws = _quant_grad(nv, torch, *args.dims[:2], args.warm)
+    torch.cuda.synchronize()
+    status = nv.nvfp4_workspace_status(ws)
+    print(f"{args.case} {args.dims}: status {nv.status_string(status)}")
+    return 0 if status == 0 else 1
+
+
+if __name__ == "__main__":
+    sys.exit(main())
