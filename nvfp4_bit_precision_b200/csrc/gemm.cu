@@ -8,17 +8,21 @@
 // Machines uskorila obuchenie Inkling 2 Small 4-bitnymi chislami", section
 // "Details": NVFP4 in the expert layers -> the grouped form).
 //
-// Structure (one persistent CTA per SM, 320 threads):
+// Structure (one persistent CTA per SM, 448 threads):
 //   warp 0      TMA producer: A/B tiles (128-byte swizzled, 4-bit codes packed
 //               two per byte) by cp.async.bulk.tensor, scale atoms by
 //               cp.async.bulk, into a 4-stage ring guarded by mbarriers.
-//   warp 1      one elected thread moves the stage's scale factors into tensor
-//               memory (tcgen05.cp 32x128b.warpx4) and issues 4 MMAs of
-//               128x256x64, then commits the stage back to the producer and,
-//               after the last K stage, the accumulator to the epilogue.
-//   warps 2..9  epilogue: tcgen05.ld of the 128x256 FP32 accumulator (two
-//               warps per lane quadrant), release of the accumulator, then
-//               times ga*gb, conversion and stores to global memory.
+//   warps 2..5  scale writers, one per tensor-memory lane quadrant: each lane
+//               loads row i of the stage's 512-byte scale atoms from shared
+//               memory and writes them into its quadrant with tcgen05.st, so
+//               the tensor pipe spends no cycles on scale copies.
+//   warp 1      one elected thread waits for a stage's tiles and scales and
+//               issues 4 MMAs of 128x256x64, then commits the stage back to
+//               the producer and, after the last K stage, the accumulator to
+//               the epilogue.
+//   warps 6..13 epilogue: tcgen05.ld of the 128x256 FP32 accumulator (two
+//               warps per lane quadrant, converted as it is loaded), release
+//               of the accumulator, then stores to global memory.
 // Every mbarrier wait is bounded (2 s); a timeout sets the workspace status
 // word and the kernel winds down instead of hanging.
 #include <cudaTypedefs.h>
@@ -39,9 +43,13 @@ constexpr int kB_Bytes = BN * BK / 2;      // 32 KB
 constexpr int kSFA_Bytes = BM * BK / 16;   // 2 KB: 4 atoms of 512 B
 constexpr int kSFB_Bytes = BN * BK / 16;   // 4 KB: 2 row blocks x 4 atoms
 constexpr int kStageBytes = kA_Bytes + kB_Bytes + kSFA_Bytes + kSFB_Bytes;
-constexpr int kGemmThreads = 320;  // producer, MMA, 8 epilogue warps
+constexpr int kGemmThreads = 448;  // producer, MMA, 4 scale writers, 8 epilogue warps
 // Tensor memory: the 128x256 FP32 accumulator in columns 0..255, then one
 // 48-column scale region per pipeline stage (SFA 4 x 4 columns, SFB 4 x 8).
+// Within a region, column 4j + c of every lane quadrant holds, in lane i, the
+// four scales of row 32c + i for K-group j (SFA) -- row i of the K-group's
+// 512-byte atom; SFB keeps rows 0..127 at 16 + 8j + c, rows 128..255 at
+// 16 + 8j + 4 + c.
 constexpr int kTmemCols = 512;
 constexpr int kTmemSF = 256;
 constexpr int kTmemSFStage = 48;
@@ -68,6 +76,7 @@ struct GemmArgs {
 struct GemmShared {
     uint64_t full[kGemmStages];
     uint64_t empty[kGemmStages];
+    uint64_t sf_ready[kGemmStages];
     uint64_t acc_full;
     uint64_t acc_empty;
     uint32_t tmem_base;
@@ -111,20 +120,6 @@ __device__ __forceinline__ uint64_t desc_sw128(const void* p)
     return start | (1ull << 16) | (64ull << 32) | (1ull << 46) | (2ull << 61);
 }
 
-// Descriptor of one 512-byte scale atom: 32 rows of 16 bytes, no swizzle,
-// 8-row groups 128 bytes apart.
-__device__ __forceinline__ uint64_t desc_sf_atom(const void* p)
-{
-    const uint64_t start = (smem_addr(p) >> 4) & 0x3FFFu;
-    return start | (1ull << 16) | (8ull << 32) | (1ull << 46);
-}
-
-__device__ __forceinline__ void tc_cp_sf(uint32_t taddr, uint64_t desc)
-{
-    asm volatile("tcgen05.cp.cta_group::1.32x128b.warpx4 [%0], %1;" ::"r"(taddr), "l"(desc)
-                 : "memory");
-}
-
 // Instruction descriptor: kind::mxf4nvf4, A/B E2M1 (format 1), UE4M3 scales,
 // both K-major, M = 128, N = 256, dense, K = 64 per instruction.
 __host__ __device__ constexpr uint32_t make_idesc()
@@ -157,6 +152,15 @@ __device__ __forceinline__ void tc_mma(uint32_t d_tmem, uint64_t adesc, uint64_t
                    "=r"(r[30]), "=r"(r[31])                                                        \
                  : "r"(taddr))
 
+
+__device__ __forceinline__ uint4 lds128(const void* p)
+{
+    uint4 r;
+    asm volatile("ld.shared.v4.u32 {%0,%1,%2,%3}, [%4];" : "=r"(r.x), "=r"(r.y), "=r"(r.z), "=r"(r.w) : "r"(smem_addr(p)));
+    return r;
+}
+#define TMEM_ST_16(taddr, v) asm volatile("tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16};" ::"r"(taddr), "r"((v)[0]), "r"((v)[1]), "r"((v)[2]), "r"((v)[3]), "r"((v)[4]), "r"((v)[5]), "r"((v)[6]), "r"((v)[7]), "r"((v)[8]), "r"((v)[9]), "r"((v)[10]), "r"((v)[11]), "r"((v)[12]), "r"((v)[13]), "r"((v)[14]), "r"((v)[15]) : "memory")
+#define TMEM_ST_32(taddr, v) asm volatile("tcgen05.st.sync.aligned.32x32b.x32.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31,%32};" ::"r"(taddr), "r"((v)[0]), "r"((v)[1]), "r"((v)[2]), "r"((v)[3]), "r"((v)[4]), "r"((v)[5]), "r"((v)[6]), "r"((v)[7]), "r"((v)[8]), "r"((v)[9]), "r"((v)[10]), "r"((v)[11]), "r"((v)[12]), "r"((v)[13]), "r"((v)[14]), "r"((v)[15]), "r"((v)[16]), "r"((v)[17]), "r"((v)[18]), "r"((v)[19]), "r"((v)[20]), "r"((v)[21]), "r"((v)[22]), "r"((v)[23]), "r"((v)[24]), "r"((v)[25]), "r"((v)[26]), "r"((v)[27]), "r"((v)[28]), "r"((v)[29]), "r"((v)[30]), "r"((v)[31]) : "memory")
 __device__ __forceinline__ void tmem_ld_wait() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory"); }
 
 // ---------------------------------------------------------------- scheduling
@@ -219,6 +223,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         for (int s = 0; s < kGemmStages; ++s) {
             mbar_init(&sh->full[s], 1);
             mbar_init(&sh->empty[s], 1);
+            mbar_init(&sh->sf_ready[s], 4);
         }
         mbar_init(&sh->acc_full, 1);
         mbar_init(&sh->acc_empty, 8);
@@ -312,20 +317,15 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
                         failed = true;
                         break;
                     }
+                    if (!mbar_wait(&sh->sf_ready[s], ph)) {
+                        record_status(a.status, NVFP4_ERR_TIMEOUT);
+                        failed = true;
+                        break;
+                    }
                     tc_fence_after();
                     uint8_t* st = smem + s * kStageBytes;
-                    const uint8_t* sfa_s = st + kA_Bytes + kB_Bytes;
-                    const uint8_t* sfb_s = sfa_s + kSFA_Bytes;
-                    // this stage's own scale columns: no overwrite of scales that
-                    // the previous stages' MMAs may still be reading
                     const uint32_t t_sfa = tmem + kTmemSF + (uint32_t)s * kTmemSFStage;
                     const uint32_t t_sfb = t_sfa + 16;
-#pragma unroll
-                    for (int j = 0; j < 4; ++j) {
-                        tc_cp_sf(t_sfa + 4 * j, desc_sf_atom(sfa_s + j * 512));
-                        tc_cp_sf(t_sfb + 8 * j, desc_sf_atom(sfb_s + j * 512));
-                        tc_cp_sf(t_sfb + 8 * j + 4, desc_sf_atom(sfb_s + kSFB_Bytes / 2 + j * 512));
-                    }
                     const uint64_t ad = desc_sw128(st), bd = desc_sw128(st + kA_Bytes);
 #pragma unroll
                     for (int j = 0; j < 4; ++j) {
@@ -339,14 +339,50 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
                 tc_commit(&sh->acc_full);
             }
         }
+    } else if (warp < 6) {
+        // ------------------------------------------------ scale writers (warps 2..5)
+        // Each warp writes its lane quadrant of the stage's scale columns with
+        // tcgen05.st: lane i gets row i of every 512-byte atom (the layout the
+        // broadcast copy would produce in each quadrant).
+        const uint32_t lane_base = (uint32_t)(32 * (warp & 3)) << 16;
+        uint32_t it = 0;
+        for (int t = blockIdx.x; t < total && !failed; t += gridDim.x) {
+            for (int64_t ks = 0; ks < kstages; ++ks, ++it) {
+                const int s = (int)(it % kGemmStages);
+                const uint32_t ph = (it / kGemmStages) & 1u;
+                bool ok = true;
+                if (lane == 0) ok = mbar_wait(&sh->full[s], ph);
+                ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
+                if (!ok) {
+                    if (lane == 0) record_status(a.status, NVFP4_ERR_TIMEOUT);
+                    failed = true;
+                    break;
+                }
+                const uint8_t* sfa_s = smem + s * kStageBytes + kA_Bytes + kB_Bytes;
+                const uint8_t* sfb_s = sfa_s + kSFA_Bytes;
+                uint32_t v[48];
+#pragma unroll
+                for (int j = 0; j < 4; ++j) {
+                    const uint4 x = lds128(sfa_s + j * 512 + lane * 16);
+                    v[4 * j] = x.x, v[4 * j + 1] = x.y, v[4 * j + 2] = x.z, v[4 * j + 3] = x.w;
+                    const uint4 lo = lds128(sfb_s + j * 512 + lane * 16);
+                    const uint4 hi = lds128(sfb_s + kSFB_Bytes / 2 + j * 512 + lane * 16);
+                    v[16 + 8 * j] = lo.x, v[17 + 8 * j] = lo.y, v[18 + 8 * j] = lo.z, v[19 + 8 * j] = lo.w;
+                    v[20 + 8 * j] = hi.x, v[21 + 8 * j] = hi.y, v[22 + 8 * j] = hi.z, v[23 + 8 * j] = hi.w;
+                }
+                const uint32_t taddr = tmem + lane_base + kTmemSF + (uint32_t)s * kTmemSFStage;
+                TMEM_ST_16(taddr, v);
+                TMEM_ST_32(taddr + 16, (v + 16));
+                asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&sh->sf_ready[s]);
+            }
+        }
     } else {
-        // ------------------------------------------------ epilogue (warps 2..9)
-        // Two warps per TMEM lane quadrant, 128 accumulator columns each.  All
-        // of a warp's tcgen05.ld are issued before one wait, and the accumulator
-        // is handed back to the MMA thread before the conversion and stores, so
-        // the next tile's MMAs overlap this tile's stores.
+        // ------------------------------------------------ epilogue (warps 6..13)
         const int quad = warp & 3;                   // TMEM lanes 32*quad .. 32*quad+31
-        const int col0 = ((warp - 2) >> 2) * (BN / 2);  // 0 or 128
+        const int col0 = ((warp - 6) >> 2) * (BN / 2);  // 0 or 128
         float out_max = 0.0f;                            // max |D| stored by this thread
         uint32_t tcount = 0;
         for (int t = blockIdx.x; t < total; t += gridDim.x, ++tcount) {
@@ -358,58 +394,79 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
             }
             tc_fence_after();
             const uint32_t tbase = tmem + ((uint32_t)(32 * quad) << 16) + (uint32_t)col0;
-            uint32_t r[4][32];
-            TMEM_LD_32(tbase + 0, r[0]);
-            TMEM_LD_32(tbase + 32, r[1]);
-            TMEM_LD_32(tbase + 64, r[2]);
-            TMEM_LD_32(tbase + 96, r[3]);
-            tmem_ld_wait();
-            tc_fence_before();
-            __syncwarp();
-            if (lane == 0) mbar_arrive(&sh->acc_empty);  // accumulator drained
-
             const float alpha = __fmul_rn(a.ga[0], a.gb[c.group]);
             const int64_t row = c.row0 + 32 * quad + lane;
-            if (row >= c.row_end) continue;
-            const int64_t cbase = c.n0 + col0;
+            const bool row_ok = row < c.row_end;
             if (a.bf16_out) {
-                uint16_t* drow = static_cast<uint16_t*>(a.D) + row * a.ldd + cbase;
+                // 128 columns in four 32-column loads, each converted to bf16
+                // pairs at once: the accumulator is released before any store
+                // with at most 32 + 64 registers of data live.
+                uint32_t packed[64];
+                float m_all = 0.0f;  // max |x| over the 128 columns (before rounding)
 #pragma unroll
-                for (int ch = 0; ch < 4; ++ch) {
+                for (int hh = 0; hh < 4; ++hh) {
+                    uint32_t r[32];
+                    TMEM_LD_32(tbase + 32 * hh, r);
+                    tmem_ld_wait();
 #pragma unroll
-                    for (int v = 0; v < 4; ++v) {
-                        uint32_t w[4];
-                        float vm = 0.0f;
+                    for (int i = 0; i < 16; ++i) {
+                        const float x0 = __fmul_rn(__uint_as_float(r[2 * i]), alpha);
+                        const float x1 = __fmul_rn(__uint_as_float(r[2 * i + 1]), alpha);
+                        m_all = absmax3(m_all, x0, x1);
+                        const __nv_bfloat162 p = __floats2bfloat162_rn(x0, x1);
+                        packed[16 * hh + i] = *reinterpret_cast<const uint32_t*>(&p);
+                    }
+                }
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&sh->acc_empty);  // accumulator drained
+                if (row_ok) {
+                    const int64_t cbase = c.n0 + col0;
+                    uint16_t* drow = static_cast<uint16_t*>(a.D) + row * a.ldd + cbase;
+                    const bool whole = cbase + 128 <= a.N;
+                    if (whole) out_max = fmaxf(out_max, m_all);
 #pragma unroll
-                        for (int i = 0; i < 4; ++i) {
-                            const float x0 = __fmul_rn(__uint_as_float(r[ch][8 * v + 2 * i]), alpha);
-                            const float x1 = __fmul_rn(__uint_as_float(r[ch][8 * v + 2 * i + 1]), alpha);
-                            vm = absmax3(vm, x0, x1);
-                            const __nv_bfloat162 p = __floats2bfloat162_rn(x0, x1);
-                            w[i] = *reinterpret_cast<const uint32_t*>(&p);
-                        }
-                        if (cbase + 32 * ch + 8 * v < a.N) {
-                            *reinterpret_cast<uint4*>(drow + 32 * ch + 8 * v) =
-                                make_uint4(w[0], w[1], w[2], w[3]);
-                            out_max = fmaxf(out_max, vm);
+                    for (int g = 0; g < 16; ++g) {  // 8 columns per 16-byte store
+                        if (cbase + 8 * g < a.N) {
+                            *reinterpret_cast<uint4*>(drow + 8 * g) = make_uint4(
+                                packed[4 * g], packed[4 * g + 1], packed[4 * g + 2], packed[4 * g + 3]);
+                            if (!whole) {  // N tail: the max of the stored (rounded) values
+#pragma unroll
+                                for (int i = 0; i < 4; ++i) {
+                                    const uint32_t w = packed[4 * g + i];
+                                    out_max = absmax3(out_max, __uint_as_float(w << 16),
+                                                      __uint_as_float(w & 0xFFFF0000u));
+                                }
+                            }
                         }
                     }
                 }
-            } else {
+                continue;
+            }
+            // FP32 output: four rounds of 32 columns, each stored before the
+            // next load; the accumulator is released after the last load.
+#pragma unroll 1
+            for (int hh = 0; hh < 4; ++hh) {
+                uint32_t r[32];
+                TMEM_LD_32(tbase + 32 * hh, r);
+                tmem_ld_wait();
+                if (hh == 3) {
+                    tc_fence_before();
+                    __syncwarp();
+                    if (lane == 0) mbar_arrive(&sh->acc_empty);  // accumulator drained
+                }
+                if (!row_ok) continue;
+                const int64_t cbase = c.n0 + col0 + 32 * hh;
                 float* drow = static_cast<float*>(a.D) + row * a.ldd + cbase;
 #pragma unroll
-                for (int ch = 0; ch < 4; ++ch) {
-#pragma unroll
-                    for (int v = 0; v < 8; ++v) {
-                        const float x0 = __fmul_rn(__uint_as_float(r[ch][4 * v]), alpha);
-                        const float x1 = __fmul_rn(__uint_as_float(r[ch][4 * v + 1]), alpha);
-                        const float x2 = __fmul_rn(__uint_as_float(r[ch][4 * v + 2]), alpha);
-                        const float x3 = __fmul_rn(__uint_as_float(r[ch][4 * v + 3]), alpha);
-                        if (cbase + 32 * ch + 4 * v < a.N) {
-                            *reinterpret_cast<float4*>(drow + 32 * ch + 4 * v) =
-                                make_float4(x0, x1, x2, x3);
-                            out_max = absmax3(out_max, absmax3(x0, x1, x2), x3);
-                        }
+                for (int v = 0; v < 8; ++v) {
+                    const float x0 = __fmul_rn(__uint_as_float(r[4 * v]), alpha);
+                    const float x1 = __fmul_rn(__uint_as_float(r[4 * v + 1]), alpha);
+                    const float x2 = __fmul_rn(__uint_as_float(r[4 * v + 2]), alpha);
+                    const float x3 = __fmul_rn(__uint_as_float(r[4 * v + 3]), alpha);
+                    if (cbase + 4 * v < a.N) {
+                        *reinterpret_cast<float4*>(drow + 4 * v) = make_float4(x0, x1, x2, x3);
+                        out_max = absmax3(out_max, absmax3(x0, x1, x2), x3);
                     }
                 }
             }
