@@ -42,6 +42,13 @@ DENSE_FLOP = 3 * 2 * TOKENS * FFN * HIDDEN
 DENSE_FLOP_PER_GEMM = 2 * TOKENS * FFN * HIDDEN
 
 
+# DRAM traffic per launch (dram__bytes_read.sum + dram__bytes_write.sum) from one
+# ncu --set full capture of each kernel as it stands -- the forward GEMM
+# 16384x20480x5120, and the amax + fused pass on dY 16384x20480; set to None
+# whenever the kernel changes.
+TRAFFIC_BYTES = {"gemm_dense_fwd": 1313.4e6, "quant_dy": 2236.3e6}
+
+
 def peaks():
     p = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0,
          "source": "fallback"}
@@ -547,14 +554,18 @@ def main():
                          "16384x20480x5120 class, mean of fwd/dgrad/wgrad launches)",
                          "achieved": round(gemm_tflops, 1), "peak": round(fp4_peak, 1),
                          "unit": "TFLOP/s", "frac": round(gemm_tflops / fp4_peak, 4),
-                         "traffic": None,
+                         "traffic": TRAFFIC_BYTES["gemm_dense_fwd"],
+                         "traffic_note": "bytes per launch of the forward GEMM 16384x20480x5120 "
+                                         "(ncu capture); algorithmic operand bytes 104 MB + "
+                                         "output 671 MB",
                          "peak_note": f"4 x {pk['bf16_tflops_sustained']} sustained bf16 "
                                       f"(fp4/bf16 nominal ratio 9/2.25), of {pk['source']}"},
             "quantize_roofline": {"bound": "hbm", "kernel": "amax_kernel + quant_kernel on dY "
                                   "16384x20480 (row SR, col RHT+SR, MXFP8 col)",
                                   "achieved": round(qgbs, 1), "peak": pk["hbm_gbs"],
                                   "unit": "GB/s", "frac": round(qgbs / pk["hbm_gbs"], 4),
-                                  "algorithmic_bytes": qbytes, "traffic": None,
+                                  "algorithmic_bytes": qbytes,
+                                  "traffic": TRAFFIC_BYTES["quant_dy"],
                                   "peak_note": f"of {pk['source']}"},
             "breakdown_ms_per_step": breakdown,
             "e2e": {"value": round(value_e2e, 2), "unit": "TFLOP/s",
