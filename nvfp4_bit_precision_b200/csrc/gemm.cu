@@ -8,21 +8,28 @@
 // Machines uskorila obuchenie Inkling 2 Small 4-bitnymi chislami", section
 // "Details": NVFP4 in the expert layers -> the grouped form).
 //
-// Structure (one persistent CTA per SM, 448 threads):
-//   warp 0      TMA producer: A/B tiles (128-byte swizzled, 4-bit codes packed
-//               two per byte) by cp.async.bulk.tensor, scale atoms by
-//               cp.async.bulk, into a 4-stage ring guarded by mbarriers.
+// Structure: persistent CTA pairs (clusters of 2, one CTA per SM, 448
+// threads each).  A pair computes a 256x256 output tile with the two-SM form
+// of the MMA (cta_group::2): each CTA stages its own 128 rows of A and 128 of
+// the 256 rows of B, so each SM moves half the B tile and the tensor cores of
+// the pair read one copy of it.  Per CTA:
+//   warp 0      TMA producer: this CTA's A/B boxes (128-byte swizzled, 4-bit
+//               codes two per byte; completing on the leader CTA's barrier,
+//               which expects both CTAs' bytes) and its scale atoms (own 128
+//               A rows; all 256 B rows; 1D bulk copies on its own barrier)
+//               into a 5-stage ring.
 //   warps 2..5  scale writers, one per tensor-memory lane quadrant: each lane
 //               loads row i of the stage's 512-byte scale atoms from shared
-//               memory and writes them into its quadrant with tcgen05.st, so
-//               the tensor pipe spends no cycles on scale copies.
-//   warp 1      one elected thread waits for a stage's tiles and scales and
-//               issues 4 MMAs of 128x256x64, then commits the stage back to
-//               the producer and, after the last K stage, the accumulator to
-//               the epilogue.
-//   warps 6..13 epilogue: tcgen05.ld of the 128x256 FP32 accumulator (two
-//               warps per lane quadrant, converted as it is loaded), release
-//               of the accumulator, then stores to global memory.
+//               memory and writes them into its quadrant of this CTA's tensor
+//               memory with tcgen05.st, then reports to the leader.  The
+//               tensor pipe spends no cycles on scale copies.
+//   warp 1      leader CTA only: one elected thread waits for a stage's tiles
+//               and both CTAs' scales and issues 4 MMAs of 256x256x64, then
+//               commits the stage to both CTAs' producers and, after the last
+//               K stage, the accumulator to both epilogues.
+//   warps 6..13 epilogue: tcgen05.ld of this CTA's 128x256 FP32 accumulator
+//               half (two warps per lane quadrant, converted as it is loaded),
+//               release of the accumulator to the leader, then stores.
 // Every mbarrier wait is bounded (2 s); a timeout sets the workspace status
 // word and the kernel winds down instead of hanging.
 #include <cudaTypedefs.h>
@@ -34,15 +41,17 @@
 
 namespace nvfp4 {
 
-constexpr int BM = 128;
-constexpr int BN = 256;
+constexpr int BM = 128;                    // A rows per CTA; a CTA pair covers 2 * BM
+constexpr int kMmaM = 2 * BM;              // M of the two-SM MMA
+constexpr int BN = 256;                    // output columns per tile
 constexpr int BK = 256;                    // elements per stage (128 bytes per row)
-constexpr int kGemmStages = 4;
-constexpr int kA_Bytes = BM * BK / 2;      // 16 KB
-constexpr int kB_Bytes = BN * BK / 2;      // 32 KB
-constexpr int kSFA_Bytes = BM * BK / 16;   // 2 KB: 4 atoms of 512 B
-constexpr int kSFB_Bytes = BN * BK / 16;   // 4 KB: 2 row blocks x 4 atoms
+constexpr int kGemmStages = 5;
+constexpr int kA_Bytes = BM * BK / 2;          // 16 KB
+constexpr int kB_Bytes = (BN / 2) * BK / 2;    // 16 KB: this CTA's half of the B tile
+constexpr int kSFA_Bytes = BM * BK / 16;       // 2 KB: 4 atoms of 512 B (this CTA's rows)
+constexpr int kSFB_Bytes = BN * BK / 16;       // 4 KB: 2 row blocks x 4 atoms (all of B)
 constexpr int kStageBytes = kA_Bytes + kB_Bytes + kSFA_Bytes + kSFB_Bytes;
+constexpr uint32_t kPairCodeTx = 2u * (kA_Bytes + kB_Bytes);  // the leader's full barrier
 constexpr int kGemmThreads = 448;  // producer, MMA, 4 scale writers, 8 epilogue warps
 // Tensor memory: the 128x256 FP32 accumulator in columns 0..255, then one
 // 48-column scale region per pipeline stage (SFA 4 x 4 columns, SFB 4 x 8).
@@ -74,9 +83,10 @@ struct GemmArgs {
 };
 
 struct GemmShared {
-    uint64_t full[kGemmStages];
-    uint64_t empty[kGemmStages];
-    uint64_t sf_ready[kGemmStages];
+    uint64_t full[kGemmStages];      // leader: A/B codes of both CTAs landed
+    uint64_t sf_full[kGemmStages];   // this CTA's scale atoms landed
+    uint64_t empty[kGemmStages];     // the stage's MMAs completed (both CTAs)
+    uint64_t sf_ready[kGemmStages];  // leader: both CTAs' scales are in tensor memory
     uint64_t acc_full;
     uint64_t acc_empty;
     uint32_t tmem_base;
@@ -87,29 +97,78 @@ struct GemmShared {
 };
 
 // ---------------------------------------------------------------- PTX wrappers
-__device__ __forceinline__ void tmem_alloc(uint32_t* dst_smem, uint32_t ncols)
+__device__ __forceinline__ uint32_t cluster_rank()
 {
-    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
+    uint32_t r;
+    asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
+    return r;
+}
+
+// Address, in the cluster's shared window, of the variable at p in CTA `rank`.
+__device__ __forceinline__ uint32_t cluster_addr(const void* p, uint32_t rank)
+{
+    uint32_t out;
+    asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(out) : "r"(smem_addr(p)), "r"(rank));
+    return out;
+}
+
+// All threads of both CTAs: arrive and wait (release / acquire at cluster scope).
+__device__ __forceinline__ void cluster_sync()
+{
+    asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::
+                     : "memory");
+}
+
+// Arrive on a barrier of either CTA of the pair (release at CTA scope, as the
+// tcgen05 fences around it order the tensor-memory work; a cluster-scope
+// release would add a memory barrier to every stage).
+__device__ __forceinline__ void mbar_arrive_cluster(uint32_t bar_cluster_addr)
+{
+    asm volatile("mbarrier.arrive.shared::cluster.b64 _, [%0];" ::"r"(bar_cluster_addr)
+                 : "memory");
+}
+
+// Pair-form TMA load: the box lands in this CTA's shared memory and its bytes
+// are counted on the barrier at `bar` (a cluster address: the leader's).  No
+// multicast.  x is a multiple of 128 bytes at every call site.
+__device__ __forceinline__ void tma_load_2d_pair(void* dst, const CUtensorMap* map, int32_t x,
+                                                 int32_t y, uint32_t bar)
+{
+    asm volatile(
+        "cp.async.bulk.tensor.2d.cta_group::2.shared::cluster.global.mbarrier::complete_tx::bytes "
+        "[%0], [%1, {%2, %3}], [%4];" ::"r"(smem_addr(dst)),
+        "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(bar)
+        : "memory");
+}
+
+// Tensor memory of the pair: one warp with the same index in each CTA.
+__device__ __forceinline__ void tmem_alloc_pair(uint32_t* dst_smem, uint32_t ncols)
+{
+    asm volatile("tcgen05.alloc.cta_group::2.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
                      smem_addr(dst_smem)),
                  "r"(ncols)
                  : "memory");
-    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::2.sync.aligned;" ::: "memory");
 }
 
-__device__ __forceinline__ void tmem_dealloc(uint32_t taddr, uint32_t ncols)
+__device__ __forceinline__ void tmem_dealloc_pair(uint32_t taddr, uint32_t ncols)
 {
-    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(taddr), "r"(ncols)
+    asm volatile("tcgen05.dealloc.cta_group::2.sync.aligned.b32 %0, %1;" ::"r"(taddr), "r"(ncols)
                  : "memory");
 }
 
 __device__ __forceinline__ void tc_fence_before() { asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory"); }
 __device__ __forceinline__ void tc_fence_after() { asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory"); }
 
-__device__ __forceinline__ void tc_commit(uint64_t* bar)
+// Arrive (once the issuing thread's earlier tcgen05 operations completed) on
+// the barrier at the same offset in both CTAs of the pair.
+__device__ __forceinline__ void tc_commit_pair(uint64_t* bar)
 {
-    asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(
-                     smem_addr(bar))
-                 : "memory");
+    asm volatile(
+        "tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.multicast::cluster.b64 "
+        "[%0], %1;" ::"r"(smem_addr(bar)),
+        "h"((uint16_t)0x3)
+        : "memory");
 }
 
 // Shared-memory matrix descriptor: K-major operand, 128-byte swizzle, 8-row
@@ -121,10 +180,10 @@ __device__ __forceinline__ uint64_t desc_sw128(const void* p)
 }
 
 // Instruction descriptor: kind::mxf4nvf4, A/B E2M1 (format 1), UE4M3 scales,
-// both K-major, M = 128, N = 256, dense, K = 64 per instruction.
+// both K-major, M = 256 (the pair), N = 256, dense, K = 64 per instruction.
 __host__ __device__ constexpr uint32_t make_idesc()
 {
-    return (1u << 7) | (1u << 10) | ((uint32_t)(BN >> 3) << 17) | ((uint32_t)(BM >> 4) << 24);
+    return (1u << 7) | (1u << 10) | ((uint32_t)(BN >> 3) << 17) | ((uint32_t)(kMmaM >> 4) << 24);
 }
 
 __device__ __forceinline__ void tc_mma(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc,
@@ -134,7 +193,7 @@ __device__ __forceinline__ void tc_mma(uint32_t d_tmem, uint64_t adesc, uint64_t
     asm volatile(
         "{\n\t.reg .pred p;\n\t"
         "setp.ne.b32 p, %4, 0;\n\t"
-        "tcgen05.mma.cta_group::1.kind::mxf4nvf4.block_scale.block16 [%0], %1, %2, %3, [%5], [%6], p;\n\t"
+        "tcgen05.mma.cta_group::2.kind::mxf4nvf4.block_scale.block16 [%0], %1, %2, %3, [%5], [%6], p;\n\t"
         "}" ::"r"(d_tmem),
         "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate), "r"(sfa_tmem), "r"(sfb_tmem)
         : "memory");
@@ -166,9 +225,9 @@ __device__ __forceinline__ void tmem_ld_wait() { asm volatile("tcgen05.wait::ld.
 // ---------------------------------------------------------------- scheduling
 struct TileCoord {
     int group;       // expert (0 when dense)
-    int64_t row0;    // first A row of the tile
+    int64_t row0;    // first A row of the pair's 256-row tile
     int64_t row_end; // one past the last valid A row
-    int64_t sf_blk;  // 128-row scale block of the tile
+    int64_t sf_blk;  // 128-row scale block of the tile's first half
     int64_t n0;
 };
 
@@ -177,16 +236,16 @@ __device__ __forceinline__ TileCoord tile_coord(const GemmArgs& a, const GemmSha
     TileCoord c;
     const int64_t tiles_n = (a.N + BN - 1) / BN;
     if (!a.grouped) {
-        const int64_t tiles_m = (a.M + BM - 1) / BM;
+        const int64_t tiles_m = (a.M + kMmaM - 1) / kMmaM;
         const int64_t band = 8 * tiles_n;  // 8 M tiles share a band: B tiles reused from L2
         const int64_t g = t / band, first_m = g * 8;
         const int64_t gm = min((int64_t)8, tiles_m - first_m);
         const int64_t r = t - g * band;
         const int64_t mt = first_m + r % gm, nt = r / gm;
         c.group = 0;
-        c.row0 = mt * BM;
+        c.row0 = mt * kMmaM;
         c.row_end = a.M;
-        c.sf_blk = mt;
+        c.sf_blk = 2 * mt;
         c.n0 = nt * BN;
     } else {
         int lo = 0, hi = a.G - 1;  // e with cum[e] <= t < cum[e+1]
@@ -200,16 +259,16 @@ __device__ __forceinline__ TileCoord tile_coord(const GemmArgs& a, const GemmSha
         const int64_t local = t - sh->cum_tiles[lo];
         const int64_t mt = local / tiles_n, nt = local - mt * tiles_n;
         c.group = lo;
-        c.row0 = sh->group_start[lo] + mt * BM;
+        c.row0 = sh->group_start[lo] + mt * kMmaM;
         c.row_end = sh->group_start[lo + 1];
-        c.sf_blk = sh->group_sfblk[lo] + mt;
+        c.sf_blk = sh->group_sfblk[lo] + 2 * mt;
         c.n0 = nt * BN;
     }
     return c;
 }
 
 // ---------------------------------------------------------------- kernel
-__global__ void __launch_bounds__(kGemmThreads, 1)
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
     gemm_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_constant__ CUtensorMap map_b,
                 GemmArgs a)
 {
@@ -218,20 +277,24 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
                                                ~uintptr_t(1023));
     GemmShared* sh = reinterpret_cast<GemmShared*>(smem + kGemmStages * kStageBytes);
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const uint32_t rank = cluster_rank();  // 0: leader (issues the MMAs), 1: peer
+    const bool leader = rank == 0;
+    const int pair = blockIdx.x >> 1, n_pairs = gridDim.x >> 1;
 
     if (threadIdx.x == 0) {
         for (int s = 0; s < kGemmStages; ++s) {
-            mbar_init(&sh->full[s], 1);
-            mbar_init(&sh->empty[s], 1);
-            mbar_init(&sh->sf_ready[s], 4);
+            mbar_init(&sh->full[s], 1);      // leader: its producer's expect_tx; peer: unused
+            mbar_init(&sh->sf_full[s], 1);   // this CTA's producer
+            mbar_init(&sh->empty[s], 1);     // the leader's MMA commit, multicast to both
+            mbar_init(&sh->sf_ready[s], 8);  // leader: 4 scale writers of each CTA
         }
         mbar_init(&sh->acc_full, 1);
-        mbar_init(&sh->acc_empty, 8);
+        mbar_init(&sh->acc_empty, 16);       // leader: 8 epilogue warps of each CTA
         fence_barrier_init();
-        // tile table
+        // tile table (both CTAs compute the same one)
         const int64_t tiles_n = (a.N + BN - 1) / BN;
         if (!a.grouped) {
-            sh->total_tiles = (int32_t)(((a.M + BM - 1) / BM) * tiles_n);
+            sh->total_tiles = (int32_t)(((a.M + kMmaM - 1) / kMmaM) * tiles_n);
         } else {
             int32_t cum = 0, blk = 0;
             for (int e = 0; e <= a.G; ++e) {
@@ -241,17 +304,18 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
                 sh->group_sfblk[e] = blk;
                 if (e < a.G) {
                     const int32_t cnt = a.group_offsets[e + 1] - st;
-                    const int32_t mt = cnt > 0 ? (cnt + BM - 1) / BM : 0;
+                    const int32_t mt = cnt > 0 ? (cnt + kMmaM - 1) / kMmaM : 0;
                     cum += mt * (int32_t)tiles_n;
-                    blk += mt;
+                    blk += cnt > 0 ? (cnt + BM - 1) / BM : 0;
                 }
             }
             sh->total_tiles = cum;
         }
     }
-    if (warp == 1) tmem_alloc(&sh->tmem_base, kTmemCols);
+    if (warp == 1) tmem_alloc_pair(&sh->tmem_base, kTmemCols);
     tc_fence_before();
     __syncthreads();
+    cluster_sync();  // both CTAs' barriers initialised and tensor memory allocated
     tc_fence_after();
     const uint32_t tmem = sh->tmem_base;
     const int total = sh->total_tiles;
@@ -260,18 +324,23 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     bool failed = false;
 
     if (warp == 0) {
-        // ------------------------------------------------ TMA producer
+        // ------------------------------------------------ TMA producer (both CTAs)
         if (lane == 0) {
             asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&map_a)) : "memory");
             asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&map_b)) : "memory");
-            const int64_t n_blocks_valid = (a.N + 127) / 128;  // scale row blocks that exist
+            const int64_t nblk = (a.N + 127) / 128;  // 128-row scale blocks of one B operand
             uint32_t it = 0;
-            for (int t = blockIdx.x; t < total && !failed; t += gridDim.x) {
+            for (int t = pair; t < total && !failed; t += n_pairs) {
                 const TileCoord c = tile_coord(a, sh, t);
-                const int64_t b_row0 = (int64_t)c.group * a.N + c.n0;
+                // This CTA's A rows; a half past the group's (or matrix's) end
+                // reads rows it never stores, and the leader's scale block
+                // instead of one that may not exist.
+                const int64_t a_row = c.row0 + (int64_t)BM * rank;
+                const int64_t sfa_blk = c.sf_blk + ((rank == 1 && a_row < c.row_end) ? 1 : 0);
+                const int64_t b_row = (int64_t)c.group * a.N + c.n0 + (int64_t)(BN / 2) * rank;
                 const int64_t nb0 = c.n0 / 128;
-                const int nsfb = (int)min((int64_t)2, n_blocks_valid - nb0);
-                const uint8_t* sfb_base = a.sfb + (int64_t)c.group * ((a.N + 127) / 128) * k64 * 512;
+                const int64_t nb1 = c.n0 + 128 < a.N ? nb0 + 1 : nb0;
+                const uint8_t* sfb_base = a.sfb + (int64_t)c.group * nblk * k64 * 512;
                 for (int64_t ks = 0; ks < kstages; ++ks, ++it) {
                     const int s = (int)(it % kGemmStages);
                     const uint32_t ph = (it / kGemmStages) & 1u;
@@ -281,28 +350,33 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
                         break;
                     }
                     uint8_t* st = smem + s * kStageBytes;
-                    const uint32_t bytes = kA_Bytes + kB_Bytes + kSFA_Bytes + nsfb * (kSFB_Bytes / 2);
-                    mbar_arrive_expect_tx(&sh->full[s], bytes);
-                    tma_load_2d(st, &map_a, (int32_t)(ks * (BK / 2)), (int32_t)c.row0, &sh->full[s]);
-                    tma_load_2d(st + kA_Bytes, &map_b, (int32_t)(ks * (BK / 2)), (int32_t)b_row0,
-                                &sh->full[s]);
-                    // 4 consecutive scale atoms (K/64 groups ks*4 .. ks*4+3) per 128-row block
-                    bulk_copy_g2s(st + kA_Bytes + kB_Bytes, a.sfa + (c.sf_blk * k64 + ks * 4) * 512,
-                                  kSFA_Bytes, &sh->full[s]);
-                    for (int h = 0; h < nsfb; ++h)
-                        bulk_copy_g2s(st + kA_Bytes + kB_Bytes + kSFA_Bytes + h * (kSFB_Bytes / 2),
-                                      sfb_base + ((nb0 + h) * k64 + ks * 4) * 512, kSFB_Bytes / 2,
-                                      &sh->full[s]);
+                    if (leader) mbar_arrive_expect_tx(&sh->full[s], kPairCodeTx);
+                    const uint32_t fb = cluster_addr(&sh->full[s], 0);
+                    tma_load_2d_pair(st, &map_a, (int32_t)(ks * (BK / 2)), (int32_t)a_row, fb);
+                    tma_load_2d_pair(st + kA_Bytes, &map_b, (int32_t)(ks * (BK / 2)), (int32_t)b_row, fb);
+                    // this CTA's scale atoms: 4 consecutive atoms (2 KB) per 128-row block
+                    uint8_t* sf = st + kA_Bytes + kB_Bytes;
+                    mbar_arrive_expect_tx(&sh->sf_full[s], kSFA_Bytes + kSFB_Bytes);
+                    bulk_copy_g2s(sf, a.sfa + (sfa_blk * k64 + ks * 4) * 512, kSFA_Bytes, &sh->sf_full[s]);
+                    bulk_copy_g2s(sf + kSFA_Bytes, sfb_base + (nb0 * k64 + ks * 4) * 512, kSFB_Bytes / 2,
+                                  &sh->sf_full[s]);
+                    bulk_copy_g2s(sf + kSFA_Bytes + kSFB_Bytes / 2, sfb_base + (nb1 * k64 + ks * 4) * 512,
+                                  kSFB_Bytes / 2, &sh->sf_full[s]);
                 }
             }
+            // Drain: the last stages' copies have landed once their MMAs
+            // completed (the CTA's shared memory must outlive them).
+            const uint32_t first = it > (uint32_t)kGemmStages ? it - kGemmStages : 0u;
+            for (uint32_t j = first; j < it; ++j)
+                (void)mbar_wait(&sh->empty[j % kGemmStages], (j / kGemmStages) & 1u);
         }
     } else if (warp == 1) {
-        // ------------------------------------------------ MMA issuer
-        if (lane == 0) {
+        // ------------------------------------------------ MMA issuer (leader CTA)
+        if (leader && lane == 0) {
             const uint32_t idesc = make_idesc();
             uint32_t it = 0, tcount = 0;
-            for (int t = blockIdx.x; t < total && !failed; t += gridDim.x, ++tcount) {
-                // wait until the epilogue drained the accumulator of the previous tile
+            for (int t = pair; t < total && !failed; t += n_pairs, ++tcount) {
+                // wait until both epilogues drained the accumulator of the previous tile
                 if (!mbar_wait(&sh->acc_empty, (tcount & 1u) ^ 1u)) {
                     record_status(a.status, NVFP4_ERR_TIMEOUT);
                     failed = true;
@@ -312,12 +386,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
                 for (int64_t ks = 0; ks < kstages; ++ks, ++it) {
                     const int s = (int)(it % kGemmStages);
                     const uint32_t ph = (it / kGemmStages) & 1u;
-                    if (!mbar_wait(&sh->full[s], ph)) {
-                        record_status(a.status, NVFP4_ERR_TIMEOUT);
-                        failed = true;
-                        break;
-                    }
-                    if (!mbar_wait(&sh->sf_ready[s], ph)) {
+                    if (!mbar_wait(&sh->full[s], ph) || !mbar_wait(&sh->sf_ready[s], ph)) {
                         record_status(a.status, NVFP4_ERR_TIMEOUT);
                         failed = true;
                         break;
@@ -333,25 +402,27 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
                         tc_mma(tmem, ad + 2 * j, bd + 2 * j, idesc, t_sfa + 4 * j, t_sfb + 8 * j,
                                (ks > 0 || j > 0) ? 1u : 0u);
                     }
-                    tc_commit(&sh->empty[s]);  // stage free once these MMAs completed
+                    tc_commit_pair(&sh->empty[s]);  // both CTAs' stage free once these MMAs completed
                 }
                 if (failed) break;
-                tc_commit(&sh->acc_full);
+                tc_commit_pair(&sh->acc_full);
             }
         }
     } else if (warp < 6) {
-        // ------------------------------------------------ scale writers (warps 2..5)
-        // Each warp writes its lane quadrant of the stage's scale columns with
-        // tcgen05.st: lane i gets row i of every 512-byte atom (the layout the
-        // broadcast copy would produce in each quadrant).
+        // ------------------------------------------------ scale writers (warps 2..5, both CTAs)
+        // Each warp writes its lane quadrant of the stage's scale columns in
+        // this CTA's tensor memory with tcgen05.st: lane i gets row i of every
+        // 512-byte atom (the layout a broadcast copy would produce in each
+        // quadrant).  Completion is reported to the leader, whose MMAs read
+        // both CTAs' scales.
         const uint32_t lane_base = (uint32_t)(32 * (warp & 3)) << 16;
         uint32_t it = 0;
-        for (int t = blockIdx.x; t < total && !failed; t += gridDim.x) {
+        for (int t = pair; t < total && !failed; t += n_pairs) {
             for (int64_t ks = 0; ks < kstages; ++ks, ++it) {
                 const int s = (int)(it % kGemmStages);
                 const uint32_t ph = (it / kGemmStages) & 1u;
                 bool ok = true;
-                if (lane == 0) ok = mbar_wait(&sh->full[s], ph);
+                if (lane == 0) ok = mbar_wait(&sh->sf_full[s], ph);
                 ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
                 if (!ok) {
                     if (lane == 0) record_status(a.status, NVFP4_ERR_TIMEOUT);
@@ -376,16 +447,17 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
                 asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
                 tc_fence_before();
                 __syncwarp();
-                if (lane == 0) mbar_arrive(&sh->sf_ready[s]);
+                if (lane == 0) mbar_arrive_cluster(cluster_addr(&sh->sf_ready[s], 0));
             }
         }
     } else {
-        // ------------------------------------------------ epilogue (warps 6..13)
+        // ------------------------------------------------ epilogue (warps 6..13, both CTAs)
         const int quad = warp & 3;                   // TMEM lanes 32*quad .. 32*quad+31
         const int col0 = ((warp - 6) >> 2) * (BN / 2);  // 0 or 128
+        const uint32_t acc_empty_leader = cluster_addr(&sh->acc_empty, 0);
         float out_max = 0.0f;                            // max |D| stored by this thread
         uint32_t tcount = 0;
-        for (int t = blockIdx.x; t < total; t += gridDim.x, ++tcount) {
+        for (int t = pair; t < total; t += n_pairs, ++tcount) {
             const TileCoord c = tile_coord(a, sh, t);
             const bool ok = mbar_wait(&sh->acc_full, tcount & 1u);
             if (!ok) {
@@ -395,7 +467,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
             tc_fence_after();
             const uint32_t tbase = tmem + ((uint32_t)(32 * quad) << 16) + (uint32_t)col0;
             const float alpha = __fmul_rn(a.ga[0], a.gb[c.group]);
-            const int64_t row = c.row0 + 32 * quad + lane;
+            const int64_t row = c.row0 + (int64_t)BM * rank + 32 * quad + lane;
             const bool row_ok = row < c.row_end;
             if (a.bf16_out) {
                 // 128 columns in four 32-column loads, each converted to bf16
@@ -419,7 +491,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
                 }
                 tc_fence_before();
                 __syncwarp();
-                if (lane == 0) mbar_arrive(&sh->acc_empty);  // accumulator drained
+                if (lane == 0) mbar_arrive_cluster(acc_empty_leader);  // accumulator drained
                 if (row_ok) {
                     const int64_t cbase = c.n0 + col0;
                     uint16_t* drow = static_cast<uint16_t*>(a.D) + row * a.ldd + cbase;
@@ -453,7 +525,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
                 if (hh == 3) {
                     tc_fence_before();
                     __syncwarp();
-                    if (lane == 0) mbar_arrive(&sh->acc_empty);  // accumulator drained
+                    if (lane == 0) mbar_arrive_cluster(acc_empty_leader);  // accumulator drained
                 }
                 if (!row_ok) continue;
                 const int64_t cbase = c.n0 + col0 + 32 * hh;
@@ -482,10 +554,12 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         }
     }
 
+    // Neither CTA leaves (or frees the pair's tensor memory) before both are done.
     tc_fence_before();
     __syncthreads();
+    cluster_sync();
     tc_fence_after();
-    if (warp == 1) tmem_dealloc(tmem, kTmemCols);
+    if (warp == 1) tmem_dealloc_pair(tmem, kTmemCols);
 }
 
 // ---------------------------------------------------------------- host side
@@ -522,6 +596,7 @@ static size_t gemm_smem_bytes() { return (size_t)kGemmStages * kStageBytes + siz
 
 struct GemmDevice {
     int sms = 0;
+    int pairs = 0;  // CTA pairs that are resident at once
     bool ok = false;
 };
 
@@ -537,6 +612,16 @@ static GemmDevice& gemm_device(int dev)
                                  (int)gemm_smem_bytes()) != cudaSuccess)
             return;
         d.sms = prop.multiProcessorCount;
+        // Pairs need two SMs of one cluster-capable group: ask how many fit
+        // at once, so that the persistent grid never waits for a second wave.
+        cudaLaunchConfig_t cfg = {};
+        cfg.gridDim = dim3((unsigned)(d.sms & ~1));
+        cfg.blockDim = dim3(kGemmThreads);
+        cfg.dynamicSmemBytes = gemm_smem_bytes();
+        int clusters = 0;
+        if (cudaOccupancyMaxActiveClusters(&clusters, gemm_kernel, &cfg) != cudaSuccess || clusters < 1)
+            return;
+        d.pairs = std::min(clusters, d.sms / 2);
         d.ok = true;
     });
     return infos[dev & 63];
@@ -562,8 +647,8 @@ static nvfp4_status launch_gemm(const CUtensorMap& ma, const CUtensorMap& mb, Ge
     // the status word reports this call only; the output amax starts at 0
     if (cudaMemsetAsync(a.status, 0, 4, st) != cudaSuccess) return NVFP4_ERR_CUDA;
     if (a.amax_out && cudaMemsetAsync(a.amax_out, 0, 4, st) != cudaSuccess) return NVFP4_ERR_CUDA;
-    const int grid = (int)std::max<int64_t>(1, std::min<int64_t>(max_tiles, info.sms));
-    gemm_kernel<<<grid, kGemmThreads, gemm_smem_bytes(), st>>>(ma, mb, a);
+    const int pairs = (int)std::max<int64_t>(1, std::min<int64_t>(max_tiles, info.pairs));
+    gemm_kernel<<<2 * pairs, kGemmThreads, gemm_smem_bytes(), st>>>(ma, mb, a);
     return cudaGetLastError() == cudaSuccess ? NVFP4_OK : NVFP4_ERR_CUDA;
 }
 
@@ -584,7 +669,7 @@ extern "C" nvfp4_status nvfp4_gemm(const uint8_t* qa, const uint8_t* sfa, const 
     if (!workspace || ws_bytes < kGemmWorkspace) return NVFP4_ERR_WORKSPACE;
     if (!al16(workspace)) return NVFP4_ERR_ALIGN;
     CUtensorMap ma, mb;
-    if (!make_map(&ma, qa, M, K / 2, BM) || !make_map(&mb, qb, N, K / 2, BN)) return NVFP4_ERR_CUDA;
+    if (!make_map(&ma, qa, M, K / 2, BM) || !make_map(&mb, qb, N, K / 2, BN / 2)) return NVFP4_ERR_CUDA;
     GemmArgs a{};
     a.sfa = sfa;
     a.sfb = sfb;
@@ -600,7 +685,7 @@ extern "C" nvfp4_status nvfp4_gemm(const uint8_t* qa, const uint8_t* sfa, const 
     a.G = 1;
     a.status = static_cast<uint32_t*>(workspace) + 2;
     a.amax_out = amax_out;
-    const int64_t tiles = ((M + BM - 1) / BM) * ((N + BN - 1) / BN);
+    const int64_t tiles = ((M + kMmaM - 1) / kMmaM) * ((N + BN - 1) / BN);
     return launch_gemm(ma, mb, a, tiles, static_cast<cudaStream_t>(stream));
 }
 
@@ -623,7 +708,7 @@ extern "C" nvfp4_status nvfp4_grouped_gemm(int G, const int32_t* group_offsets, 
     if (!workspace || ws_bytes < kGemmWorkspace) return NVFP4_ERR_WORKSPACE;
     if (!al16(workspace)) return NVFP4_ERR_ALIGN;
     CUtensorMap ma, mb;
-    if (!make_map(&ma, qa, total_rows, K / 2, BM) || !make_map(&mb, qb, (int64_t)G * N, K / 2, BN))
+    if (!make_map(&ma, qa, total_rows, K / 2, BM) || !make_map(&mb, qb, (int64_t)G * N, K / 2, BN / 2))
         return NVFP4_ERR_CUDA;
     GemmArgs a{};
     a.sfa = sfa;
@@ -643,6 +728,6 @@ extern "C" nvfp4_status nvfp4_grouped_gemm(int G, const int32_t* group_offsets, 
     a.status = static_cast<uint32_t*>(workspace) + 2;
     a.amax_out = amax_out;
     // upper bound on tiles: every group may add one partial M tile
-    const int64_t tiles = ((total_rows + BM - 1) / BM + G) * (N / BN + 1);
+    const int64_t tiles = ((total_rows + kMmaM - 1) / kMmaM + G) * ((N + BN - 1) / BN);
     return launch_gemm(ma, mb, a, tiles, static_cast<cudaStream_t>(stream));
 }
