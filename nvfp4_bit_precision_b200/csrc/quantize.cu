@@ -1,7 +1,7 @@
 // quantize.cu -- NVFP4 / MXFP8 quantisation and NVFP4 dequantisation on sm_100a.
 //
 // Two HBM-bound passes over 128x128 bf16 tiles, each a persistent grid whose
-// warp 0 keeps a 3-stage ring of tiles in flight (TMA boxes with the 128-byte
+// warp 0 keeps a 2-stage ring of tiles in flight (TMA boxes with the 128-byte
 // swizzle for dense input, per-row bulk copies for a gather) while all eight
 // warps compute from shared memory:
 //   1. amax_kernel: max |x| and, when the columnwise Hadamard is on, max
@@ -11,7 +11,9 @@
 //      pass 1 left in L2 is read first) and produces, from one staged copy,
 //      the rowwise codes/scales, the columnwise (transposed, optionally
 //      Hadamard-rotated) codes/scales and the MXFP8 copies, with Philox
-//      stochastic rounding in registers and 8/16-byte vector stores.
+//      stochastic rounding in registers, 16-byte vector stores, and the
+//      transposed MXFP8 codes written through per-warp shared-memory staging
+//      and TMA stores.
 //
 // Format and steps: asector.ru, "Nvidia dobivaetsya uspekha s 4-bitnym
 // formatom NVFP4" ("NVFP4 and Blackwell": E2M1, 16-element local scale plus a
@@ -32,7 +34,10 @@ constexpr int kTileRows = 128;
 constexpr int kTileCols = 128;
 constexpr int kPitch = kTileCols * 2 + 16;  // bytes per staged row (+16 breaks bank aliasing)
 constexpr int kTileBytes = kTileRows * kPitch;
-constexpr int kStages = 3;
+constexpr int kStages = 2;
+// Per-warp staging of MXFP8 columnwise codes: 64 columns x 32 rows (bytes),
+// written out with one TMA store per warp and tile.
+constexpr int kMxStageBytes = 64 * 32;
 constexpr int kQuantThreads = 256;
 constexpr int kMaxGroups = 256;  // MoE groups per call (the grouped GEMM's limit too)
 
@@ -56,6 +61,7 @@ struct QArgs {
     uint8_t *mx_q_row, *mx_sf_row, *mx_q_col, *mx_sf_col;
     uint32_t* status;
     int64_t tiles_c, n_tiles;
+    int mx_staged;  // MXFP8 columnwise codes go through shared memory and TMA stores
 };
 
 __device__ __forceinline__ uint4 ld_global_v4(const void* p)
@@ -297,7 +303,7 @@ __device__ __forceinline__ void store_codes32(uint8_t* dst, const uint32_t (&c)[
 }
 
 // --------------------------------------------------------------------------
-// Pass 1: global amax (dense input).  The same 128x128 TMA tiles and 3-stage
+// Pass 1: global amax (dense input).  The same 128x128 TMA tiles and 2-stage
 // copy ring as pass 2, walked in the opposite order; each thread takes one column pair over 32
 // rows (two 16-row blocks): max |x| for the rowwise and 2D scales and, with the
 // Hadamard on, max |RHT(x)| over the columnwise 16-vectors.  One atomicMax per
@@ -496,7 +502,8 @@ __host__ __device__ constexpr bool spec_pick(int8_t s, bool run_time)
 
 template <bool kTma, int kSpec>
 __global__ void __launch_bounds__(kQuantThreads, 2)
-    quant_kernel(const __grid_constant__ CUtensorMap map_x, QArgs a)
+    quant_kernel(const __grid_constant__ CUtensorMap map_x, const __grid_constant__ CUtensorMap map_mx,
+                 QArgs a)
 {
     constexpr QSpec sp = kSpecs[kSpec];
     extern __shared__ uint8_t smem_raw[];
@@ -504,8 +511,9 @@ __global__ void __launch_bounds__(kQuantThreads, 2)
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                                ~uintptr_t(1023));
     uint8_t* tiles = smem;
-    uint64_t* bars = reinterpret_cast<uint64_t*>(smem + kStages * kTileBytes);
-    QShared* sh = reinterpret_cast<QShared*>(smem + kStages * kTileBytes + 64);
+    uint8_t* mx_stage_all = smem + kStages * kTileBytes;
+    uint64_t* bars = reinterpret_cast<uint64_t*>(mx_stage_all + (kQuantThreads / 32) * kMxStageBytes);
+    QShared* sh = reinterpret_cast<QShared*>(reinterpret_cast<uint8_t*>(bars) + 64);
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     if (threadIdx.x == 0) {
@@ -781,7 +789,56 @@ __global__ void __launch_bounds__(kQuantThreads, 2)
                     }
                 }
             }
-            if (mx_col && cvalid && rbase < a.rows) {
+            if (kTma && mx_col && a.mx_staged) {
+                // This warp's 64 columns x 32 rows of codes go to its staging
+                // buffer (row 2*lane + h of the buffer = column cg0 + h) and out
+                // with one TMA store; the store clips what lies past the tensor.
+                const int64_t cwarp = c0 + 64 * (warp & 1);  // first column of the warp
+                if (rbase < a.rows && cwarp < a.cols) {
+                    uint8_t* stg = mx_stage_all + warp * kMxStageBytes;
+                    if (lane == 0) bulk_wait_read0();  // the previous store has read stg
+                    __syncwarp();
+                    float sa, sb;
+                    const int ea = mx_exponent(mxa, sa), eb = mx_exponent(mxb, sb);
+                    const int64_t ia = cg0 * a.rows + rbase, ib = ia + a.rows;  // element indices
+#pragma unroll
+                    for (int g2 = 0; g2 < 2; ++g2) {  // 16 rows per pass
+                        uint2 ca[2], cb[2];
+#pragma unroll
+                        for (int gg = 0; gg < 2; ++gg) {
+                            const int g = 2 * g2 + gg;
+                            float va[8], vb[8];
+#pragma unroll
+                            for (int i = 0; i < 8; ++i) {
+                                const uint32_t w = pair_word(8 * g + i);
+                                va[i] = bf16_lo(w);
+                                vb[i] = bf16_hi(w);
+                            }
+                            U4 wa{}, wb{};
+                            if (mx_sr) {
+                                wa = sr_block8(a.seed, a.offset, 2u, (uint64_t)(ia >> 3) + g);
+                                wb = sr_block8(a.seed, a.offset, 2u, (uint64_t)(ib >> 3) + g);
+                            }
+                            ca[gg] = mx_convert8(va, sa, mx_sr, wa);
+                            cb[gg] = mx_convert8(vb, sb, mx_sr, wb);
+                        }
+                        st_shared_v4(stg + (2 * lane) * 32 + 16 * g2,
+                                     make_uint4(ca[0].x, ca[0].y, ca[1].x, ca[1].y));
+                        st_shared_v4(stg + (2 * lane + 1) * 32 + 16 * g2,
+                                     make_uint4(cb[0].x, cb[0].y, cb[1].x, cb[1].y));
+                    }
+                    if (cvalid) {
+                        a.mx_sf_col[cg0 * (a.rows / 32) + rbase / 32] = (uint8_t)(ea + 127);
+                        a.mx_sf_col[(cg0 + 1) * (a.rows / 32) + rbase / 32] = (uint8_t)(eb + 127);
+                    }
+                    fence_proxy_async_smem();
+                    __syncwarp();
+                    if (lane == 0) {
+                        tma_store_2d(&map_mx, stg, (int32_t)rbase, (int32_t)cwarp);
+                        bulk_commit();
+                    }
+                }
+            } else if (mx_col && cvalid && rbase < a.rows) {
                 float sa, sb;
                 const int ea = mx_exponent(mxa, sa), eb = mx_exponent(mxb, sb);
                 const int64_t ia = cg0 * a.rows + rbase, ib = ia + a.rows;  // element indices
@@ -811,6 +868,9 @@ __global__ void __launch_bounds__(kQuantThreads, 2)
         __syncwarp();
         if (lane == 0) mbar_arrive(&empty[stage]);  // this warp is done with the stage
     }
+    // This warp's staged stores must finish before the CTA's shared memory
+    // goes away.
+    if (kTma && lane == 0) bulk_wait_all();
     // Copies issued for tiles this CTA did not consume (only after a timeout)
     // must land before the CTA's shared memory goes away.
     if (warp == 0) {
@@ -955,7 +1015,8 @@ struct DeviceInfo {
 
 static size_t quant_smem_bytes()
 {
-    return (size_t)kStages * kTileBytes + 64 + sizeof(QShared) + 1024;  // + alignment slack
+    return (size_t)kStages * kTileBytes + (kQuantThreads / 32) * kMxStageBytes + 64 + sizeof(QShared) +
+           1024;  // + alignment slack
 }
 
 // Tensor map of the bf16 input for the TMA tile path: boxes of 128 rows x 64
@@ -973,7 +1034,7 @@ static bool make_input_map(CUtensorMap* m, const void* x, int64_t rows, int64_t 
               CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-using QuantKernel = void (*)(const CUtensorMap, QArgs);
+using QuantKernel = void (*)(const CUtensorMap, const CUtensorMap, QArgs);
 
 // The compiled variants: TMA tiles for dense input, row copies for the gather
 // (which only variants 0 and 4 serve).  nullptr where none is built.
@@ -1006,6 +1067,21 @@ static int pick_variant(const QArgs& a, bool tma)
             return v;
     }
     return 0;
+}
+
+// Store map of the MXFP8 columnwise codes [cols, rows] (u8, rows contiguous):
+// boxes of 32 bytes (rows) x 64 columns, no swizzle.  rows is a multiple of 32.
+static bool make_mx_store_map(CUtensorMap* m, const void* q, int64_t rows, int64_t cols)
+{
+    auto fn = encode_tiled_fn();
+    if (!fn) return false;
+    cuuint64_t dims[2] = {(cuuint64_t)rows, (cuuint64_t)cols};
+    cuuint64_t strides[1] = {(cuuint64_t)rows};
+    cuuint32_t box[2] = {32u, 64u};
+    cuuint32_t estr[2] = {1u, 1u};
+    return fn(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void*>(q), dims, strides, box, estr,
+              CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
+              CU_TENSOR_MAP_L2_PROMOTION_NONE, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
 static DeviceInfo& device_info(int dev)
@@ -1109,7 +1185,14 @@ static nvfp4_status launch_quant(QArgs& a, bool need_amax, void* workspace, cuda
         if (cudaGetLastError() != cudaSuccess) return NVFP4_ERR_CUDA;
     }
     const QuantKernel fn = quant_variant(tma, pick_variant(a, tma));
-    void* args[] = {&map, &a};
+    CUtensorMap map_mx;
+    memset(&map_mx, 0, sizeof(map_mx));
+    a.mx_staged = 0;
+    if (tma && (a.mx_outputs & NVFP4_COLWISE)) {
+        if (!make_mx_store_map(&map_mx, a.mx_q_col, a.rows, a.cols)) return NVFP4_ERR_CUDA;
+        a.mx_staged = 1;
+    }
+    void* args[] = {&map, &map_mx, &a};
     if (cudaLaunchKernel(reinterpret_cast<const void*>(fn), dim3((unsigned)grid), dim3(kQuantThreads),
                          args, quant_smem_bytes(), st) != cudaSuccess)
         return NVFP4_ERR_CUDA;
