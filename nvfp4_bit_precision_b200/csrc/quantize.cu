@@ -35,9 +35,11 @@ constexpr int kTileCols = 128;
 constexpr int kPitch = kTileCols * 2 + 16;  // bytes per staged row (+16 breaks bank aliasing)
 constexpr int kTileBytes = kTileRows * kPitch;
 constexpr int kStages = 2;
-// Per-warp staging of MXFP8 columnwise codes: 64 columns x 32 rows (bytes),
-// written out with one TMA store per warp and tile.
+// Per-warp staging of the transposed outputs of a warp's 64 columns x 32 rows,
+// each written out with one TMA store per warp and tile: MXFP8 codes (32
+// bytes per column) and NVFP4 columnwise codes (16 bytes per column).
 constexpr int kMxStageBytes = 64 * 32;
+constexpr int kQcStageBytes = 64 * 16;
 constexpr int kQuantThreads = 256;
 constexpr int kMaxGroups = 256;  // MoE groups per call (the grouped GEMM's limit too)
 
@@ -62,6 +64,7 @@ struct QArgs {
     uint32_t* status;
     int64_t tiles_c, n_tiles;
     int mx_staged;  // MXFP8 columnwise codes go through shared memory and TMA stores
+    int qc_staged;  // NVFP4 columnwise codes likewise (rows a multiple of 32)
 };
 
 __device__ __forceinline__ uint4 ld_global_v4(const void* p)
@@ -503,7 +506,7 @@ __host__ __device__ constexpr bool spec_pick(int8_t s, bool run_time)
 template <bool kTma, int kSpec>
 __global__ void __launch_bounds__(kQuantThreads, 2)
     quant_kernel(const __grid_constant__ CUtensorMap map_x, const __grid_constant__ CUtensorMap map_mx,
-                 QArgs a)
+                 const __grid_constant__ CUtensorMap map_qc, QArgs a)
 {
     constexpr QSpec sp = kSpecs[kSpec];
     extern __shared__ uint8_t smem_raw[];
@@ -512,7 +515,8 @@ __global__ void __launch_bounds__(kQuantThreads, 2)
                                                ~uintptr_t(1023));
     uint8_t* tiles = smem;
     uint8_t* mx_stage_all = smem + kStages * kTileBytes;
-    uint64_t* bars = reinterpret_cast<uint64_t*>(mx_stage_all + (kQuantThreads / 32) * kMxStageBytes);
+    uint8_t* qc_stage_all = mx_stage_all + (kQuantThreads / 32) * kMxStageBytes;
+    uint64_t* bars = reinterpret_cast<uint64_t*>(qc_stage_all + (kQuantThreads / 32) * kQcStageBytes);
     QShared* sh = reinterpret_cast<QShared*>(reinterpret_cast<uint8_t*>(bars) + 64);
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -712,6 +716,13 @@ __global__ void __launch_bounds__(kQuantThreads, 2)
             // Hadamard's sign flips leave |x| alone); the conversion then
             // re-reads the rows 8 at a time.  rows is a multiple of 32 here.
             float mxa = 0.0f, mxb = 0.0f;
+            const int64_t cwarp = c0 + 64 * (warp & 1);  // first column of the warp
+            uint8_t* stg_qc = qc_stage_all + warp * kQcStageBytes;
+            const bool qc_staged = kTma && nv_col && a.qc_staged;
+            if (kTma && (a.mx_staged || qc_staged)) {
+                if (lane == 0) bulk_wait_read0();  // this warp's previous stores have read its staging
+                __syncwarp();
+            }
             if (rbase < a.rows) {
                 // rows is a multiple of 16: both 16-row blocks exist, or (at the
                 // bottom edge) only the first.  The first block's codes wait in
@@ -766,7 +777,10 @@ __global__ void __launch_bounds__(kQuantThreads, 2)
                         a.sf_col[offa] = (uint8_t)ba;
                         a.sf_col[offb] = (uint8_t)bb;
                     } else {
-                        if (q_col_vec) {
+                        if (qc_staged) {  // buffer row 2*lane + h = column cg0 + h
+                            st_shared_v4(stg_qc + (2 * lane) * 16, make_uint4(keep0, keep1, ca0, ca1));
+                            st_shared_v4(stg_qc + (2 * lane + 1) * 16, make_uint4(keep2, keep3, cb0, cb1));
+                        } else if (q_col_vec) {
                             *reinterpret_cast<uint4*>(da) = make_uint4(keep0, keep1, ca0, ca1);
                             *reinterpret_cast<uint4*>(db) = make_uint4(keep2, keep3, cb0, cb1);
                         } else {
@@ -789,15 +803,22 @@ __global__ void __launch_bounds__(kQuantThreads, 2)
                     }
                 }
             }
+            if (qc_staged && rbase < a.rows && cwarp < a.cols) {
+                // this warp's 64 columns x 32 rows of NVFP4 codes (16 bytes per
+                // column) out with one TMA store, clipped at the tensor edge
+                fence_proxy_async_smem();
+                __syncwarp();
+                if (lane == 0) {
+                    tma_store_2d(&map_qc, stg_qc, (int32_t)(rbase / 2), (int32_t)cwarp);
+                    bulk_commit();
+                }
+            }
             if (kTma && mx_col && a.mx_staged) {
                 // This warp's 64 columns x 32 rows of codes go to its staging
                 // buffer (row 2*lane + h of the buffer = column cg0 + h) and out
                 // with one TMA store; the store clips what lies past the tensor.
-                const int64_t cwarp = c0 + 64 * (warp & 1);  // first column of the warp
                 if (rbase < a.rows && cwarp < a.cols) {
                     uint8_t* stg = mx_stage_all + warp * kMxStageBytes;
-                    if (lane == 0) bulk_wait_read0();  // the previous store has read stg
-                    __syncwarp();
                     float sa, sb;
                     const int ea = mx_exponent(mxa, sa), eb = mx_exponent(mxb, sb);
                     const int64_t ia = cg0 * a.rows + rbase, ib = ia + a.rows;  // element indices
@@ -1015,8 +1036,8 @@ struct DeviceInfo {
 
 static size_t quant_smem_bytes()
 {
-    return (size_t)kStages * kTileBytes + (kQuantThreads / 32) * kMxStageBytes + 64 + sizeof(QShared) +
-           1024;  // + alignment slack
+    return (size_t)kStages * kTileBytes + (kQuantThreads / 32) * (kMxStageBytes + kQcStageBytes) + 64 +
+           sizeof(QShared) + 1024;  // + alignment slack
 }
 
 // Tensor map of the bf16 input for the TMA tile path: boxes of 128 rows x 64
@@ -1034,7 +1055,7 @@ static bool make_input_map(CUtensorMap* m, const void* x, int64_t rows, int64_t 
               CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-using QuantKernel = void (*)(const CUtensorMap, const CUtensorMap, QArgs);
+using QuantKernel = void (*)(const CUtensorMap, const CUtensorMap, const CUtensorMap, QArgs);
 
 // The compiled variants: TMA tiles for dense input, row copies for the gather
 // (which only variants 0 and 4 serve).  nullptr where none is built.
@@ -1069,15 +1090,16 @@ static int pick_variant(const QArgs& a, bool tma)
     return 0;
 }
 
-// Store map of the MXFP8 columnwise codes [cols, rows] (u8, rows contiguous):
-// boxes of 32 bytes (rows) x 64 columns, no swizzle.  rows is a multiple of 32.
-static bool make_mx_store_map(CUtensorMap* m, const void* q, int64_t rows, int64_t cols)
+// Store map of a transposed output [cols, inner] (u8, inner bytes contiguous):
+// boxes of box_inner bytes x 64 columns, no swizzle.  inner is a multiple of
+// 16 (MXFP8 codes: inner = rows, box 32; NVFP4 codes: inner = rows / 2, box 16).
+static bool make_store_map(CUtensorMap* m, const void* q, int64_t inner, int64_t cols, uint32_t box_inner)
 {
     auto fn = encode_tiled_fn();
     if (!fn) return false;
-    cuuint64_t dims[2] = {(cuuint64_t)rows, (cuuint64_t)cols};
-    cuuint64_t strides[1] = {(cuuint64_t)rows};
-    cuuint32_t box[2] = {32u, 64u};
+    cuuint64_t dims[2] = {(cuuint64_t)inner, (cuuint64_t)cols};
+    cuuint64_t strides[1] = {(cuuint64_t)inner};
+    cuuint32_t box[2] = {box_inner, 64u};
     cuuint32_t estr[2] = {1u, 1u};
     return fn(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void*>(q), dims, strides, box, estr,
               CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
@@ -1189,10 +1211,17 @@ static nvfp4_status launch_quant(QArgs& a, bool need_amax, void* workspace, cuda
     memset(&map_mx, 0, sizeof(map_mx));
     a.mx_staged = 0;
     if (tma && (a.mx_outputs & NVFP4_COLWISE)) {
-        if (!make_mx_store_map(&map_mx, a.mx_q_col, a.rows, a.cols)) return NVFP4_ERR_CUDA;
+        if (!make_store_map(&map_mx, a.mx_q_col, a.rows, a.cols, 32)) return NVFP4_ERR_CUDA;
         a.mx_staged = 1;
     }
-    void* args[] = {&map, &map_mx, &a};
+    CUtensorMap map_qc;
+    memset(&map_qc, 0, sizeof(map_qc));
+    a.qc_staged = 0;
+    if (tma && (a.outputs & NVFP4_COLWISE) && a.rows % 32 == 0) {
+        if (!make_store_map(&map_qc, a.q_col, a.rows / 2, a.cols, 16)) return NVFP4_ERR_CUDA;
+        a.qc_staged = 1;
+    }
+    void* args[] = {&map, &map_mx, &map_qc, &a};
     if (cudaLaunchKernel(reinterpret_cast<const void*>(fn), dim3((unsigned)grid), dim3(kQuantThreads),
                          args, quant_smem_bytes(), st) != cudaSuccess)
         return NVFP4_ERR_CUDA;
