@@ -198,22 +198,59 @@ __device__ __forceinline__ U4 philox4x32_10(uint32_t c0, uint32_t c1, uint32_t c
     return U4{c0, c1, c2, c3};
 }
 
+// The ten round keys of one seed (key words after 0..9 Weyl steps), computed
+// once on the host and passed as kernel parameters, so each round's XOR reads
+// its key from the constant bank instead of recomputing it.
+struct PhiloxKeys {
+    uint32_t k0[10], k1[10];
+};
+
+inline void philox_round_keys(uint64_t seed, PhiloxKeys* k)
+{
+    uint32_t k0 = static_cast<uint32_t>(seed), k1 = static_cast<uint32_t>(seed >> 32);
+    for (int r = 0; r < 10; ++r) {
+        k->k0[r] = k0;
+        k->k1[r] = k1;
+        k0 += 0x9E3779B9u;
+        k1 += 0xBB67AE85u;
+    }
+}
+
+// Philox4x32-10 with precomputed round keys (same result as philox4x32_10
+// with key (k->k0[0], k->k1[0])).
+__device__ __forceinline__ U4 philox4x32_10_keyed(uint32_t c0, uint32_t c1, uint32_t c2, uint32_t c3,
+                                                   const PhiloxKeys& k)
+{
+#pragma unroll
+    for (int r = 0; r < 10; ++r) {
+        const uint64_t p0 = static_cast<uint64_t>(c0) * 0xD2511F53u;
+        const uint64_t p1 = static_cast<uint64_t>(c2) * 0xCD9E8D57u;
+        const uint32_t n0 = static_cast<uint32_t>(p1 >> 32) ^ c1 ^ k.k0[r];
+        const uint32_t n2 = static_cast<uint32_t>(p0 >> 32) ^ c3 ^ k.k1[r];
+        c0 = n0;
+        c1 = static_cast<uint32_t>(p1);
+        c2 = n2;
+        c3 = static_cast<uint32_t>(p0);
+    }
+    return U4{c0, c1, c2, c3};
+}
+
 // MXFP8 stream: random bits for elements idx8*8 .. idx8*8+7; element j takes
 // the 16-bit half (j % 2) of word j / 2.
-__device__ __forceinline__ U4 sr_block8(uint64_t seed, uint32_t offset, uint32_t stream,
+__device__ __forceinline__ U4 sr_block8(const PhiloxKeys& k, uint32_t offset, uint32_t stream,
                                         uint64_t idx8)
 {
-    return philox4x32_10(static_cast<uint32_t>(idx8), static_cast<uint32_t>(idx8 >> 32), stream,
-                         offset, static_cast<uint32_t>(seed), static_cast<uint32_t>(seed >> 32));
+    return philox4x32_10_keyed(static_cast<uint32_t>(idx8), static_cast<uint32_t>(idx8 >> 32), stream,
+                               offset, k);
 }
 
 // NVFP4 streams: the four words for elements idx16*16 .. idx16*16+15; word q
 // drives elements 4q .. 4q+3 through the stochastic-rounding conversion.
-__device__ __forceinline__ U4 sr_block16(uint64_t seed, uint32_t offset, uint32_t stream,
+__device__ __forceinline__ U4 sr_block16(const PhiloxKeys& k, uint32_t offset, uint32_t stream,
                                          uint64_t idx16)
 {
-    return philox4x32_10(static_cast<uint32_t>(idx16), static_cast<uint32_t>(idx16 >> 32), stream,
-                         offset, static_cast<uint32_t>(seed), static_cast<uint32_t>(seed >> 32));
+    return philox4x32_10_keyed(static_cast<uint32_t>(idx16), static_cast<uint32_t>(idx16 >> 32),
+                               stream, offset, k);
 }
 
 // Stochastic rounding of four scaled values onto E2M1 with Blackwell's

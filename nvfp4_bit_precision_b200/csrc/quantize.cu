@@ -63,6 +63,7 @@ struct QArgs {
     uint8_t *mx_q_row, *mx_sf_row, *mx_q_col, *mx_sf_col;
     uint32_t* status;
     int64_t tiles_c, n_tiles;
+    PhiloxKeys pk;  // round keys of `seed`
     int mx_staged;  // MXFP8 columnwise codes go through shared memory and TMA stores
     int qc_staged;  // NVFP4 columnwise codes likewise (rows a multiple of 32)
 };
@@ -201,7 +202,7 @@ __device__ __forceinline__ void unpack8(const uint4& p, float* v)
 // applied here exactly: amax_b/4 never rounds, and v*(r/4) == (v/4)*r whenever
 // r/4 is a normal float (otherwise the division is done per element).
 __device__ __forceinline__ uint32_t quant_block16(float (&v)[16], float amax_b, float S,
-                                                  bool times4, bool sr, uint64_t seed,
+                                                  bool times4, bool sr, const PhiloxKeys& pk,
                                                   uint32_t offset, uint32_t stream, uint64_t idx,
                                                   uint32_t& c0, uint32_t& c1)
 {
@@ -222,7 +223,7 @@ __device__ __forceinline__ uint32_t quant_block16(float (&v)[16], float amax_b, 
     for (int i = 0; i < 16; i += 2) mul2(v[i], v[i + 1], v[i], v[i + 1], r, r);
     if (sr) {
         // one Philox call per 16-element block: word q drives elements 4q..4q+3
-        const U4 w = sr_block16(seed, offset, stream, idx >> 4);
+        const U4 w = sr_block16(pk, offset, stream, idx >> 4);
         c0 = e2m1x4_sr(v + 0, w.x) | (e2m1x4_sr(v + 4, w.y) << 16);
         c1 = e2m1x4_sr(v + 8, w.z) | (e2m1x4_sr(v + 12, w.w) << 16);
     } else {
@@ -233,7 +234,7 @@ __device__ __forceinline__ uint32_t quant_block16(float (&v)[16], float amax_b, 
 }
 
 // MXFP8 of 32 values: returns the E8M0 byte, writes 32 code bytes to out[8].
-__device__ __forceinline__ uint32_t mx_block32(const float* v, bool sr, uint64_t seed,
+__device__ __forceinline__ uint32_t mx_block32(const float* v, bool sr, const PhiloxKeys& pk,
                                                uint32_t offset, uint64_t idx, uint32_t* out)
 {
     const float am = absmax16(v + 16, absmax16(v, 0.0f));
@@ -244,7 +245,7 @@ __device__ __forceinline__ uint32_t mx_block32(const float* v, bool sr, uint64_t
     if (sr) {
         U4 w[4];
 #pragma unroll
-        for (int q = 0; q < 4; ++q) w[q] = sr_block8(seed, offset, 2u, (idx >> 3) + q);
+        for (int q = 0; q < 4; ++q) w[q] = sr_block8(pk, offset, 2u, (idx >> 3) + q);
 #pragma unroll
         for (int k = 0; k < 8; ++k) {
             float y[4];
@@ -506,7 +507,7 @@ __host__ __device__ constexpr bool spec_pick(int8_t s, bool run_time)
 template <bool kTma, int kSpec>
 __global__ void __launch_bounds__(kQuantThreads, 2)
     quant_kernel(const __grid_constant__ CUtensorMap map_x, const __grid_constant__ CUtensorMap map_mx,
-                 const __grid_constant__ CUtensorMap map_qc, QArgs a)
+                 const __grid_constant__ CUtensorMap map_qc, const __grid_constant__ QArgs a)
 {
     constexpr QSpec sp = kSpecs[kSpec];
     extern __shared__ uint8_t smem_raw[];
@@ -647,7 +648,7 @@ __global__ void __launch_bounds__(kQuantThreads, 2)
                     float am = absmax16(v, 0.0f);
                     if (two_d) am = warp_max16(am);
                     uint32_t cw0, cw1;
-                    const uint32_t byte = quant_block16(v, am, S_row, false, sr && valid, a.seed,
+                    const uint32_t byte = quant_block16(v, am, S_row, false, sr && valid, a.pk,
                                                         a.offset, 0u,
                                                         (uint64_t)(rg * a.cols + cg), cw0, cw1);
                     codes[2 * blk] = cw0;
@@ -688,7 +689,7 @@ __global__ void __launch_bounds__(kQuantThreads, 2)
                     for (int q = 0; q < 4; ++q)
                         unpack8(ld_shared_v4(chunk_addr<kTma>(T, rl, 8 * h + 4 * part + q)), v + 8 * q);
                     uint32_t out[8];
-                    const uint32_t e8 = mx_block32(v, mx_sr, a.seed, a.offset,
+                    const uint32_t e8 = mx_block32(v, mx_sr, a.pk, a.offset,
                                                    (uint64_t)(rg * a.cols + cg), out);
                     uint4* dst = reinterpret_cast<uint4*>(a.mx_q_row + rg * a.cols + cg);
                     dst[0] = make_uint4(out[0], out[1], out[2], out[3]);
@@ -753,10 +754,10 @@ __global__ void __launch_bounds__(kQuantThreads, 2)
                         ama = amb = m;
                     }
                     uint32_t ca0, ca1, cb0, cb1;
-                    const uint32_t ba = quant_block16(va, ama, S_col, rht, sr && cvalid, a.seed,
+                    const uint32_t ba = quant_block16(va, ama, S_col, rht, sr && cvalid, a.pk,
                                                       a.offset, 1u, (uint64_t)(cg0 * a.rows + rg),
                                                       ca0, ca1);
-                    const uint32_t bb = quant_block16(vb, amb, S_col, rht, sr && cvalid, a.seed,
+                    const uint32_t bb = quant_block16(vb, amb, S_col, rht, sr && cvalid, a.pk,
                                                       a.offset, 1u,
                                                       (uint64_t)((cg0 + 1) * a.rows + rg), cb0, cb1);
                     if (!cvalid) continue;
@@ -837,8 +838,8 @@ __global__ void __launch_bounds__(kQuantThreads, 2)
                             }
                             U4 wa{}, wb{};
                             if (mx_sr) {
-                                wa = sr_block8(a.seed, a.offset, 2u, (uint64_t)(ia >> 3) + g);
-                                wb = sr_block8(a.seed, a.offset, 2u, (uint64_t)(ib >> 3) + g);
+                                wa = sr_block8(a.pk, a.offset, 2u, (uint64_t)(ia >> 3) + g);
+                                wb = sr_block8(a.pk, a.offset, 2u, (uint64_t)(ib >> 3) + g);
                             }
                             ca[gg] = mx_convert8(va, sa, mx_sr, wa);
                             cb[gg] = mx_convert8(vb, sb, mx_sr, wb);
@@ -876,8 +877,8 @@ __global__ void __launch_bounds__(kQuantThreads, 2)
                     }
                     U4 wa{}, wb{};
                     if (mx_sr) {
-                        wa = sr_block8(a.seed, a.offset, 2u, (uint64_t)(ia >> 3) + g);
-                        wb = sr_block8(a.seed, a.offset, 2u, (uint64_t)(ib >> 3) + g);
+                        wa = sr_block8(a.pk, a.offset, 2u, (uint64_t)(ia >> 3) + g);
+                        wb = sr_block8(a.pk, a.offset, 2u, (uint64_t)(ib >> 3) + g);
                     }
                     *reinterpret_cast<uint2*>(qa + 8 * g) = mx_convert8(va, sa, mx_sr, wa);
                     *reinterpret_cast<uint2*>(qb + 8 * g) = mx_convert8(vb, sb, mx_sr, wb);
@@ -1176,6 +1177,7 @@ extern "C" size_t nvfp4_quantize_workspace_size(int64_t, int64_t, const nvfp4_qu
 
 static nvfp4_status launch_quant(QArgs& a, bool need_amax, void* workspace, cudaStream_t st)
 {
+    philox_round_keys(a.seed, &a.pk);
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess) return NVFP4_ERR_CUDA;
     DeviceInfo& info = device_info(dev);
