@@ -124,6 +124,10 @@ __device__ __forceinline__ float warp_max16(float v)
 // Tile staging and block quantisation, shared by the passes.
 // --------------------------------------------------------------------------
 struct QShared {
+    // RN(S / d) for every scale byte (d its E4M3 value; 0 where d = 0), for
+    // the rowwise [0] and columnwise [1] global scales: the per-block
+    // division becomes a table lookup with the same result.
+    float rtab[2][128];
     int32_t n_groups;
     int32_t group_start[kMaxGroups + 1];   // output-row offsets
     int32_t group_padded[kMaxGroups + 1];  // padded scale-row offsets
@@ -202,15 +206,15 @@ __device__ __forceinline__ void unpack8(const uint4& p, float* v)
 // applied here exactly: amax_b/4 never rounds, and v*(r/4) == (v/4)*r whenever
 // r/4 is a normal float (otherwise the division is done per element).
 __device__ __forceinline__ uint32_t quant_block16(float (&v)[16], float amax_b, float S,
-                                                  bool times4, bool sr, const PhiloxKeys& pk,
-                                                  uint32_t offset, uint32_t stream, uint64_t idx,
-                                                  uint32_t& c0, uint32_t& c1)
+                                                  const float* rtab, bool times4, bool sr,
+                                                  const PhiloxKeys& pk, uint32_t offset,
+                                                  uint32_t stream, uint64_t idx, uint32_t& c0,
+                                                  uint32_t& c1)
 {
     if (times4) amax_b = __fmul_rn(amax_b, 0.25f);
     const float s = __fmul_rn(__fdiv_rn(amax_b, 6.0f), S);
     const uint32_t byte = e4m3_rne_sat(s);
-    const float d = e4m3_value(byte);
-    float r = (d != 0.0f) ? __fdiv_rn(S, d) : 0.0f;  // d = 0: every y is +-0
+    float r = rtab[byte];  // RN(S / d); 0 when d = 0, so every y is +-0
     if (times4) {
         if (r >= 7.52316384526264005100e-37f) {  // 2^-120: r/4 stays normal
             r = __fmul_rn(r, 0.25f);
@@ -572,6 +576,11 @@ __global__ void __launch_bounds__(kQuantThreads, 2)
             if (nv_row) *a.g_row = g_row;
             if (nv_col) *a.g_col = g_col;
         }
+        for (int t = threadIdx.x; t < 256; t += blockDim.x) {
+            const float d = e4m3_value((uint32_t)(t & 127));
+            sh->rtab[t >> 7][t & 127] = d != 0.0f ? __fdiv_rn(t < 128 ? S_row : S_col, d) : 0.0f;
+        }
+        __syncthreads();
     }
     const uint32_t signs = (nv_col && rht) ? rht_sign_bits(a.seed) : 0u;
 
@@ -648,7 +657,7 @@ __global__ void __launch_bounds__(kQuantThreads, 2)
                     float am = absmax16(v, 0.0f);
                     if (two_d) am = warp_max16(am);
                     uint32_t cw0, cw1;
-                    const uint32_t byte = quant_block16(v, am, S_row, false, sr && valid, a.pk,
+                    const uint32_t byte = quant_block16(v, am, S_row, sh->rtab[0], false, sr && valid, a.pk,
                                                         a.offset, 0u,
                                                         (uint64_t)(rg * a.cols + cg), cw0, cw1);
                     codes[2 * blk] = cw0;
@@ -754,10 +763,10 @@ __global__ void __launch_bounds__(kQuantThreads, 2)
                         ama = amb = m;
                     }
                     uint32_t ca0, ca1, cb0, cb1;
-                    const uint32_t ba = quant_block16(va, ama, S_col, rht, sr && cvalid, a.pk,
+                    const uint32_t ba = quant_block16(va, ama, S_col, sh->rtab[1], rht, sr && cvalid, a.pk,
                                                       a.offset, 1u, (uint64_t)(cg0 * a.rows + rg),
                                                       ca0, ca1);
-                    const uint32_t bb = quant_block16(vb, amb, S_col, rht, sr && cvalid, a.pk,
+                    const uint32_t bb = quant_block16(vb, amb, S_col, sh->rtab[1], rht, sr && cvalid, a.pk,
                                                       a.offset, 1u,
                                                       (uint64_t)((cg0 + 1) * a.rows + rg), cb0, cb1);
                     if (!cvalid) continue;
