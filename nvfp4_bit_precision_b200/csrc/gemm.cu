@@ -29,7 +29,10 @@
 //               K stage, the accumulator to both epilogues.
 //   warps 6..13 epilogue: tcgen05.ld of this CTA's 128x256 FP32 accumulator
 //               half (two warps per lane quadrant, converted as it is loaded),
-//               release of the accumulator to the leader, then stores.
+//               release of the accumulator to the leader, then stores.  BF16
+//               rows are turned around in a 2 KB staging block per warp so
+//               that each store instruction writes whole 32-byte sectors of 8
+//               rows instead of a 16-byte piece of 32 rows.
 // Every mbarrier wait is bounded (2 s); a timeout sets the workspace status
 // word and the kernel winds down instead of hanging.
 #include <cudaTypedefs.h>
@@ -64,6 +67,7 @@ constexpr int kTmemSF = 256;
 constexpr int kTmemSFStage = 48;
 static_assert(kTmemSF + kGemmStages * kTmemSFStage <= kTmemCols, "tensor memory overflow");
 constexpr int kMaxGemmGroups = 256;
+constexpr int kEpiStageBytes = 2048;  // per epilogue warp: 32 rows x 64 bytes of BF16
 
 struct GemmArgs {
     const uint8_t* sfa;
@@ -95,6 +99,8 @@ struct GemmShared {
     int32_t group_start[kMaxGemmGroups + 1];
     int32_t group_sfblk[kMaxGemmGroups + 1];  // first padded 128-row scale block of a group
 };
+
+constexpr int kSmemShared = (int)((sizeof(GemmShared) + 1023) / 1024 * 1024);
 
 // ---------------------------------------------------------------- PTX wrappers
 __device__ __forceinline__ uint32_t cluster_rank()
@@ -280,6 +286,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
     const uint32_t rank = cluster_rank();  // 0: leader (issues the MMAs), 1: peer
     const bool leader = rank == 0;
     const int pair = blockIdx.x >> 1, n_pairs = gridDim.x >> 1;
+    uint8_t* epi_stage = smem + kGemmStages * kStageBytes + kSmemShared;
 
     if (threadIdx.x == 0) {
         for (int s = 0; s < kGemmStages; ++s) {
@@ -455,6 +462,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
         const int quad = warp & 3;                   // TMEM lanes 32*quad .. 32*quad+31
         const int col0 = ((warp - 6) >> 2) * (BN / 2);  // 0 or 128
         const uint32_t acc_empty_leader = cluster_addr(&sh->acc_empty, 0);
+        uint8_t* stg = epi_stage + (warp - 6) * kEpiStageBytes;
         float out_max = 0.0f;                            // max |D| stored by this thread
         uint32_t tcount = 0;
         for (int t = pair; t < total; t += n_pairs, ++tcount) {
@@ -492,17 +500,15 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
                 tc_fence_before();
                 __syncwarp();
                 if (lane == 0) mbar_arrive_cluster(acc_empty_leader);  // accumulator drained
+                const int64_t cbase = c.n0 + col0;
+                // max |D| of this lane's row (rounded values where the N tail cuts the row)
                 if (row_ok) {
-                    const int64_t cbase = c.n0 + col0;
-                    uint16_t* drow = static_cast<uint16_t*>(a.D) + row * a.ldd + cbase;
-                    const bool whole = cbase + 128 <= a.N;
-                    if (whole) out_max = fmaxf(out_max, m_all);
+                    if (cbase + 128 <= a.N) {
+                        out_max = fmaxf(out_max, m_all);
+                    } else {
 #pragma unroll
-                    for (int g = 0; g < 16; ++g) {  // 8 columns per 16-byte store
-                        if (cbase + 8 * g < a.N) {
-                            *reinterpret_cast<uint4*>(drow + 8 * g) = make_uint4(
-                                packed[4 * g], packed[4 * g + 1], packed[4 * g + 2], packed[4 * g + 3]);
-                            if (!whole) {  // N tail: the max of the stored (rounded) values
+                        for (int g = 0; g < 16; ++g)
+                            if (cbase + 8 * g < a.N) {
 #pragma unroll
                                 for (int i = 0; i < 4; ++i) {
                                     const uint32_t w = packed[4 * g + i];
@@ -510,8 +516,29 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
                                                       __uint_as_float(w & 0xFFFF0000u));
                                 }
                             }
-                        }
                     }
+                }
+                const int64_t rowbase = c.row0 + (int64_t)BM * rank + 32 * quad;
+                // 32-column chunks through a 64-byte-swizzled 32x64-byte staging
+                // block: each lane writes its row, then 8 rows x 64 bytes leave
+                // per store instruction (whole 32-byte sectors).
+#pragma unroll
+                for (int hh = 0; hh < 4; ++hh) {
+#pragma unroll
+                    for (int q = 0; q < 4; ++q)
+                        st_shared_v4(stg + lane * 64 + 16 * (q ^ ((lane >> 1) & 3)),
+                                     make_uint4(packed[16 * hh + 4 * q], packed[16 * hh + 4 * q + 1],
+                                                packed[16 * hh + 4 * q + 2], packed[16 * hh + 4 * q + 3]));
+                    __syncwarp();
+#pragma unroll
+                    for (int i = 0; i < 4; ++i) {
+                        const int r = 8 * i + (lane >> 2), q = lane & 3;
+                        const uint4 v = lds128(stg + r * 64 + 16 * (q ^ ((r >> 1) & 3)));
+                        const int64_t grow = rowbase + r, col = cbase + 32 * hh + 8 * q;
+                        if (grow < c.row_end && col < a.N)
+                            *reinterpret_cast<uint4*>(static_cast<uint16_t*>(a.D) + grow * a.ldd + col) = v;
+                    }
+                    __syncwarp();
                 }
                 continue;
             }
@@ -592,7 +619,7 @@ static bool make_map(CUtensorMap* m, const void* base, int64_t rows, int64_t kby
               CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-static size_t gemm_smem_bytes() { return (size_t)kGemmStages * kStageBytes + sizeof(GemmShared) + 1024; }
+static size_t gemm_smem_bytes() { return (size_t)kGemmStages * kStageBytes + kSmemShared + 8 * kEpiStageBytes + 1024; }
 
 struct GemmDevice {
     int sms = 0;
