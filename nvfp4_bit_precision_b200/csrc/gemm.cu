@@ -16,8 +16,8 @@
 //   warp 0      TMA producer: this CTA's A/B boxes (128-byte swizzled, 4-bit
 //               codes two per byte; completing on the leader CTA's barrier,
 //               which expects both CTAs' bytes) and its scale atoms (own 128
-//               A rows; all 256 B rows; 1D bulk copies on its own barrier)
-//               into a 5-stage ring.
+//               A rows: one 1D bulk copy; all 256 B rows: one 4D box; both on
+//               its own barrier) into a 5-stage ring.
 //   warps 2..5  scale writers, one per tensor-memory lane quadrant: each lane
 //               loads row i of the stage's 512-byte scale atoms from shared
 //               memory and writes them into its quadrant of this CTA's tensor
@@ -144,6 +144,17 @@ __device__ __forceinline__ void tma_load_2d_pair(void* dst, const CUtensorMap* m
         "cp.async.bulk.tensor.2d.cta_group::2.shared::cluster.global.mbarrier::complete_tx::bytes "
         "[%0], [%1, {%2, %3}], [%4];" ::"r"(smem_addr(dst)),
         "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(bar)
+        : "memory");
+}
+
+// Four-dimensional TMA tile load completing on `bar` (x = 0 at every call site).
+__device__ __forceinline__ void tma_load_4d(void* dst, const CUtensorMap* map, int32_t x, int32_t y,
+                                            int32_t z, int32_t w, uint64_t* bar)
+{
+    asm volatile(
+        "cp.async.bulk.tensor.4d.shared::cluster.global.tile.mbarrier::complete_tx::bytes [%0], "
+        "[%1, {%2, %3, %4, %5}], [%6];" ::"r"(smem_addr(dst)),
+        "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(z), "r"(w), "r"(smem_addr(bar))
         : "memory");
 }
 
@@ -276,7 +287,7 @@ __device__ __forceinline__ TileCoord tile_coord(const GemmArgs& a, const GemmSha
 // ---------------------------------------------------------------- kernel
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
     gemm_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_constant__ CUtensorMap map_b,
-                GemmArgs a)
+                const __grid_constant__ CUtensorMap map_sfb, GemmArgs a)
 {
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
@@ -335,7 +346,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
         if (lane == 0) {
             asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&map_a)) : "memory");
             asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&map_b)) : "memory");
-            const int64_t nblk = (a.N + 127) / 128;  // 128-row scale blocks of one B operand
+            asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&map_sfb)) : "memory");
             uint32_t it = 0;
             for (int t = pair; t < total && !failed; t += n_pairs) {
                 const TileCoord c = tile_coord(a, sh, t);
@@ -346,8 +357,6 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
                 const int64_t sfa_blk = c.sf_blk + ((rank == 1 && a_row < c.row_end) ? 1 : 0);
                 const int64_t b_row = (int64_t)c.group * a.N + c.n0 + (int64_t)(BN / 2) * rank;
                 const int64_t nb0 = c.n0 / 128;
-                const int64_t nb1 = c.n0 + 128 < a.N ? nb0 + 1 : nb0;
-                const uint8_t* sfb_base = a.sfb + (int64_t)c.group * nblk * k64 * 512;
                 for (int64_t ks = 0; ks < kstages; ++ks, ++it) {
                     const int s = (int)(it % kGemmStages);
                     const uint32_t ph = (it / kGemmStages) & 1u;
@@ -365,10 +374,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
                     uint8_t* sf = st + kA_Bytes + kB_Bytes;
                     mbar_arrive_expect_tx(&sh->sf_full[s], kSFA_Bytes + kSFB_Bytes);
                     bulk_copy_g2s(sf, a.sfa + (sfa_blk * k64 + ks * 4) * 512, kSFA_Bytes, &sh->sf_full[s]);
-                    bulk_copy_g2s(sf + kSFA_Bytes, sfb_base + (nb0 * k64 + ks * 4) * 512, kSFB_Bytes / 2,
-                                  &sh->sf_full[s]);
-                    bulk_copy_g2s(sf + kSFA_Bytes + kSFB_Bytes / 2, sfb_base + (nb1 * k64 + ks * 4) * 512,
-                                  kSFB_Bytes / 2, &sh->sf_full[s]);
+                    // both 128-row blocks of B's scales in one box (a block past
+                    // the operand's end reads as zeros)
+                    tma_load_4d(sf + kSFA_Bytes, &map_sfb, 0, (int32_t)ks, (int32_t)nb0, c.group,
+                                &sh->sf_full[s]);
                 }
             }
             // Drain: the last stages' copies have landed once their MMAs
@@ -619,6 +628,23 @@ static bool make_map(CUtensorMap* m, const void* base, int64_t rows, int64_t kby
               CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// B's scales in the tensor-core layout, [G][nblk][K/64 atoms][512 bytes], seen
+// as 8-byte elements: {256 (one K stage's 4 atoms), K/256 stages, nblk, G}; a
+// box is one stage of two consecutive row blocks.
+static bool make_sfb_map(CUtensorMap* m, const void* sfb, int64_t G, int64_t N, int64_t K)
+{
+    auto fn = encode_tiled();
+    if (!fn) return false;
+    const int64_t nblk = (N + 127) / 128, k64 = K / 64;
+    cuuint64_t dims[4] = {256u, (cuuint64_t)(K / BK), (cuuint64_t)nblk, (cuuint64_t)G};
+    cuuint64_t strides[3] = {2048u, (cuuint64_t)(k64 * 512), (cuuint64_t)(nblk * k64 * 512)};
+    cuuint32_t box[4] = {256u, 1u, 2u, 1u};
+    cuuint32_t estr[4] = {1u, 1u, 1u, 1u};
+    return fn(m, CU_TENSOR_MAP_DATA_TYPE_UINT64, 4, const_cast<void*>(sfb), dims, strides, box, estr,
+              CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
+              CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 static size_t gemm_smem_bytes() { return (size_t)kGemmStages * kStageBytes + kSmemShared + 8 * kEpiStageBytes + 1024; }
 
 struct GemmDevice {
@@ -664,7 +690,7 @@ using namespace nvfp4;
 
 extern "C" size_t nvfp4_gemm_workspace_size(int64_t, int64_t, int64_t) { return kGemmWorkspace; }
 
-static nvfp4_status launch_gemm(const CUtensorMap& ma, const CUtensorMap& mb, GemmArgs& a,
+static nvfp4_status launch_gemm(const CUtensorMap& ma, const CUtensorMap& mb, const CUtensorMap& msf, GemmArgs& a,
                                 int64_t max_tiles, cudaStream_t st)
 {
     int dev = 0;
@@ -675,7 +701,7 @@ static nvfp4_status launch_gemm(const CUtensorMap& ma, const CUtensorMap& mb, Ge
     if (cudaMemsetAsync(a.status, 0, 4, st) != cudaSuccess) return NVFP4_ERR_CUDA;
     if (a.amax_out && cudaMemsetAsync(a.amax_out, 0, 4, st) != cudaSuccess) return NVFP4_ERR_CUDA;
     const int pairs = (int)std::max<int64_t>(1, std::min<int64_t>(max_tiles, info.pairs));
-    gemm_kernel<<<2 * pairs, kGemmThreads, gemm_smem_bytes(), st>>>(ma, mb, a);
+    gemm_kernel<<<2 * pairs, kGemmThreads, gemm_smem_bytes(), st>>>(ma, mb, msf, a);
     return cudaGetLastError() == cudaSuccess ? NVFP4_OK : NVFP4_ERR_CUDA;
 }
 
@@ -712,8 +738,10 @@ extern "C" nvfp4_status nvfp4_gemm(const uint8_t* qa, const uint8_t* sfa, const 
     a.G = 1;
     a.status = static_cast<uint32_t*>(workspace) + 2;
     a.amax_out = amax_out;
+    CUtensorMap msf;
+    if (!make_sfb_map(&msf, sfb, 1, N, K)) return NVFP4_ERR_CUDA;
     const int64_t tiles = ((M + kMmaM - 1) / kMmaM) * ((N + BN - 1) / BN);
-    return launch_gemm(ma, mb, a, tiles, static_cast<cudaStream_t>(stream));
+    return launch_gemm(ma, mb, msf, a, tiles, static_cast<cudaStream_t>(stream));
 }
 
 extern "C" nvfp4_status nvfp4_grouped_gemm(int G, const int32_t* group_offsets, int64_t total_rows,
@@ -755,6 +783,8 @@ extern "C" nvfp4_status nvfp4_grouped_gemm(int G, const int32_t* group_offsets, 
     a.status = static_cast<uint32_t*>(workspace) + 2;
     a.amax_out = amax_out;
     // upper bound on tiles: every group may add one partial M tile
+    CUtensorMap msf;
+    if (!make_sfb_map(&msf, sfb, G, N, K)) return NVFP4_ERR_CUDA;
     const int64_t tiles = ((total_rows + kMmaM - 1) / kMmaM + G) * ((N + BN - 1) / BN);
-    return launch_gemm(ma, mb, a, tiles, static_cast<cudaStream_t>(stream));
+    return launch_gemm(ma, mb, msf, a, tiles, static_cast<cudaStream_t>(stream));
 }
