@@ -46,7 +46,7 @@ DENSE_FLOP_PER_GEMM = 2 * TOKENS * FFN * HIDDEN
 # ncu --set full capture of each kernel as it stands -- the forward GEMM
 # 16384x20480x5120, and the amax + fused pass on dY 16384x20480; set to None
 # whenever the kernel changes.
-TRAFFIC_BYTES = {"gemm_dense_fwd": 1142.9e6, "quant_dy": None}
+TRAFFIC_BYTES = {"gemm_dense_fwd": 1147.1e6, "quant_dy": 2069.2e6}
 
 
 def peaks():
@@ -234,6 +234,25 @@ class Step:
             s = self.nv.nvfp4_workspace_status(w)
             if s != 0:
                 raise RuntimeError(f"device status {self.nv.status_string(s)}")
+
+
+# The tensor pipe's own FP4 rate as ncu reports it (sm__ops_path_tensor_op_utcomma
+# _src_fp4_dst_fp32: 32768 FLOP per SM per cycle, dense).  Context beside the
+# derived peak above, which a library FP4 GEMM exceeds on these shapes.
+HW_FP4_FLOP_PER_SM_CYCLE = 32768
+NUM_SMS = 148
+
+
+def hw_fp4_context(gemm_tflops, clocks):
+    mhz = (clocks or {}).get("sm_mhz")
+    if not mhz:
+        return {}
+    peak = HW_FP4_FLOP_PER_SM_CYCLE * NUM_SMS * mhz * 1e6 / 1e12
+    return {"hw_fp4_peak_at_clock": round(peak, 1),
+            "frac_of_hw_fp4_peak": round(gemm_tflops / peak, 4),
+            "hw_note": "ncu's dense FP4 tensor rate at the median SM clock of the timed region; "
+                       "the ncu capture of the forward GEMM reads 64.9% of it (at the profiler's "
+                       "1.55 GHz)"}
 
 
 def quant_algorithmic_bytes():
@@ -559,13 +578,15 @@ def main():
                                          "(ncu capture); algorithmic operand bytes 104 MB + "
                                          "output 671 MB",
                          "peak_note": f"4 x {pk['bf16_tflops_sustained']} sustained bf16 "
-                                      f"(fp4/bf16 nominal ratio 9/2.25), of {pk['source']}"},
+                                      f"(fp4/bf16 nominal ratio 9/2.25), of {pk['source']}",
+                         **hw_fp4_context(gemm_tflops, clocks)},
             "quantize_roofline": {"bound": "hbm", "kernel": "amax_kernel + quant_kernel on dY "
                                   "16384x20480 (row SR, col RHT+SR, MXFP8 col)",
                                   "achieved": round(qgbs, 1), "peak": pk["hbm_gbs"],
                                   "unit": "GB/s", "frac": round(qgbs / pk["hbm_gbs"], 4),
                                   "algorithmic_bytes": qbytes,
                                   "traffic": TRAFFIC_BYTES["quant_dy"],
+                                  "traffic_note": "amax + fused pass, DRAM bytes of one ncu capture",
                                   "peak_note": f"of {pk['source']}"},
             "breakdown_ms_per_step": breakdown,
             "e2e": {"value": round(value_e2e, 2), "unit": "TFLOP/s",
