@@ -366,11 +366,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
                         break;
                     }
                     uint8_t* st = smem + s * kStageBytes;
-                    if (leader) mbar_arrive_expect_tx(&sh->full[s], kPairCodeTx);
-                    const uint32_t fb = cluster_addr(&sh->full[s], 0);
-                    tma_load_2d_pair(st, &map_a, (int32_t)(ks * (BK / 2)), (int32_t)a_row, fb);
-                    tma_load_2d_pair(st + kA_Bytes, &map_b, (int32_t)(ks * (BK / 2)), (int32_t)b_row, fb);
-                    // this CTA's scale atoms: 4 consecutive atoms (2 KB) per 128-row block
+                    // this CTA's scale atoms first (they land first, and the scale
+                    // writers' work overlaps the code tiles' flight): 4 consecutive
+                    // atoms (2 KB) per 128-row block
                     uint8_t* sf = st + kA_Bytes + kB_Bytes;
                     mbar_arrive_expect_tx(&sh->sf_full[s], kSFA_Bytes + kSFB_Bytes);
                     bulk_copy_g2s(sf, a.sfa + (sfa_blk * k64 + ks * 4) * 512, kSFA_Bytes, &sh->sf_full[s]);
@@ -378,6 +376,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
                     // the operand's end reads as zeros)
                     tma_load_4d(sf + kSFA_Bytes, &map_sfb, 0, (int32_t)ks, (int32_t)nb0, c.group,
                                 &sh->sf_full[s]);
+                    if (leader) mbar_arrive_expect_tx(&sh->full[s], kPairCodeTx);
+                    const uint32_t fb = cluster_addr(&sh->full[s], 0);
+                    tma_load_2d_pair(st, &map_a, (int32_t)(ks * (BK / 2)), (int32_t)a_row, fb);
+                    tma_load_2d_pair(st + kA_Bytes, &map_b, (int32_t)(ks * (BK / 2)), (int32_t)b_row, fb);
                 }
             }
             // Drain: the last stages' copies have landed once their MMAs
