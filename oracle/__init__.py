@@ -75,6 +75,8 @@ def lib():
         L.orc_amax.argtypes = [P, i64, i64, i64, ctypes.c_int, ctypes.c_int, u64]
         L.orc_amax.restype = ctypes.c_float
         L.orc_mxfp8_quantize.restype = ctypes.c_int
+        L.orc_mxfp4_quantize.argtypes = [P, i64, i64, i64, ctypes.c_int, P, P]
+        L.orc_mxfp4_quantize.restype = ctypes.c_int
         L.orc_nvfp4_dequant_f64.argtypes = [P, P, ctypes.c_float, i64, i64, P]
         L.orc_nvfp4_dequant_f32.argtypes = [P, P, ctypes.c_float, i64, i64, P]
         L.orc_nvfp4_gemm_rows.argtypes = [P, P, ctypes.c_float, P, P, ctypes.c_float, i64, i64,
@@ -202,6 +204,32 @@ def mxfp8_quantize(x_bf16: np.ndarray, direction: int, rounding: int = 0, seed: 
     if rc != 0:
         raise ValueError("oracle mxfp8_quantize: invalid arguments")
     return q, e8
+
+
+def mxfp4_quantize(x_bf16: np.ndarray, direction: int):
+    """MXFP4 (OCP MX, E2M1 elements, E8M0 scale per 32): codes [rows, cols/2] +
+    E8M0 [rows, cols/32] (direction 0) or the same on x^T (direction 1)."""
+    x = np.ascontiguousarray(x_bf16, dtype=np.uint16)
+    rows, cols = x.shape
+    nr, nc = (cols, rows) if direction else (rows, cols)
+    q = np.zeros((nr, nc // 2), dtype=np.uint8)
+    e8 = np.zeros((nr, nc // 32), dtype=np.uint8)
+    rc = lib().orc_mxfp4_quantize(_p(x), rows, cols, cols, direction, _p(q), _p(e8))
+    if rc != 0:
+        raise ValueError("oracle mxfp4_quantize: invalid arguments")
+    return q, e8
+
+
+def mxfp4_dequant(q: np.ndarray, e8: np.ndarray) -> np.ndarray:
+    """x_hat = e2m1(code) * 2^(e8 - 127), exact in binary64."""
+    q = np.ascontiguousarray(q, dtype=np.uint8)
+    rows, half = q.shape
+    codes = np.empty((rows, half * 2), dtype=np.uint8)
+    codes[:, 0::2] = q & 0xF
+    codes[:, 1::2] = q >> 4
+    mag = np.array([e2m1_decode(c) for c in range(16)], dtype=np.float64)
+    scale = np.ldexp(1.0, np.repeat(np.asarray(e8, dtype=np.int64) - 127, 32, axis=1))
+    return mag[codes] * scale
 
 
 def nvfp4_dequant(q: np.ndarray, sf: np.ndarray, g: float, f64: bool = True) -> np.ndarray:

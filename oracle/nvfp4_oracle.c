@@ -18,7 +18,8 @@
  *             (hightech.plus, 2025-10-30).
  *   Philox4x32-10: J. K. Salmon, M. A. Moraes, R. O. Dror, D. E. Shaw,
  *             "Parallel random numbers: as easy as 1, 2, 3", SC'11.
- *   MXFP8 scale rule: OCP Microscaling Formats (MX) v1.0 specification.
+ *   MXFP8 and MXFP4 scale rule: OCP Microscaling Formats (MX) v1.0
+ *             specification.
  *
  * Arithmetic: decisions that pick a code (block scale, element scaling) are
  * taken in IEEE binary32, in the stated order, because the quantised code is
@@ -494,6 +495,62 @@ int orc_mxfp8_quantize(const uint16_t* x, int64_t rows, int64_t cols, int64_t ld
                 q[idx] = rounding ? orc_e4m3_sr_sat(y, orc_sr_bits(seed, offset, 2,
                                                                  idx_base + (uint64_t)idx))
                                   : orc_e4m3_rne_sat(y);
+            }
+        }
+    }
+    return ORC_OK;
+}
+
+/* ------------------------------------------------------------------------ */
+/* MXFP4: the Open Compute Project 4-bit format the pages compare NVFP4 with */
+/* [hightech: existing 4-bit formats such as MXFP4 fall short of 8-bit       */
+/* accuracy; asector, "NVFP4 and Blackwell": the tensor cores take MXFP4,    */
+/* and NVFP4 beat the OCP's MXFP4].  The pages do not restate the format;    */
+/* the OCP MX v1.0 rule is used, as for MXFP8 above with the element format  */
+/* E2M1: e = floor(log2(amax_32)) - 2 (2 = largest E2M1 exponent, 6 = 1.5 *  */
+/* 2^2), clamped to [-127, 127], stored as e + 127; amax 0 gives e = -127.    */
+/* Element = E2M1 RNE of x * 2^-e, saturating at 6 (the same RNE search as   */
+/* NVFP4's).  Codes two per byte, even index in the low nibble.              */
+/* direction 0: blocks along cols, codes [rows, cols/2], scales [rows,       */
+/* cols/32]; direction 1: on x^T, codes [cols, rows/2], scales [cols,        */
+/* rows/32].  No tensor scale, no stochastic rounding.                       */
+/* ------------------------------------------------------------------------ */
+int orc_mxfp4_quantize(const uint16_t* x, int64_t rows, int64_t cols, int64_t ld,
+                       int direction, uint8_t* q, uint8_t* e8)
+{
+    int64_t nr = direction ? cols : rows, nc = direction ? rows : cols;
+    if (rows <= 0 || cols <= 0 || nc % 32 || ld < cols) return ORC_EINVAL;
+    for (int64_t r = 0; r < nr; ++r) {
+        for (int64_t b = 0; b < nc / 32; ++b) {
+            double vals[32];
+            double amax = 0.0;
+            for (int i = 0; i < 32; ++i) {
+                int64_t c = b * 32 + i;
+                uint16_t raw = direction ? x[c * ld + r] : x[r * ld + c];
+                vals[i] = (double)bf16_to_float(raw);
+                if (fabs(vals[i]) > amax) amax = fabs(vals[i]);
+            }
+            int e;
+            if (amax == 0.0) {
+                e = -127;
+            } else {
+                int k;
+                frexp(amax, &k); /* amax = m 2^k, m in [0.5, 1): floor(log2) = k-1 */
+                e = (k - 1) - 2;
+                if (e < -127) e = -127;
+                if (e > 127) e = 127;
+            }
+            e8[r * (nc / 32) + b] = (uint8_t)(e + 127);
+            for (int i = 0; i < 32; ++i) {
+                /* y is exact in binary64; as a float it is exact whenever it is
+                 * a normal float, and smaller values all round to code 0 */
+                uint8_t code = orc_e2m1_rne((float)ldexp(vals[i], -e));
+                int64_t idx = r * nc + b * 32 + i;
+                uint8_t* byte = &q[idx / 2];
+                if (idx % 2 == 0)
+                    *byte = (uint8_t)((*byte & 0xF0) | code);
+                else
+                    *byte = (uint8_t)((*byte & 0x0F) | (code << 4));
             }
         }
     }
