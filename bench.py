@@ -255,6 +255,34 @@ def hw_fp4_context(gemm_tflops, clocks):
                        "1.55 GHz)"}
 
 
+def time_mxfp4(step, steps, warmup):
+    """MXFP4 (OCP: 32-blocks, E8M0, E2M1) of the resident dY, both directions from one
+    call, timed apart from the step: mean ms per launch over `steps` launches after
+    `warmup`, CUDA events on the launching stream.  dY (671 MB) is larger than L2."""
+    nv, torch = step.nv, step.torch
+    dy = step.inputs[0]["dy"]
+    R, C = dy.shape
+    u8 = dict(dtype=torch.uint8, device=dy.device)
+    qr, er = torch.empty((R, C // 2), **u8), torch.empty((R, C // 32), **u8)
+    qc, ec = torch.empty((C, R // 2), **u8), torch.empty((C, R // 32), **u8)
+    both = nv.NVFP4_ROWWISE | nv.NVFP4_COLWISE
+    run = lambda: nv.mxfp4_quantize(dy, R, C, dy.stride(0), both, qr, er, qc, ec)
+    for _ in range(max(warmup, 3)):
+        run()
+    stream = torch.cuda.current_stream()
+    torch.cuda.synchronize()
+    s, e = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    s.record(stream)
+    for _ in range(steps):
+        run()
+    e.record(stream)
+    torch.cuda.synchronize()
+    ms = s.elapsed_time(e) / steps
+    n = R * C
+    nbytes = 2 * n + 2 * (n // 2 + n // 32)  # one bf16 read, codes + scales both ways
+    return ms, nbytes
+
+
 def quant_algorithmic_bytes():
     """Bytes the dY quantisation must move: two reads of the bf16 input (amax pass and
     quantise pass), NVFP4 codes and scales in both directions, MXFP8 codes and scales."""
@@ -542,6 +570,7 @@ def main():
     barrier()
     ms_e2e = e0.elapsed_time(e1)
 
+    mx4_ms, mx4_bytes = time_mxfp4(step, args.steps, args.warmup)
     ms, ms_e2e = max_over_ranks([ms, ms_e2e], world, dev)
     value = job_tflops(step.flops(), world, args.steps, ms)
     value_e2e = job_tflops(step.flops(), world, args.steps, ms_e2e)
@@ -589,6 +618,13 @@ def main():
                                   "traffic_note": "amax + fused pass, DRAM bytes of one ncu capture",
                                   "peak_note": f"of {pk['source']}"},
             "breakdown_ms_per_step": breakdown,
+            "next_rows": {"mxfp4_quantize": {
+                "bound": "hbm", "kernel": "mxfp4_kernel on dY 16384x20480, both directions "
+                "(timed apart from the step)", "ms": round(mx4_ms, 4),
+                "achieved": round(mx4_bytes / (mx4_ms / 1e3) / 1e9, 1), "peak": pk["hbm_gbs"],
+                "unit": "GB/s",
+                "frac": round(mx4_bytes / (mx4_ms / 1e3) / 1e9 / pk["hbm_gbs"], 4),
+                "algorithmic_bytes": mx4_bytes, "peak_note": f"of {pk['source']}"}},
             "e2e": {"value": round(value_e2e, 2), "unit": "TFLOP/s",
                     "h2d_bytes_per_step": step.h2d_bytes(), "d2h_bytes_per_step": d2h},
             "gpu_launches": Step.LAUNCHES_PER_STEP * args.steps,

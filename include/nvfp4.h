@@ -201,6 +201,25 @@ nvfp4_status mxfp8_quantize(const void* x_bf16, int64_t rows, int64_t cols, int6
                             void* stream);
 
 /*
+ * mxfp4_quantize -- MXFP4, the Open Compute Project 4-bit format the pages
+ * compare NVFP4 against (hightech; asector, "NVFP4 and Blackwell" and the
+ * comparison with MXFP4).  The pages do not restate it; the OCP MX v1.0 rule
+ * is used: per 32-element block e = clamp(floor(log2 amax) - 2, -127, 127)
+ * (2 = largest E2M1 exponent), E8M0 byte e + 127 (amax 0 -> byte 0), element =
+ * E2M1 of x * 2^-e, round-to-nearest-even saturating at +-6.  No tensor scale.
+ * Codes two per byte, even index in the low nibble.
+ * directions: NVFP4_ROWWISE (codes [rows, cols/2], scales [rows, cols/32])
+ * and/or NVFP4_COLWISE (codes [cols, rows/2], scales [cols, rows/32]); both
+ * come from one read of x.  rows and cols multiples of 32 (NVFP4_ERR_SHAPE);
+ * x, q_row, q_col 16-byte aligned and ld a multiple of 8 (NVFP4_ERR_ALIGN);
+ * a requested direction with a NULL output -> NVFP4_ERR_INVALID_ARG.  All
+ * buffers are device memory owned by the caller; asynchronous on `stream`.
+ */
+nvfp4_status mxfp4_quantize(const void* x_bf16, int64_t rows, int64_t cols, int64_t ld,
+                            int directions, uint8_t* q_row, uint8_t* e8_row, uint8_t* q_col,
+                            uint8_t* e8_col, void* stream);
+
+/*
  * nvfp4_gather_rows -- MoE dispatch of quantised rows (iitak, "Details" and
  * "But": tokens travel to the expert layers, where NVFP4 is used).  Output row
  * i is source row row_index[i]: its codes [k/2 bytes] and its scale bytes,

@@ -2,14 +2,14 @@
 block-scaled GEMM.
 
 The C functions keep their names (``nvfp4_quantize``, ``nvfp4_dequantize``,
-``mxfp8_quantize``, ``nvfp4_gemm``, ``nvfp4_grouped_gemm``); this module only
+``mxfp8_quantize``, ``mxfp4_quantize``, ``nvfp4_gemm``, ``nvfp4_grouped_gemm``); this module only
 marshals arguments: torch tensors become device pointers and the current torch
 stream becomes the ``cudaStream_t``.  Every arithmetic step runs in the CUDA
 kernels of ``libnvfp4.so``.  There is no fallback: importing this package
 raises if the library is missing, and every call raises ``NVFP4Error`` on a
 non-zero status.
 
-The convenience wrappers (``quantize``, ``dequantize``, ``mxfp8``, ``gemm``,
+The convenience wrappers (``quantize``, ``dequantize``, ``mxfp8``, ``mxfp4``, ``gemm``,
 ``grouped_gemm``) allocate their outputs with torch and call the C functions.
 """
 from __future__ import annotations
@@ -45,7 +45,7 @@ EXPORTED = [
     "nvfp4_quantize", "nvfp4_dequantize", "mxfp8_quantize", "nvfp4_gemm", "nvfp4_grouped_gemm",
     "nvfp4_quantize_workspace_size", "nvfp4_gemm_workspace_size", "nvfp4_sf_mma_bytes",
     "nvfp4_sf_mma_grouped_bytes", "nvfp4_workspace_status", "nvfp4_status_string",
-    "nvfp4_version", "nvfp4_quantize_noalloc", "nvfp4_gather_rows",
+    "nvfp4_version", "nvfp4_quantize_noalloc", "nvfp4_gather_rows", "mxfp4_quantize",
 ]
 
 
@@ -71,6 +71,7 @@ _lib.nvfp4_quantize_noalloc.argtypes = [_P, _I64, _I64, _I64, ctypes.POINTER(Qua
                                         _P, _P, _P, _P, _P, _P]
 _lib.mxfp8_quantize.argtypes = [_P, _I64, _I64, _I64, ctypes.c_int, ctypes.c_int,
                                 ctypes.c_uint64, ctypes.c_uint32, _P, _P, _P, _P, _P]
+_lib.mxfp4_quantize.argtypes = [_P, _I64, _I64, _I64, ctypes.c_int, _P, _P, _P, _P, _P]
 _lib.nvfp4_dequantize.argtypes = [_P, _P, _P, _I64, _I64, ctypes.c_int, ctypes.c_int, _P, _P]
 _lib.nvfp4_gemm.argtypes = [_P, _P, _P, _P, _P, _P, _I64, _I64, _I64, ctypes.c_int, _P, _I64, _P,
                             _P, _SZ, _P]
@@ -90,7 +91,8 @@ _lib.nvfp4_workspace_status.argtypes = [_P, _P]
 _lib.nvfp4_status_string.argtypes = [ctypes.c_int]
 _lib.nvfp4_status_string.restype = ctypes.c_char_p
 _lib.nvfp4_version.restype = ctypes.c_int
-for _n in ("nvfp4_quantize", "nvfp4_quantize_noalloc", "mxfp8_quantize", "nvfp4_dequantize", "nvfp4_gemm",
+for _n in ("nvfp4_quantize", "nvfp4_quantize_noalloc", "mxfp8_quantize", "mxfp4_quantize",
+           "nvfp4_dequantize", "nvfp4_gemm",
            "nvfp4_grouped_gemm", "nvfp4_gather_rows", "nvfp4_workspace_status"):
     getattr(_lib, _n).restype = ctypes.c_int
 
@@ -149,6 +151,12 @@ def mxfp8_quantize(x, rows, cols, ld, directions, rounding, seed, offset, q_row,
     _check(_lib.mxfp8_quantize(_ptr(x), rows, cols, ld, directions, rounding, seed, offset,
                                _ptr(q_row), _ptr(e8_row), _ptr(q_col), _ptr(e8_col),
                                _stream(stream)), "mxfp8_quantize")
+
+
+def mxfp4_quantize(x, rows, cols, ld, directions, q_row, e8_row, q_col, e8_col,
+                   stream=None) -> None:
+    _check(_lib.mxfp4_quantize(_ptr(x), rows, cols, ld, directions, _ptr(q_row), _ptr(e8_row),
+                               _ptr(q_col), _ptr(e8_col), _stream(stream)), "mxfp4_quantize")
 
 
 def nvfp4_dequantize(q, sf, g, rows, cols, sf_layout, out_dtype, out, stream=None) -> None:
@@ -297,6 +305,22 @@ def mxfp8(x, directions: int = NVFP4_COLWISE, rounding: int = NVFP4_RNE, seed: i
         qc, ec = torch.empty((cols, rows), **u8), torch.empty((cols, rows // 32), **u8)
     mxfp8_quantize(x, rows, cols, x.stride(0), directions, rounding, seed, offset, qr, er, qc, ec,
                    stream)
+    return (qr, er), (qc, ec)
+
+
+def mxfp4(x, directions: int = NVFP4_ROWWISE | NVFP4_COLWISE, stream=None):
+    """MXFP4 codes and E8M0 scales of a bf16 [rows, cols] tensor:
+    ((q_row [rows, cols/2], e8 [rows, cols/32]) or (None, None),
+     (q_col [cols, rows/2], e8 [cols, rows/32]) or (None, None))."""
+    import torch
+    rows, cols = x.shape
+    u8 = dict(dtype=torch.uint8, device=x.device)
+    qr = er = qc = ec = None
+    if directions & NVFP4_ROWWISE:
+        qr, er = torch.empty((rows, cols // 2), **u8), torch.empty((rows, cols // 32), **u8)
+    if directions & NVFP4_COLWISE:
+        qc, ec = torch.empty((cols, rows // 2), **u8), torch.empty((cols, rows // 32), **u8)
+    mxfp4_quantize(x, rows, cols, x.stride(0), directions, qr, er, qc, ec, stream)
     return (qr, er), (qc, ec)
 
 

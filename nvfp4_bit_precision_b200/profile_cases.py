@@ -3,6 +3,7 @@
     python -m nvfp4_bit_precision_b200.profile_cases gemm M N K [--warm W]
     python -m nvfp4_bit_precision_b200.profile_cases grouped-gemm N K [--warm W]
     python -m nvfp4_bit_precision_b200.profile_cases quant-grad ROWS COLS [--warm W]
+    python -m nvfp4_bit_precision_b200.profile_cases mxfp4 ROWS COLS [--warm W]
 
 Each runs W untimed launches of the case, then one more, on synthetic operands
 (codes and in-range scale bytes drawn on the device; bf16 inputs ~N(0, 1e-3)),
@@ -68,9 +69,20 @@ def _quant_grad(nv, torch, rows, cols, warm):
     return ws
 
 
+def _mxfp4(nv, torch, rows, cols, warm):
+    """MXFP4 of a bf16 ~N(0, 1) tensor, both directions."""
+    dev = torch.device("cuda")
+    g = torch.Generator(device=dev)
+    g.manual_seed(2)
+    x = torch.randn((rows, cols), generator=g, device=dev).to(torch.bfloat16)
+    for _ in range(warm + 1):
+        nv.mxfp4(x, nv.NVFP4_ROWWISE | nv.NVFP4_COLWISE)
+    return None
+
+
 def main(argv=None) -> int:
     ap = argparse.ArgumentParser()
-    ap.add_argument("case", choices=["gemm", "grouped-gemm", "quant-grad"])
+    ap.add_argument("case", choices=["gemm", "grouped-gemm", "quant-grad", "mxfp4"])
     ap.add_argument("dims", type=int, nargs="+")
     ap.add_argument("--warm", type=int, default=3)
     args = ap.parse_args(argv)
@@ -81,10 +93,12 @@ def main(argv=None) -> int:
         ws = _gemm(nv, torch, *args.dims[:3], args.warm)
     elif args.case == "grouped-gemm":
         ws = _grouped(nv, torch, *args.dims[:2], args.warm)
-    else:
+    elif args.case == "quant-grad":
         ws = _quant_grad(nv, torch, *args.dims[:2], args.warm)
+    else:
+        ws = _mxfp4(nv, torch, *args.dims[:2], args.warm)
     torch.cuda.synchronize()
-    status = nv.nvfp4_workspace_status(ws)
+    status = nv.nvfp4_workspace_status(ws) if ws is not None else 0
     print(f"{args.case} {args.dims}: status {nv.status_string(status)}")
     return 0 if status == 0 else 1
 

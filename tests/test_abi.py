@@ -116,3 +116,17 @@ def test_mxfp8_and_dequant_argument_errors(nv):
     assert L.mxfp8_quantize(FAKE, 32, 48, 48, 1, 0, 0, 0, FAKE, FAKE, None, None, None) == 2
     assert L.nvfp4_dequantize(FAKE, FAKE, FAKE, 16, 24, 0, 0, FAKE, None) == 2
     assert L.nvfp4_dequantize(FAKE, FAKE, FAKE, 16, 32, 0, 3, FAKE, None) == 1
+
+
+def test_mxfp4_argument_errors(nv):
+    L = nv._lib
+    assert L.mxfp4_quantize(None, 32, 32, 32, 1, FAKE, FAKE, None, None, None) == 1
+    assert L.mxfp4_quantize(FAKE, 32, 32, 32, 0, FAKE, FAKE, FAKE, FAKE, None) == 1   # no direction
+    assert L.mxfp4_quantize(FAKE, 32, 32, 32, 4, FAKE, FAKE, FAKE, FAKE, None) == 1   # unknown bit
+    assert L.mxfp4_quantize(FAKE, 32, 32, 32, 2, FAKE, FAKE, None, FAKE, None) == 1   # col output NULL
+    assert L.mxfp4_quantize(FAKE, 48, 32, 32, 1, FAKE, FAKE, None, None, None) == 2   # rows % 32
+    assert L.mxfp4_quantize(FAKE, 32, 48, 48, 1, FAKE, FAKE, None, None, None) == 2   # cols % 32
+    assert L.mxfp4_quantize(FAKE, 32, 64, 32, 1, FAKE, FAKE, None, None, None) == 2   # ld < cols
+    assert L.mxfp4_quantize(FAKE + 8, 32, 32, 32, 1, FAKE, FAKE, None, None, None) == 3
+    assert L.mxfp4_quantize(FAKE, 32, 32, 36, 1, FAKE, FAKE, None, None, None) == 3   # ld % 8
+    assert L.mxfp4_quantize(FAKE, 32, 32, 32, 2, None, None, FAKE + 4, FAKE, None) == 3
