@@ -13,13 +13,17 @@
 // element = E2M1 of x * 2^-e, round-to-nearest-even, saturating at +-6.
 // There is no tensor scale.
 //
-// One CTA per 64 x 128 tile: the tile is loaded once into shared memory with
-// coalesced 16-byte loads; warps 0..3 quantise its columns (thread = column
-// pair x 32-row block, one 32-bit shared load per row gives both columns),
-// warps 4..7 its rows (thread = row x 64-column half, two blocks).  The
-// kernel is HBM-bound: 2 bytes read and 0.5 + 1/32 written per element and
-// direction.
+// Persistent CTAs walk 64 x 128 tiles; each tile is copied into one of two
+// shared-memory buffers with 16-byte cp.async while the CTA quantises the
+// other.  Warps 0..3 quantise the tile's columns (thread = column pair x
+// 32-row block, one 32-bit shared load per row gives both columns), warps
+// 4..7 its rows (thread = one 32-block of a row; four lanes cover a row's 64
+// code bytes, so every store instruction writes whole sectors).  Values stay
+// packed as bf16 pairs and are unpacked where they are used.  The kernel is
+// HBM-bound: 2 bytes read and 0.5 + 1/32 written per element and direction.
 #include "common.cuh"
+
+#include <mutex>
 
 namespace nvfp4 {
 namespace {
@@ -36,17 +40,8 @@ struct Mx4Args {
     uint8_t* e8_row;
     uint8_t* q_col;
     uint8_t* e8_col;
-    int64_t tiles_c;
+    int64_t tiles_r, tiles_c;
 };
-
-__device__ __forceinline__ uint4 ldg_nc_v4(const void* p)
-{
-    uint4 r;
-    asm volatile("ld.global.nc.v4.u32 {%0,%1,%2,%3}, [%4];"
-                 : "=r"(r.x), "=r"(r.y), "=r"(r.z), "=r"(r.w)
-                 : "l"(p));
-    return r;
-}
 
 // E8M0 byte of a block with absolute maximum am, and the exact factor 2^-e
 // its elements are multiplied by.  floor(log2 am) is the unbiased exponent
@@ -60,90 +55,155 @@ __device__ __forceinline__ uint32_t mx4_scale(float am, float& factor)
     return (uint32_t)(e + 127);
 }
 
-// 32 values -> 16 code bytes (element 0 in the low nibble of byte 0).
-__device__ __forceinline__ uint4 mx4_codes(const float (&v)[32], float factor)
+// Eight values, given as four bf16 pairs (element 0 in the low half), times
+// the block factor -> eight codes (element 0 in the low nibble).
+__device__ __forceinline__ uint32_t mx4_codes8(uint32_t w0, uint32_t w1, uint32_t w2, uint32_t w3,
+                                               float f)
 {
-    uint32_t c[4];
-#pragma unroll
-    for (int g = 0; g < 4; ++g) {
-        float y[8];
-#pragma unroll
-        for (int i = 0; i < 8; i += 2) mul2(y[i], y[i + 1], v[8 * g + i], v[8 * g + i + 1], factor, factor);
-        c[g] = e2m1x8_rne(y);
-    }
-    return make_uint4(c[0], c[1], c[2], c[3]);
+    float y[8];
+    mul2(y[0], y[1], bf16_lo(w0), bf16_hi(w0), f, f);
+    mul2(y[2], y[3], bf16_lo(w1), bf16_hi(w1), f, f);
+    mul2(y[4], y[5], bf16_lo(w2), bf16_hi(w2), f, f);
+    mul2(y[6], y[7], bf16_lo(w3), bf16_hi(w3), f, f);
+    return e2m1x8_rne(y);
 }
 
-__global__ void __launch_bounds__(kMx4Threads) mxfp4_kernel(const Mx4Args a)
+// Copy tile t into `buf` (64 rows of 16 chunks of 8 elements); chunks past the
+// tensor are zero-filled without reading and only feed blocks never stored.
+__device__ __forceinline__ void mx4_issue_tile(const Mx4Args& a, int64_t t, uint8_t* buf)
 {
-    __shared__ __align__(16) uint8_t tile[kMx4TileRows * kMx4Pitch];
-    const int64_t tr = blockIdx.x / a.tiles_c, tcol = blockIdx.x - tr * a.tiles_c;
+    const int64_t tr = t / a.tiles_c, tcol = t - tr * a.tiles_c;
+    const int64_t r0 = tr * kMx4TileRows, c0 = tcol * kMx4TileCols;
+#pragma unroll
+    for (int i = threadIdx.x; i < kMx4TileRows * 16; i += kMx4Threads) {
+        const int r = i >> 4, q = i & 15;
+        const bool in = r0 + r < a.rows && c0 + 8 * q < a.cols;
+        const uint16_t* src = in ? a.x + (r0 + r) * a.ld + c0 + 8 * q : a.x;
+        asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(
+                         smem_addr(buf + r * kMx4Pitch + 16 * q)),
+                     "l"(src), "r"(in ? 16 : 0)
+                     : "memory");
+    }
+    asm volatile("cp.async.commit_group;" ::: "memory");
+}
+
+__device__ __forceinline__ void mx4_tile(const Mx4Args& a, int64_t t, const uint8_t* tile)
+{
+    const int64_t tr = t / a.tiles_c, tcol = t - tr * a.tiles_c;
     const int64_t r0 = tr * kMx4TileRows, c0 = tcol * kMx4TileCols;
     // valid extent of the tile: multiples of 32 (rows and cols are)
     const int nr = a.rows - r0 < kMx4TileRows ? (int)(a.rows - r0) : kMx4TileRows;
     const int nc = a.cols - c0 < kMx4TileCols ? (int)(a.cols - c0) : kMx4TileCols;
-
-    // 64 rows x 16 chunks of 8 elements; chunks past the tensor are zeros
-    // and only ever feed blocks that are not stored.
-#pragma unroll
-    for (int i = threadIdx.x; i < kMx4TileRows * 16; i += kMx4Threads) {
-        const int r = i >> 4, q = i & 15;
-        uint4 v = make_uint4(0u, 0u, 0u, 0u);
-        if (r < nr && 8 * q < nc) v = ldg_nc_v4(a.x + (r0 + r) * a.ld + c0 + 8 * q);
-        *reinterpret_cast<uint4*>(tile + r * kMx4Pitch + 16 * q) = v;
-    }
-    __syncthreads();
-
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     if (warp < 4) {
         if (!a.q_col) return;
         // columnwise: column pair cp (columns 2cp, 2cp + 1), 32-row block rb
         const int cp = 32 * (warp & 1) + lane, rb = warp >> 1;
         if (2 * cp >= nc || 32 * rb >= nr) return;
-        float va[32], vb[32];
+        uint32_t w[32];
+        float ma = 0.0f, mb = 0.0f;
 #pragma unroll
         for (int i = 0; i < 32; ++i) {
-            const uint32_t w = *reinterpret_cast<const uint32_t*>(tile + (32 * rb + i) * kMx4Pitch + 4 * cp);
-            va[i] = bf16_lo(w);
-            vb[i] = bf16_hi(w);
+            w[i] = *reinterpret_cast<const uint32_t*>(tile + (32 * rb + i) * kMx4Pitch + 4 * cp);
+            ma = absmax3(ma, bf16_lo(w[i]), 0.0f);
+            mb = absmax3(mb, bf16_hi(w[i]), 0.0f);
         }
         float fa, fb;
-        const uint32_t ea = mx4_scale(absmax16(va + 16, absmax16(va, 0.0f)), fa);
-        const uint32_t eb = mx4_scale(absmax16(vb + 16, absmax16(vb, 0.0f)), fb);
+        const uint32_t ea = mx4_scale(ma, fa), eb = mx4_scale(mb, fb);
+        uint32_t ca[4], cb[4];
+#pragma unroll
+        for (int g = 0; g < 4; ++g) {
+            // column a = low halves, column b = high halves of rows 8g .. 8g+7
+            float y[8];
+#pragma unroll
+            for (int i = 0; i < 8; i += 2)
+                mul2(y[i], y[i + 1], bf16_lo(w[8 * g + i]), bf16_lo(w[8 * g + i + 1]), fa, fa);
+            ca[g] = e2m1x8_rne(y);
+#pragma unroll
+            for (int i = 0; i < 8; i += 2)
+                mul2(y[i], y[i + 1], bf16_hi(w[8 * g + i]), bf16_hi(w[8 * g + i + 1]), fb, fb);
+            cb[g] = e2m1x8_rne(y);
+        }
         const int64_t col = c0 + 2 * cp, rr = r0 + 32 * rb;
-        *reinterpret_cast<uint4*>(a.q_col + col * (a.rows / 2) + rr / 2) = mx4_codes(va, fa);
-        *reinterpret_cast<uint4*>(a.q_col + (col + 1) * (a.rows / 2) + rr / 2) = mx4_codes(vb, fb);
+        *reinterpret_cast<uint4*>(a.q_col + col * (a.rows / 2) + rr / 2) =
+            make_uint4(ca[0], ca[1], ca[2], ca[3]);
+        *reinterpret_cast<uint4*>(a.q_col + (col + 1) * (a.rows / 2) + rr / 2) =
+            make_uint4(cb[0], cb[1], cb[2], cb[3]);
         a.e8_col[col * (a.rows / 32) + rr / 32] = (uint8_t)ea;
         a.e8_col[(col + 1) * (a.rows / 32) + rr / 32] = (uint8_t)eb;
     } else {
         if (!a.q_row) return;
-        // rowwise: row r, 64-column half h (two 32-blocks)
-        const int t = threadIdx.x - 128;
-        const int r = t >> 1, h = t & 1;
-        if (r >= nr) return;
+        // rowwise: block blk (32 columns) of row r, for r = t/4 and t/4 + 32
+        const int u = threadIdx.x - 128;
+        const int blk = u & 3;
+        if (32 * blk >= nc) return;
 #pragma unroll
-        for (int blk = 0; blk < 2; ++blk) {
-            const int cb = 64 * h + 32 * blk;
-            if (cb >= nc) break;
-            float v[32];
+        for (int pass = 0; pass < 2; ++pass) {
+            const int r = (u >> 2) + 32 * pass;
+            if (r >= nr) break;
+            uint4 p[4];
+            float m = 0.0f;
 #pragma unroll
             for (int q = 0; q < 4; ++q) {
-                const uint4 p = *reinterpret_cast<const uint4*>(tile + r * kMx4Pitch + 2 * cb + 16 * q);
-                v[8 * q + 0] = bf16_lo(p.x), v[8 * q + 1] = bf16_hi(p.x);
-                v[8 * q + 2] = bf16_lo(p.y), v[8 * q + 3] = bf16_hi(p.y);
-                v[8 * q + 4] = bf16_lo(p.z), v[8 * q + 5] = bf16_hi(p.z);
-                v[8 * q + 6] = bf16_lo(p.w), v[8 * q + 7] = bf16_hi(p.w);
+                p[q] = *reinterpret_cast<const uint4*>(tile + r * kMx4Pitch + 64 * blk + 16 * q);
+                m = absmax3(m, bf16_lo(p[q].x), bf16_hi(p[q].x));
+                m = absmax3(m, bf16_lo(p[q].y), bf16_hi(p[q].y));
+                m = absmax3(m, bf16_lo(p[q].z), bf16_hi(p[q].z));
+                m = absmax3(m, bf16_lo(p[q].w), bf16_hi(p[q].w));
             }
             float f;
-            const uint32_t e8 = mx4_scale(absmax16(v + 16, absmax16(v, 0.0f)), f);
-            const int64_t row = r0 + r, cg = c0 + cb;
-            *reinterpret_cast<uint4*>(a.q_row + row * (a.cols / 2) + cg / 2) = mx4_codes(v, f);
+            const uint32_t e8 = mx4_scale(m, f);
+            const int64_t row = r0 + r, cg = c0 + 32 * blk;
+            *reinterpret_cast<uint4*>(a.q_row + row * (a.cols / 2) + cg / 2) =
+                make_uint4(mx4_codes8(p[0].x, p[0].y, p[0].z, p[0].w, f),
+                           mx4_codes8(p[1].x, p[1].y, p[1].z, p[1].w, f),
+                           mx4_codes8(p[2].x, p[2].y, p[2].z, p[2].w, f),
+                           mx4_codes8(p[3].x, p[3].y, p[3].z, p[3].w, f));
             a.e8_row[row * (a.cols / 32) + cg / 32] = (uint8_t)e8;
         }
     }
 }
 
+__global__ void __launch_bounds__(kMx4Threads, 3) mxfp4_kernel(const Mx4Args a)
+{
+    __shared__ __align__(16) uint8_t tiles[2][kMx4TileRows * kMx4Pitch];
+    const int64_t n_tiles = a.tiles_r * a.tiles_c;
+    int64_t t = blockIdx.x;
+    if (t >= n_tiles) return;
+    mx4_issue_tile(a, t, tiles[0]);
+    for (int k = 0; t < n_tiles; ++k, t += gridDim.x) {
+        const int64_t nt = t + gridDim.x;
+        if (nt < n_tiles) {
+            mx4_issue_tile(a, nt, tiles[(k + 1) & 1]);
+            asm volatile("cp.async.wait_group 1;" ::: "memory");  // tile t has landed
+        } else {
+            asm volatile("cp.async.wait_group 0;" ::: "memory");
+        }
+        __syncthreads();
+        mx4_tile(a, t, tiles[k & 1]);
+        __syncthreads();  // buffer k & 1 is refilled two tiles later
+    }
+}
+
 bool aligned16_ptr(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+// Resident CTAs per device (the persistent grid); 0 when the device is not sm_100.
+int mx4_grid(int dev)
+{
+    static int grids[64];
+    static std::once_flag flags[64];
+    std::call_once(flags[dev & 63], [dev]() {
+        int major = 0, sms = 0, per_sm = 0;
+        if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess ||
+            major != 10 ||
+            cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess ||
+            cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, mxfp4_kernel, kMx4Threads, 0) !=
+                cudaSuccess)
+            return;
+        grids[dev & 63] = sms * (per_sm > 0 ? per_sm : 1);
+    });
+    return grids[dev & 63];
+}
 
 }  // namespace
 }  // namespace nvfp4
@@ -165,11 +225,10 @@ extern "C" nvfp4_status mxfp4_quantize(const void* x_bf16, int64_t rows, int64_t
     const int64_t tiles_r = (rows + kMx4TileRows - 1) / kMx4TileRows;
     const int64_t tiles_c = (cols + kMx4TileCols - 1) / kMx4TileCols;
     if (tiles_r * tiles_c > 0x7FFFFFFFll) return NVFP4_ERR_SHAPE;
-    int dev = 0, major = 0;
-    if (cudaGetDevice(&dev) != cudaSuccess ||
-        cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess)
-        return NVFP4_ERR_CUDA;
-    if (major != 10) return NVFP4_ERR_UNSUPPORTED;
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return NVFP4_ERR_CUDA;
+    const int grid = mx4_grid(dev);
+    if (grid <= 0) return NVFP4_ERR_UNSUPPORTED;
     Mx4Args a{};
     a.x = static_cast<const uint16_t*>(x_bf16);
     a.rows = rows;
@@ -179,7 +238,10 @@ extern "C" nvfp4_status mxfp4_quantize(const void* x_bf16, int64_t rows, int64_t
     a.e8_row = row ? e8_row : nullptr;
     a.q_col = col ? q_col : nullptr;
     a.e8_col = col ? e8_col : nullptr;
+    a.tiles_r = tiles_r;
     a.tiles_c = tiles_c;
-    mxfp4_kernel<<<(unsigned)(tiles_r * tiles_c), kMx4Threads, 0, static_cast<cudaStream_t>(stream)>>>(a);
+    const int64_t n_tiles = tiles_r * tiles_c;
+    mxfp4_kernel<<<(unsigned)(n_tiles < grid ? n_tiles : grid), kMx4Threads, 0,
+                   static_cast<cudaStream_t>(stream)>>>(a);
     return cudaGetLastError() == cudaSuccess ? NVFP4_OK : NVFP4_ERR_CUDA;
 }
