@@ -16,10 +16,12 @@
 // Persistent CTAs walk 64 x 128 tiles; each tile is copied into one of two
 // shared-memory buffers with 16-byte cp.async while the CTA quantises the
 // other.  Warps 0..3 quantise the tile's columns (thread = column pair x
-// 32-row block, one 32-bit shared load per row gives both columns), warps
-// 4..7 its rows (thread = one 32-block of a row; four lanes cover a row's 64
-// code bytes, so every store instruction writes whole sectors).  Values stay
-// packed as bf16 pairs and are unpacked where they are used.  The kernel is
+// 32-row block, one 32-bit shared load per row gives both columns) into a
+// staging block, from which lane pairs store each column's 32 code bytes as
+// one whole sector; warps 4..7 quantise its rows (thread = one 32-block of a
+// row; four lanes cover a row's 64 code bytes, so every store instruction
+// writes whole sectors).  Values stay packed as bf16 pairs and are unpacked
+// where they are used.  The kernel is
 // HBM-bound: 2 bytes read and 0.5 + 1/32 written per element and direction.
 #include "common.cuh"
 
@@ -87,7 +89,10 @@ __device__ __forceinline__ void mx4_issue_tile(const Mx4Args& a, int64_t t, uint
     asm volatile("cp.async.commit_group;" ::: "memory");
 }
 
-__device__ __forceinline__ void mx4_tile(const Mx4Args& a, int64_t t, const uint8_t* tile)
+constexpr int kMx4StgPitch = 48;  // bytes per staged column: 32 code bytes + 16 (banks)
+
+__device__ __forceinline__ void mx4_tile(const Mx4Args& a, int64_t t, const uint8_t* tile,
+                                         uint8_t* stg, uint8_t* stg_e8)
 {
     const int64_t tr = t / a.tiles_c, tcol = t - tr * a.tiles_c;
     const int64_t r0 = tr * kMx4TileRows, c0 = tcol * kMx4TileCols;
@@ -99,7 +104,7 @@ __device__ __forceinline__ void mx4_tile(const Mx4Args& a, int64_t t, const uint
         if (!a.q_col) return;
         // columnwise: column pair cp (columns 2cp, 2cp + 1), 32-row block rb
         const int cp = 32 * (warp & 1) + lane, rb = warp >> 1;
-        if (2 * cp >= nc || 32 * rb >= nr) return;
+        if (2 * cp < nc && 32 * rb < nr) {
         uint32_t w[32];
         float ma = 0.0f, mb = 0.0f;
 #pragma unroll
@@ -124,13 +129,31 @@ __device__ __forceinline__ void mx4_tile(const Mx4Args& a, int64_t t, const uint
                 mul2(y[i], y[i + 1], bf16_hi(w[8 * g + i]), bf16_hi(w[8 * g + i + 1]), fb, fb);
             cb[g] = e2m1x8_rne(y);
         }
-        const int64_t col = c0 + 2 * cp, rr = r0 + 32 * rb;
-        *reinterpret_cast<uint4*>(a.q_col + col * (a.rows / 2) + rr / 2) =
-            make_uint4(ca[0], ca[1], ca[2], ca[3]);
-        *reinterpret_cast<uint4*>(a.q_col + (col + 1) * (a.rows / 2) + rr / 2) =
-            make_uint4(cb[0], cb[1], cb[2], cb[3]);
-        a.e8_col[col * (a.rows / 32) + rr / 32] = (uint8_t)ea;
-        a.e8_col[(col + 1) * (a.rows / 32) + rr / 32] = (uint8_t)eb;
+        // stage: column 2cp + h, rows 32rb .. 32rb+31 -> 16 bytes at 16 rb
+        *reinterpret_cast<uint4*>(stg + (2 * cp) * kMx4StgPitch + 16 * rb) = make_uint4(ca[0], ca[1], ca[2], ca[3]);
+        *reinterpret_cast<uint4*>(stg + (2 * cp + 1) * kMx4StgPitch + 16 * rb) = make_uint4(cb[0], cb[1], cb[2], cb[3]);
+        stg_e8[(2 * cp) * 2 + rb] = (uint8_t)ea;
+        stg_e8[(2 * cp + 1) * 2 + rb] = (uint8_t)eb;
+        }
+        // the four column warps' staged codes -> whole 32-byte sectors: lanes
+        // 2k and 2k+1 store the two halves of one column's 64 rows
+        asm volatile("bar.sync 1, 128;" ::: "memory");
+#pragma unroll
+        for (int j = 0; j < 2; ++j) {
+            const int i = threadIdx.x + 128 * j;  // 16-byte chunk: column i/2, half i%2
+            const int c = i >> 1, h = i & 1;
+            if (c < nc && 32 * h < nr)
+                *reinterpret_cast<uint4*>(a.q_col + (c0 + c) * (a.rows / 2) + r0 / 2 + 16 * h) =
+                    *reinterpret_cast<const uint4*>(stg + c * kMx4StgPitch + 16 * h);
+        }
+        {
+            const int c = threadIdx.x;  // 0..127: column c's scale bytes
+            if (c < nc) {
+                uint8_t* e = a.e8_col + (c0 + c) * (a.rows / 32) + r0 / 32;
+                e[0] = stg_e8[2 * c];
+                if (nr > 32) e[1] = stg_e8[2 * c + 1];
+            }
+        }
     } else {
         if (!a.q_row) return;
         // rowwise: block blk (32 columns) of row r, for r = t/4 and t/4 + 32
@@ -167,6 +190,8 @@ __device__ __forceinline__ void mx4_tile(const Mx4Args& a, int64_t t, const uint
 __global__ void __launch_bounds__(kMx4Threads, 3) mxfp4_kernel(const Mx4Args a)
 {
     __shared__ __align__(16) uint8_t tiles[2][kMx4TileRows * kMx4Pitch];
+    __shared__ __align__(16) uint8_t stg[kMx4TileCols * kMx4StgPitch];
+    __shared__ uint8_t stg_e8[kMx4TileCols * 2];
     const int64_t n_tiles = a.tiles_r * a.tiles_c;
     int64_t t = blockIdx.x;
     if (t >= n_tiles) return;
@@ -180,7 +205,7 @@ __global__ void __launch_bounds__(kMx4Threads, 3) mxfp4_kernel(const Mx4Args a)
             asm volatile("cp.async.wait_group 0;" ::: "memory");
         }
         __syncthreads();
-        mx4_tile(a, t, tiles[k & 1]);
+        mx4_tile(a, t, tiles[k & 1], stg, stg_e8);
         __syncthreads();  // buffer k & 1 is refilled two tiles later
     }
 }
