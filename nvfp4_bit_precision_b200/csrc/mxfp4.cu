@@ -74,7 +74,7 @@ __device__ __forceinline__ uint32_t mx4_codes8(uint32_t w0, uint32_t w1, uint32_
 // tensor are zero-filled without reading and only feed blocks never stored.
 __device__ __forceinline__ void mx4_issue_tile(const Mx4Args& a, int64_t t, uint8_t* buf)
 {
-    const int64_t tr = t / a.tiles_c, tcol = t - tr * a.tiles_c;
+    const int64_t tr = (uint32_t)t / (uint32_t)a.tiles_c, tcol = t - tr * a.tiles_c;  // t < 2^31
     const int64_t r0 = tr * kMx4TileRows, c0 = tcol * kMx4TileCols;
 #pragma unroll
     for (int i = threadIdx.x; i < kMx4TileRows * 16; i += kMx4Threads) {
@@ -94,7 +94,7 @@ constexpr int kMx4StgPitch = 48;  // bytes per staged column: 32 code bytes + 16
 __device__ __forceinline__ void mx4_tile(const Mx4Args& a, int64_t t, const uint8_t* tile,
                                          uint8_t* stg, uint8_t* stg_e8)
 {
-    const int64_t tr = t / a.tiles_c, tcol = t - tr * a.tiles_c;
+    const int64_t tr = (uint32_t)t / (uint32_t)a.tiles_c, tcol = t - tr * a.tiles_c;  // t < 2^31
     const int64_t r0 = tr * kMx4TileRows, c0 = tcol * kMx4TileCols;
     // valid extent of the tile: multiples of 32 (rows and cols are)
     const int nr = a.rows - r0 < kMx4TileRows ? (int)(a.rows - r0) : kMx4TileRows;

@@ -113,6 +113,13 @@ __device__ __forceinline__ int64_t source_row(const QArgs& a, int64_t r)
     return s;
 }
 
+// Tile row of a tile index: the host caps the tile count at 2^31 - 1, so a
+// 32-bit division does (a 64-bit one costs several times the instructions).
+__device__ __forceinline__ int64_t tile_row(const QArgs& a, int64_t tile)
+{
+    return (int64_t)((uint32_t)tile / (uint32_t)a.tiles_c);
+}
+
 __device__ __forceinline__ float warp_max16(float v)
 {
 #pragma unroll
@@ -166,7 +173,7 @@ template <bool kTma>
 __device__ __forceinline__ void issue_tile(const QArgs& a, const CUtensorMap* map, int64_t tile,
                                            uint8_t* buf, uint64_t* bar, int lane)
 {
-    const int64_t tr = tile / a.tiles_c, tc = tile - tr * a.tiles_c;
+    const int64_t tr = tile_row(a, tile), tc = tile - tr * a.tiles_c;
     const int64_t r0 = tr * kTileRows, c0 = tc * kTileCols;
     if (kTma) {
         // one box per 64-column panel; rows and columns past the tensor read as 0
@@ -370,7 +377,7 @@ __global__ void __launch_bounds__(kQuantThreads, 2)
         }
         const uint8_t* T = tiles + stage * kTileBytes;
         const int64_t tile = tile_of(k);
-        const int64_t tr = tile / a.tiles_c, tc = tile - tr * a.tiles_c;
+        const int64_t tr = tile_row(a, tile), tc = tile - tr * a.tiles_c;
         const int64_t cg0 = tc * kTileCols + 2 * cp;
         const int64_t rbase = tr * kTileRows + 32 * rgrp;
 #pragma unroll
@@ -628,7 +635,7 @@ __global__ void __launch_bounds__(kQuantThreads, 2)
         }
         const uint8_t* T = tiles + stage * kTileBytes;
         const int64_t tile = tile_of(k);
-        const int64_t tr = tile / a.tiles_c, tc = tile - tr * a.tiles_c;
+        const int64_t tr = tile_row(a, tile), tc = tile - tr * a.tiles_c;
         const int64_t r0 = tr * kTileRows, c0 = tc * kTileCols;
 
         // ---------------- rowwise: thread = (row, 64-column half) ----------
@@ -1193,6 +1200,7 @@ static nvfp4_status launch_quant(QArgs& a, bool need_amax, void* workspace, cuda
     if (!info.ok) return NVFP4_ERR_UNSUPPORTED;
     a.tiles_c = (a.cols + kTileCols - 1) / kTileCols;
     a.n_tiles = ((a.rows + kTileRows - 1) / kTileRows) * a.tiles_c;
+    if (a.n_tiles > 0x7FFFFFFFll) return NVFP4_ERR_SHAPE;  // tile indices are 31-bit on the device
     if (workspace) {
         // amax words (when computed) and the status word start at zero on every call
         uint32_t* ws = static_cast<uint32_t*>(workspace);
