@@ -195,11 +195,13 @@ def test_grouped_gemm_amax_out(nv, orc):
 
 def test_requantize_with_gemm_amax(nv, orc):
     """Quantising the up projection's output with the GEMM's amax_out as amax_in gives the
-    same bytes as the quantiser's own amax pass (and the oracle's quantisation)."""
+    same bytes as the quantiser's own amax pass; and that amax_in path matches the oracle
+    on an output the oracle computed itself (its FP64 grouped GEMM, rounded to bf16)."""
     import torch
     N, K = 256, 512
     counts = [0, 150, 7, 0, 33, 130]
-    offsets, _, _, A, qb_d, sfb_d, gb_d, off_d = _grouped_case(orc, nv, counts, N, K, seed=9)
+    offsets, (qa, sa, ga), (qb, sb, gb), A, qb_d, sfb_d, gb_d, off_d = _grouped_case(
+        orc, nv, counts, N, K, seed=9)
     am = torch.zeros(2, dtype=torch.float32, device="cuda")
     H = nv.grouped_gemm(off_d, A, qb_d, sfb_d, gb_d, N, amax_out=am)
     kw = dict(group_offsets=off_d, num_groups=len(counts), sf_layout=nv.NVFP4_SF_MMA)
@@ -207,7 +209,14 @@ def test_requantize_with_gemm_amax(nv, orc):
     own = nv.quantize(H, **kw)["row"]
     for f in ("q", "sf", "g"):
         assert np.array_equal(host(getattr(fused, f)), host(getattr(own, f)))
-    q, sf, g = orc.nvfp4_quantize(host(H), 0)
-    assert np.array_equal(host(fused.q), q)
-    assert np.array_equal(sf_mma_to_rowmajor(host(fused.sf), int(offsets[-1]), N,
+    total = int(offsets[-1])
+    Dr, _ = orc.nvfp4_grouped_gemm_rows(offsets, qa, sa, ga, qb, sb, gb, np.arange(total))
+    h = W.f32_to_bf16_bits(Dr.astype(np.float32))
+    amax_h = float(np.max(np.abs(W.bf16_bits_to_f32(h))))
+    amd = torch.tensor([amax_h, amax_h], dtype=torch.float32, device="cuda")
+    got = nv.quantize(to_dev(h), amax=amd, **kw)["row"]
+    q, sf, g = orc.nvfp4_quantize(h, 0, amax=(amax_h, amax_h))
+    assert np.array_equal(host(got.q), q)
+    assert np.array_equal(sf_mma_to_rowmajor(host(got.sf), total, N,
                                              grouped_padded_rows(offsets)), sf)
+    assert float(host(got.g)[0]) == g
