@@ -17,7 +17,9 @@
 //               codes two per byte; completing on the leader CTA's barrier,
 //               which expects both CTAs' bytes) and its scale atoms (own 128
 //               A rows: one 1D bulk copy; all 256 B rows: one 4D box; both on
-//               its own barrier) into a 5-stage ring.
+//               its own barrier, issued before the stage's code tiles so the
+//               scale writers' work overlaps the tiles' flight) into a 5-stage
+//               ring.
 //   warps 2..5  scale writers, one per tensor-memory lane quadrant: each lane
 //               loads row i of the stage's 512-byte scale atoms from shared
 //               memory and writes them into its quadrant of this CTA's tensor
