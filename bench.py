@@ -283,6 +283,35 @@ def time_mxfp4(step, steps, warmup):
     return ms, nbytes
 
 
+def time_linear(step, steps, warmup):
+    """The NVFP4 linear autograd op, forward + backward, on the dense layer's resident
+    x [16384, 5120], W [20480, 5120] and dY [16384, 20480]: 9 launches of ours per pass
+    (x, W and dY each amax + fused quantisation; the forward, dgrad and wgrad GEMMs),
+    timed apart from the step with CUDA events.  Returns mean ms per pass."""
+    torch = step.torch
+    from nvfp4_bit_precision_b200.linear import nvfp4_linear
+    inp = step.inputs[0]
+    x = inp["x"].detach().requires_grad_(True)
+    w = inp["w"].detach().requires_grad_(True)
+    dy = inp["dy"]
+
+    def run(i):
+        x.grad = w.grad = None
+        nvfp4_linear(x, w, seed=20251030, offset=i).backward(dy)
+
+    for i in range(max(warmup, 3)):
+        run(i)
+    stream = torch.cuda.current_stream()
+    torch.cuda.synchronize()
+    s, e = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    s.record(stream)
+    for i in range(steps):
+        run(i)
+    e.record(stream)
+    torch.cuda.synchronize()
+    return s.elapsed_time(e) / steps
+
+
 def quant_algorithmic_bytes():
     """Bytes the dY quantisation must move: two reads of the bf16 input (amax pass and
     quantise pass), NVFP4 codes and scales in both directions, MXFP8 codes and scales."""
@@ -571,6 +600,7 @@ def main():
     ms_e2e = e0.elapsed_time(e1)
 
     mx4_ms, mx4_bytes = time_mxfp4(step, args.steps, args.warmup)
+    lin_ms = time_linear(step, args.steps, args.warmup)
     ms, ms_e2e = max_over_ranks([ms, ms_e2e], world, dev)
     value = job_tflops(step.flops(), world, args.steps, ms)
     value_e2e = job_tflops(step.flops(), world, args.steps, ms_e2e)
@@ -624,7 +654,13 @@ def main():
                 "achieved": round(mx4_bytes / (mx4_ms / 1e3) / 1e9, 1), "peak": pk["hbm_gbs"],
                 "unit": "GB/s",
                 "frac": round(mx4_bytes / (mx4_ms / 1e3) / 1e9 / pk["hbm_gbs"], 4),
-                "algorithmic_bytes": mx4_bytes, "peak_note": f"of {pk['source']}"}},
+                "algorithmic_bytes": mx4_bytes, "peak_note": f"of {pk['source']}"},
+                "nvfp4_linear": {
+                    "kernel": "NVFP4LinearFunction forward + backward on the dense layer "
+                    "(x 16384x5120, W 20480x5120, dY 16384x20480; 9 launches per pass; timed "
+                    "apart from the step)", "ms": round(lin_ms, 4),
+                    "value": round(3 * DENSE_FLOP_PER_GEMM / (lin_ms / 1e3) / 1e12, 1),
+                    "unit": "TFLOP/s"}},
             "e2e": {"value": round(value_e2e, 2), "unit": "TFLOP/s",
                     "h2d_bytes_per_step": step.h2d_bytes(), "d2h_bytes_per_step": d2h},
             "gpu_launches": Step.LAUNCHES_PER_STEP * args.steps,
