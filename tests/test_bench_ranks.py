@@ -67,3 +67,14 @@ def test_clock_summary_decodes_reasons():
     assert s["reasons"] == ["sw_power_cap"]
     c.samples.append((1200, 0x40))
     assert bench.ClockSampler.summary(c)["reasons"] == ["hw_thermal_slowdown", "sw_power_cap"]
+
+
+def test_hw_fp4_context_uses_the_sampled_clock():
+    """The FP4 tensor rate is 32768 FLOP per SM per cycle on 148 SMs at the sampled
+    clock; without a clock sample the context is left out."""
+    import bench
+    ctx = bench.hw_fp4_context(4765.0, {"sm_mhz": 1965.0})
+    assert abs(ctx["hw_fp4_peak_at_clock"] - 32768 * 148 * 1965e6 / 1e12) < 0.1
+    assert abs(ctx["frac_of_hw_fp4_peak"] - 4765.0 / ctx["hw_fp4_peak_at_clock"]) < 1e-4
+    assert bench.hw_fp4_context(4765.0, None) == {}
+    assert bench.hw_fp4_context(4765.0, {"sm_mhz": None}) == {}
