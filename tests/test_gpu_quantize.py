@@ -249,3 +249,29 @@ def test_gather_rows_bad_index_reports(nv):
     ws = torch.zeros(256, dtype=torch.uint8, device="cuda")
     nv.gather_rows(src, idx, workspace=ws)
     assert nv.nvfp4_workspace_status(ws) == 8
+
+
+@pytest.mark.parametrize("c0", [0, 64])
+def test_quantize_column_slice_of_wider_tensor(nv, orc, c0):
+    """ld > cols: the input is a 320-column slice (at column c0) of a 400-column tensor,
+    quantised with every output of the gradient recipe in tiled and row-major layouts."""
+    full = edge_tensor(192, 400, seed=31 + c0)
+    xs = to_dev(full)[:, c0:c0 + 320]
+    assert xs.stride(0) == 400
+    x = np.ascontiguousarray(full[:, c0:c0 + 320])
+    for layout in (nv.NVFP4_SF_ROWMAJOR, nv.NVFP4_SF_MMA):
+        out = nv.quantize(xs, rowwise=True, colwise=True, rounding=1, rht=True, seed=9,
+                          mx_outputs=nv.NVFP4_COLWISE, sf_layout=layout)
+        qr, sr, gr = orc.nvfp4_quantize(x, 0, 1, 0, 0, 9)
+        qc, sc, gc = orc.nvfp4_quantize(x, 1, 1, 0, 1, 9)
+        mq, me = orc.mxfp8_quantize(x, 1, 0, 9)
+        to_rm = (lambda sf, r, k: sf_mma_to_rowmajor(host(sf), r, k)) if layout else \
+            (lambda sf, r, k: host(sf))
+        np.testing.assert_array_equal(host(out["row"].q), qr)
+        np.testing.assert_array_equal(to_rm(out["row"].sf, 192, 320), sr)
+        np.testing.assert_array_equal(host(out["col"].q), qc)
+        np.testing.assert_array_equal(to_rm(out["col"].sf, 320, 192), sc)
+        assert float(host(out["row"].g)[0]) == gr and float(host(out["col"].g)[0]) == gc
+        np.testing.assert_array_equal(host(out["mx_col"][0]), mq)
+        np.testing.assert_array_equal(host(out["mx_col"][1]), me)
+        assert nv.nvfp4_workspace_status(out["workspace"]) == 0
