@@ -220,3 +220,33 @@ def test_requantize_with_gemm_amax(nv, orc):
     assert np.array_equal(sf_mma_to_rowmajor(host(got.sf), total, N,
                                              grouped_padded_rows(offsets)), sf)
     assert float(host(got.g)[0]) == g
+
+def test_grouped_gemm_max_groups(nv, orc):
+    """256 groups (the limit), many of them empty, ragged counts; every row checked."""
+    rng = np.random.default_rng(256)
+    counts = [int(c) if rng.random() > 0.3 else 0 for c in rng.integers(1, 40, 256)]
+    counts[-1] += (16 - sum(counts) % 16) % 16  # the oracle quantises whole 16-row tiles
+    N, K = 256, 256
+    offsets, (qa, sa, ga), (qb, sb, gb), A, qb_d, sfb_d, gb_d, off_d = _grouped_case(
+        orc, nv, counts, N, K, seed=256)
+    D = W.bf16_bits_to_f32(host(nv.grouped_gemm(off_d, A, qb_d, sfb_d, gb_d, N)))
+    Dr, Ar = orc.nvfp4_grouped_gemm_rows(offsets, qa, sa, ga, qb, sb, gb,
+                                         np.arange(int(offsets[-1])))
+    check_gemm(D, Dr, Ar, True)
+
+
+def test_all_zero_operands(nv, orc):
+    """amax 0: S = g = 1, every code and scale byte is the oracle's (zeros), and the
+    GEMM of zero operands is exactly zero (with amax_out 0)."""
+    import torch
+    x = np.zeros((256, 512), dtype=np.uint16)
+    out = nv.quantize(to_dev(x), rowwise=True, colwise=True, rounding=nv.NVFP4_SR, rht=True,
+                      seed=3, sf_layout=nv.NVFP4_SF_MMA)
+    for d, t in ((0, out["row"]), (1, out["col"])):
+        q, sf, g = orc.nvfp4_quantize(x, d, 1, 0, d, 3)
+        assert g == 1.0 and float(host(t.g)[0]) == g
+        np.testing.assert_array_equal(host(t.q), q)
+        np.testing.assert_array_equal(sf_mma_to_rowmajor(host(t.sf), t.rows, t.k), sf)
+    am = torch.full((1,), 7.0, dtype=torch.float32, device="cuda")
+    D = host(nv.gemm(out["row"], out["row"], nv.NVFP4_OUT_F32, amax_out=am))
+    assert not np.any(D) and host(am)[0] == 0.0
