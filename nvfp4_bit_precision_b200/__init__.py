@@ -45,7 +45,8 @@ EXPORTED = [
     "nvfp4_quantize", "nvfp4_dequantize", "mxfp8_quantize", "nvfp4_gemm", "nvfp4_grouped_gemm",
     "nvfp4_quantize_workspace_size", "nvfp4_gemm_workspace_size", "nvfp4_sf_mma_bytes",
     "nvfp4_sf_mma_grouped_bytes", "nvfp4_workspace_status", "nvfp4_status_string",
-    "nvfp4_version", "nvfp4_quantize_noalloc", "nvfp4_gather_rows", "mxfp4_quantize",
+    "nvfp4_version", "nvfp4_quantize_noalloc", "nvfp4_quantize_noalloc_status",
+    "nvfp4_gather_rows", "mxfp4_quantize",
 ]
 
 
@@ -88,12 +89,14 @@ _lib.nvfp4_sf_mma_bytes.restype = _SZ
 _lib.nvfp4_sf_mma_grouped_bytes.argtypes = [_I64, ctypes.c_int, _I64]
 _lib.nvfp4_sf_mma_grouped_bytes.restype = _SZ
 _lib.nvfp4_workspace_status.argtypes = [_P, _P]
+_lib.nvfp4_quantize_noalloc_status.argtypes = [_P]
 _lib.nvfp4_status_string.argtypes = [ctypes.c_int]
 _lib.nvfp4_status_string.restype = ctypes.c_char_p
 _lib.nvfp4_version.restype = ctypes.c_int
 for _n in ("nvfp4_quantize", "nvfp4_quantize_noalloc", "mxfp8_quantize", "mxfp4_quantize",
            "nvfp4_dequantize", "nvfp4_gemm",
-           "nvfp4_grouped_gemm", "nvfp4_gather_rows", "nvfp4_workspace_status"):
+           "nvfp4_grouped_gemm", "nvfp4_gather_rows", "nvfp4_workspace_status",
+           "nvfp4_quantize_noalloc_status"):
     getattr(_lib, _n).restype = ctypes.c_int
 
 
@@ -191,6 +194,10 @@ def nvfp4_gather_rows(q_src, sf_src, src_rows, k, row_index, rows, group_offsets
 
 def nvfp4_workspace_status(workspace, stream=None) -> int:
     return int(_lib.nvfp4_workspace_status(_ptr(workspace), _stream(stream)))
+
+
+def nvfp4_quantize_noalloc_status(stream=None) -> int:
+    return int(_lib.nvfp4_quantize_noalloc_status(_stream(stream)))
 
 
 def nvfp4_sf_mma_bytes(rows: int, k: int) -> int:

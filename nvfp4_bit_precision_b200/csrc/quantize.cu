@@ -23,6 +23,7 @@
 // ("Details": -54 -> -6 with multiplier 9; "How it works": transposed blocks,
 // 16x16 squares, random re-rounding, MXFP8 backward).
 #include <algorithm>
+#include <atomic>
 #include <cstdio>
 #include <mutex>
 
@@ -1338,18 +1339,22 @@ extern "C" nvfp4_status nvfp4_quantize(const void* x_bf16, int64_t rows, int64_t
 constexpr size_t kNoAllocScratchBytes = 256;
 static __device__ __align__(256) uint8_t g_noalloc_scratch[kNoAllocScratchBytes];
 
-// Device address of the array on device `dev`, looked up once per device with
-// that device current (host code only sees a stand-in symbol, never the
-// device address).
+// Device address of the array on device `dev`, looked up with that device
+// current (host code only sees a stand-in symbol, never the device address).
+// Only a successful lookup is kept: a failed one (for example, attempted during
+// a stream capture) is tried again on the next call instead of failing every
+// later call on that device.
 static void* noalloc_scratch(int dev)
 {
-    static void* ptrs[64];
-    static cudaError_t errs[64];
-    static std::once_flag flags[64];
-    std::call_once(flags[dev], [dev]() {
-        errs[dev] = cudaGetSymbolAddress(&ptrs[dev], g_noalloc_scratch);
-    });
-    return errs[dev] == cudaSuccess ? ptrs[dev] : nullptr;
+    static std::atomic<void*> ptrs[64];
+    void* p = ptrs[dev].load(std::memory_order_acquire);
+    if (p) return p;
+    static std::mutex mu;
+    std::lock_guard<std::mutex> lock(mu);
+    p = ptrs[dev].load(std::memory_order_relaxed);
+    if (!p && cudaGetSymbolAddress(&p, g_noalloc_scratch) == cudaSuccess && p)
+        ptrs[dev].store(p, std::memory_order_release);
+    return ptrs[dev].load(std::memory_order_relaxed);
 }
 
 extern "C" nvfp4_status nvfp4_quantize_noalloc(const void* x_bf16, int64_t rows, int64_t cols,
@@ -1367,6 +1372,16 @@ extern "C" nvfp4_status nvfp4_quantize_noalloc(const void* x_bf16, int64_t rows,
     if (!scratch) return NVFP4_ERR_CUDA;
     return nvfp4_quantize(x_bf16, rows, cols, ld, p, q_row, sf_row, g_row, q_col, sf_col, g_col,
                           scratch, kNoAllocScratchBytes, stream);
+}
+
+extern "C" nvfp4_status nvfp4_quantize_noalloc_status(void* stream)
+{
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return NVFP4_ERR_CUDA;
+    if (dev < 0 || dev >= 64) return NVFP4_ERR_UNSUPPORTED;
+    void* scratch = noalloc_scratch(dev);
+    if (!scratch) return NVFP4_ERR_CUDA;
+    return nvfp4_workspace_status(scratch, stream);
 }
 
 extern "C" nvfp4_status mxfp8_quantize(const void* x_bf16, int64_t rows, int64_t cols, int64_t ld,

@@ -329,6 +329,83 @@ def test_sr_bits_nvfp4_mapping(orc):
         assert np.all(np.abs(bits.mean(axis=0) - 0.5) < 0.03)
 
 
+# Largest |P(up_2k and up_2k+1) - P(up_2k) P(up_2k+1)| over every pair of thresholds,
+# found by exact enumeration (attained at t = 21845 = 65535/3 for both elements).
+SR_PAIR_MAX_COV = 5.444 / 65536
+
+
+def test_sr_bits_nvfp4_joint_law(orc):
+    """Exact joint law of the two draws that share a byte pair.  Over all 2^16 values
+    of (B0, B2) -- the two bytes elements 0 and 1 of a 4-group read -- each element's u
+    takes every 16-bit value exactly once (uniform marginals, so every element rounds up
+    with probability exactly floor(f 2^16)/2^16), and the two rounding decisions are
+    nearly but not exactly independent: the covariance of 'u0 < t0' and 'u1 < t1' never
+    exceeds SR_PAIR_MAX_COV (correlation <= 3.8e-4 at P(up) = 1/3).  Elements 0 and 2
+    (disjoint bytes) are exactly independent.  The oracle's stream obeys this law."""
+    rev = np.array([int(f"{b:08b}"[::-1], 2) for b in range(256)])
+    B0, B2 = np.meshgrid(np.arange(256), np.arange(256), indexing="ij")
+    u0 = (65535 - ((B2 << 8) | B0)).ravel()
+    u1 = (65535 - ((rev[B0] << 8) | rev[B2])).ravel()
+    np.testing.assert_array_equal(np.sort(u0), np.arange(65536))
+    np.testing.assert_array_equal(np.sort(u1), np.arange(65536))
+    # the oracle's draws for elements 4g and 4g+1 (and 4g+2, 4g+3) are pairs of this law
+    pair_of = np.empty(65536, dtype=np.int64)
+    pair_of[u0] = u1
+    for idx0 in range(0, 4 * 3000, 4):
+        d = [orc.sr_bits_nvfp4(99, 5, 0, idx0 + k) for k in range(4)]
+        assert pair_of[d[0]] == d[1] and pair_of[d[2]] == d[3]
+
+    def cov(t0, t1):
+        return np.mean((u0 < t0) & (u1 < t1)) - (t0 / 65536) * (t1 / 65536)
+
+    worst = cov(21845, 21845)
+    assert abs(worst - SR_PAIR_MAX_COV) < 1e-3 / 65536
+    rng = np.random.default_rng(21)
+    ts = np.concatenate([rng.integers(0, 65537, (3000, 2)),
+                         [[t, t] for t in (1, 255, 256, 4096, 16384, 32768, 49152, 65535)]])
+    for t0, t1 in ts:
+        assert abs(cov(t0, t1)) <= SR_PAIR_MAX_COV + 1e-12
+
+
+def test_e4m3_sr_sat_enumerated(orc):
+    """Stochastic rounding onto the E4M3 grid (MXFP8 with stochastic rounding), over
+    all 2^16 draws u for a value inside every kind of E4M3 interval: the subnormal
+    steps of 2^-9, the interval starting at the smallest normal 2^-6, ordinary binades
+    and the top interval below 448.  Grid neighbours come from the bit-field
+    enumeration in brute.py: only the two neighbours occur, exactly the draws
+    u < floor(f 2^16) round up (f = exact rational position between them), the rule
+    is sign-symmetric, grid values never move and everything >= 448 saturates."""
+    grid = brute.e4m3_grid()[:0x7F]            # magnitudes of codes 0x00 .. 0x7E
+    us = np.arange(65536)
+    sub = 2.0 ** -9
+    ys = [0.3 * sub, sub + 0.3 * sub, 3 * sub + 0.71 * sub, 7 * sub + 0.5 * sub + sub / 1024,
+          2.0 ** -6 + 0.3 * sub, 2.0 ** -6 * 1.875 + 0.41 * 2.0 ** -9,
+          1.03, 2.25 + 0.0421, 9.7, 250.3, 270.0, 440.0, 447.9]
+    for y in ys:
+        c = int(np.searchsorted(grid, y, side="right") - 1)
+        lo, hi = Fraction(float(grid[c])), Fraction(float(grid[c + 1]))
+        t = int((Fraction(y) - lo) / (hi - lo) * 65536)      # floor: the value is positive
+        assert 0 < t < 65536
+        codes = np.array([orc.e4m3_sr_sat(y, int(u)) for u in us])
+        expect = np.where(us < t, c + 1, c)
+        np.testing.assert_array_equal(codes, expect)
+        neg = np.array([orc.e4m3_sr_sat(-y, int(u)) for u in us[::97]])
+        np.testing.assert_array_equal(neg, expect[::97] | 0x80)
+    for c in range(0x7F):                       # grid values stay put for every u
+        for u in (0, 1, 0x7FFF, 0xFFFF):
+            assert orc.e4m3_sr_sat(float(grid[c]), u) == c
+            assert orc.e4m3_sr_sat(-float(grid[c]), u) == 0x80 | c
+    for y in (448.0, 448.5, 464.0, 1e6):        # satfinite: 448 = code 0x7E
+        for u in (0, 0x8000, 0xFFFF):
+            assert orc.e4m3_sr_sat(y, u) == 0x7E
+            assert orc.e4m3_sr_sat(-y, u) == 0xFE
+    # the mean over all draws is the value itself, up to the 2^-16 resolution
+    for y in ys:
+        c = int(np.searchsorted(grid, y, side="right") - 1)
+        vals = grid[[orc.e4m3_sr_sat(y, int(u)) for u in us[::1]]]
+        assert abs(vals.mean() - y) <= (grid[c + 1] - grid[c]) / 65536
+
+
 # ------------------------------------------------------------------ global scale
 def test_global_scale(orc):
     assert orc.global_scale(0.0) == (1.0, 1.0)

@@ -45,3 +45,4 @@ def test_noalloc_matches_workspace_entry_point_twice():
         for a, b in zip(got, ref):
             np.testing.assert_array_equal(host(a), host(b))
         assert nv.nvfp4_workspace_status(ws) == 0
+        assert nv.nvfp4_quantize_noalloc_status() == 0  # the shared array's status word
