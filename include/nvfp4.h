@@ -134,10 +134,20 @@ typedef struct {
     uint8_t* mx_sf_row;
     uint8_t* mx_q_col;
     uint8_t* mx_sf_col;
+    /* Layout of the MXFP8 scale bytes: NVFP4_SF_ROWMAJOR ([rows, K/32]) or
+     * NVFP4_SF_MMA, the 128x4 atoms of the NVFP4 tiled layout with 32-element
+     * blocks (byte of block b of row r at ((r/128)*(K/128) + b/4)*512 +
+     * (r%32)*16 + ((r%128)/32)*4 + b%4; bytes = mxfp8_sf_mma_bytes), which
+     * mxfp8_gemm reads.  NVFP4_SF_MMA needs the block axis a multiple of 128. */
+    int mx_sf_layout;
 } nvfp4_quant_params;
 
 /* Bytes of scale storage in NVFP4_SF_MMA layout for a [rows, k] operand. */
 size_t nvfp4_sf_mma_bytes(int64_t rows, int64_t k);
+
+/* Bytes of MXFP8 scale storage in NVFP4_SF_MMA layout for a [rows, k] operand
+ * (one E8M0 byte per 32 elements; ceil(rows/128)*128 rows). */
+size_t mxfp8_sf_mma_bytes(int64_t rows, int64_t k);
 
 /* Bytes of scale storage in NVFP4_SF_MMA layout for the grouped (MoE) layout:
  * sum over groups of ceil(rows_e/128)*128 rows; bounded by
@@ -305,6 +315,25 @@ nvfp4_status nvfp4_gemm(const uint8_t* qa, const uint8_t* sfa, const float* ga,
                         float* amax_out, void* workspace, size_t ws_bytes, void* stream);
 
 /*
+ * mxfp8_gemm -- block-scaled MXFP8 GEMM on the tcgen05 tensor cores, for the
+ * backward pass of the recipe on the iitak page ("How it works": the backward
+ * pass runs in 8-bit MXFP8; "But": 8 bits per element plus one 8-bit scale per
+ * 32, 8.25 bits per number):
+ *   D[i][j] = sum_k (e4m3(a_ik) * 2^(ea(i, k/32) - 127)) * (e4m3(b_jk) * 2^(eb(j, k/32) - 127))
+ * with FP32 accumulation, no tensor scale.  "TN": qa [M, K] and qb [N, K] E4M3
+ * codes (one byte each, K-contiguous); sfa / sfb E8M0 bytes in the
+ * NVFP4_SF_MMA layout with 32-element blocks (mx_sf_layout of
+ * nvfp4_quant_params).  D [M, ldd] FP32 or bf16 (RNE); amax_out as for
+ * nvfp4_gemm.  Shapes: K a multiple of 128 (one pipeline stage), M and N
+ * multiples of 16; ldd >= N with ldd * element size a multiple of 16 bytes;
+ * every pointer 16-byte aligned (amax_out 4).  Errors as for nvfp4_gemm.
+ */
+nvfp4_status mxfp8_gemm(const uint8_t* qa, const uint8_t* sfa, const uint8_t* qb,
+                        const uint8_t* sfb, int64_t M, int64_t N, int64_t K, int out_dtype,
+                        void* D, int64_t ldd, float* amax_out, void* workspace, size_t ws_bytes,
+                        void* stream);
+
+/*
  * nvfp4_grouped_gemm -- MoE grouped form (iitak, "Details": NVFP4 in the
  * expert layers): rows [off[e], off[e+1]) of the stacked A [total_rows, K]
  * are multiplied by expert e's B_e [N, K]:
@@ -329,7 +358,8 @@ nvfp4_status nvfp4_workspace_status(void* workspace, void* stream);
 /* Text of a status code (static storage). */
 const char* nvfp4_status_string(nvfp4_status s);
 
-/* Library version: major * 10000 + minor * 100 + patch. */
+/* Library version: major * 10000 + minor * 100 + patch (200: adds mx_sf_layout
+ * to nvfp4_quant_params, mxfp8_gemm and mxfp8_sf_mma_bytes). */
 int nvfp4_version(void);
 
 #ifdef __cplusplus

@@ -46,7 +46,7 @@ EXPORTED = [
     "nvfp4_quantize_workspace_size", "nvfp4_gemm_workspace_size", "nvfp4_sf_mma_bytes",
     "nvfp4_sf_mma_grouped_bytes", "nvfp4_workspace_status", "nvfp4_status_string",
     "nvfp4_version", "nvfp4_quantize_noalloc", "nvfp4_quantize_noalloc_status",
-    "nvfp4_gather_rows", "mxfp4_quantize",
+    "nvfp4_gather_rows", "mxfp4_quantize", "mxfp8_gemm", "mxfp8_sf_mma_bytes",
 ]
 
 
@@ -62,6 +62,7 @@ class QuantParams(ctypes.Structure):
         ("mx_outputs", ctypes.c_int), ("mx_rounding", ctypes.c_int),
         ("mx_q_row", ctypes.c_void_p), ("mx_sf_row", ctypes.c_void_p),
         ("mx_q_col", ctypes.c_void_p), ("mx_sf_col", ctypes.c_void_p),
+        ("mx_sf_layout", ctypes.c_int),
     ]
 
 
@@ -76,6 +77,10 @@ _lib.mxfp4_quantize.argtypes = [_P, _I64, _I64, _I64, ctypes.c_int, _P, _P, _P, 
 _lib.nvfp4_dequantize.argtypes = [_P, _P, _P, _I64, _I64, ctypes.c_int, ctypes.c_int, _P, _P]
 _lib.nvfp4_gemm.argtypes = [_P, _P, _P, _P, _P, _P, _I64, _I64, _I64, ctypes.c_int, _P, _I64, _P,
                             _P, _SZ, _P]
+_lib.mxfp8_gemm.argtypes = [_P, _P, _P, _P, _I64, _I64, _I64, ctypes.c_int, _P, _I64, _P, _P, _SZ,
+                            _P]
+_lib.mxfp8_sf_mma_bytes.argtypes = [_I64, _I64]
+_lib.mxfp8_sf_mma_bytes.restype = _SZ
 _lib.nvfp4_grouped_gemm.argtypes = [ctypes.c_int, _P, _I64, _P, _P, _P, _P, _P, _P, _I64, _I64,
                                     ctypes.c_int, _P, _P, _P, _SZ, _P]
 _lib.nvfp4_gather_rows.argtypes = [_P, _P, _I64, _I64, _P, _I64, _P, ctypes.c_int, _P, _P, _P,
@@ -94,7 +99,7 @@ _lib.nvfp4_status_string.argtypes = [ctypes.c_int]
 _lib.nvfp4_status_string.restype = ctypes.c_char_p
 _lib.nvfp4_version.restype = ctypes.c_int
 for _n in ("nvfp4_quantize", "nvfp4_quantize_noalloc", "mxfp8_quantize", "mxfp4_quantize",
-           "nvfp4_dequantize", "nvfp4_gemm",
+           "nvfp4_dequantize", "nvfp4_gemm", "mxfp8_gemm",
            "nvfp4_grouped_gemm", "nvfp4_gather_rows", "nvfp4_workspace_status",
            "nvfp4_quantize_noalloc_status"):
     getattr(_lib, _n).restype = ctypes.c_int
@@ -175,6 +180,13 @@ def nvfp4_gemm(qa, sfa, ga, qb, sfb, gb, M, N, K, out_dtype, D, ldd, amax_out, w
            "nvfp4_gemm")
 
 
+def mxfp8_gemm(qa, sfa, qb, sfb, M, N, K, out_dtype, D, ldd, amax_out, workspace, ws_bytes,
+               stream=None) -> None:
+    _check(_lib.mxfp8_gemm(_ptr(qa), _ptr(sfa), _ptr(qb), _ptr(sfb), M, N, K, out_dtype, _ptr(D),
+                           ldd, _ptr(amax_out), _ptr(workspace), ws_bytes, _stream(stream)),
+           "mxfp8_gemm")
+
+
 def nvfp4_grouped_gemm(G, group_offsets, total_rows, qa, sfa, ga, qb, sfb, gb, N, K, out_dtype, D,
                        amax_out, workspace, ws_bytes, stream=None) -> None:
     _check(_lib.nvfp4_grouped_gemm(G, _ptr(group_offsets), total_rows, _ptr(qa), _ptr(sfa),
@@ -202,6 +214,10 @@ def nvfp4_quantize_noalloc_status(stream=None) -> int:
 
 def nvfp4_sf_mma_bytes(rows: int, k: int) -> int:
     return int(_lib.nvfp4_sf_mma_bytes(rows, k))
+
+
+def mxfp8_sf_mma_bytes(rows: int, k: int) -> int:
+    return int(_lib.mxfp8_sf_mma_bytes(rows, k))
 
 
 def nvfp4_sf_mma_grouped_bytes(total_rows: int, num_groups: int, k: int) -> int:
@@ -240,9 +256,9 @@ def _workspace(device, nbytes: int = 256):
 def quantize(x, *, rowwise: bool = True, colwise: bool = False, rounding: int = NVFP4_RNE,
              scaling: int = NVFP4_1D16, rht: bool = False, sf_layout: int = NVFP4_SF_ROWMAJOR,
              seed: int = 0, offset: int = 0, amax=None, mx_outputs: int = 0,
-             mx_rounding: int = NVFP4_RNE, row_index=None, src_rows: int = 0,
-             group_offsets=None, num_groups: int = 0, rows: Optional[int] = None,
-             workspace=None, stream=None):
+             mx_rounding: int = NVFP4_RNE, mx_sf_layout: int = NVFP4_SF_ROWMAJOR,
+             row_index=None, src_rows: int = 0, group_offsets=None, num_groups: int = 0,
+             rows: Optional[int] = None, workspace=None, stream=None):
     """Quantise a bf16 [rows, cols] CUDA tensor.  Returns dict with 'row', 'col'
     (NVFP4Tensor or None), 'mx_row', 'mx_col' ((codes, e8m0) or None)."""
     import torch
@@ -284,13 +300,19 @@ def quantize(x, *, rowwise: bool = True, colwise: bool = False, rounding: int = 
     p.src_rows = src_rows if row_index is not None else 0
     p.group_offsets = _ptr(group_offsets)
     p.num_groups = num_groups
-    p.mx_outputs, p.mx_rounding = mx_outputs, mx_rounding
+    p.mx_outputs, p.mx_rounding, p.mx_sf_layout = mx_outputs, mx_rounding, mx_sf_layout
+
+    def mx_sf_alloc(r, k):
+        if mx_sf_layout == NVFP4_SF_MMA:
+            return torch.zeros(mxfp8_sf_mma_bytes(r, k), **u8)
+        return torch.empty((r, k // 32), **u8)
+
     if mx_outputs & NVFP4_ROWWISE:
-        mq, me = torch.empty((n_rows, cols), **u8), torch.empty((n_rows, cols // 32), **u8)
+        mq, me = torch.empty((n_rows, cols), **u8), mx_sf_alloc(n_rows, cols)
         p.mx_q_row, p.mx_sf_row = mq.data_ptr(), me.data_ptr()
         out["mx_row"] = (mq, me)
     if mx_outputs & NVFP4_COLWISE:
-        mq, me = torch.empty((cols, n_rows), **u8), torch.empty((cols, n_rows // 32), **u8)
+        mq, me = torch.empty((cols, n_rows), **u8), mx_sf_alloc(cols, n_rows)
         p.mx_q_col, p.mx_sf_col = mq.data_ptr(), me.data_ptr()
         out["mx_col"] = (mq, me)
     ws = workspace if workspace is not None else _workspace(dev)
@@ -353,6 +375,21 @@ def gemm(a: NVFP4Tensor, b: NVFP4Tensor, out_dtype: int = NVFP4_OUT_BF16, out=No
     nvfp4_gemm(a.q, a.sf, a.g, b.q, b.sf, b.g, M, N, K, out_dtype, out, out.stride(0), amax_out,
                ws, ws.numel(), stream)
     return out
+
+
+def mx_gemm(qa, sfa, qb, sfb, out_dtype: int = NVFP4_OUT_BF16, out=None, amax_out=None,
+            workspace=None, stream=None):
+    """D = A_hat B_hat^T of MXFP8 operands: qa [M, K], qb [N, K] E4M3 codes with E8M0
+    scales in the tiled layout (quantize(..., mx_sf_layout=NVFP4_SF_MMA))."""
+    import torch
+    M, K = qa.shape
+    N = qb.shape[0]
+    dt = torch.bfloat16 if out_dtype == NVFP4_OUT_BF16 else torch.float32
+    D = out if out is not None else torch.empty((M, N), dtype=dt, device=qa.device)
+    ws = workspace if workspace is not None else _workspace(qa.device)
+    mxfp8_gemm(qa, sfa, qb, sfb, M, N, K, out_dtype, D, D.stride(0), amax_out, ws, ws.numel(),
+               stream)
+    return D
 
 
 def grouped_gemm(group_offsets, a: NVFP4Tensor, qb, sfb, gb, N: int, out_dtype: int = NVFP4_OUT_BF16,

@@ -40,41 +40,95 @@
 #include <cudaTypedefs.h>
 
 #include <algorithm>
+#include <cstdlib>
+#include <cstring>
 #include <mutex>
 
 #include "common.cuh"
 
 namespace nvfp4 {
 
+// Operand formats.  NVFP4: E2M1 codes, one UE4M3 scale per 16 elements
+// (kind::mxf4nvf4, block16).  MXFP8: E4M3 codes, one UE8M0 scale per 32
+// elements (kind::mxf8f6f4, block32) -- the backward-pass format of the
+// recipe on the iitak page, "How it works".
+enum : int { kFmtNVFP4 = 0, kFmtMXFP8 = 1 };
+
 constexpr int BM = 128;                    // A rows per CTA; a CTA pair covers 2 * BM
 constexpr int kMmaM = 2 * BM;              // M of the two-SM MMA
-constexpr int BN = 256;                    // output columns per tile
-constexpr int BK = 256;                    // elements per stage (128 bytes per row)
-constexpr int kGemmStages = 5;
-constexpr int kA_Bytes = BM * BK / 2;          // 16 KB
-constexpr int kB_Bytes = (BN / 2) * BK / 2;    // 16 KB: this CTA's half of the B tile
-constexpr int kSFA_Bytes = BM * BK / 16;       // 2 KB: 4 atoms of 512 B (this CTA's rows)
-constexpr int kSFB_Bytes = BN * BK / 16;       // 4 KB: 2 row blocks x 4 atoms (all of B)
-constexpr int kStageBytes = kA_Bytes + kB_Bytes + kSFA_Bytes + kSFB_Bytes;
-constexpr uint32_t kPairCodeTx = 2u * (kA_Bytes + kB_Bytes);  // the leader's full barrier
+constexpr int kMaxStages = 8;
+constexpr int kMaxAccStages = 2;
 constexpr int kGemmThreads = 448;  // producer, MMA, 4 scale writers, 8 epilogue warps
-// Tensor memory: the 128x256 FP32 accumulator in columns 0..255, then one
-// 48-column scale region per pipeline stage (SFA 4 x 4 columns, SFB 4 x 8).
-// Within a region, column 4j + c of every lane quadrant holds, in lane i, the
-// four scales of row 32c + i for K-group j (SFA) -- row i of the K-group's
-// 512-byte atom; SFB keeps rows 0..127 at 16 + 8j + c, rows 128..255 at
-// 16 + 8j + 4 + c.
 constexpr int kTmemCols = 512;
-constexpr int kTmemSF = 256;
-constexpr int kTmemSFStage = 48;
-static_assert(kTmemSF + kGemmStages * kTmemSFStage <= kTmemCols, "tensor memory overflow");
 constexpr int kMaxGemmGroups = 256;
 constexpr int kEpiStageBytes = 2048;  // per epilogue warp: 32 rows x 64 bytes of BF16
+constexpr int kSmemLimit = 232448;    // 227 KB of dynamic shared memory per CTA
+
+struct GemmShared {
+    uint64_t full[kMaxStages];      // leader: A/B codes of both CTAs landed
+    uint64_t sf_full[kMaxStages];   // this CTA's scale atoms landed
+    uint64_t empty[kMaxStages];     // the stage's MMAs completed (both CTAs)
+    uint64_t sf_ready[kMaxStages];  // leader: both CTAs' scales are in tensor memory
+    uint64_t acc_full[kMaxAccStages];
+    uint64_t acc_empty[kMaxAccStages];
+    uint32_t tmem_base;
+    int32_t total_tiles;
+    int32_t cum_tiles[kMaxGemmGroups + 1];
+    int32_t group_start[kMaxGemmGroups + 1];
+    int32_t group_sfblk[kMaxGemmGroups + 1];  // first padded 128-row scale block of a group
+};
+
+constexpr int kSmemShared = (int)((sizeof(GemmShared) + 1023) / 1024 * 1024);
+
+// Tile and pipeline geometry of one (format, tile width) variant.  Every stage
+// holds 128 bytes of K per operand row -- one 128-byte swizzle row, 256 FP4 or
+// 128 FP8 elements -- and is consumed by 4 MMAs that each step 32 bytes along K
+// (K = 64 for FP4, K = 32 for FP8).
+//  - kBN = 256: one 256x256 FP32 accumulator (256 tensor-memory columns) per
+//    pair; the next tile's MMAs wait until the epilogue has read it.
+//  - kBN = 128: two 256x128 accumulators used in turn, so the MMAs of tile t+1
+//    run while the epilogue drains tile t.
+// Scale atoms (512 bytes: 128 rows x 4 scale bytes) per 128 rows and stage:
+// four for NVFP4 (16 scales per row), one for MXFP8 (4 scales per row).  In
+// tensor memory each atom takes 4 columns per 128 rows (column c, lane i: row
+// 32c + i's 4 bytes, in every lane quadrant).
+template <int kFmt, int kBN>
+struct GemmCfg {
+    static constexpr int BN = kBN;
+    static constexpr int kBRows = kBN / 2;  // B rows staged by each CTA
+    static constexpr int kBlocksN = kBN / 128;
+    static constexpr int kSfAtoms = kFmt == kFmtNVFP4 ? 4 : 1;
+    static constexpr int kKStage = kFmt == kFmtNVFP4 ? 256 : 128;  // K elements per stage
+    static constexpr int kKAtom = kFmt == kFmtNVFP4 ? 64 : 128;    // K elements per scale atom
+    static constexpr int kA_Bytes = BM * 128;
+    static constexpr int kB_Bytes = kBRows * 128;
+    static constexpr int kSFA_Bytes = kSfAtoms * 512;
+    static constexpr int kSFB_Bytes = kSfAtoms * 512 * kBlocksN;
+    // stages start on 1024-byte boundaries (the 128-byte swizzle repeats every 1024)
+    static constexpr int kStageBytes = (kA_Bytes + kB_Bytes + kSFA_Bytes + kSFB_Bytes + 1023) / 1024 * 1024;
+    static constexpr uint32_t kPairCodeTx = 2u * (kA_Bytes + kB_Bytes);  // the leader's full barrier
+    static constexpr int kAccStages = kBN == 256 ? 1 : 2;
+    static constexpr int kTmemSF = kAccStages * kBN;  // scale regions follow the accumulators
+    static constexpr int kSfColsA = kSfAtoms * 4;
+    static constexpr int kSfCols = kSfColsA + kSfAtoms * 4 * kBlocksN;  // written per stage
+    static constexpr int kSfStride = (kSfCols + 15) / 16 * 16;            // columns per stage region
+    static constexpr int kStagesBySmem =
+        (kSmemLimit - kSmemShared - 8 * kEpiStageBytes - 1024) / kStageBytes;
+    static constexpr int kStagesByTmem = (kTmemCols - kTmemSF) / kSfStride;
+    static constexpr int kStages = kStagesBySmem < kStagesByTmem
+                                       ? (kStagesBySmem < kMaxStages ? kStagesBySmem : kMaxStages)
+                                       : (kStagesByTmem < kMaxStages ? kStagesByTmem : kMaxStages);
+    static constexpr size_t kSmemBytes =
+        (size_t)kStages * kStageBytes + kSmemShared + 8 * kEpiStageBytes + 1024;
+    static_assert(kStages >= 4, "pipeline too shallow");
+    static_assert(kTmemSF + kStages * kSfStride <= kTmemCols, "tensor memory overflow");
+    static_assert(kSmemBytes <= (size_t)kSmemLimit, "shared memory overflow");
+};
 
 struct GemmArgs {
     const uint8_t* sfa;
     const uint8_t* sfb;
-    const float* ga;
+    const float* ga;  // NVFP4 tensor scales (unused for MXFP8)
     const float* gb;
     void* D;
     int64_t M, N, K, ldd;
@@ -86,23 +140,9 @@ struct GemmArgs {
     int64_t total_rows;
     uint32_t* status;
     float* amax_out;  // optional: max |D| (as stored), atomically accumulated
+    uint64_t wait_ns;  // limit of every barrier wait (2 s; shorter under the test hook)
+    int no_copies;     // test hook: the producers issue no copy (see wait_test_hook)
 };
-
-struct GemmShared {
-    uint64_t full[kGemmStages];      // leader: A/B codes of both CTAs landed
-    uint64_t sf_full[kGemmStages];   // this CTA's scale atoms landed
-    uint64_t empty[kGemmStages];     // the stage's MMAs completed (both CTAs)
-    uint64_t sf_ready[kGemmStages];  // leader: both CTAs' scales are in tensor memory
-    uint64_t acc_full;
-    uint64_t acc_empty;
-    uint32_t tmem_base;
-    int32_t total_tiles;
-    int32_t cum_tiles[kMaxGemmGroups + 1];
-    int32_t group_start[kMaxGemmGroups + 1];
-    int32_t group_sfblk[kMaxGemmGroups + 1];  // first padded 128-row scale block of a group
-};
-
-constexpr int kSmemShared = (int)((sizeof(GemmShared) + 1023) / 1024 * 1024);
 
 // ---------------------------------------------------------------- PTX wrappers
 __device__ __forceinline__ uint32_t cluster_rank()
@@ -198,24 +238,42 @@ __device__ __forceinline__ uint64_t desc_sw128(const void* p)
     return start | (1ull << 16) | (64ull << 32) | (1ull << 46) | (2ull << 61);
 }
 
-// Instruction descriptor: kind::mxf4nvf4, A/B E2M1 (format 1), UE4M3 scales,
-// both K-major, M = 256 (the pair), N = 256, dense, K = 64 per instruction.
-__host__ __device__ constexpr uint32_t make_idesc()
+// Instruction descriptor of a block-scaled MMA, M = 256 (the pair), N = kBN,
+// both operands K-major, dense.  NVFP4: A/B format E2M1 (1), UE4M3 scales
+// (bit 23 clear).  MXFP8: A/B format E4M3 (0), UE8M0 scales (bit 23 set).
+// sf_id picks the byte of each 32-bit scale column an MXFP8 MMA reads (its
+// 32-element block within the atom's 128); NVFP4 reads all four bytes.
+template <int kFmt, int kBN>
+__host__ __device__ constexpr uint32_t make_idesc(uint32_t sf_id)
 {
-    return (1u << 7) | (1u << 10) | ((uint32_t)(BN >> 3) << 17) | ((uint32_t)(kMmaM >> 4) << 24);
+    const uint32_t fmt = kFmt == kFmtNVFP4 ? 1u : 0u;
+    const uint32_t e8m0 = kFmt == kFmtNVFP4 ? 0u : 1u;
+    return (sf_id << 4) | (fmt << 7) | (fmt << 10) | ((uint32_t)(kBN >> 3) << 17) | (e8m0 << 23) |
+           ((uint32_t)(kMmaM >> 4) << 24) | (sf_id << 29);
 }
 
+template <int kFmt>
 __device__ __forceinline__ void tc_mma(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc,
                                        uint32_t idesc, uint32_t sfa_tmem, uint32_t sfb_tmem,
                                        uint32_t accumulate)
 {
-    asm volatile(
-        "{\n\t.reg .pred p;\n\t"
-        "setp.ne.b32 p, %4, 0;\n\t"
-        "tcgen05.mma.cta_group::2.kind::mxf4nvf4.block_scale.block16 [%0], %1, %2, %3, [%5], [%6], p;\n\t"
-        "}" ::"r"(d_tmem),
-        "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate), "r"(sfa_tmem), "r"(sfb_tmem)
-        : "memory");
+    if constexpr (kFmt == kFmtNVFP4) {
+        asm volatile(
+            "{\n\t.reg .pred p;\n\t"
+            "setp.ne.b32 p, %4, 0;\n\t"
+            "tcgen05.mma.cta_group::2.kind::mxf4nvf4.block_scale.block16 [%0], %1, %2, %3, [%5], [%6], p;\n\t"
+            "}" ::"r"(d_tmem),
+            "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate), "r"(sfa_tmem), "r"(sfb_tmem)
+            : "memory");
+    } else {
+        asm volatile(
+            "{\n\t.reg .pred p;\n\t"
+            "setp.ne.b32 p, %4, 0;\n\t"
+            "tcgen05.mma.cta_group::2.kind::mxf8f6f4.block_scale.block32 [%0], %1, %2, %3, [%5], [%6], p;\n\t"
+            "}" ::"r"(d_tmem),
+            "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate), "r"(sfa_tmem), "r"(sfb_tmem)
+            : "memory");
+    }
 }
 
 #define TMEM_LD_32(taddr, r)                                                                       \
@@ -239,6 +297,28 @@ __device__ __forceinline__ uint4 lds128(const void* p)
 }
 #define TMEM_ST_16(taddr, v) asm volatile("tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16};" ::"r"(taddr), "r"((v)[0]), "r"((v)[1]), "r"((v)[2]), "r"((v)[3]), "r"((v)[4]), "r"((v)[5]), "r"((v)[6]), "r"((v)[7]), "r"((v)[8]), "r"((v)[9]), "r"((v)[10]), "r"((v)[11]), "r"((v)[12]), "r"((v)[13]), "r"((v)[14]), "r"((v)[15]) : "memory")
 #define TMEM_ST_32(taddr, v) asm volatile("tcgen05.st.sync.aligned.32x32b.x32.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31,%32};" ::"r"(taddr), "r"((v)[0]), "r"((v)[1]), "r"((v)[2]), "r"((v)[3]), "r"((v)[4]), "r"((v)[5]), "r"((v)[6]), "r"((v)[7]), "r"((v)[8]), "r"((v)[9]), "r"((v)[10]), "r"((v)[11]), "r"((v)[12]), "r"((v)[13]), "r"((v)[14]), "r"((v)[15]), "r"((v)[16]), "r"((v)[17]), "r"((v)[18]), "r"((v)[19]), "r"((v)[20]), "r"((v)[21]), "r"((v)[22]), "r"((v)[23]), "r"((v)[24]), "r"((v)[25]), "r"((v)[26]), "r"((v)[27]), "r"((v)[28]), "r"((v)[29]), "r"((v)[30]), "r"((v)[31]) : "memory")
+#define TMEM_ST_8(taddr, v) asm volatile("tcgen05.st.sync.aligned.32x32b.x8.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8};" ::"r"(taddr), "r"((v)[0]), "r"((v)[1]), "r"((v)[2]), "r"((v)[3]), "r"((v)[4]), "r"((v)[5]), "r"((v)[6]), "r"((v)[7]) : "memory")
+#define TMEM_ST_4(taddr, v) asm volatile("tcgen05.st.sync.aligned.32x32b.x4.b32 [%0], {%1,%2,%3,%4};" ::"r"(taddr), "r"((v)[0]), "r"((v)[1]), "r"((v)[2]), "r"((v)[3]) : "memory")
+
+// One lane's N consecutive 32-bit tensor-memory columns from v (warp-wide).
+template <int N>
+__device__ __forceinline__ void tmem_store_words(uint32_t taddr, const uint32_t* v)
+{
+    if constexpr (N == 48) {
+        TMEM_ST_16(taddr, v);
+        TMEM_ST_32(taddr + 16, (v + 16));
+    } else if constexpr (N == 32) {
+        TMEM_ST_32(taddr, v);
+    } else if constexpr (N == 12) {
+        TMEM_ST_8(taddr, v);
+        TMEM_ST_4(taddr + 8, (v + 8));
+    } else if constexpr (N == 8) {
+        TMEM_ST_8(taddr, v);
+    } else {
+        static_assert(N == 0, "unsupported scale-column count");
+    }
+}
+
 __device__ __forceinline__ void tmem_ld_wait() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory"); }
 
 // ---------------------------------------------------------------- scheduling
@@ -250,10 +330,11 @@ struct TileCoord {
     int64_t n0;
 };
 
+template <int kBN>
 __device__ __forceinline__ TileCoord tile_coord(const GemmArgs& a, const GemmShared* sh, int t)
 {
     TileCoord c;
-    const int64_t tiles_n = (a.N + BN - 1) / BN;
+    const int64_t tiles_n = (a.N + kBN - 1) / kBN;
     if (!a.grouped) {
         const int64_t tiles_m = (a.M + kMmaM - 1) / kMmaM;
         const int64_t band = 8 * tiles_n;  // 8 M tiles share a band: B tiles reused from L2
@@ -265,7 +346,7 @@ __device__ __forceinline__ TileCoord tile_coord(const GemmArgs& a, const GemmSha
         c.row0 = mt * kMmaM;
         c.row_end = a.M;
         c.sf_blk = 2 * mt;
-        c.n0 = nt * BN;
+        c.n0 = nt * kBN;
     } else {
         int lo = 0, hi = a.G - 1;  // e with cum[e] <= t < cum[e+1]
         while (lo < hi) {
@@ -281,38 +362,44 @@ __device__ __forceinline__ TileCoord tile_coord(const GemmArgs& a, const GemmSha
         c.row0 = sh->group_start[lo] + mt * kMmaM;
         c.row_end = sh->group_start[lo + 1];
         c.sf_blk = sh->group_sfblk[lo] + 2 * mt;
-        c.n0 = nt * BN;
+        c.n0 = nt * kBN;
     }
     return c;
 }
 
 // ---------------------------------------------------------------- kernel
+template <int kFmt, int kBN>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
     gemm_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_constant__ CUtensorMap map_b,
                 const __grid_constant__ CUtensorMap map_sfb, GemmArgs a)
 {
+    using C = GemmCfg<kFmt, kBN>;
+    constexpr int kS = C::kStages;
+    constexpr int kAcc = C::kAccStages;
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                                ~uintptr_t(1023));
-    GemmShared* sh = reinterpret_cast<GemmShared*>(smem + kGemmStages * kStageBytes);
+    GemmShared* sh = reinterpret_cast<GemmShared*>(smem + kS * C::kStageBytes);
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const uint32_t rank = cluster_rank();  // 0: leader (issues the MMAs), 1: peer
     const bool leader = rank == 0;
     const int pair = blockIdx.x >> 1, n_pairs = gridDim.x >> 1;
-    uint8_t* epi_stage = smem + kGemmStages * kStageBytes + kSmemShared;
+    uint8_t* epi_stage = smem + kS * C::kStageBytes + kSmemShared;
 
     if (threadIdx.x == 0) {
-        for (int s = 0; s < kGemmStages; ++s) {
+        for (int s = 0; s < kS; ++s) {
             mbar_init(&sh->full[s], 1);      // leader: its producer's expect_tx; peer: unused
             mbar_init(&sh->sf_full[s], 1);   // this CTA's producer
             mbar_init(&sh->empty[s], 1);     // the leader's MMA commit, multicast to both
             mbar_init(&sh->sf_ready[s], 8);  // leader: 4 scale writers of each CTA
         }
-        mbar_init(&sh->acc_full, 1);
-        mbar_init(&sh->acc_empty, 16);       // leader: 8 epilogue warps of each CTA
+        for (int b = 0; b < kAcc; ++b) {
+            mbar_init(&sh->acc_full[b], 1);
+            mbar_init(&sh->acc_empty[b], 16);  // leader: 8 epilogue warps of each CTA
+        }
         fence_barrier_init();
         // tile table (both CTAs compute the same one)
-        const int64_t tiles_n = (a.N + BN - 1) / BN;
+        const int64_t tiles_n = (a.N + kBN - 1) / kBN;
         if (!a.grouped) {
             sh->total_tiles = (int32_t)(((a.M + kMmaM - 1) / kMmaM) * tiles_n);
         } else {
@@ -339,8 +426,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
     tc_fence_after();
     const uint32_t tmem = sh->tmem_base;
     const int total = sh->total_tiles;
-    const int64_t kstages = a.K / BK;
-    const int64_t k64 = a.K / 64;  // scale atoms per 128-row block
+    const int64_t kstages = a.K / C::kKStage;
+    const int64_t k_atoms = a.K / C::kKAtom;  // scale atoms per 128-row block
     bool failed = false;
 
     if (warp == 0) {
@@ -348,84 +435,102 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
         if (lane == 0) {
             asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&map_a)) : "memory");
             asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&map_b)) : "memory");
-            asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&map_sfb)) : "memory");
+            if (kBN == 256)
+                asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&map_sfb)) : "memory");
+            const int64_t nblk = (a.N + 127) / 128;  // 128-row scale blocks per group of B
             uint32_t it = 0;
-            for (int t = pair; t < total && !failed; t += n_pairs) {
-                const TileCoord c = tile_coord(a, sh, t);
+            for (int t = pair; t < total && !failed && !a.no_copies; t += n_pairs) {
+                const TileCoord c = tile_coord<kBN>(a, sh, t);
                 // This CTA's A rows; a half past the group's (or matrix's) end
                 // reads rows it never stores, and the leader's scale block
                 // instead of one that may not exist.
                 const int64_t a_row = c.row0 + (int64_t)BM * rank;
                 const int64_t sfa_blk = c.sf_blk + ((rank == 1 && a_row < c.row_end) ? 1 : 0);
-                const int64_t b_row = (int64_t)c.group * a.N + c.n0 + (int64_t)(BN / 2) * rank;
+                const int64_t b_row = (int64_t)c.group * a.N + c.n0 + (int64_t)C::kBRows * rank;
                 const int64_t nb0 = c.n0 / 128;
                 for (int64_t ks = 0; ks < kstages; ++ks, ++it) {
-                    const int s = (int)(it % kGemmStages);
-                    const uint32_t ph = (it / kGemmStages) & 1u;
-                    if (!mbar_wait(&sh->empty[s], ph ^ 1u)) {
+                    const int s = (int)(it % kS);
+                    const uint32_t ph = (it / kS) & 1u;
+                    if (!mbar_wait(&sh->empty[s], ph ^ 1u, a.wait_ns)) {
                         record_status(a.status, NVFP4_ERR_TIMEOUT);
                         failed = true;
                         break;
                     }
-                    uint8_t* st = smem + s * kStageBytes;
+                    uint8_t* st = smem + s * C::kStageBytes;
                     // this CTA's scale atoms first (they land first, and the scale
-                    // writers' work overlaps the code tiles' flight): 4 consecutive
-                    // atoms (2 KB) per 128-row block
-                    uint8_t* sf = st + kA_Bytes + kB_Bytes;
-                    mbar_arrive_expect_tx(&sh->sf_full[s], kSFA_Bytes + kSFB_Bytes);
-                    bulk_copy_g2s(sf, a.sfa + (sfa_blk * k64 + ks * 4) * 512, kSFA_Bytes, &sh->sf_full[s]);
-                    // both 128-row blocks of B's scales in one box (a block past
-                    // the operand's end reads as zeros)
-                    tma_load_4d(sf + kSFA_Bytes, &map_sfb, 0, (int32_t)ks, (int32_t)nb0, c.group,
-                                &sh->sf_full[s]);
-                    if (leader) mbar_arrive_expect_tx(&sh->full[s], kPairCodeTx);
+                    // writers' work overlaps the code tiles' flight): kSfAtoms
+                    // consecutive atoms per 128-row block
+                    uint8_t* sf = st + C::kA_Bytes + C::kB_Bytes;
+                    mbar_arrive_expect_tx(&sh->sf_full[s], C::kSFA_Bytes + C::kSFB_Bytes);
+                    bulk_copy_g2s(sf, a.sfa + (sfa_blk * k_atoms + ks * C::kSfAtoms) * 512,
+                                  C::kSFA_Bytes, &sh->sf_full[s]);
+                    if constexpr (kBN == 256) {
+                        // both 128-row blocks of B's scales in one box (a block past
+                        // the operand's end reads as zeros)
+                        tma_load_4d(sf + C::kSFA_Bytes, &map_sfb, 0, (int32_t)ks, (int32_t)nb0,
+                                    c.group, &sh->sf_full[s]);
+                    } else {
+                        // the tile's one 128-row block (n0 is a multiple of 128 and
+                        // below N, so the block exists)
+                        bulk_copy_g2s(sf + C::kSFA_Bytes,
+                                      a.sfb + (((int64_t)c.group * nblk + nb0) * k_atoms +
+                                               ks * C::kSfAtoms) * 512,
+                                      C::kSFB_Bytes, &sh->sf_full[s]);
+                    }
+                    if (leader) mbar_arrive_expect_tx(&sh->full[s], C::kPairCodeTx);
                     const uint32_t fb = cluster_addr(&sh->full[s], 0);
-                    tma_load_2d_pair(st, &map_a, (int32_t)(ks * (BK / 2)), (int32_t)a_row, fb);
-                    tma_load_2d_pair(st + kA_Bytes, &map_b, (int32_t)(ks * (BK / 2)), (int32_t)b_row, fb);
+                    tma_load_2d_pair(st, &map_a, (int32_t)(ks * 128), (int32_t)a_row, fb);
+                    tma_load_2d_pair(st + C::kA_Bytes, &map_b, (int32_t)(ks * 128), (int32_t)b_row, fb);
                 }
             }
             // Drain: the last stages' copies have landed once their MMAs
             // completed (the CTA's shared memory must outlive them).
-            const uint32_t first = it > (uint32_t)kGemmStages ? it - kGemmStages : 0u;
+            const uint32_t first = it > (uint32_t)kS ? it - kS : 0u;
             for (uint32_t j = first; j < it; ++j)
-                (void)mbar_wait(&sh->empty[j % kGemmStages], (j / kGemmStages) & 1u);
+                (void)mbar_wait(&sh->empty[j % kS], (j / kS) & 1u, a.wait_ns);
         }
     } else if (warp == 1) {
         // ------------------------------------------------ MMA issuer (leader CTA)
         if (leader && lane == 0) {
-            const uint32_t idesc = make_idesc();
             uint32_t it = 0, tcount = 0;
             for (int t = pair; t < total && !failed; t += n_pairs, ++tcount) {
-                // wait until both epilogues drained the accumulator of the previous tile
-                if (!mbar_wait(&sh->acc_empty, (tcount & 1u) ^ 1u)) {
+                const uint32_t buf = tcount % kAcc, aph = (tcount / kAcc) & 1u;
+                // wait until both epilogues drained this accumulator's previous tile
+                if (!mbar_wait(&sh->acc_empty[buf], aph ^ 1u, a.wait_ns)) {
                     record_status(a.status, NVFP4_ERR_TIMEOUT);
                     failed = true;
                     break;
                 }
                 tc_fence_after();
+                const uint32_t d_tmem = tmem + buf * (uint32_t)kBN;
                 for (int64_t ks = 0; ks < kstages; ++ks, ++it) {
-                    const int s = (int)(it % kGemmStages);
-                    const uint32_t ph = (it / kGemmStages) & 1u;
-                    if (!mbar_wait(&sh->full[s], ph) || !mbar_wait(&sh->sf_ready[s], ph)) {
+                    const int s = (int)(it % kS);
+                    const uint32_t ph = (it / kS) & 1u;
+                    if (!mbar_wait(&sh->full[s], ph, a.wait_ns) || !mbar_wait(&sh->sf_ready[s], ph, a.wait_ns)) {
                         record_status(a.status, NVFP4_ERR_TIMEOUT);
                         failed = true;
                         break;
                     }
                     tc_fence_after();
-                    uint8_t* st = smem + s * kStageBytes;
-                    const uint32_t t_sfa = tmem + kTmemSF + (uint32_t)s * kTmemSFStage;
-                    const uint32_t t_sfb = t_sfa + 16;
-                    const uint64_t ad = desc_sw128(st), bd = desc_sw128(st + kA_Bytes);
+                    uint8_t* st = smem + s * C::kStageBytes;
+                    const uint32_t t_sfa = tmem + C::kTmemSF + (uint32_t)s * C::kSfStride;
+                    const uint32_t t_sfb = t_sfa + C::kSfColsA;
+                    const uint64_t ad = desc_sw128(st), bd = desc_sw128(st + C::kA_Bytes);
 #pragma unroll
                     for (int j = 0; j < 4; ++j) {
-                        // +32 bytes (64 four-bit elements) along K inside the swizzled row
-                        tc_mma(tmem, ad + 2 * j, bd + 2 * j, idesc, t_sfa + 4 * j, t_sfb + 8 * j,
-                               (ks > 0 || j > 0) ? 1u : 0u);
+                        // +32 bytes along K inside the swizzled row: 64 FP4 or 32 FP8
+                        // elements.  NVFP4: atom j's columns; MXFP8: byte j of the
+                        // stage's one atom.
+                        const uint32_t aj = kFmt == kFmtNVFP4 ? (uint32_t)j : 0u;
+                        tc_mma<kFmt>(d_tmem, ad + 2 * j, bd + 2 * j,
+                                     make_idesc<kFmt, kBN>(kFmt == kFmtNVFP4 ? 0u : (uint32_t)j),
+                                     t_sfa + 4 * aj, t_sfb + 4 * C::kBlocksN * aj,
+                                     (ks > 0 || j > 0) ? 1u : 0u);
                     }
                     tc_commit_pair(&sh->empty[s]);  // both CTAs' stage free once these MMAs completed
                 }
                 if (failed) break;
-                tc_commit_pair(&sh->acc_full);
+                tc_commit_pair(&sh->acc_full[buf]);
             }
         }
     } else if (warp < 6) {
@@ -439,31 +544,31 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
         uint32_t it = 0;
         for (int t = pair; t < total && !failed; t += n_pairs) {
             for (int64_t ks = 0; ks < kstages; ++ks, ++it) {
-                const int s = (int)(it % kGemmStages);
-                const uint32_t ph = (it / kGemmStages) & 1u;
+                const int s = (int)(it % kS);
+                const uint32_t ph = (it / kS) & 1u;
                 bool ok = true;
-                if (lane == 0) ok = mbar_wait(&sh->sf_full[s], ph);
+                if (lane == 0) ok = mbar_wait(&sh->sf_full[s], ph, a.wait_ns);
                 ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
                 if (!ok) {
                     if (lane == 0) record_status(a.status, NVFP4_ERR_TIMEOUT);
                     failed = true;
                     break;
                 }
-                const uint8_t* sfa_s = smem + s * kStageBytes + kA_Bytes + kB_Bytes;
-                const uint8_t* sfb_s = sfa_s + kSFA_Bytes;
-                uint32_t v[48];
+                const uint8_t* sfa_s = smem + s * C::kStageBytes + C::kA_Bytes + C::kB_Bytes;
+                const uint8_t* sfb_s = sfa_s + C::kSFA_Bytes;  // [block][atom][512]
+                uint32_t v[C::kSfCols];
 #pragma unroll
-                for (int j = 0; j < 4; ++j) {
+                for (int j = 0; j < C::kSfAtoms; ++j) {
                     const uint4 x = lds128(sfa_s + j * 512 + lane * 16);
                     v[4 * j] = x.x, v[4 * j + 1] = x.y, v[4 * j + 2] = x.z, v[4 * j + 3] = x.w;
-                    const uint4 lo = lds128(sfb_s + j * 512 + lane * 16);
-                    const uint4 hi = lds128(sfb_s + kSFB_Bytes / 2 + j * 512 + lane * 16);
-                    v[16 + 8 * j] = lo.x, v[17 + 8 * j] = lo.y, v[18 + 8 * j] = lo.z, v[19 + 8 * j] = lo.w;
-                    v[20 + 8 * j] = hi.x, v[21 + 8 * j] = hi.y, v[22 + 8 * j] = hi.z, v[23 + 8 * j] = hi.w;
+#pragma unroll
+                    for (int bb = 0; bb < C::kBlocksN; ++bb) {
+                        const uint4 y = lds128(sfb_s + (bb * C::kSfAtoms + j) * 512 + lane * 16);
+                        const int o = C::kSfColsA + 4 * (j * C::kBlocksN + bb);
+                        v[o] = y.x, v[o + 1] = y.y, v[o + 2] = y.z, v[o + 3] = y.w;
+                    }
                 }
-                const uint32_t taddr = tmem + lane_base + kTmemSF + (uint32_t)s * kTmemSFStage;
-                TMEM_ST_16(taddr, v);
-                TMEM_ST_32(taddr + 16, (v + 16));
+                tmem_store_words<C::kSfCols>(tmem + lane_base + C::kTmemSF + (uint32_t)s * C::kSfStride, v);
                 asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
                 tc_fence_before();
                 __syncwarp();
@@ -472,37 +577,42 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
         }
     } else {
         // ------------------------------------------------ epilogue (warps 6..13, both CTAs)
+        constexpr int kCols = kBN / 2;     // accumulator columns per warp
+        constexpr int kChunks = kCols / 32;
         const int quad = warp & 3;                   // TMEM lanes 32*quad .. 32*quad+31
-        const int col0 = ((warp - 6) >> 2) * (BN / 2);  // 0 or 128
-        const uint32_t acc_empty_leader = cluster_addr(&sh->acc_empty, 0);
+        const int col0 = ((warp - 6) >> 2) * kCols;
         uint8_t* stg = epi_stage + (warp - 6) * kEpiStageBytes;
         float out_max = 0.0f;                            // max |D| stored by this thread
         uint32_t tcount = 0;
         for (int t = pair; t < total; t += n_pairs, ++tcount) {
-            const TileCoord c = tile_coord(a, sh, t);
-            const bool ok = mbar_wait(&sh->acc_full, tcount & 1u);
+            const TileCoord c = tile_coord<kBN>(a, sh, t);
+            const uint32_t buf = tcount % kAcc, aph = (tcount / kAcc) & 1u;
+            const bool ok = mbar_wait(&sh->acc_full[buf], aph, a.wait_ns);
             if (!ok) {
                 if (lane == 0) record_status(a.status, NVFP4_ERR_TIMEOUT);
                 break;
             }
             tc_fence_after();
-            const uint32_t tbase = tmem + ((uint32_t)(32 * quad) << 16) + (uint32_t)col0;
-            const float alpha = __fmul_rn(a.ga[0], a.gb[c.group]);
+            const uint32_t tbase =
+                tmem + ((uint32_t)(32 * quad) << 16) + buf * (uint32_t)kBN + (uint32_t)col0;
+            const float alpha = kFmt == kFmtNVFP4 ? __fmul_rn(a.ga[0], a.gb[c.group]) : 1.0f;
             const int64_t row = c.row0 + (int64_t)BM * rank + 32 * quad + lane;
             const bool row_ok = row < c.row_end;
             if (a.bf16_out) {
-                // 128 columns in four 32-column loads, each converted to bf16
-                // pairs at once: the accumulator is released before any store
-                // with at most 32 + 64 registers of data live.
-                uint32_t packed[64];
-                float m_all = 0.0f;  // max |x| over the 128 columns (before rounding)
+                // kCols columns in 32-column loads, converted to bf16 pairs as they
+                // arrive (two loads in flight per wait for 64-column warps): the
+                // accumulator is released before any store.
+                uint32_t packed[16 * kChunks];
+                float m_all = 0.0f;  // max |x| over the warp's columns (before rounding)
+                constexpr int kPer = kChunks == 2 ? 2 : 1;
 #pragma unroll
-                for (int hh = 0; hh < 4; ++hh) {
-                    uint32_t r[32];
-                    TMEM_LD_32(tbase + 32 * hh, r);
+                for (int hh = 0; hh < kChunks; hh += kPer) {
+                    uint32_t r[32 * kPer];
+#pragma unroll
+                    for (int q = 0; q < kPer; ++q) TMEM_LD_32(tbase + 32 * (hh + q), (r + 32 * q));
                     tmem_ld_wait();
 #pragma unroll
-                    for (int i = 0; i < 16; ++i) {
+                    for (int i = 0; i < 16 * kPer; ++i) {
                         const float x0 = __fmul_rn(__uint_as_float(r[2 * i]), alpha);
                         const float x1 = __fmul_rn(__uint_as_float(r[2 * i + 1]), alpha);
                         m_all = absmax3(m_all, x0, x1);
@@ -512,15 +622,15 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
                 }
                 tc_fence_before();
                 __syncwarp();
-                if (lane == 0) mbar_arrive_cluster(acc_empty_leader);  // accumulator drained
+                if (lane == 0) mbar_arrive_cluster(cluster_addr(&sh->acc_empty[buf], 0));  // accumulator drained
                 const int64_t cbase = c.n0 + col0;
                 // max |D| of this lane's row (rounded values where the N tail cuts the row)
                 if (row_ok) {
-                    if (cbase + 128 <= a.N) {
+                    if (cbase + kCols <= a.N) {
                         out_max = fmaxf(out_max, m_all);
                     } else {
 #pragma unroll
-                        for (int g = 0; g < 16; ++g)
+                        for (int g = 0; g < 4 * kChunks; ++g)
                             if (cbase + 8 * g < a.N) {
 #pragma unroll
                                 for (int i = 0; i < 4; ++i) {
@@ -536,7 +646,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
                 // block: each lane writes its row, then 8 rows x 64 bytes leave
                 // per store instruction (whole 32-byte sectors).
 #pragma unroll
-                for (int hh = 0; hh < 4; ++hh) {
+                for (int hh = 0; hh < kChunks; ++hh) {
 #pragma unroll
                     for (int q = 0; q < 4; ++q)
                         st_shared_v4(stg + lane * 64 + 16 * (q ^ ((lane >> 1) & 3)),
@@ -555,17 +665,17 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
                 }
                 continue;
             }
-            // FP32 output: four rounds of 32 columns, each stored before the
-            // next load; the accumulator is released after the last load.
+            // FP32 output: rounds of 32 columns, each stored before the next
+            // load; the accumulator is released after the last load.
 #pragma unroll 1
-            for (int hh = 0; hh < 4; ++hh) {
+            for (int hh = 0; hh < kChunks; ++hh) {
                 uint32_t r[32];
                 TMEM_LD_32(tbase + 32 * hh, r);
                 tmem_ld_wait();
-                if (hh == 3) {
+                if (hh == kChunks - 1) {
                     tc_fence_before();
                     __syncwarp();
-                    if (lane == 0) mbar_arrive_cluster(acc_empty_leader);  // accumulator drained
+                    if (lane == 0) mbar_arrive_cluster(cluster_addr(&sh->acc_empty[buf], 0));  // accumulator drained
                 }
                 if (!row_ok) continue;
                 const int64_t cbase = c.n0 + col0 + 32 * hh;
@@ -632,24 +742,25 @@ static bool make_map(CUtensorMap* m, const void* base, int64_t rows, int64_t kby
               CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-// B's scales in the tensor-core layout, [G][nblk][K/64 atoms][512 bytes], seen
-// as 8-byte elements: {256 (one K stage's 4 atoms), K/256 stages, nblk, G}; a
-// box is one stage of two consecutive row blocks.
-static bool make_sfb_map(CUtensorMap* m, const void* sfb, int64_t G, int64_t N, int64_t K)
+// B's scales in the tensor-core layout, [G][nblk][k_atoms][512 bytes], seen
+// as 8-byte elements: {one K stage's atoms, K stages, nblk, G}; a box is one
+// stage of two consecutive row blocks (the 256-wide tile).
+static bool make_sfb_map(CUtensorMap* m, const void* sfb, int64_t G, int64_t N, int64_t K,
+                         int k_stage, int k_atom, int stage_atoms)
 {
     auto fn = encode_tiled();
     if (!fn) return false;
-    const int64_t nblk = (N + 127) / 128, k64 = K / 64;
-    cuuint64_t dims[4] = {256u, (cuuint64_t)(K / BK), (cuuint64_t)nblk, (cuuint64_t)G};
-    cuuint64_t strides[3] = {2048u, (cuuint64_t)(k64 * 512), (cuuint64_t)(nblk * k64 * 512)};
-    cuuint32_t box[4] = {256u, 1u, 2u, 1u};
+    const int64_t nblk = (N + 127) / 128, k_atoms = K / k_atom;
+    const cuuint32_t inner = (cuuint32_t)(stage_atoms * 64);  // 8-byte elements per stage
+    cuuint64_t dims[4] = {inner, (cuuint64_t)(K / k_stage), (cuuint64_t)nblk, (cuuint64_t)G};
+    cuuint64_t strides[3] = {(cuuint64_t)stage_atoms * 512u, (cuuint64_t)(k_atoms * 512),
+                             (cuuint64_t)(nblk * k_atoms * 512)};
+    cuuint32_t box[4] = {inner, 1u, 2u, 1u};
     cuuint32_t estr[4] = {1u, 1u, 1u, 1u};
     return fn(m, CU_TENSOR_MAP_DATA_TYPE_UINT64, 4, const_cast<void*>(sfb), dims, strides, box, estr,
               CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
               CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
-
-static size_t gemm_smem_bytes() { return (size_t)kGemmStages * kStageBytes + kSmemShared + 8 * kEpiStageBytes + 1024; }
 
 struct GemmDevice {
     int sms = 0;
@@ -657,16 +768,19 @@ struct GemmDevice {
     bool ok = false;
 };
 
+template <int kFmt, int kBN>
 static GemmDevice& gemm_device(int dev)
 {
     static GemmDevice infos[64];
     static std::once_flag flags[64];
     std::call_once(flags[dev & 63], [dev]() {
         GemmDevice& d = infos[dev & 63];
+        using C = GemmCfg<kFmt, kBN>;
+        auto fn = gemm_kernel<kFmt, kBN>;
         cudaDeviceProp prop;
         if (cudaGetDeviceProperties(&prop, dev) != cudaSuccess || prop.major != 10) return;
-        if (cudaFuncSetAttribute(gemm_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                 (int)gemm_smem_bytes()) != cudaSuccess)
+        if (cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 (int)C::kSmemBytes) != cudaSuccess)
             return;
         d.sms = prop.multiProcessorCount;
         // Pairs need two SMs of one cluster-capable group: ask how many fit
@@ -674,9 +788,9 @@ static GemmDevice& gemm_device(int dev)
         cudaLaunchConfig_t cfg = {};
         cfg.gridDim = dim3((unsigned)(d.sms & ~1));
         cfg.blockDim = dim3(kGemmThreads);
-        cfg.dynamicSmemBytes = gemm_smem_bytes();
+        cfg.dynamicSmemBytes = C::kSmemBytes;
         int clusters = 0;
-        if (cudaOccupancyMaxActiveClusters(&clusters, gemm_kernel, &cfg) != cudaSuccess || clusters < 1)
+        if (cudaOccupancyMaxActiveClusters(&clusters, fn, &cfg) != cudaSuccess || clusters < 1)
             return;
         d.pairs = std::min(clusters, d.sms / 2);
         d.ok = true;
@@ -688,25 +802,80 @@ static bool al16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) 
 
 constexpr size_t kGemmWorkspace = 256;
 
+// Output-tile width.  256 (one accumulator) moves the fewest operand bytes per
+// FLOP; 128 (two accumulators) hides the epilogue's drain, which matters when
+// tiles are short along K.  NVFP4_GEMM_TILE_N=128 or 256 in the environment
+// overrides the choice (read on every call).
+static int pick_tile_n(bool grouped, int64_t K, int k_stage)
+{
+    if (const char* e = getenv("NVFP4_GEMM_TILE_N")) {
+        if (!strcmp(e, "128")) return 128;
+        if (!strcmp(e, "256")) return 256;
+    }
+    (void)K;
+    (void)k_stage;
+    return grouped ? 128 : 256;
+}
+
+template <int kFmt, int kBN>
+static nvfp4_status launch_variant(const void* qa, const void* qb, GemmArgs& a, int64_t a_rows,
+                                   int64_t b_rows, int64_t max_tiles_m, cudaStream_t st)
+{
+    using C = GemmCfg<kFmt, kBN>;
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return NVFP4_ERR_CUDA;
+    wait_test_hook(&a.wait_ns, &a.no_copies);
+    GemmDevice& info = gemm_device<kFmt, kBN>(dev);
+    if (!info.ok) return NVFP4_ERR_UNSUPPORTED;
+    const int64_t kbytes = kFmt == kFmtNVFP4 ? a.K / 2 : a.K;
+    CUtensorMap ma, mb, msf;
+    memset(&msf, 0, sizeof(msf));
+    if (!make_map(&ma, qa, a_rows, kbytes, BM) || !make_map(&mb, qb, b_rows, kbytes, C::kBRows))
+        return NVFP4_ERR_CUDA;
+    if (kBN == 256 &&
+        !make_sfb_map(&msf, a.sfb, a.G, a.N, a.K, C::kKStage, C::kKAtom, C::kSfAtoms))
+        return NVFP4_ERR_CUDA;
+    // the status word reports this call only; the output amax starts at 0
+    if (cudaMemsetAsync(a.status, 0, 4, st) != cudaSuccess) return NVFP4_ERR_CUDA;
+    if (a.amax_out && cudaMemsetAsync(a.amax_out, 0, 4, st) != cudaSuccess) return NVFP4_ERR_CUDA;
+    const int64_t tiles = max_tiles_m * ((a.N + kBN - 1) / kBN);
+    const int pairs = (int)std::max<int64_t>(1, std::min<int64_t>(tiles, info.pairs));
+    gemm_kernel<kFmt, kBN><<<2 * pairs, kGemmThreads, C::kSmemBytes, st>>>(ma, mb, msf, a);
+    return cudaGetLastError() == cudaSuccess ? NVFP4_OK : NVFP4_ERR_CUDA;
+}
+
+template <int kFmt>
+static nvfp4_status launch_gemm(const void* qa, const void* qb, GemmArgs& a, int64_t a_rows,
+                                int64_t b_rows, int64_t max_tiles_m, cudaStream_t st)
+{
+    if (pick_tile_n(a.grouped != 0, a.K, GemmCfg<kFmt, 256>::kKStage) == 128)
+        return launch_variant<kFmt, 128>(qa, qb, a, a_rows, b_rows, max_tiles_m, st);
+    return launch_variant<kFmt, 256>(qa, qb, a, a_rows, b_rows, max_tiles_m, st);
+}
+
 }  // namespace nvfp4
 
 using namespace nvfp4;
 
 extern "C" size_t nvfp4_gemm_workspace_size(int64_t, int64_t, int64_t) { return kGemmWorkspace; }
 
-static nvfp4_status launch_gemm(const CUtensorMap& ma, const CUtensorMap& mb, const CUtensorMap& msf, GemmArgs& a,
-                                int64_t max_tiles, cudaStream_t st)
+// Checks shared by the dense GEMMs; k_mult is the K granularity of a stage.
+static nvfp4_status check_dense(const uint8_t* qa, const uint8_t* sfa, const uint8_t* qb,
+                                const uint8_t* sfb, int64_t M, int64_t N, int64_t K, int64_t k_mult,
+                                int out_dtype, void* D, int64_t ldd, float* amax_out,
+                                void* workspace, size_t ws_bytes)
 {
-    int dev = 0;
-    if (cudaGetDevice(&dev) != cudaSuccess) return NVFP4_ERR_CUDA;
-    GemmDevice& info = gemm_device(dev);
-    if (!info.ok) return NVFP4_ERR_UNSUPPORTED;
-    // the status word reports this call only; the output amax starts at 0
-    if (cudaMemsetAsync(a.status, 0, 4, st) != cudaSuccess) return NVFP4_ERR_CUDA;
-    if (a.amax_out && cudaMemsetAsync(a.amax_out, 0, 4, st) != cudaSuccess) return NVFP4_ERR_CUDA;
-    const int pairs = (int)std::max<int64_t>(1, std::min<int64_t>(max_tiles, info.pairs));
-    gemm_kernel<<<2 * pairs, kGemmThreads, gemm_smem_bytes(), st>>>(ma, mb, msf, a);
-    return cudaGetLastError() == cudaSuccess ? NVFP4_OK : NVFP4_ERR_CUDA;
+    if (!qa || !sfa || !qb || !sfb || !D) return NVFP4_ERR_INVALID_ARG;
+    if (out_dtype != NVFP4_OUT_F32 && out_dtype != NVFP4_OUT_BF16) return NVFP4_ERR_INVALID_ARG;
+    if (M <= 0 || N <= 0 || K <= 0 || M % 16 || N % 16 || K % k_mult || ldd < N) return NVFP4_ERR_SHAPE;
+    if (M > (int64_t)1 << 31 || N > (int64_t)1 << 31) return NVFP4_ERR_SHAPE;
+    const int esz = out_dtype == NVFP4_OUT_BF16 ? 2 : 4;
+    if (!al16(qa) || !al16(qb) || !al16(sfa) || !al16(sfb) || !al16(D) || (ldd * esz) % 16 ||
+        (reinterpret_cast<uintptr_t>(amax_out) & 3u))
+        return NVFP4_ERR_ALIGN;
+    if (!workspace || ws_bytes < kGemmWorkspace) return NVFP4_ERR_WORKSPACE;
+    if (!al16(workspace)) return NVFP4_ERR_ALIGN;
+    return NVFP4_OK;
 }
 
 extern "C" nvfp4_status nvfp4_gemm(const uint8_t* qa, const uint8_t* sfa, const float* ga,
@@ -715,18 +884,10 @@ extern "C" nvfp4_status nvfp4_gemm(const uint8_t* qa, const uint8_t* sfa, const 
                                    int64_t ldd, float* amax_out, void* workspace, size_t ws_bytes,
                                    void* stream)
 {
-    if (!qa || !sfa || !ga || !qb || !sfb || !gb || !D) return NVFP4_ERR_INVALID_ARG;
-    if (out_dtype != NVFP4_OUT_F32 && out_dtype != NVFP4_OUT_BF16) return NVFP4_ERR_INVALID_ARG;
-    if (M <= 0 || N <= 0 || K <= 0 || M % 16 || N % 16 || K % BK || ldd < N) return NVFP4_ERR_SHAPE;
-    if (M > (int64_t)1 << 31 || N > (int64_t)1 << 31) return NVFP4_ERR_SHAPE;
-    const int esz = out_dtype == NVFP4_OUT_BF16 ? 2 : 4;
-    if (!al16(qa) || !al16(qb) || !al16(sfa) || !al16(sfb) || !al16(D) || (ldd * esz) % 16 ||
-        (reinterpret_cast<uintptr_t>(amax_out) & 3u))
-        return NVFP4_ERR_ALIGN;
-    if (!workspace || ws_bytes < kGemmWorkspace) return NVFP4_ERR_WORKSPACE;
-    if (!al16(workspace)) return NVFP4_ERR_ALIGN;
-    CUtensorMap ma, mb;
-    if (!make_map(&ma, qa, M, K / 2, BM) || !make_map(&mb, qb, N, K / 2, BN / 2)) return NVFP4_ERR_CUDA;
+    if (!ga || !gb) return NVFP4_ERR_INVALID_ARG;
+    const nvfp4_status chk = check_dense(qa, sfa, qb, sfb, M, N, K, 256, out_dtype, D, ldd,
+                                         amax_out, workspace, ws_bytes);
+    if (chk != NVFP4_OK) return chk;
     GemmArgs a{};
     a.sfa = sfa;
     a.sfb = sfb;
@@ -742,10 +903,33 @@ extern "C" nvfp4_status nvfp4_gemm(const uint8_t* qa, const uint8_t* sfa, const 
     a.G = 1;
     a.status = static_cast<uint32_t*>(workspace) + 2;
     a.amax_out = amax_out;
-    CUtensorMap msf;
-    if (!make_sfb_map(&msf, sfb, 1, N, K)) return NVFP4_ERR_CUDA;
-    const int64_t tiles = ((M + kMmaM - 1) / kMmaM) * ((N + BN - 1) / BN);
-    return launch_gemm(ma, mb, msf, a, tiles, static_cast<cudaStream_t>(stream));
+    return launch_gemm<kFmtNVFP4>(qa, qb, a, M, N, (M + kMmaM - 1) / kMmaM,
+                                  static_cast<cudaStream_t>(stream));
+}
+
+extern "C" nvfp4_status mxfp8_gemm(const uint8_t* qa, const uint8_t* sfa, const uint8_t* qb,
+                                   const uint8_t* sfb, int64_t M, int64_t N, int64_t K,
+                                   int out_dtype, void* D, int64_t ldd, float* amax_out,
+                                   void* workspace, size_t ws_bytes, void* stream)
+{
+    const nvfp4_status chk = check_dense(qa, sfa, qb, sfb, M, N, K, 128, out_dtype, D, ldd,
+                                         amax_out, workspace, ws_bytes);
+    if (chk != NVFP4_OK) return chk;
+    GemmArgs a{};
+    a.sfa = sfa;
+    a.sfb = sfb;
+    a.D = D;
+    a.M = M;
+    a.N = N;
+    a.K = K;
+    a.ldd = ldd;
+    a.bf16_out = out_dtype == NVFP4_OUT_BF16;
+    a.grouped = 0;
+    a.G = 1;
+    a.status = static_cast<uint32_t*>(workspace) + 2;
+    a.amax_out = amax_out;
+    return launch_gemm<kFmtMXFP8>(qa, qb, a, M, N, (M + kMmaM - 1) / kMmaM,
+                                  static_cast<cudaStream_t>(stream));
 }
 
 extern "C" nvfp4_status nvfp4_grouped_gemm(int G, const int32_t* group_offsets, int64_t total_rows,
@@ -759,16 +943,13 @@ extern "C" nvfp4_status nvfp4_grouped_gemm(int G, const int32_t* group_offsets, 
         !gb || !D)
         return NVFP4_ERR_INVALID_ARG;
     if (out_dtype != NVFP4_OUT_F32 && out_dtype != NVFP4_OUT_BF16) return NVFP4_ERR_INVALID_ARG;
-    if (total_rows <= 0 || N <= 0 || K <= 0 || N % 128 || K % BK) return NVFP4_ERR_SHAPE;
+    if (total_rows <= 0 || N <= 0 || K <= 0 || N % 128 || K % 256) return NVFP4_ERR_SHAPE;
     if (total_rows > (int64_t)1 << 31 || (int64_t)G * N > (int64_t)1 << 31) return NVFP4_ERR_SHAPE;
     if (!al16(qa) || !al16(qb) || !al16(sfa) || !al16(sfb) || !al16(D) ||
         (reinterpret_cast<uintptr_t>(amax_out) & 3u))
         return NVFP4_ERR_ALIGN;
     if (!workspace || ws_bytes < kGemmWorkspace) return NVFP4_ERR_WORKSPACE;
     if (!al16(workspace)) return NVFP4_ERR_ALIGN;
-    CUtensorMap ma, mb;
-    if (!make_map(&ma, qa, total_rows, K / 2, BM) || !make_map(&mb, qb, (int64_t)G * N, K / 2, BN / 2))
-        return NVFP4_ERR_CUDA;
     GemmArgs a{};
     a.sfa = sfa;
     a.sfb = sfb;
@@ -786,9 +967,8 @@ extern "C" nvfp4_status nvfp4_grouped_gemm(int G, const int32_t* group_offsets, 
     a.total_rows = total_rows;
     a.status = static_cast<uint32_t*>(workspace) + 2;
     a.amax_out = amax_out;
-    // upper bound on tiles: every group may add one partial M tile
-    CUtensorMap msf;
-    if (!make_sfb_map(&msf, sfb, G, N, K)) return NVFP4_ERR_CUDA;
-    const int64_t tiles = ((total_rows + kMmaM - 1) / kMmaM + G) * ((N + BN - 1) / BN);
-    return launch_gemm(ma, mb, msf, a, tiles, static_cast<cudaStream_t>(stream));
+    // upper bound on M tiles: every group may add one partial tile
+    return launch_gemm<kFmtNVFP4>(qa, qb, a, total_rows, (int64_t)G * N,
+                                  (total_rows + kMmaM - 1) / kMmaM + G,
+                                  static_cast<cudaStream_t>(stream));
 }

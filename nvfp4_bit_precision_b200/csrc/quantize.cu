@@ -41,7 +41,14 @@ constexpr int kStages = 2;
 // bytes per column) and NVFP4 columnwise codes (16 bytes per column).
 constexpr int kMxStageBytes = 64 * 32;
 constexpr int kQcStageBytes = 64 * 16;
-constexpr int kQuantThreads = 256;
+// The fused pass runs 12 warps per CTA (2 CTAs, 24 warps per SM at <= 80
+// registers a thread): when a tile feeds both directions, warps 0..7 take the
+// columnwise work (one column pair x 32 rows each) and warps 8..11 the rowwise
+// work (two row halves each); with one direction only, warps 0..7 take it and
+// warps 8..11 only release the stage.  The amax pass keeps 8 warps.
+constexpr int kQuantThreads = 384;
+constexpr int kColWarps = 8;
+constexpr int kAmaxThreads = 256;
 constexpr int kMaxGroups = 256;  // MoE groups per call (the grouped GEMM's limit too)
 
 struct QArgs {
@@ -67,7 +74,18 @@ struct QArgs {
     PhiloxKeys pk;  // round keys of `seed`
     int mx_staged;  // MXFP8 columnwise codes go through shared memory and TMA stores
     int qc_staged;  // NVFP4 columnwise codes likewise (rows a multiple of 32)
+    int mx_mma;     // MXFP8 scale bytes in the tensor-core tiled layout
+    uint64_t wait_ns;  // limit of every barrier wait (2 s; shorter under the test hook)
+    int no_copies;     // test hook: the producer issues no copy (see wait_test_hook)
 };
+
+// Offset of the E8M0 byte of 32-block b of row r, in a [rows, nblk] scale
+// tensor: row-major, or the tensor cores' 128x4 atoms (the NVFP4 tiled layout
+// with 32-element blocks).
+__device__ __forceinline__ int64_t mx_sf_off(const QArgs& a, int64_t r, int64_t b, int64_t nblk)
+{
+    return a.mx_mma ? sf_mma_offset(r, b, nblk) : r * nblk + b;
+}
 
 __device__ __forceinline__ uint4 ld_global_v4(const void* p)
 {
@@ -325,7 +343,7 @@ __device__ __forceinline__ void store_codes32(uint8_t* dst, const uint32_t (&c)[
 // Hadamard on, max |RHT(x)| over the columnwise 16-vectors.  One atomicMax per
 // CTA on the float bit pattern.
 // --------------------------------------------------------------------------
-__global__ void __launch_bounds__(kQuantThreads, 2)
+__global__ void __launch_bounds__(kAmaxThreads, 2)
     amax_kernel(const __grid_constant__ CUtensorMap map_x, QArgs a, uint32_t* amax_out)
 {
     extern __shared__ uint8_t smem_raw[];
@@ -338,7 +356,7 @@ __global__ void __launch_bounds__(kQuantThreads, 2)
     if (threadIdx.x == 0) {
         for (int s = 0; s < kStages; ++s) {
             mbar_init(&full[s], 1);
-            mbar_init(&empty[s], kQuantThreads / 32);
+            mbar_init(&empty[s], kAmaxThreads / 32);
         }
         fence_barrier_init();
     }
@@ -350,7 +368,8 @@ __global__ void __launch_bounds__(kQuantThreads, 2)
         first < a.n_tiles ? (a.n_tiles - first + gridDim.x - 1) / gridDim.x : 0;
     auto tile_of = [&](int64_t k) { return first + k * (int64_t)gridDim.x; };
     int64_t issued = 0;
-    if (warp == 0) {
+    const bool produce = warp == 0 && !a.no_copies;
+    if (produce) {
         for (; issued < my_count && issued < kStages - 1; ++issued)
             issue_tile<true>(a, &map_x, tile_of(issued), tiles + (issued % kStages) * kTileBytes,
                              &full[issued % kStages], lane);
@@ -361,10 +380,10 @@ __global__ void __launch_bounds__(kQuantThreads, 2)
     int64_t k = 0;
     for (; k < my_count; ++k) {
         const int stage = (int)(k % kStages);
-        if (warp == 0 && issued < my_count) {
+        if (produce && issued < my_count) {
             const int s = (int)(issued % kStages);
             bool ok = true;
-            if (issued >= kStages) ok = mbar_wait(&empty[s], (uint32_t)((issued / kStages - 1) & 1));
+            if (issued >= kStages) ok = mbar_wait(&empty[s], (uint32_t)((issued / kStages - 1) & 1), a.wait_ns);
             if (!ok) {
                 if (lane == 0) record_status(a.status, NVFP4_ERR_TIMEOUT);
                 break;
@@ -372,7 +391,7 @@ __global__ void __launch_bounds__(kQuantThreads, 2)
             issue_tile<true>(a, &map_x, tile_of(issued), tiles + s * kTileBytes, &full[s], lane);
             ++issued;
         }
-        if (!mbar_wait(&full[stage], (uint32_t)((k / kStages) & 1))) {
+        if (!mbar_wait(&full[stage], (uint32_t)((k / kStages) & 1), a.wait_ns)) {
             if (lane == 0) record_status(a.status, NVFP4_ERR_TIMEOUT);
             break;
         }
@@ -404,21 +423,21 @@ __global__ void __launch_bounds__(kQuantThreads, 2)
     }
     if (warp == 0) {
         for (int64_t j = k + 1; j < issued; ++j)
-            (void)mbar_wait(&full[j % kStages], (uint32_t)((j / kStages) & 1));
+            (void)mbar_wait(&full[j % kStages], (uint32_t)((j / kStages) & 1), a.wait_ns);
     }
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) {
         mr = fmaxf(mr, __shfl_xor_sync(0xffffffffu, mr, o));
         mc = fmaxf(mc, __shfl_xor_sync(0xffffffffu, mc, o));
     }
-    __shared__ float red[2][kQuantThreads / 32];
+    __shared__ float red[2][kAmaxThreads / 32];
     if (lane == 0) {
         red[0][warp] = mr;
         red[1][warp] = mc;
     }
     __syncthreads();
     if (threadIdx.x == 0) {
-        for (int w = 1; w < kQuantThreads / 32; ++w) {
+        for (int w = 1; w < kAmaxThreads / 32; ++w) {
             mr = fmaxf(mr, red[0][w]);
             mc = fmaxf(mc, red[1][w]);
         }
@@ -528,8 +547,8 @@ __global__ void __launch_bounds__(kQuantThreads, 2)
                                                ~uintptr_t(1023));
     uint8_t* tiles = smem;
     uint8_t* mx_stage_all = smem + kStages * kTileBytes;
-    uint8_t* qc_stage_all = mx_stage_all + (kQuantThreads / 32) * kMxStageBytes;
-    uint64_t* bars = reinterpret_cast<uint64_t*>(qc_stage_all + (kQuantThreads / 32) * kQcStageBytes);
+    uint8_t* qc_stage_all = mx_stage_all + kColWarps * kMxStageBytes;
+    uint64_t* bars = reinterpret_cast<uint64_t*>(qc_stage_all + kColWarps * kQcStageBytes);
     QShared* sh = reinterpret_cast<QShared*>(reinterpret_cast<uint8_t*>(bars) + 64);
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -603,7 +622,8 @@ __global__ void __launch_bounds__(kQuantThreads, 2)
     uint64_t* full = bars;
     uint64_t* empty = bars + kStages;
     int64_t issued = 0;  // tiles whose copies warp 0 has issued
-    if (warp == 0) {
+    const bool produce = warp == 0 && !a.no_copies;
+    if (produce) {
         for (; issued < my_count && issued < kStages - 1; ++issued)
             issue_tile<kTma>(a, &map_x, tile_of(issued), tiles + (issued % kStages) * kTileBytes,
                              &full[issued % kStages], lane);
@@ -617,12 +637,12 @@ __global__ void __launch_bounds__(kQuantThreads, 2)
     int64_t k = 0;
     for (; k < my_count; ++k) {
         const int stage = (int)(k % kStages);
-        if (warp == 0 && issued < my_count) {
+        if (produce && issued < my_count) {
             // refill the stage tile `issued - kStages` used, once every warp released it
             const int s = (int)(issued % kStages);
             bool ok = true;
             if (issued >= kStages)
-                ok = mbar_wait(&empty[s], (uint32_t)((issued / kStages - 1) & 1));
+                ok = mbar_wait(&empty[s], (uint32_t)((issued / kStages - 1) & 1), a.wait_ns);
             if (!ok) {
                 if (lane == 0) record_status(a.status, NVFP4_ERR_TIMEOUT);
                 break;
@@ -630,7 +650,7 @@ __global__ void __launch_bounds__(kQuantThreads, 2)
             issue_tile<kTma>(a, &map_x, tile_of(issued), tiles + s * kTileBytes, &full[s], lane);
             ++issued;
         }
-        if (!mbar_wait(&full[stage], (uint32_t)((k / kStages) & 1))) {
+        if (!mbar_wait(&full[stage], (uint32_t)((k / kStages) & 1), a.wait_ns)) {
             if (lane == 0) record_status(a.status, NVFP4_ERR_TIMEOUT);
             break;
         }
@@ -639,9 +659,18 @@ __global__ void __launch_bounds__(kQuantThreads, 2)
         const int64_t tr = tile_row(a, tile), tc = tile - tr * a.tiles_c;
         const int64_t r0 = tr * kTileRows, c0 = tc * kTileCols;
 
-        // ---------------- rowwise: thread = (row, 64-column half) ----------
-        if (nv_row || mx_row) {
-            const int rl = 16 * warp + (lane & 15);
+        // ---------------- rowwise: item = (row, 64-column half) ------------
+        // Item i (0..255) is row 16*(i/32) + i%16, half (i%32)/16, so the 16
+        // lanes of a half-warp hold 16 consecutive rows (a 16x16 tile for 2D).
+        // Both directions: warps 8..11 take items i and i + 128; rowwise
+        // only: warps 0..7 take one item each.
+        const bool both_dirs = (nv_row || mx_row) && (nv_col || mx_col);
+        const int row_warp0 = both_dirs ? kColWarps : 0;
+        const int row_items = both_dirs ? 2 : 1;
+        if ((nv_row || mx_row) && warp >= row_warp0 && warp < row_warp0 + 8 / row_items)
+#pragma unroll 1
+        for (int ri = 0; ri < row_items; ++ri) {
+            const int rl = 16 * (warp - row_warp0 + 4 * ri) + (lane & 15);
             const int h = lane >> 4;
             const int64_t rg = r0 + rl;
             const bool rvalid = rg < a.rows;
@@ -711,15 +740,16 @@ __global__ void __launch_bounds__(kQuantThreads, 2)
                     uint4* dst = reinterpret_cast<uint4*>(a.mx_q_row + rg * a.cols + cg);
                     dst[0] = make_uint4(out[0], out[1], out[2], out[3]);
                     dst[1] = make_uint4(out[4], out[5], out[6], out[7]);
-                    a.mx_sf_row[rg * (a.cols / 32) + cg / 32] = (uint8_t)e8;
+                    a.mx_sf_row[mx_sf_off(a, rg, cg / 32, a.cols / 32)] = (uint8_t)e8;
                 }
             }
         }
 
         // ---------------- columnwise: thread = (column pair, 32-row group) --
-        // One 32-bit shared load per row gives both columns of the pair; the
-        // pair's two Hadamard transforms run in the two lanes of f32x2.
-        if (nv_col || mx_col) {
+        // Warps 0..7.  One 32-bit shared load per row gives both columns of
+        // the pair; the pair's two Hadamard transforms run in the two lanes of
+        // f32x2.
+        if ((nv_col || mx_col) && warp < kColWarps) {
             const int cp = 32 * (warp & 1) + lane;  // column pair 0..63
             const int rgrp = warp >> 1;              // 32-row group 0..3
             const int64_t cg0 = c0 + 2 * cp;         // columns cg0, cg0 + 1
@@ -867,8 +897,8 @@ __global__ void __launch_bounds__(kQuantThreads, 2)
                                      make_uint4(cb[0].x, cb[0].y, cb[1].x, cb[1].y));
                     }
                     if (cvalid) {
-                        a.mx_sf_col[cg0 * (a.rows / 32) + rbase / 32] = (uint8_t)(ea + 127);
-                        a.mx_sf_col[(cg0 + 1) * (a.rows / 32) + rbase / 32] = (uint8_t)(eb + 127);
+                        a.mx_sf_col[mx_sf_off(a, cg0, rbase / 32, a.rows / 32)] = (uint8_t)(ea + 127);
+                        a.mx_sf_col[mx_sf_off(a, cg0 + 1, rbase / 32, a.rows / 32)] = (uint8_t)(eb + 127);
                     }
                     fence_proxy_async_smem();
                     __syncwarp();
@@ -900,8 +930,8 @@ __global__ void __launch_bounds__(kQuantThreads, 2)
                     *reinterpret_cast<uint2*>(qa + 8 * g) = mx_convert8(va, sa, mx_sr, wa);
                     *reinterpret_cast<uint2*>(qb + 8 * g) = mx_convert8(vb, sb, mx_sr, wb);
                 }
-                a.mx_sf_col[cg0 * (a.rows / 32) + rbase / 32] = (uint8_t)(ea + 127);
-                a.mx_sf_col[(cg0 + 1) * (a.rows / 32) + rbase / 32] = (uint8_t)(eb + 127);
+                a.mx_sf_col[mx_sf_off(a, cg0, rbase / 32, a.rows / 32)] = (uint8_t)(ea + 127);
+                a.mx_sf_col[mx_sf_off(a, cg0 + 1, rbase / 32, a.rows / 32)] = (uint8_t)(eb + 127);
             }
         }
         __syncwarp();
@@ -914,7 +944,7 @@ __global__ void __launch_bounds__(kQuantThreads, 2)
     // must land before the CTA's shared memory goes away.
     if (warp == 0) {
         for (int64_t j = k + 1; j < issued; ++j)
-            (void)mbar_wait(&full[j % kStages], (uint32_t)((j / kStages) & 1));
+            (void)mbar_wait(&full[j % kStages], (uint32_t)((j / kStages) & 1), a.wait_ns);
     }
 }
 
@@ -1054,7 +1084,7 @@ struct DeviceInfo {
 
 static size_t quant_smem_bytes()
 {
-    return (size_t)kStages * kTileBytes + (kQuantThreads / 32) * (kMxStageBytes + kQcStageBytes) + 64 +
+    return (size_t)kStages * kTileBytes + kColWarps * (kMxStageBytes + kQcStageBytes) + 64 +
            sizeof(QShared) + 1024;  // + alignment slack
 }
 
@@ -1154,7 +1184,7 @@ static DeviceInfo& device_info(int dev)
             int nb = 0;
             if (cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                      (int)quant_smem_bytes()) != cudaSuccess ||
-                cudaOccupancyMaxActiveBlocksPerMultiprocessor(&nb, fn, kQuantThreads,
+                cudaOccupancyMaxActiveBlocksPerMultiprocessor(&nb, fn, kAmaxThreads,
                                                               quant_smem_bytes()) != cudaSuccess ||
                 nb < 1)
                 return;
@@ -1180,6 +1210,12 @@ extern "C" size_t nvfp4_sf_mma_bytes(int64_t rows, int64_t k)
     return (size_t)((rows + 127) / 128) * 128 * (size_t)(((k / 16) + 3) / 4) * 4;
 }
 
+extern "C" size_t mxfp8_sf_mma_bytes(int64_t rows, int64_t k)
+{
+    if (rows <= 0 || k <= 0) return 0;
+    return (size_t)((rows + 127) / 128) * 128 * (size_t)(((k / 32) + 3) / 4) * 4;
+}
+
 extern "C" size_t nvfp4_sf_mma_grouped_bytes(int64_t total_rows, int num_groups, int64_t k)
 {
     if (total_rows < 0 || num_groups <= 0 || k <= 0) return 0;
@@ -1195,6 +1231,7 @@ extern "C" size_t nvfp4_quantize_workspace_size(int64_t, int64_t, const nvfp4_qu
 static nvfp4_status launch_quant(QArgs& a, bool need_amax, void* workspace, cudaStream_t st)
 {
     philox_round_keys(a.seed, &a.pk);
+    wait_test_hook(&a.wait_ns, &a.no_copies);
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess) return NVFP4_ERR_CUDA;
     DeviceInfo& info = device_info(dev);
@@ -1217,7 +1254,7 @@ static nvfp4_status launch_quant(QArgs& a, bool need_amax, void* workspace, cuda
         uint32_t* amax = static_cast<uint32_t*>(workspace);
         a.amax_ws = amax;
         if (tma) {
-            amax_kernel<<<(int)grid, kQuantThreads, quant_smem_bytes(), st>>>(map, a, amax);
+            amax_kernel<<<(int)grid, kAmaxThreads, quant_smem_bytes(), st>>>(map, a, amax);
         } else {
             const int64_t units = (a.rows / 16) * (a.cols / 4);  // 16 rows x 4 columns each
             const int blocks = (int)std::max<int64_t>(
@@ -1272,6 +1309,11 @@ extern "C" nvfp4_status nvfp4_quantize(const void* x_bf16, int64_t rows, int64_t
         return NVFP4_ERR_ALIGN;
     if (p->sf_layout == NVFP4_SF_MMA && ((nv_row && cols % 64) || (nv_col && rows % 64)))
         return NVFP4_ERR_SHAPE;
+    if (p->mx_sf_layout != NVFP4_SF_ROWMAJOR && p->mx_sf_layout != NVFP4_SF_MMA)
+        return NVFP4_ERR_INVALID_ARG;
+    if (p->mx_sf_layout == NVFP4_SF_MMA &&
+        (((p->mx_outputs & NVFP4_ROWWISE) && cols % 128) || ((p->mx_outputs & NVFP4_COLWISE) && rows % 128)))
+        return NVFP4_ERR_SHAPE;
     if (p->mx_outputs & NVFP4_ROWWISE) {
         if (cols % 32) return NVFP4_ERR_SHAPE;
         if (!p->mx_q_row || !p->mx_sf_row) return NVFP4_ERR_INVALID_ARG;
@@ -1321,6 +1363,7 @@ extern "C" nvfp4_status nvfp4_quantize(const void* x_bf16, int64_t rows, int64_t
     a.mx_sf_row = p->mx_sf_row;
     a.mx_q_col = p->mx_q_col;
     a.mx_sf_col = p->mx_sf_col;
+    a.mx_mma = p->mx_sf_layout == NVFP4_SF_MMA;
     a.status = workspace ? static_cast<uint32_t*>(workspace) + 2 : nullptr;
     return launch_quant(a, need_amax, workspace, static_cast<cudaStream_t>(stream));
 }
@@ -1479,4 +1522,4 @@ extern "C" const char* nvfp4_status_string(nvfp4_status s)
     return "unknown status";
 }
 
-extern "C" int nvfp4_version(void) { return 100; }
+extern "C" int nvfp4_version(void) { return 200; }

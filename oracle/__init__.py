@@ -85,6 +85,9 @@ def lib():
         L.orc_nvfp4_grouped_gemm_rows.argtypes = [ctypes.c_int, P, P, P, ctypes.c_float, P, P, P,
                                                   i64, i64, P, i64, P, P]
         L.orc_nvfp4_grouped_gemm_rows.restype = ctypes.c_int
+        L.orc_mxfp8_dequant_f64.argtypes = [P, P, i64, i64, P]
+        L.orc_mxfp8_gemm_rows.argtypes = [P, P, P, P, i64, i64, i64, P, i64, P, P]
+        L.orc_mxfp8_gemm_rows.restype = ctypes.c_int
         _lib = L
     return _lib
 
@@ -282,4 +285,34 @@ def nvfp4_grouped_gemm_rows(offsets, qa, sfa, ga, qb, sfb, gb, rows_sel):
                                            _p(out), _p(absout))
     if rc != 0:
         raise ValueError("oracle grouped gemm: invalid arguments")
+    return out, absout
+
+
+def mxfp8_dequant(q: np.ndarray, e8: np.ndarray) -> np.ndarray:
+    """Binary64 values of MXFP8 codes [rows, cols] with row-major E8M0 scales [rows, cols/32]."""
+    q = np.ascontiguousarray(q, dtype=np.uint8)
+    e8 = np.ascontiguousarray(e8, dtype=np.uint8)
+    rows, cols = q.shape
+    out = np.zeros((rows, cols), dtype=np.float64)
+    lib().orc_mxfp8_dequant_f64(_p(q), _p(e8), rows, cols, _p(out))
+    return out
+
+
+def mxfp8_gemm_rows(qa, e8a, qb, e8b, rows_sel=None):
+    """FP64 D = A_hat B_hat^T of MXFP8 operands for the selected rows of A; also
+    sum |a_hat||b_hat|."""
+    qa = np.ascontiguousarray(qa, dtype=np.uint8)
+    qb = np.ascontiguousarray(qb, dtype=np.uint8)
+    e8a = np.ascontiguousarray(e8a, dtype=np.uint8)
+    e8b = np.ascontiguousarray(e8b, dtype=np.uint8)
+    M, K = qa.shape
+    N = qb.shape[0]
+    sel = np.arange(M, dtype=np.int64) if rows_sel is None else np.ascontiguousarray(
+        rows_sel, dtype=np.int64)
+    out = np.zeros((len(sel), N), dtype=np.float64)
+    absout = np.zeros((len(sel), N), dtype=np.float64)
+    rc = lib().orc_mxfp8_gemm_rows(_p(qa), _p(e8a), _p(qb), _p(e8b), M, N, K, _p(sel), len(sel),
+                                   _p(out), _p(absout))
+    if rc != 0:
+        raise ValueError("oracle mxfp8 gemm: invalid arguments")
     return out, absout

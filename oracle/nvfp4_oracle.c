@@ -655,3 +655,59 @@ int orc_nvfp4_grouped_gemm_rows(int G, const int64_t* off, const uint8_t* qa,
     }
     return ORC_OK;
 }
+
+/* ------------------------------------------------------------------------ */
+/* MXFP8 GEMM reference (the backward-pass format of the recipe [iitak,     */
+/* "How it works"]).  An MXFP8 element stands for its E4M3 value times      */
+/* 2^(byte - 127), byte being the E8M0 scale of its 32-element block (OCP MX */
+/* v1.0); the oracle multiplies the dequantised operands in binary64, where  */
+/* every product of two such values is exact.                               */
+/* ------------------------------------------------------------------------ */
+void orc_mxfp8_dequant_f64(const uint8_t* q, const uint8_t* e8, int64_t rows, int64_t cols,
+                           double* out)
+{
+    for (int64_t r = 0; r < rows; ++r)
+        for (int64_t c = 0; c < cols; ++c)
+            out[r * cols + c] = ldexp(orc_e4m3_decode(q[r * cols + c]),
+                                      (int)e8[r * (cols / 32) + c / 32] - 127);
+}
+
+/* D[s][j] = sum_k a_hat[rows_sel[s]][k] * b_hat[j][k] (binary64), and the same
+ * sum of absolute products (the tolerance's scale).  A [M, K], B [N, K] codes
+ * with row-major E8M0 scales [M, K/32], [N, K/32]. */
+int orc_mxfp8_gemm_rows(const uint8_t* qa, const uint8_t* e8a, const uint8_t* qb,
+                        const uint8_t* e8b, int64_t M, int64_t N, int64_t K,
+                        const int64_t* rows_sel, int64_t n_sel, double* out, double* absout)
+{
+    if (K % 32) return ORC_EINVAL;
+    double* a = (double*)malloc(sizeof(double) * (size_t)K);
+    double* bt = (double*)malloc(sizeof(double) * (size_t)(N * K));
+    if (!a || !bt) {
+        free(a);
+        free(bt);
+        return ORC_EINVAL;
+    }
+    orc_mxfp8_dequant_f64(qb, e8b, N, K, bt);
+    for (int64_t s = 0; s < n_sel; ++s) {
+        int64_t i = rows_sel[s];
+        if (i < 0 || i >= M) {
+            free(a);
+            free(bt);
+            return ORC_EINVAL;
+        }
+        orc_mxfp8_dequant_f64(qa + i * K, e8a + i * (K / 32), 1, K, a);
+        for (int64_t j = 0; j < N; ++j) {
+            double acc = 0.0, aacc = 0.0;
+            for (int64_t k = 0; k < K; ++k) {
+                double pr = a[k] * bt[j * K + k];
+                acc += pr;
+                aacc += fabs(pr);
+            }
+            out[s * N + j] = acc;
+            absout[s * N + j] = aacc;
+        }
+    }
+    free(a);
+    free(bt);
+    return ORC_OK;
+}

@@ -130,3 +130,28 @@ def test_mxfp4_argument_errors(nv):
     assert L.mxfp4_quantize(FAKE + 8, 32, 32, 32, 1, FAKE, FAKE, None, None, None) == 3
     assert L.mxfp4_quantize(FAKE, 32, 32, 36, 1, FAKE, FAKE, None, None, None) == 3   # ld % 8
     assert L.mxfp4_quantize(FAKE, 32, 32, 32, 2, None, None, FAKE + 4, FAKE, None) == 3
+
+
+def test_mxfp8_gemm_argument_errors(nv):
+    """The MXFP8 GEMM validates like the NVFP4 one, with K in stages of 128; the MXFP8
+    tiled scale layout needs the block axis a multiple of 128."""
+    L = nv._lib
+    g = L.mxfp8_gemm
+    args = (FAKE,) * 4
+    assert g(None, FAKE, FAKE, FAKE, 128, 128, 128, 0, FAKE, 128, None, FAKE, 256, None) == 1
+    assert g(*args, 128, 128, 96, 0, FAKE, 128, None, FAKE, 256, None) == 2      # K % 128
+    assert g(*args, 120, 128, 128, 0, FAKE, 128, None, FAKE, 256, None) == 2     # M % 16
+    assert g(*args, 128, 128, 128, 0, FAKE, 100, None, FAKE, 256, None) == 2     # ldd < N
+    assert g(*args, 128, 128, 128, 1, FAKE, 132, None, FAKE, 256, None) == 3     # ldd align
+    assert g(FAKE + 8, FAKE, FAKE, FAKE, 128, 128, 128, 0, FAKE, 128, None, FAKE, 256, None) == 3
+    assert g(*args, 128, 128, 128, 0, FAKE, 128, None, FAKE, 8, None) == 7       # workspace
+    assert g(*args, 128, 128, 128, 9, FAKE, 128, None, FAKE, 256, None) == 1     # dtype
+    assert nv.mxfp8_sf_mma_bytes(128, 128) == 128 * 4
+    assert nv.mxfp8_sf_mma_bytes(129, 512) == 256 * 16
+    p = nv.QuantParams()
+    p.mx_outputs = nv.NVFP4_ROWWISE
+    p.mx_q_row = p.mx_sf_row = FAKE
+    p.mx_sf_layout = nv.NVFP4_SF_MMA
+    assert q(nv, 32, 96, 96, p) == 2                    # tiled MXFP8 scales need K % 128
+    p.mx_sf_layout = 3
+    assert q(nv, 32, 128, 128, p) == 1

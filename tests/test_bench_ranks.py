@@ -69,12 +69,31 @@ def test_clock_summary_decodes_reasons():
     assert bench.ClockSampler.summary(c)["reasons"] == ["hw_thermal_slowdown", "sw_power_cap"]
 
 
-def test_hw_fp4_context_uses_the_sampled_clock():
-    """The FP4 tensor rate is 32768 FLOP per SM per cycle on 148 SMs at the sampled
-    clock; without a clock sample the context is left out."""
+def test_hw_fp4_peak_uses_the_sampled_clock():
+    """The GEMM roofline's peak: 32768 FP4 FLOP per SM per cycle on 148 SMs at the
+    median clock of the timed region, falling back to the maximum clock (then 1965
+    MHz) when nothing was sampled."""
     import bench
-    ctx = bench.hw_fp4_context(4765.0, {"sm_mhz": 1965.0})
-    assert abs(ctx["hw_fp4_peak_at_clock"] - 32768 * 148 * 1965e6 / 1e12) < 0.1
-    assert abs(ctx["frac_of_hw_fp4_peak"] - 4765.0 / ctx["hw_fp4_peak_at_clock"]) < 1e-4
-    assert bench.hw_fp4_context(4765.0, None) == {}
-    assert bench.hw_fp4_context(4765.0, {"sm_mhz": None}) == {}
+    peak, mhz = bench.hw_fp4_peak({"sm_mhz": 1965.0, "sm_max_mhz": 1965})
+    assert mhz == 1965.0 and abs(peak - 32768 * 148 * 1965e6 / 1e12) < 0.1
+    peak, mhz = bench.hw_fp4_peak({"sm_mhz": 1500.0, "sm_max_mhz": 1965})
+    assert mhz == 1500.0 and abs(peak - 32768 * 148 * 1500e6 / 1e12) < 0.1
+    assert bench.hw_fp4_peak({"sm_mhz": None, "sm_max_mhz": 1800})[1] == 1800
+    assert bench.hw_fp4_peak(None)[1] == 1965
+
+
+def test_grouped_roofline_bytes_and_flops():
+    """The MoE grouped GEMMs' roofline: the up projection (K 4096 -> N 1536) and the
+    down projection (K 1536 -> N 4096) over 65536 routed rows move 578.8 MB and
+    820.0 MB (codes, scales, bf16 output) and each does 824.6 GFLOP."""
+    import types
+
+    import bench
+    step = types.SimpleNamespace(routed=65536)
+    pk = {"hbm_gbs": 6550.4, "source": "measured"}
+    r = bench.grouped_roofline([0.1, 0.2, 0.1, 0.2], 2, step, pk, 9529.6)
+    assert r["up"]["algorithmic_bytes"] == 578813952
+    assert r["down"]["algorithmic_bytes"] == 819986432
+    up_roof = max(2 * 65536 * 1536 * 4096 / 9529.6e12, 578813952 / 6550.4e9) * 1e6
+    assert abs(r["up"]["roofline_us"] - round(up_roof, 1)) < 0.11
+    assert abs(r["up"]["frac"] - up_roof / 100.0) < 1e-4

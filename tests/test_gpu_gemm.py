@@ -19,6 +19,14 @@ def nv():
     return nv
 
 
+@pytest.fixture(params=["256", "128"])
+def tile_n(request, monkeypatch):
+    """Both output-tile widths of the GEMM kernel: 256 (one accumulator) and 128 (two
+    accumulators in turn), forced through the library's tile override."""
+    monkeypatch.setenv("NVFP4_GEMM_TILE_N", request.param)
+    return int(request.param)
+
+
 def _operands(orc, nv, x, w, scaling_w=0):
     qa, sa, ga = orc.nvfp4_quantize(x, 0)
     qb, sb, gb = orc.nvfp4_quantize(w, 0, scaling=scaling_w)
@@ -27,7 +35,7 @@ def _operands(orc, nv, x, w, scaling_w=0):
     return (qa, sa, ga), (qb, sb, gb), A, B
 
 
-def test_tiny_linear_fp32(nv, orc):
+def test_tiny_linear_fp32(nv, orc, tile_n):
     """X 128x256 (1% outliers x50) times W^T 128x256, FP32 out, checked in full."""
     x, w = W.tiny_linear(0)
     (qa, sa, ga), (qb, sb, gb), A, B = _operands(orc, nv, x, w)
@@ -39,7 +47,7 @@ def test_tiny_linear_fp32(nv, orc):
 @pytest.mark.parametrize("mnk", [(256, 512, 512), (272, 400, 768), (128, 256, 256),
                                  (384, 128, 1024), (16, 16, 256)])
 @pytest.mark.parametrize("bf16_out", [False, True])
-def test_gemm_shapes(nv, orc, mnk, bf16_out):
+def test_gemm_shapes(nv, orc, tile_n, mnk, bf16_out):
     M, N, K = mnk
     rng = np.random.default_rng(M + N + K)
     x = W.f32_to_bf16_bits(W.student_t(rng, (M, K), 3.0, 1.0))
@@ -52,7 +60,7 @@ def test_gemm_shapes(nv, orc, mnk, bf16_out):
     check_gemm(D, Dr, Ar, bf16_out)
 
 
-def test_gemm_padded_ldd(nv, orc):
+def test_gemm_padded_ldd(nv, orc, tile_n):
     """Output with a leading dimension larger than N: the padding is left untouched."""
     import torch
     M, N, K = 128, 256, 512
@@ -117,7 +125,7 @@ def _grouped_case(orc, nv, counts, N, K, seed):
 
 @pytest.mark.parametrize("counts", [[0, 150, 7, 0, 33, 130], [128, 256], [1, 0, 303]])
 @pytest.mark.parametrize("bf16_out", [False, True])
-def test_grouped_gemm(nv, orc, counts, bf16_out):
+def test_grouped_gemm(nv, orc, tile_n, counts, bf16_out):
     N, K = 256, 512
     offsets, (qa, sa, ga), (qb, sb, gb), A, qb_d, sfb_d, gb_d, off_d = _grouped_case(
         orc, nv, counts, N, K, seed=sum(counts))
@@ -166,7 +174,7 @@ def test_grouped_gemm_moe_up_sampled(nv, orc):
 
 
 @pytest.mark.parametrize("bf16_out", [False, True])
-def test_gemm_amax_out(nv, orc, bf16_out):
+def test_gemm_amax_out(nv, orc, tile_n, bf16_out):
     """amax_out holds max |D| over the stored output, exactly, and replaces a stale value."""
     import torch
     M, N, K = 272, 400, 512
@@ -181,7 +189,7 @@ def test_gemm_amax_out(nv, orc, bf16_out):
     assert host(am)[0] == np.max(np.abs(D)).astype(np.float32)
 
 
-def test_grouped_gemm_amax_out(nv, orc):
+def test_grouped_gemm_amax_out(nv, orc, tile_n):
     """Grouped: the max covers every group's rows and nothing from padding tiles."""
     import torch
     N, K = 256, 512
@@ -221,7 +229,7 @@ def test_requantize_with_gemm_amax(nv, orc):
                                              grouped_padded_rows(offsets)), sf)
     assert float(host(got.g)[0]) == g
 
-def test_grouped_gemm_max_groups(nv, orc):
+def test_grouped_gemm_max_groups(nv, orc, tile_n):
     """256 groups (the limit), many of them empty, ragged counts; every row checked."""
     rng = np.random.default_rng(256)
     counts = [int(c) if rng.random() > 0.3 else 0 for c in rng.integers(1, 40, 256)]

@@ -572,6 +572,56 @@ def test_gemm_oracle_vs_numpy(orc):
     assert rel < 0.2
 
 
+def _mx_hat(q, e8):
+    """MXFP8 values from the bit-field grid of brute.py: E4M3 value x 2^(byte - 127)."""
+    grid = brute.e4m3_grid()
+    return grid[q] * np.repeat(2.0 ** (e8.astype(np.int64) - 127), 32, axis=1)
+
+
+def test_mxfp8_gemm_oracle_closed_form(orc):
+    """Hand-built MXFP8 operands whose product is known in closed form: every A
+    element is +-1.0 (E4M3 0x38 / 0xB8) and every B element 2.0 (0x40); block b of
+    A row i has scale 2^(i-b) and block b of B row j has 2^(j+b-1), so
+    D[i][j] = sum over blocks of 32 * s * 2^(i+j), s the block's sign."""
+    M, N, K = 3, 4, 128
+    signs = np.array([1, -1, 1, 1])
+    qa = np.repeat(np.where(signs > 0, 0x38, 0xB8), 32)[None, :].repeat(M, 0).astype(np.uint8)
+    e8a = np.array([[127 + i - b for b in range(4)] for i in range(M)], dtype=np.uint8)
+    qb = np.full((N, K), 0x40, dtype=np.uint8)
+    e8b = np.array([[127 + j + b - 1 for b in range(4)] for j in range(N)], dtype=np.uint8)
+    D, A = orc.mxfp8_gemm_rows(qa, e8a, qb, e8b)
+    for i in range(M):
+        for j in range(N):
+            assert D[i, j] == 32 * signs.sum() * 2.0 ** (i + j)
+            assert A[i, j] == 32 * 4 * 2.0 ** (i + j)
+    np.testing.assert_array_equal(orc.mxfp8_dequant(qa, e8a), _mx_hat(qa, e8a))
+
+
+def test_mxfp8_gemm_oracle_exact_and_numpy(orc):
+    """The MXFP8 GEMM reference on quantised heavy-tailed data: against exact rational
+    sums for sampled entries and against numpy on the brute-force dequantisation."""
+    rng = np.random.default_rng(31)
+    x = W.f32_to_bf16_bits(W.student_t(rng, (16, 96), 3.0))
+    w = W.f32_to_bf16_bits(W.normal(rng, (24, 96), 0.02))
+    qa, ea = orc.mxfp8_quantize(x, 0)
+    qb, eb = orc.mxfp8_quantize(w, 0)
+    D, A = orc.mxfp8_gemm_rows(qa, ea, qb, eb)
+    ah, bh = _mx_hat(qa, ea), _mx_hat(qb, eb)
+    for i in (0, 7, 15):
+        for j in (0, 11, 23):
+            exact = sum(Fraction(float(ah[i, k])) * Fraction(float(bh[j, k])) for k in range(96))
+            assert Fraction(D[i, j]) == exact       # every partial sum here is exact in FP64
+    np.testing.assert_allclose(D, ah @ bh.T, rtol=0, atol=1e-13 * A.max())
+    np.testing.assert_allclose(A, np.abs(ah) @ np.abs(bh).T, rtol=1e-13)
+    sel = np.array([9, 2])
+    Ds, _ = orc.mxfp8_gemm_rows(qa, ea, qb, eb, rows_sel=sel)
+    np.testing.assert_array_equal(Ds, D[sel])
+    xf = W.bf16_bits_to_f32(x).astype(np.float64)
+    wf = W.bf16_bits_to_f32(w).astype(np.float64)
+    rel = np.linalg.norm(D - xf @ wf.T) / np.linalg.norm(xf @ wf.T)
+    assert rel < 0.05                                # 8-bit operands track the bf16 product
+
+
 def test_grouped_gemm_oracle_matches_dense(orc):
     rng = np.random.default_rng(16)
     x = W.f32_to_bf16_bits(rng.standard_normal((40, 32)).astype(np.float32))
