@@ -444,6 +444,105 @@ def time_configs(dev, reps, warmup, pk, fp4_peak):
     return out
 
 
+def time_mxfp8_backward(step, steps, warmup, fp8_peak):
+    """The backward GEMMs of the dense layer in MXFP8 (the recipe on the iitak page,
+    "How it works": the backward pass in 8-bit MXFP8): dgrad dX = dY W (A = dY
+    rowwise, B = W columnwise) and wgrad dW = dY^T X (A = dY columnwise, B = X
+    columnwise), 16384 x 5120 x 20480 and 20480 x 5120 x 16384, on operands the
+    quantiser writes with tiled E8M0 scales from the resident bf16 tensors.  Each
+    GEMM launch and the dY quantisation (both directions, one pass) are timed apart
+    from the step with CUDA events after warm-up; inputs are larger than L2."""
+    nv, torch = step.nv, step.torch
+    inp = step.inputs[0]
+    T, H, F = TOKENS, HIDDEN, FFN
+    dev = inp["dy"].device
+    u8 = dict(dtype=torch.uint8, device=dev)
+    mk = lambda r, k: (torch.empty((r, k), **u8), torch.zeros(nv.mxfp8_sf_mma_bytes(r, k), **u8))
+    dyr, dyc, wc, xc = mk(T, F), mk(F, T), mk(H, F), mk(H, T)
+
+    def mxq(x, rows, cols, row, col):
+        p = nv.QuantParams()
+        p.mx_outputs = (nv.NVFP4_ROWWISE if row else 0) | (nv.NVFP4_COLWISE if col else 0)
+        p.mx_sf_layout = nv.NVFP4_SF_MMA
+        if row:
+            p.mx_q_row, p.mx_sf_row = row[0].data_ptr(), row[1].data_ptr()
+        if col:
+            p.mx_q_col, p.mx_sf_col = col[0].data_ptr(), col[1].data_ptr()
+        nv.nvfp4_quantize(x, rows, cols, cols, p, None, None, None, None, None, None,
+                          step.ws[0], 256)
+
+    mxq(inp["w"], F, H, None, wc)
+    mxq(inp["x"], T, H, None, xc)
+    stream = torch.cuda.current_stream()
+    runs = {"quant_dy": lambda: mxq(inp["dy"], T, F, dyr, dyc),
+            "dgrad": lambda: nv.mxfp8_gemm(dyr[0], dyr[1], wc[0], wc[1], T, H, F,
+                                           nv.NVFP4_OUT_BF16, step.dX, H, None, step.ws[4], 256),
+            "wgrad": lambda: nv.mxfp8_gemm(dyc[0], dyc[1], xc[0], xc[1], F, H, T,
+                                           nv.NVFP4_OUT_BF16, step.dW, H, None, step.ws[5], 256)}
+    ms = {}
+    for name, fn in runs.items():
+        for _ in range(max(warmup, 3)):
+            fn()
+        evs = []
+        for _ in range(steps):
+            s_, e_ = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            s_.record(stream)
+            fn()
+            e_.record(stream)
+            evs.append((s_, e_))
+        torch.cuda.synchronize()
+        ms[name] = sum(a.elapsed_time(b) for a, b in evs) / steps
+    step.check_status()
+    flop = 2 * T * H * F
+    tf = {k: flop / (ms[k] / 1e3) / 1e12 for k in ("dgrad", "wgrad")}
+    mean_tf = 2 * flop / ((ms["dgrad"] + ms["wgrad"]) / 1e3) / 1e12
+    n = T * F
+    qbytes = 2 * n + 2 * (n + n // 32)
+    return {"kernel": "gemm_kernel<MXFP8> (tcgen05 kind::mxf8f6f4, UE8M0 block-32 scales): dgrad "
+                      "16384x5120x20480 and wgrad 20480x5120x16384, bf16 out, timed apart from "
+                      "the step", "bound": "tensor",
+            "dgrad_us": round(ms["dgrad"] * 1e3, 1), "wgrad_us": round(ms["wgrad"] * 1e3, 1),
+            "dgrad_tflops": round(tf["dgrad"], 1), "wgrad_tflops": round(tf["wgrad"], 1),
+            "achieved": round(mean_tf, 1), "peak": round(fp8_peak, 1), "unit": "TFLOP/s",
+            "frac": round(mean_tf / fp8_peak, 4),
+            "peak_note": "dense FP8 tensor rate (half the FP4 rate: 16384 FLOP per SM per cycle) "
+                         "at the sampled SM clock",
+            "quant_dy_mxfp8_both_us": round(ms["quant_dy"] * 1e3, 1),
+            "quant_dy_mxfp8_both_gbs": round(qbytes / (ms["quant_dy"] / 1e3) / 1e9, 1)}
+
+
+def time_mxfp4_gemm(step, steps, warmup, fp4_peak):
+    """The dense layer's forward GEMM (16384 x 20480 x 5120) in MXFP4 (kind::mxf4, E8M0
+    scales per 32) on the resident x and W quantised by mxfp4_quantize with tiled scales,
+    timed apart from the step with CUDA events after warm-up; the OCP format the pages
+    set NVFP4 against."""
+    nv, torch = step.nv, step.torch
+    inp = step.inputs[0]
+    T, H, F = TOKENS, HIDDEN, FFN
+    (qa, sa), _ = nv.mxfp4(inp["x"], nv.NVFP4_ROWWISE, sf_layout=nv.NVFP4_SF_MMA)
+    (qb, sb), _ = nv.mxfp4(inp["w"], nv.NVFP4_ROWWISE, sf_layout=nv.NVFP4_SF_MMA)
+    run = lambda: nv.mxfp4_gemm(qa, sa, qb, sb, T, F, H, nv.NVFP4_OUT_BF16, step.Y, F, None,
+                                step.ws[2], 256)
+    for _ in range(max(warmup, 3)):
+        run()
+    stream = torch.cuda.current_stream()
+    evs = []
+    for _ in range(steps):
+        s_, e_ = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        s_.record(stream)
+        run()
+        e_.record(stream)
+        evs.append((s_, e_))
+    torch.cuda.synchronize()
+    step.check_status()
+    ms = sum(a.elapsed_time(b) for a, b in evs) / steps
+    tf = DENSE_FLOP_PER_GEMM / (ms / 1e3) / 1e12
+    return {"kernel": "gemm_kernel<MXFP4> (tcgen05 kind::mxf4, UE8M0 block-32 scales), "
+                      "16384x20480x5120, bf16 out, timed apart from the step", "bound": "tensor",
+            "us": round(ms * 1e3, 1), "achieved": round(tf, 1), "peak": round(fp4_peak, 1),
+            "unit": "TFLOP/s", "frac": round(tf / fp4_peak, 4)}
+
+
 def quant_algorithmic_bytes():
     """Bytes the dY quantisation must move: two reads of the bf16 input (amax pass and
     quantise pass), NVFP4 codes and scales in both directions, MXFP8 codes and scales."""
@@ -544,6 +643,7 @@ class ClockSampler:
 
 # ----------------------------------------------------------------------------- CPU oracle
 _SAMPLE_INPUTS = {}
+GEMM_SAMPLE_N = 2048
 
 
 def _sample_inputs():
@@ -559,7 +659,9 @@ def _sample_inputs():
     d["ws"] = W.f32_to_bf16_bits(W.normal(rng, (32, HIDDEN), 0.02))
     d["dys"] = W.f32_to_bf16_bits(W.student_t(rng, (32, FFN), 3.0))
     d["qa"] = orc.nvfp4_quantize(d["xs"], 0, amax=am)
-    d["qb"] = orc.nvfp4_quantize(W.f32_to_bf16_bits(W.normal(rng, (FFN, HIDDEN), 0.02)), 0)
+    # 2048 of the FFN rows of W: the GEMM piece's time scales with the rows it spans
+    d["qb"] = orc.nvfp4_quantize(W.f32_to_bf16_bits(W.normal(rng, (GEMM_SAMPLE_N, HIDDEN), 0.02)),
+                                 0)
     d["acts"] = W.f32_to_bf16_bits(W.normal(rng, (32, MOE_HIDDEN)))
     d["hs"] = W.f32_to_bf16_bits(W.normal(rng, (32, MOE_FFN)))
     d["qa2"] = orc.nvfp4_quantize(d["acts"], 0, amax=am)
@@ -600,7 +702,8 @@ def oracle_sample():
     # GEMM reference: 2 rows of each dense GEMM (same cost for the three shapes' K*N)
     qa, sa, ga = d["qa"]
     qb, sb, gb = d["qb"]
-    tq(lambda: orc.nvfp4_gemm_rows(qa, sa, ga, qb, sb, gb, rows_sel=[0, 1]), 3 * TOKENS / 2)
+    tq(lambda: orc.nvfp4_gemm_rows(qa, sa, ga, qb, sb, gb, rows_sel=[0, 1]),
+       3 * TOKENS / 2 * FFN / GEMM_SAMPLE_N)
     routed = MOE_TOKENS * TOPK
     # the tokens are quantised once, then dispatched; the up output is requantised
     tq(lambda: orc.nvfp4_quantize(d["acts"], 0, amax=am), MOE_TOKENS / 32)
@@ -612,8 +715,9 @@ def oracle_sample():
        2 * routed / 2)
     flops = DENSE_FLOP + 2 * 2 * routed * MOE_FFN * MOE_HIDDEN
     return {"value": flops / t_full / 1e12, "unit": "TFLOP/s", "cores": 1, "kind": "oracle",
-            "sample": ("each quantisation on 32-row slices, each GEMM on 2 output rows; per-piece "
-                       "time scaled to the full step"),
+            "sample": ("each quantisation on 32-row slices, each GEMM on 2 output rows (the dense "
+                       "GEMMs over 2048 of their output columns); per-piece time scaled to the "
+                       "full step"),
             "sample_seconds": round(sum(pieces), 2), "extrapolated_step_s": round(t_full, 1)}
 
 
@@ -826,6 +930,8 @@ def main():
     fp4_peak, fp4_mhz = hw_fp4_peak(clocks)
     derived_peak = 4.0 * pk["bf16_tflops"]
     cfgs = time_configs(dev, max(args.steps, 10), args.warmup, pk, fp4_peak)
+    mx8 = time_mxfp8_backward(step, args.steps, args.warmup, fp4_peak / 2)
+    mx4g = time_mxfp4_gemm(step, args.steps, args.warmup, fp4_peak)
     gd = per_kernel["gemm_dense"]
     gemm_ms = sum(gd) / len(gd)
     gemm_tflops = DENSE_FLOP_PER_GEMM / (gemm_ms / 1e3) / 1e12
@@ -876,7 +982,7 @@ def main():
             "grouped_gemm_roofline": grouped_roofline(per_kernel["gemm_grouped"], args.steps,
                                                       step, pk, fp4_peak),
             "configs": cfgs,
-            "next_rows": {"mxfp4_quantize": {
+            "next_rows": {"mxfp8_backward_gemm": mx8, "mxfp4_gemm": mx4g, "mxfp4_quantize": {
                 "bound": "hbm", "kernel": "mxfp4_kernel on dY 16384x20480, both directions "
                 "(timed apart from the step)", "ms": round(mx4_ms, 4),
                 "achieved": round(mx4_bytes / (mx4_ms / 1e3) / 1e9, 1), "peak": pk["hbm_gbs"],

@@ -252,14 +252,17 @@ nvfp4_status mxfp8_quantize(const void* x_bf16, int64_t rows, int64_t cols, int6
  * Codes two per byte, even index in the low nibble.
  * directions: NVFP4_ROWWISE (codes [rows, cols/2], scales [rows, cols/32])
  * and/or NVFP4_COLWISE (codes [cols, rows/2], scales [cols, rows/32]); both
- * come from one read of x.  rows and cols multiples of 32 (NVFP4_ERR_SHAPE);
+ * come from one read of x.  sf_layout: NVFP4_SF_ROWMAJOR, or NVFP4_SF_MMA (the
+ * 128x4 atoms of 32-blocks that mxfp4_gemm reads; bytes = mxfp8_sf_mma_bytes
+ * of the same shape; the block axis a multiple of 128).  rows and cols
+ * multiples of 32 (NVFP4_ERR_SHAPE);
  * x, q_row, q_col 16-byte aligned and ld a multiple of 8 (NVFP4_ERR_ALIGN);
  * a requested direction with a NULL output -> NVFP4_ERR_INVALID_ARG.  All
  * buffers are device memory owned by the caller; asynchronous on `stream`.
  */
 nvfp4_status mxfp4_quantize(const void* x_bf16, int64_t rows, int64_t cols, int64_t ld,
-                            int directions, uint8_t* q_row, uint8_t* e8_row, uint8_t* q_col,
-                            uint8_t* e8_col, void* stream);
+                            int directions, int sf_layout, uint8_t* q_row, uint8_t* e8_row,
+                            uint8_t* q_col, uint8_t* e8_col, void* stream);
 
 /*
  * nvfp4_gather_rows -- MoE dispatch of quantised rows (iitak, "Details" and
@@ -334,6 +337,23 @@ nvfp4_status mxfp8_gemm(const uint8_t* qa, const uint8_t* sfa, const uint8_t* qb
                         void* stream);
 
 /*
+ * mxfp4_gemm -- block-scaled MXFP4 GEMM on the tcgen05 tensor cores
+ * (kind::mxf4), the OCP format the pages compare NVFP4 against (hightech;
+ * asector, "NVFP4 and Blackwell"):
+ *   D[i][j] = sum_k (e2m1(a_ik) * 2^(ea(i, k/32) - 127)) * (e2m1(b_jk) * 2^(eb(j, k/32) - 127))
+ * with FP32 accumulation, no tensor scale.  "TN": qa [M, K/2], qb [N, K/2]
+ * E2M1 codes (even element in the low nibble); sfa / sfb E8M0 bytes in the
+ * tiled layout of mxfp4_quantize(..., NVFP4_SF_MMA, ...).  D [M, ldd] FP32 or
+ * bf16 (RNE); amax_out as for nvfp4_gemm.  Shapes: K a multiple of 256, M and
+ * N multiples of 16, ldd >= N with ldd * element size a multiple of 16 bytes;
+ * pointers 16-byte aligned (amax_out 4).  Errors as for nvfp4_gemm.
+ */
+nvfp4_status mxfp4_gemm(const uint8_t* qa, const uint8_t* sfa, const uint8_t* qb,
+                        const uint8_t* sfb, int64_t M, int64_t N, int64_t K, int out_dtype,
+                        void* D, int64_t ldd, float* amax_out, void* workspace, size_t ws_bytes,
+                        void* stream);
+
+/*
  * nvfp4_grouped_gemm -- MoE grouped form (iitak, "Details": NVFP4 in the
  * expert layers): rows [off[e], off[e+1]) of the stacked A [total_rows, K]
  * are multiplied by expert e's B_e [N, K]:
@@ -359,7 +379,8 @@ nvfp4_status nvfp4_workspace_status(void* workspace, void* stream);
 const char* nvfp4_status_string(nvfp4_status s);
 
 /* Library version: major * 10000 + minor * 100 + patch (200: adds mx_sf_layout
- * to nvfp4_quant_params, mxfp8_gemm and mxfp8_sf_mma_bytes). */
+ * to nvfp4_quant_params, the sf_layout argument of mxfp4_quantize, mxfp8_gemm,
+ * mxfp4_gemm and mxfp8_sf_mma_bytes). */
 int nvfp4_version(void);
 
 #ifdef __cplusplus

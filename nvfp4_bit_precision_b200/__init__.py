@@ -46,7 +46,7 @@ EXPORTED = [
     "nvfp4_quantize_workspace_size", "nvfp4_gemm_workspace_size", "nvfp4_sf_mma_bytes",
     "nvfp4_sf_mma_grouped_bytes", "nvfp4_workspace_status", "nvfp4_status_string",
     "nvfp4_version", "nvfp4_quantize_noalloc", "nvfp4_quantize_noalloc_status",
-    "nvfp4_gather_rows", "mxfp4_quantize", "mxfp8_gemm", "mxfp8_sf_mma_bytes",
+    "nvfp4_gather_rows", "mxfp4_quantize", "mxfp8_gemm", "mxfp8_sf_mma_bytes", "mxfp4_gemm",
 ]
 
 
@@ -73,7 +73,10 @@ _lib.nvfp4_quantize_noalloc.argtypes = [_P, _I64, _I64, _I64, ctypes.POINTER(Qua
                                         _P, _P, _P, _P, _P, _P]
 _lib.mxfp8_quantize.argtypes = [_P, _I64, _I64, _I64, ctypes.c_int, ctypes.c_int,
                                 ctypes.c_uint64, ctypes.c_uint32, _P, _P, _P, _P, _P]
-_lib.mxfp4_quantize.argtypes = [_P, _I64, _I64, _I64, ctypes.c_int, _P, _P, _P, _P, _P]
+_lib.mxfp4_quantize.argtypes = [_P, _I64, _I64, _I64, ctypes.c_int, ctypes.c_int, _P, _P, _P,
+                                _P, _P]
+_lib.mxfp4_gemm.argtypes = [_P, _P, _P, _P, _I64, _I64, _I64, ctypes.c_int, _P, _I64, _P, _P, _SZ,
+                            _P]
 _lib.nvfp4_dequantize.argtypes = [_P, _P, _P, _I64, _I64, ctypes.c_int, ctypes.c_int, _P, _P]
 _lib.nvfp4_gemm.argtypes = [_P, _P, _P, _P, _P, _P, _I64, _I64, _I64, ctypes.c_int, _P, _I64, _P,
                             _P, _SZ, _P]
@@ -99,7 +102,7 @@ _lib.nvfp4_status_string.argtypes = [ctypes.c_int]
 _lib.nvfp4_status_string.restype = ctypes.c_char_p
 _lib.nvfp4_version.restype = ctypes.c_int
 for _n in ("nvfp4_quantize", "nvfp4_quantize_noalloc", "mxfp8_quantize", "mxfp4_quantize",
-           "nvfp4_dequantize", "nvfp4_gemm", "mxfp8_gemm",
+           "nvfp4_dequantize", "nvfp4_gemm", "mxfp8_gemm", "mxfp4_gemm",
            "nvfp4_grouped_gemm", "nvfp4_gather_rows", "nvfp4_workspace_status",
            "nvfp4_quantize_noalloc_status"):
     getattr(_lib, _n).restype = ctypes.c_int
@@ -162,9 +165,17 @@ def mxfp8_quantize(x, rows, cols, ld, directions, rounding, seed, offset, q_row,
 
 
 def mxfp4_quantize(x, rows, cols, ld, directions, q_row, e8_row, q_col, e8_col,
-                   stream=None) -> None:
-    _check(_lib.mxfp4_quantize(_ptr(x), rows, cols, ld, directions, _ptr(q_row), _ptr(e8_row),
-                               _ptr(q_col), _ptr(e8_col), _stream(stream)), "mxfp4_quantize")
+                   stream=None, sf_layout=NVFP4_SF_ROWMAJOR) -> None:
+    _check(_lib.mxfp4_quantize(_ptr(x), rows, cols, ld, directions, sf_layout, _ptr(q_row),
+                               _ptr(e8_row), _ptr(q_col), _ptr(e8_col), _stream(stream)),
+           "mxfp4_quantize")
+
+
+def mxfp4_gemm(qa, sfa, qb, sfb, M, N, K, out_dtype, D, ldd, amax_out, workspace, ws_bytes,
+               stream=None) -> None:
+    _check(_lib.mxfp4_gemm(_ptr(qa), _ptr(sfa), _ptr(qb), _ptr(sfb), M, N, K, out_dtype, _ptr(D),
+                           ldd, _ptr(amax_out), _ptr(workspace), ws_bytes, _stream(stream)),
+           "mxfp4_gemm")
 
 
 def nvfp4_dequantize(q, sf, g, rows, cols, sf_layout, out_dtype, out, stream=None) -> None:
@@ -337,20 +348,43 @@ def mxfp8(x, directions: int = NVFP4_COLWISE, rounding: int = NVFP4_RNE, seed: i
     return (qr, er), (qc, ec)
 
 
-def mxfp4(x, directions: int = NVFP4_ROWWISE | NVFP4_COLWISE, stream=None):
+def mxfp4(x, directions: int = NVFP4_ROWWISE | NVFP4_COLWISE, stream=None,
+          sf_layout: int = NVFP4_SF_ROWMAJOR):
     """MXFP4 codes and E8M0 scales of a bf16 [rows, cols] tensor:
     ((q_row [rows, cols/2], e8 [rows, cols/32]) or (None, None),
-     (q_col [cols, rows/2], e8 [cols, rows/32]) or (None, None))."""
+     (q_col [cols, rows/2], e8 [cols, rows/32]) or (None, None)); with
+    sf_layout = NVFP4_SF_MMA the scales are flat tiled buffers (mxfp4_gemm's layout)."""
     import torch
     rows, cols = x.shape
     u8 = dict(dtype=torch.uint8, device=x.device)
+
+    def e8(r, k):
+        if sf_layout == NVFP4_SF_MMA:
+            return torch.zeros(mxfp8_sf_mma_bytes(r, k), **u8)
+        return torch.empty((r, k // 32), **u8)
+
     qr = er = qc = ec = None
     if directions & NVFP4_ROWWISE:
-        qr, er = torch.empty((rows, cols // 2), **u8), torch.empty((rows, cols // 32), **u8)
+        qr, er = torch.empty((rows, cols // 2), **u8), e8(rows, cols)
     if directions & NVFP4_COLWISE:
-        qc, ec = torch.empty((cols, rows // 2), **u8), torch.empty((cols, rows // 32), **u8)
-    mxfp4_quantize(x, rows, cols, x.stride(0), directions, qr, er, qc, ec, stream)
+        qc, ec = torch.empty((cols, rows // 2), **u8), e8(cols, rows)
+    mxfp4_quantize(x, rows, cols, x.stride(0), directions, qr, er, qc, ec, stream, sf_layout)
     return (qr, er), (qc, ec)
+
+
+def mx4_gemm(qa, sfa, qb, sfb, out_dtype: int = NVFP4_OUT_BF16, out=None, amax_out=None,
+             workspace=None, stream=None):
+    """D = A_hat B_hat^T of MXFP4 operands: qa [M, K/2], qb [N, K/2] codes with E8M0 scales
+    in the tiled layout (mxfp4(..., sf_layout=NVFP4_SF_MMA))."""
+    import torch
+    M, K = qa.shape[0], qa.shape[1] * 2
+    N = qb.shape[0]
+    dt = torch.bfloat16 if out_dtype == NVFP4_OUT_BF16 else torch.float32
+    D = out if out is not None else torch.empty((M, N), dtype=dt, device=qa.device)
+    ws = workspace if workspace is not None else _workspace(qa.device)
+    mxfp4_gemm(qa, sfa, qb, sfb, M, N, K, out_dtype, D, D.stride(0), amax_out, ws, ws.numel(),
+               stream)
+    return D
 
 
 def dequantize(t: NVFP4Tensor, out_dtype: int = NVFP4_OUT_F32, stream=None):

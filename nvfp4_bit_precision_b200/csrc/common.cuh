@@ -258,6 +258,34 @@ __device__ __forceinline__ U4 philox4x32_10_keyed(uint32_t c0, uint32_t c1, uint
     return U4{c0, c1, c2, c3};
 }
 
+// Two Philox4x32-10 blocks that differ only in the first two counter words,
+// computed round by round side by side (two independent dependency chains for
+// the scheduler to interleave).  Same results as two philox4x32_10_keyed calls.
+__device__ __forceinline__ void philox4x32_10_keyed_x2(uint32_t a0, uint32_t a1, uint32_t b0,
+                                                       uint32_t b1, uint32_t c2, uint32_t c3,
+                                                       const PhiloxKeys& k, U4& ra, U4& rb)
+{
+    uint32_t x0 = a0, x1 = a1, x2 = c2, x3 = c3;
+    uint32_t y0 = b0, y1 = b1, y2 = c2, y3 = c3;
+#pragma unroll
+    for (int r = 0; r < 10; ++r) {
+        const uint64_t p0 = static_cast<uint64_t>(x0) * 0xD2511F53u;
+        const uint64_t p1 = static_cast<uint64_t>(x2) * 0xCD9E8D57u;
+        const uint64_t q0 = static_cast<uint64_t>(y0) * 0xD2511F53u;
+        const uint64_t q1 = static_cast<uint64_t>(y2) * 0xCD9E8D57u;
+        x0 = static_cast<uint32_t>(p1 >> 32) ^ x1 ^ k.k0[r];
+        x2 = static_cast<uint32_t>(p0 >> 32) ^ x3 ^ k.k1[r];
+        x1 = static_cast<uint32_t>(p1);
+        x3 = static_cast<uint32_t>(p0);
+        y0 = static_cast<uint32_t>(q1 >> 32) ^ y1 ^ k.k0[r];
+        y2 = static_cast<uint32_t>(q0 >> 32) ^ y3 ^ k.k1[r];
+        y1 = static_cast<uint32_t>(q1);
+        y3 = static_cast<uint32_t>(q0);
+    }
+    ra = U4{x0, x1, x2, x3};
+    rb = U4{y0, y1, y2, y3};
+}
+
 // MXFP8 stream: random bits for elements idx8*8 .. idx8*8+7; element j takes
 // the 16-bit half (j % 2) of word j / 2.
 __device__ __forceinline__ U4 sr_block8(const PhiloxKeys& k, uint32_t offset, uint32_t stream,

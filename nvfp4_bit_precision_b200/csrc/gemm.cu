@@ -51,8 +51,10 @@ namespace nvfp4 {
 // Operand formats.  NVFP4: E2M1 codes, one UE4M3 scale per 16 elements
 // (kind::mxf4nvf4, block16).  MXFP8: E4M3 codes, one UE8M0 scale per 32
 // elements (kind::mxf8f6f4, block32) -- the backward-pass format of the
-// recipe on the iitak page, "How it works".
-enum : int { kFmtNVFP4 = 0, kFmtMXFP8 = 1 };
+// recipe on the iitak page, "How it works".  MXFP4: E2M1 codes, one UE8M0
+// scale per 32 elements (kind::mxf4, block32) -- the OCP format the pages
+// compare NVFP4 against (hightech page; asector page, "NVFP4 and Blackwell").
+enum : int { kFmtNVFP4 = 0, kFmtMXFP8 = 1, kFmtMXFP4 = 2 };
 
 constexpr int BM = 128;                    // A rows per CTA; a CTA pair covers 2 * BM
 constexpr int kMmaM = 2 * BM;              // M of the two-SM MMA
@@ -89,7 +91,7 @@ constexpr int kSmemShared = (int)((sizeof(GemmShared) + 1023) / 1024 * 1024);
 //  - kBN = 128: two 256x128 accumulators used in turn, so the MMAs of tile t+1
 //    run while the epilogue drains tile t.
 // Scale atoms (512 bytes: 128 rows x 4 scale bytes) per 128 rows and stage:
-// four for NVFP4 (16 scales per row), one for MXFP8 (4 scales per row).  In
+// four for NVFP4 (16 scales per row), two for MXFP4 (8), one for MXFP8 (4).  In
 // tensor memory each atom takes 4 columns per 128 rows (column c, lane i: row
 // 32c + i's 4 bytes, in every lane quadrant).
 template <int kFmt, int kBN>
@@ -97,8 +99,8 @@ struct GemmCfg {
     static constexpr int BN = kBN;
     static constexpr int kBRows = kBN / 2;  // B rows staged by each CTA
     static constexpr int kBlocksN = kBN / 128;
-    static constexpr int kSfAtoms = kFmt == kFmtNVFP4 ? 4 : 1;
-    static constexpr int kKStage = kFmt == kFmtNVFP4 ? 256 : 128;  // K elements per stage
+    static constexpr int kSfAtoms = kFmt == kFmtNVFP4 ? 4 : kFmt == kFmtMXFP4 ? 2 : 1;
+    static constexpr int kKStage = kFmt == kFmtMXFP8 ? 128 : 256;  // K elements per stage
     static constexpr int kKAtom = kFmt == kFmtNVFP4 ? 64 : 128;    // K elements per scale atom
     static constexpr int kA_Bytes = BM * 128;
     static constexpr int kB_Bytes = kBRows * 128;
@@ -142,6 +144,7 @@ struct GemmArgs {
     float* amax_out;  // optional: max |D| (as stored), atomically accumulated
     uint64_t wait_ns;  // limit of every barrier wait (2 s; shorter under the test hook)
     int no_copies;     // test hook: the producers issue no copy (see wait_test_hook)
+    int st32;          // D and its rows are 32-byte aligned: each lane stores 32-byte pieces
 };
 
 // ---------------------------------------------------------------- PTX wrappers
@@ -241,12 +244,13 @@ __device__ __forceinline__ uint64_t desc_sw128(const void* p)
 // Instruction descriptor of a block-scaled MMA, M = 256 (the pair), N = kBN,
 // both operands K-major, dense.  NVFP4: A/B format E2M1 (1), UE4M3 scales
 // (bit 23 clear).  MXFP8: A/B format E4M3 (0), UE8M0 scales (bit 23 set).
-// sf_id picks the byte of each 32-bit scale column an MXFP8 MMA reads (its
-// 32-element block within the atom's 128); NVFP4 reads all four bytes.
+// MXFP4: E2M1 (1), UE8M0.  sf_id is the first byte of each 32-bit scale column
+// the MMA reads: an MXFP8 MMA (K 32) reads byte sf_id = 0..3, an MXFP4 MMA
+// (K 64) the two bytes from sf_id = 0 or 2; NVFP4 reads all four (sf_id 0).
 template <int kFmt, int kBN>
 __host__ __device__ constexpr uint32_t make_idesc(uint32_t sf_id)
 {
-    const uint32_t fmt = kFmt == kFmtNVFP4 ? 1u : 0u;
+    const uint32_t fmt = kFmt == kFmtMXFP8 ? 0u : 1u;
     const uint32_t e8m0 = kFmt == kFmtNVFP4 ? 0u : 1u;
     return (sf_id << 4) | (fmt << 7) | (fmt << 10) | ((uint32_t)(kBN >> 3) << 17) | (e8m0 << 23) |
            ((uint32_t)(kMmaM >> 4) << 24) | (sf_id << 29);
@@ -265,11 +269,19 @@ __device__ __forceinline__ void tc_mma(uint32_t d_tmem, uint64_t adesc, uint64_t
             "}" ::"r"(d_tmem),
             "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate), "r"(sfa_tmem), "r"(sfb_tmem)
             : "memory");
-    } else {
+    } else if constexpr (kFmt == kFmtMXFP8) {
         asm volatile(
             "{\n\t.reg .pred p;\n\t"
             "setp.ne.b32 p, %4, 0;\n\t"
             "tcgen05.mma.cta_group::2.kind::mxf8f6f4.block_scale.block32 [%0], %1, %2, %3, [%5], [%6], p;\n\t"
+            "}" ::"r"(d_tmem),
+            "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate), "r"(sfa_tmem), "r"(sfb_tmem)
+            : "memory");
+    } else {
+        asm volatile(
+            "{\n\t.reg .pred p;\n\t"
+            "setp.ne.b32 p, %4, 0;\n\t"
+            "tcgen05.mma.cta_group::2.kind::mxf4.block_scale.block32 [%0], %1, %2, %3, [%5], [%6], p;\n\t"
             "}" ::"r"(d_tmem),
             "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate), "r"(sfa_tmem), "r"(sfb_tmem)
             : "memory");
@@ -309,6 +321,11 @@ __device__ __forceinline__ void tmem_store_words(uint32_t taddr, const uint32_t*
         TMEM_ST_32(taddr + 16, (v + 16));
     } else if constexpr (N == 32) {
         TMEM_ST_32(taddr, v);
+    } else if constexpr (N == 16) {
+        TMEM_ST_16(taddr, v);
+    } else if constexpr (N == 24) {
+        TMEM_ST_16(taddr, v);
+        TMEM_ST_8(taddr + 16, (v + 16));
     } else if constexpr (N == 12) {
         TMEM_ST_8(taddr, v);
         TMEM_ST_4(taddr + 8, (v + 8));
@@ -317,6 +334,16 @@ __device__ __forceinline__ void tmem_store_words(uint32_t taddr, const uint32_t*
     } else {
         static_assert(N == 0, "unsupported scale-column count");
     }
+}
+
+// 32 bytes (8 words) to global memory in one instruction, marked to leave L2
+// first: the output streams past while the operand tiles stay resident.
+__device__ __forceinline__ void st_global_v8_ef(void* p, const uint32_t* v)
+{
+    asm volatile("st.global.L2::evict_first.v8.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8};" ::"l"(p),
+                 "r"(v[0]), "r"(v[1]), "r"(v[2]), "r"(v[3]), "r"(v[4]), "r"(v[5]), "r"(v[6]),
+                 "r"(v[7])
+                 : "memory");
 }
 
 __device__ __forceinline__ void tmem_ld_wait() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory"); }
@@ -520,10 +547,13 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
                     for (int j = 0; j < 4; ++j) {
                         // +32 bytes along K inside the swizzled row: 64 FP4 or 32 FP8
                         // elements.  NVFP4: atom j's columns; MXFP8: byte j of the
-                        // stage's one atom.
-                        const uint32_t aj = kFmt == kFmtNVFP4 ? (uint32_t)j : 0u;
-                        tc_mma<kFmt>(d_tmem, ad + 2 * j, bd + 2 * j,
-                                     make_idesc<kFmt, kBN>(kFmt == kFmtNVFP4 ? 0u : (uint32_t)j),
+                        // stage's one atom; MXFP4: bytes 2(j%2), 2(j%2)+1 of atom j/2.
+                        const uint32_t aj = kFmt == kFmtNVFP4 ? (uint32_t)j
+                                            : kFmt == kFmtMXFP4 ? (uint32_t)(j >> 1) : 0u;
+                        const uint32_t sf_id = kFmt == kFmtNVFP4 ? 0u
+                                               : kFmt == kFmtMXFP4 ? 2u * (uint32_t)(j & 1)
+                                                                   : (uint32_t)j;
+                        tc_mma<kFmt>(d_tmem, ad + 2 * j, bd + 2 * j, make_idesc<kFmt, kBN>(sf_id),
                                      t_sfa + 4 * aj, t_sfb + 4 * C::kBlocksN * aj,
                                      (ks > 0 || j > 0) ? 1u : 0u);
                     }
@@ -641,6 +671,17 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
                             }
                     }
                 }
+                if (a.st32) {
+                    // each lane stores its own row in 32-byte pieces (16 columns):
+                    // whole sectors without a shared-memory turnaround
+                    if (row_ok) {
+                        uint16_t* drow = static_cast<uint16_t*>(a.D) + row * a.ldd + cbase;
+#pragma unroll
+                        for (int g = 0; g < 2 * kChunks; ++g)
+                            if (cbase + 16 * g < a.N) st_global_v8_ef(drow + 16 * g, packed + 8 * g);
+                    }
+                    continue;
+                }
                 const int64_t rowbase = c.row0 + (int64_t)BM * rank + 32 * quad;
                 // 32-column chunks through a 64-byte-swizzled 32x64-byte staging
                 // block: each lane writes its row, then 8 rows x 64 bytes leave
@@ -686,9 +727,21 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
                     const float x1 = __fmul_rn(__uint_as_float(r[4 * v + 1]), alpha);
                     const float x2 = __fmul_rn(__uint_as_float(r[4 * v + 2]), alpha);
                     const float x3 = __fmul_rn(__uint_as_float(r[4 * v + 3]), alpha);
-                    if (cbase + 4 * v < a.N) {
-                        *reinterpret_cast<float4*>(drow + 4 * v) = make_float4(x0, x1, x2, x3);
-                        out_max = absmax3(out_max, absmax3(x0, x1, x2), x3);
+                    r[4 * v] = __float_as_uint(x0), r[4 * v + 1] = __float_as_uint(x1);
+                    r[4 * v + 2] = __float_as_uint(x2), r[4 * v + 3] = __float_as_uint(x3);
+                    if (cbase + 4 * v < a.N) out_max = absmax3(out_max, absmax3(x0, x1, x2), x3);
+                }
+                // N is a multiple of 16, so an 8-column piece is stored whole or not at all
+#pragma unroll
+                for (int v = 0; v < 4; ++v) {
+                    if (cbase + 8 * v >= a.N) continue;
+                    if (a.st32) {
+                        st_global_v8_ef(drow + 8 * v, r + 8 * v);
+                    } else {
+                        reinterpret_cast<uint4*>(drow + 8 * v)[0] =
+                            make_uint4(r[8 * v], r[8 * v + 1], r[8 * v + 2], r[8 * v + 3]);
+                        reinterpret_cast<uint4*>(drow + 8 * v)[1] =
+                            make_uint4(r[8 * v + 4], r[8 * v + 5], r[8 * v + 6], r[8 * v + 7]);
                     }
                 }
             }
@@ -799,22 +852,26 @@ static GemmDevice& gemm_device(int dev)
 }
 
 static bool al16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+static bool al32(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 31u) == 0; }
 
 constexpr size_t kGemmWorkspace = 256;
 
 // Output-tile width.  256 (one accumulator) moves the fewest operand bytes per
-// FLOP; 128 (two accumulators) hides the epilogue's drain, which matters when
-// tiles are short along K.  NVFP4_GEMM_TILE_N=128 or 256 in the environment
-// overrides the choice (read on every call).
+// FLOP; 128 (two accumulators) hides the epilogue's drain but moves 1.5x the
+// operand bytes per FLOP, and measured 30-45% slower on every shape of the
+// workloads (dense, grouped, MXFP8), so 256 is the default.
+// NVFP4_GEMM_TILE_N=128 or 256 in the environment overrides the choice (read
+// on every call).
 static int pick_tile_n(bool grouped, int64_t K, int k_stage)
 {
     if (const char* e = getenv("NVFP4_GEMM_TILE_N")) {
         if (!strcmp(e, "128")) return 128;
         if (!strcmp(e, "256")) return 256;
     }
+    (void)grouped;
     (void)K;
     (void)k_stage;
-    return grouped ? 128 : 256;
+    return 256;  // measured faster for every shape of the workloads, dense and grouped
 }
 
 template <int kFmt, int kBN>
@@ -827,7 +884,7 @@ static nvfp4_status launch_variant(const void* qa, const void* qb, GemmArgs& a, 
     wait_test_hook(&a.wait_ns, &a.no_copies);
     GemmDevice& info = gemm_device<kFmt, kBN>(dev);
     if (!info.ok) return NVFP4_ERR_UNSUPPORTED;
-    const int64_t kbytes = kFmt == kFmtNVFP4 ? a.K / 2 : a.K;
+    const int64_t kbytes = kFmt == kFmtMXFP8 ? a.K : a.K / 2;
     CUtensorMap ma, mb, msf;
     memset(&msf, 0, sizeof(msf));
     if (!make_map(&ma, qa, a_rows, kbytes, BM) || !make_map(&mb, qb, b_rows, kbytes, C::kBRows))
@@ -903,6 +960,7 @@ extern "C" nvfp4_status nvfp4_gemm(const uint8_t* qa, const uint8_t* sfa, const 
     a.G = 1;
     a.status = static_cast<uint32_t*>(workspace) + 2;
     a.amax_out = amax_out;
+    a.st32 = al32(D) && (ldd * (a.bf16_out ? 2 : 4)) % 32 == 0;
     return launch_gemm<kFmtNVFP4>(qa, qb, a, M, N, (M + kMmaM - 1) / kMmaM,
                                   static_cast<cudaStream_t>(stream));
 }
@@ -928,7 +986,34 @@ extern "C" nvfp4_status mxfp8_gemm(const uint8_t* qa, const uint8_t* sfa, const 
     a.G = 1;
     a.status = static_cast<uint32_t*>(workspace) + 2;
     a.amax_out = amax_out;
+    a.st32 = al32(D) && (ldd * (a.bf16_out ? 2 : 4)) % 32 == 0;
     return launch_gemm<kFmtMXFP8>(qa, qb, a, M, N, (M + kMmaM - 1) / kMmaM,
+                                  static_cast<cudaStream_t>(stream));
+}
+
+extern "C" nvfp4_status mxfp4_gemm(const uint8_t* qa, const uint8_t* sfa, const uint8_t* qb,
+                                   const uint8_t* sfb, int64_t M, int64_t N, int64_t K,
+                                   int out_dtype, void* D, int64_t ldd, float* amax_out,
+                                   void* workspace, size_t ws_bytes, void* stream)
+{
+    const nvfp4_status chk = check_dense(qa, sfa, qb, sfb, M, N, K, 256, out_dtype, D, ldd,
+                                         amax_out, workspace, ws_bytes);
+    if (chk != NVFP4_OK) return chk;
+    GemmArgs a{};
+    a.sfa = sfa;
+    a.sfb = sfb;
+    a.D = D;
+    a.M = M;
+    a.N = N;
+    a.K = K;
+    a.ldd = ldd;
+    a.bf16_out = out_dtype == NVFP4_OUT_BF16;
+    a.grouped = 0;
+    a.G = 1;
+    a.status = static_cast<uint32_t*>(workspace) + 2;
+    a.amax_out = amax_out;
+    a.st32 = al32(D) && (ldd * (a.bf16_out ? 2 : 4)) % 32 == 0;
+    return launch_gemm<kFmtMXFP4>(qa, qb, a, M, N, (M + kMmaM - 1) / kMmaM,
                                   static_cast<cudaStream_t>(stream));
 }
 
@@ -967,6 +1052,7 @@ extern "C" nvfp4_status nvfp4_grouped_gemm(int G, const int32_t* group_offsets, 
     a.total_rows = total_rows;
     a.status = static_cast<uint32_t*>(workspace) + 2;
     a.amax_out = amax_out;
+    a.st32 = al32(D);  // ldd = N, a multiple of 128
     // upper bound on M tiles: every group may add one partial tile
     return launch_gemm<kFmtNVFP4>(qa, qb, a, total_rows, (int64_t)G * N,
                                   (total_rows + kMmaM - 1) / kMmaM + G,

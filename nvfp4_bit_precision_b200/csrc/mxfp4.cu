@@ -43,7 +43,14 @@ struct Mx4Args {
     uint8_t* q_col;
     uint8_t* e8_col;
     int64_t tiles_r, tiles_c;
+    int mma_sf;  // scale bytes in the tensor cores' tiled layout (128x4 atoms of 32-blocks)
 };
+
+// Offset of the E8M0 byte of 32-block b of row r in a [rows, nblk] scale tensor.
+__device__ __forceinline__ int64_t mx4_sf_off(const Mx4Args& a, int64_t r, int64_t b, int64_t nblk)
+{
+    return a.mma_sf ? sf_mma_offset(r, b, nblk) : r * nblk + b;
+}
 
 // E8M0 byte of a block with absolute maximum am, and the exact factor 2^-e
 // its elements are multiplied by.  floor(log2 am) is the unbiased exponent
@@ -149,9 +156,8 @@ __device__ __forceinline__ void mx4_tile(const Mx4Args& a, int64_t t, const uint
         {
             const int c = threadIdx.x;  // 0..127: column c's scale bytes
             if (c < nc) {
-                uint8_t* e = a.e8_col + (c0 + c) * (a.rows / 32) + r0 / 32;
-                e[0] = stg_e8[2 * c];
-                if (nr > 32) e[1] = stg_e8[2 * c + 1];
+                a.e8_col[mx4_sf_off(a, c0 + c, r0 / 32, a.rows / 32)] = stg_e8[2 * c];
+                if (nr > 32) a.e8_col[mx4_sf_off(a, c0 + c, r0 / 32 + 1, a.rows / 32)] = stg_e8[2 * c + 1];
             }
         }
     } else {
@@ -182,7 +188,7 @@ __device__ __forceinline__ void mx4_tile(const Mx4Args& a, int64_t t, const uint
                            mx4_codes8(p[1].x, p[1].y, p[1].z, p[1].w, f),
                            mx4_codes8(p[2].x, p[2].y, p[2].z, p[2].w, f),
                            mx4_codes8(p[3].x, p[3].y, p[3].z, p[3].w, f));
-            a.e8_row[row * (a.cols / 32) + cg / 32] = (uint8_t)e8;
+            a.e8_row[mx4_sf_off(a, row, cg / 32, a.cols / 32)] = (uint8_t)e8;
         }
     }
 }
@@ -236,13 +242,16 @@ int mx4_grid(int dev)
 using namespace nvfp4;
 
 extern "C" nvfp4_status mxfp4_quantize(const void* x_bf16, int64_t rows, int64_t cols, int64_t ld,
-                                       int directions, uint8_t* q_row, uint8_t* e8_row,
-                                       uint8_t* q_col, uint8_t* e8_col, void* stream)
+                                       int directions, int sf_layout, uint8_t* q_row,
+                                       uint8_t* e8_row, uint8_t* q_col, uint8_t* e8_col,
+                                       void* stream)
 {
     if (!x_bf16 || directions == 0 || (directions & ~3)) return NVFP4_ERR_INVALID_ARG;
+    if (sf_layout != NVFP4_SF_ROWMAJOR && sf_layout != NVFP4_SF_MMA) return NVFP4_ERR_INVALID_ARG;
     const bool row = (directions & NVFP4_ROWWISE) != 0, col = (directions & NVFP4_COLWISE) != 0;
     if ((row && (!q_row || !e8_row)) || (col && (!q_col || !e8_col))) return NVFP4_ERR_INVALID_ARG;
     if (rows <= 0 || cols <= 0 || rows % 32 || cols % 32 || ld < cols) return NVFP4_ERR_SHAPE;
+    if (sf_layout == NVFP4_SF_MMA && ((row && cols % 128) || (col && rows % 128))) return NVFP4_ERR_SHAPE;
     if (rows > ((int64_t)1 << 31) || cols > ((int64_t)1 << 31)) return NVFP4_ERR_SHAPE;
     if (!aligned16_ptr(x_bf16) || ld % 8 || (row && !aligned16_ptr(q_row)) ||
         (col && !aligned16_ptr(q_col)))
@@ -265,6 +274,7 @@ extern "C" nvfp4_status mxfp4_quantize(const void* x_bf16, int64_t rows, int64_t
     a.e8_col = col ? e8_col : nullptr;
     a.tiles_r = tiles_r;
     a.tiles_c = tiles_c;
+    a.mma_sf = sf_layout == NVFP4_SF_MMA;
     const int64_t n_tiles = tiles_r * tiles_c;
     mxfp4_kernel<<<(unsigned)(n_tiles < grid ? n_tiles : grid), kMx4Threads, 0,
                    static_cast<cudaStream_t>(stream)>>>(a);

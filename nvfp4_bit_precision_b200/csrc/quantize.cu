@@ -41,12 +41,10 @@ constexpr int kStages = 2;
 // bytes per column) and NVFP4 columnwise codes (16 bytes per column).
 constexpr int kMxStageBytes = 64 * 32;
 constexpr int kQcStageBytes = 64 * 16;
-// The fused pass runs 12 warps per CTA (2 CTAs, 24 warps per SM at <= 80
-// registers a thread): when a tile feeds both directions, warps 0..7 take the
-// columnwise work (one column pair x 32 rows each) and warps 8..11 the rowwise
-// work (two row halves each); with one direction only, warps 0..7 take it and
-// warps 8..11 only release the stage.  The amax pass keeps 8 warps.
-constexpr int kQuantThreads = 384;
+// Both passes run 8 warps per CTA, 2 CTAs per SM.  (Measured: 12-warp CTAs at
+// 80 registers, with the rowwise and columnwise work on separate warps, made
+// the fused gradient pass 13% slower.)
+constexpr int kQuantThreads = 256;
 constexpr int kColWarps = 8;
 constexpr int kAmaxThreads = 256;
 constexpr int kMaxGroups = 256;  // MoE groups per call (the grouped GEMM's limit too)
@@ -226,41 +224,68 @@ __device__ __forceinline__ void unpack8(const uint4& p, float* v)
     v[7] = bf16_hi(p.w);
 }
 
-// Quantise one 16-value block given its (possibly 2D-reduced) amax.
-// Returns the scale byte; writes 8 code bytes to c0/c1.  times4: v and amax_b
-// hold 4x the values (Hadamard path without its factor 1/4); the factor is
-// applied here exactly: amax_b/4 never rounds, and v*(r/4) == (v/4)*r whenever
-// r/4 is a normal float (otherwise the division is done per element).
-__device__ __forceinline__ uint32_t quant_block16(float (&v)[16], float amax_b, float S,
-                                                  const float* rtab, bool times4, bool sr,
-                                                  const PhiloxKeys& pk, uint32_t offset,
-                                                  uint32_t stream, uint64_t idx, uint32_t& c0,
-                                                  uint32_t& c1)
+// Quantisation of 16-value blocks given their (possibly 2D-reduced) amax:
+// scale byte = E4M3_RNE((amax_b / 6) * S), r = RN(S / d) from the per-CTA table,
+// codes = RNE or SR of x * r.  times4: v and amax_b hold 4x the values (Hadamard
+// path without its factor 1/4); the factor is applied here exactly: amax_b/4
+// never rounds, and v*(r/4) == (v/4)*r whenever r/4 is a normal float
+// (otherwise the division is done per element).
+// Two blocks at once (v and w, with their amax): both scale bytes from one
+// paired E4M3 conversion and both Philox blocks computed side by side.  Returns
+// the scale bytes (v's in bits 0..7, w's in bits 8..15); the codes go to
+// cv0/cv1 and cw0/cw1.
+__device__ __forceinline__ uint32_t quant_block16x2(float (&v)[16], float (&w)[16], float am_v,
+                                                    float am_w, float S, const float* rtab,
+                                                    bool times4, bool sr, const PhiloxKeys& pk,
+                                                    uint32_t offset, uint32_t stream,
+                                                    uint64_t idx_v, uint64_t idx_w, uint32_t& cv0,
+                                                    uint32_t& cv1, uint32_t& cw0, uint32_t& cw1)
 {
-    if (times4) amax_b = __fmul_rn(amax_b, 0.25f);
-    const float s = __fmul_rn(__fdiv_rn(amax_b, 6.0f), S);
-    const uint32_t byte = e4m3_rne_sat(s);
-    float r = rtab[byte];  // RN(S / d); 0 when d = 0, so every y is +-0
     if (times4) {
-        if (r >= 7.52316384526264005100e-37f) {  // 2^-120: r/4 stays normal
-            r = __fmul_rn(r, 0.25f);
+        am_v = __fmul_rn(am_v, 0.25f);
+        am_w = __fmul_rn(am_w, 0.25f);
+    }
+    const float sv = __fmul_rn(__fdiv_rn(am_v, 6.0f), S);
+    const float sw = __fmul_rn(__fdiv_rn(am_w, 6.0f), S);
+    const uint32_t bytes = e4m3x2_rne_sat(sw, sv) & 0xFFFFu;
+    float rv = rtab[bytes & 0xFFu], rw = rtab[bytes >> 8];  // RN(S / d); 0 when d = 0
+    if (times4) {
+        if (rv >= 7.52316384526264005100e-37f) {  // 2^-120: r/4 stays normal
+            rv = __fmul_rn(rv, 0.25f);
         } else {
 #pragma unroll
             for (int i = 0; i < 16; ++i) v[i] = __fmul_rn(v[i], 0.25f);
         }
+        if (rw >= 7.52316384526264005100e-37f) {
+            rw = __fmul_rn(rw, 0.25f);
+        } else {
+#pragma unroll
+            for (int i = 0; i < 16; ++i) w[i] = __fmul_rn(w[i], 0.25f);
+        }
     }
 #pragma unroll
-    for (int i = 0; i < 16; i += 2) mul2(v[i], v[i + 1], v[i], v[i + 1], r, r);
+    for (int i = 0; i < 16; i += 2) {
+        mul2(v[i], v[i + 1], v[i], v[i + 1], rv, rv);
+        mul2(w[i], w[i + 1], w[i], w[i + 1], rw, rw);
+    }
     if (sr) {
         // one Philox call per 16-element block: word q drives elements 4q..4q+3
-        const U4 w = sr_block16(pk, offset, stream, idx >> 4);
-        c0 = e2m1x4_sr(v + 0, w.x) | (e2m1x4_sr(v + 4, w.y) << 16);
-        c1 = e2m1x4_sr(v + 8, w.z) | (e2m1x4_sr(v + 12, w.w) << 16);
+        U4 a, b;
+        const uint64_t jv = idx_v >> 4, jw = idx_w >> 4;
+        philox4x32_10_keyed_x2(static_cast<uint32_t>(jv), static_cast<uint32_t>(jv >> 32),
+                               static_cast<uint32_t>(jw), static_cast<uint32_t>(jw >> 32), stream,
+                               offset, pk, a, b);
+        cv0 = e2m1x4_sr(v + 0, a.x) | (e2m1x4_sr(v + 4, a.y) << 16);
+        cv1 = e2m1x4_sr(v + 8, a.z) | (e2m1x4_sr(v + 12, a.w) << 16);
+        cw0 = e2m1x4_sr(w + 0, b.x) | (e2m1x4_sr(w + 4, b.y) << 16);
+        cw1 = e2m1x4_sr(w + 8, b.z) | (e2m1x4_sr(w + 12, b.w) << 16);
     } else {
-        c0 = e2m1x8_rne(v);
-        c1 = e2m1x8_rne(v + 8);
+        cv0 = e2m1x8_rne(v);
+        cv1 = e2m1x8_rne(v + 8);
+        cw0 = e2m1x8_rne(w);
+        cw1 = e2m1x8_rne(w + 8);
     }
-    return byte;
+    return bytes;
 }
 
 // MXFP8 of 32 values: returns the E8M0 byte, writes 32 code bytes to out[8].
@@ -659,18 +684,9 @@ __global__ void __launch_bounds__(kQuantThreads, 2)
         const int64_t tr = tile_row(a, tile), tc = tile - tr * a.tiles_c;
         const int64_t r0 = tr * kTileRows, c0 = tc * kTileCols;
 
-        // ---------------- rowwise: item = (row, 64-column half) ------------
-        // Item i (0..255) is row 16*(i/32) + i%16, half (i%32)/16, so the 16
-        // lanes of a half-warp hold 16 consecutive rows (a 16x16 tile for 2D).
-        // Both directions: warps 8..11 take items i and i + 128; rowwise
-        // only: warps 0..7 take one item each.
-        const bool both_dirs = (nv_row || mx_row) && (nv_col || mx_col);
-        const int row_warp0 = both_dirs ? kColWarps : 0;
-        const int row_items = both_dirs ? 2 : 1;
-        if ((nv_row || mx_row) && warp >= row_warp0 && warp < row_warp0 + 8 / row_items)
-#pragma unroll 1
-        for (int ri = 0; ri < row_items; ++ri) {
-            const int rl = 16 * (warp - row_warp0 + 4 * ri) + (lane & 15);
+        // ---------------- rowwise: thread = (row, 64-column half) ----------
+        if (nv_row || mx_row) {
+            const int rl = 16 * warp + (lane & 15);
             const int h = lane >> 4;
             const int64_t rg = r0 + rl;
             const bool rvalid = rg < a.rows;
@@ -684,22 +700,25 @@ __global__ void __launch_bounds__(kQuantThreads, 2)
                 uint32_t sfw = 0;
                 bool all_valid = true;
 #pragma unroll
-                for (int blk = 0; blk < 4; ++blk) {
-                    const int64_t cg = cbase + 16 * blk;
-                    const bool valid = rvalid && cg < a.cols;
-                    all_valid &= valid;
-                    float v[16];
-                    unpack8(ld_shared_v4(chunk_addr<kTma>(T, rl, 8 * h + 2 * blk)), v);
-                    unpack8(ld_shared_v4(chunk_addr<kTma>(T, rl, 8 * h + 2 * blk + 1)), v + 8);
-                    float am = absmax16(v, 0.0f);
-                    if (two_d) am = warp_max16(am);
-                    uint32_t cw0, cw1;
-                    const uint32_t byte = quant_block16(v, am, S_row, sh->rtab[0], false, sr && valid, a.pk,
-                                                        a.offset, 0u,
-                                                        (uint64_t)(rg * a.cols + cg), cw0, cw1);
-                    codes[2 * blk] = cw0;
-                    codes[2 * blk + 1] = cw1;
-                    sfw |= byte << (8 * blk);
+                for (int bp = 0; bp < 4; bp += 2) {  // two 16-blocks at a time
+                    const int64_t cg = cbase + 16 * bp;
+                    all_valid &= rvalid && cg + 16 < a.cols;
+                    float v[16], w[16];
+                    unpack8(ld_shared_v4(chunk_addr<kTma>(T, rl, 8 * h + 2 * bp)), v);
+                    unpack8(ld_shared_v4(chunk_addr<kTma>(T, rl, 8 * h + 2 * bp + 1)), v + 8);
+                    unpack8(ld_shared_v4(chunk_addr<kTma>(T, rl, 8 * h + 2 * bp + 2)), w);
+                    unpack8(ld_shared_v4(chunk_addr<kTma>(T, rl, 8 * h + 2 * bp + 3)), w + 8);
+                    float amv = absmax16(v, 0.0f), amw = absmax16(w, 0.0f);
+                    if (two_d) {
+                        amv = warp_max16(amv);
+                        amw = warp_max16(amw);
+                    }
+                    const uint64_t idx = (uint64_t)(rg * a.cols + cg);
+                    const uint32_t bytes = quant_block16x2(
+                        v, w, amv, amw, S_row, sh->rtab[0], false, sr && rvalid && cg < a.cols, a.pk,
+                        a.offset, 0u, idx, idx + 16, codes[2 * bp], codes[2 * bp + 1],
+                        codes[2 * bp + 2], codes[2 * bp + 3]);
+                    sfw |= bytes << (8 * bp);
                 }
                 if (all_valid) {
                     store_codes32(a.q_row + rg * (a.cols / 2) + cbase / 2, codes, q_row_vec);
@@ -746,10 +765,9 @@ __global__ void __launch_bounds__(kQuantThreads, 2)
         }
 
         // ---------------- columnwise: thread = (column pair, 32-row group) --
-        // Warps 0..7.  One 32-bit shared load per row gives both columns of
-        // the pair; the pair's two Hadamard transforms run in the two lanes of
-        // f32x2.
-        if ((nv_col || mx_col) && warp < kColWarps) {
+        // One 32-bit shared load per row gives both columns of the pair; the
+        // pair's two Hadamard transforms run in the two lanes of f32x2.
+        if (nv_col || mx_col) {
             const int cp = 32 * (warp & 1) + lane;  // column pair 0..63
             const int rgrp = warp >> 1;              // 32-row group 0..3
             const int64_t cg0 = c0 + 2 * cp;         // columns cg0, cg0 + 1
@@ -801,12 +819,11 @@ __global__ void __launch_bounds__(kQuantThreads, 2)
                         ama = amb = m;
                     }
                     uint32_t ca0, ca1, cb0, cb1;
-                    const uint32_t ba = quant_block16(va, ama, S_col, sh->rtab[1], rht, sr && cvalid, a.pk,
-                                                      a.offset, 1u, (uint64_t)(cg0 * a.rows + rg),
-                                                      ca0, ca1);
-                    const uint32_t bb = quant_block16(vb, amb, S_col, sh->rtab[1], rht, sr && cvalid, a.pk,
-                                                      a.offset, 1u,
-                                                      (uint64_t)((cg0 + 1) * a.rows + rg), cb0, cb1);
+                    const uint32_t bab = quant_block16x2(
+                        va, vb, ama, amb, S_col, sh->rtab[1], rht, sr && cvalid, a.pk, a.offset, 1u,
+                        (uint64_t)(cg0 * a.rows + rg), (uint64_t)((cg0 + 1) * a.rows + rg), ca0, ca1,
+                        cb0, cb1);
+                    const uint32_t ba = bab & 0xFFu, bb = bab >> 8;
                     if (!cvalid) continue;
                     if (two && sub == 0) {
                         keep0 = ca0, keep1 = ca1, keep2 = cb0, keep3 = cb1;

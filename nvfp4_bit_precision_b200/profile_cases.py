@@ -1,6 +1,7 @@
 """Single-case drivers for profiling one kernel launch under ncu.
 
     python -m nvfp4_bit_precision_b200.profile_cases gemm M N K [--warm W]
+    python -m nvfp4_bit_precision_b200.profile_cases mxfp8-gemm M N K [--warm W]
     python -m nvfp4_bit_precision_b200.profile_cases grouped-gemm N K [--warm W]
     python -m nvfp4_bit_precision_b200.profile_cases quant-grad ROWS COLS [--warm W]
     python -m nvfp4_bit_precision_b200.profile_cases mxfp4 ROWS COLS [--warm W]
@@ -29,6 +30,26 @@ def _gemm(nv, torch, M, N, K, warm):
     ws = torch.zeros(256, **u8)
     for _ in range(warm + 1):
         nv.nvfp4_gemm(qa, sa, one, qb, sb, one, M, N, K, nv.NVFP4_OUT_BF16, D, N, None, ws, 256)
+    return ws
+
+
+def _mxfp8_gemm(nv, torch, M, N, K, warm):
+    """MXFP8 GEMM on random E4M3 codes (NaN codes 0x7F/0xFF mapped to 0) and E8M0
+    scale bytes near 127."""
+    dev = torch.device("cuda")
+    g = torch.Generator(device=dev)
+    g.manual_seed(0)
+    u8 = dict(dtype=torch.uint8, device=dev)
+    qa = torch.randint(0, 256, (M, K), generator=g, **u8)
+    qb = torch.randint(0, 256, (N, K), generator=g, **u8)
+    for q in (qa, qb):
+        q[(q & 0x7F) == 0x7F] = 0
+    sa = torch.randint(120, 134, (nv.mxfp8_sf_mma_bytes(M, K),), generator=g, **u8)
+    sb = torch.randint(120, 134, (nv.mxfp8_sf_mma_bytes(N, K),), generator=g, **u8)
+    D = torch.empty((M, N), dtype=torch.bfloat16, device=dev)
+    ws = torch.zeros(256, **u8)
+    for _ in range(warm + 1):
+        nv.mxfp8_gemm(qa, sa, qb, sb, M, N, K, nv.NVFP4_OUT_BF16, D, N, None, ws, 256)
     return ws
 
 
@@ -82,7 +103,7 @@ def _mxfp4(nv, torch, rows, cols, warm):
 
 def main(argv=None) -> int:
     ap = argparse.ArgumentParser()
-    ap.add_argument("case", choices=["gemm", "grouped-gemm", "quant-grad", "mxfp4"])
+    ap.add_argument("case", choices=["gemm", "mxfp8-gemm", "grouped-gemm", "quant-grad", "mxfp4"])
     ap.add_argument("dims", type=int, nargs="+")
     ap.add_argument("--warm", type=int, default=3)
     args = ap.parse_args(argv)
@@ -91,6 +112,8 @@ def main(argv=None) -> int:
     import nvfp4_bit_precision_b200 as nv
     if args.case == "gemm":
         ws = _gemm(nv, torch, *args.dims[:3], args.warm)
+    elif args.case == "mxfp8-gemm":
+        ws = _mxfp8_gemm(nv, torch, *args.dims[:3], args.warm)
     elif args.case == "grouped-gemm":
         ws = _grouped(nv, torch, *args.dims[:2], args.warm)
     elif args.case == "quant-grad":

@@ -88,6 +88,9 @@ def lib():
         L.orc_mxfp8_dequant_f64.argtypes = [P, P, i64, i64, P]
         L.orc_mxfp8_gemm_rows.argtypes = [P, P, P, P, i64, i64, i64, P, i64, P, P]
         L.orc_mxfp8_gemm_rows.restype = ctypes.c_int
+        L.orc_mxfp4_dequant_f64.argtypes = [P, P, i64, i64, P]
+        L.orc_mxfp4_gemm_rows.argtypes = [P, P, P, P, i64, i64, i64, P, i64, P, P]
+        L.orc_mxfp4_gemm_rows.restype = ctypes.c_int
         _lib = L
     return _lib
 
@@ -315,4 +318,24 @@ def mxfp8_gemm_rows(qa, e8a, qb, e8b, rows_sel=None):
                                    _p(out), _p(absout))
     if rc != 0:
         raise ValueError("oracle mxfp8 gemm: invalid arguments")
+    return out, absout
+
+
+def mxfp4_gemm_rows(qa, e8a, qb, e8b, rows_sel=None):
+    """FP64 D = A_hat B_hat^T of MXFP4 operands (codes [., K/2], row-major E8M0 [., K/32])
+    for the selected rows of A; also sum |a_hat||b_hat|."""
+    qa = np.ascontiguousarray(qa, dtype=np.uint8)
+    qb = np.ascontiguousarray(qb, dtype=np.uint8)
+    e8a = np.ascontiguousarray(e8a, dtype=np.uint8)
+    e8b = np.ascontiguousarray(e8b, dtype=np.uint8)
+    M, K = qa.shape[0], qa.shape[1] * 2
+    N = qb.shape[0]
+    sel = np.arange(M, dtype=np.int64) if rows_sel is None else np.ascontiguousarray(
+        rows_sel, dtype=np.int64)
+    out = np.zeros((len(sel), N), dtype=np.float64)
+    absout = np.zeros((len(sel), N), dtype=np.float64)
+    rc = lib().orc_mxfp4_gemm_rows(_p(qa), _p(e8a), _p(qb), _p(e8b), M, N, K, _p(sel), len(sel),
+                                   _p(out), _p(absout))
+    if rc != 0:
+        raise ValueError("oracle mxfp4 gemm: invalid arguments")
     return out, absout

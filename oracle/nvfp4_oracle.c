@@ -711,3 +711,57 @@ int orc_mxfp8_gemm_rows(const uint8_t* qa, const uint8_t* e8a, const uint8_t* qb
     free(bt);
     return ORC_OK;
 }
+
+/* ------------------------------------------------------------------------ */
+/* MXFP4 GEMM reference: the OCP MX format NVFP4 is compared with [hightech; */
+/* asector, "NVFP4 and Blackwell"].  An element stands for its E2M1 value    */
+/* times 2^(byte - 127), byte being the E8M0 scale of its 32-element block;  */
+/* binary64 products and sums as for the other GEMM references.              */
+/* ------------------------------------------------------------------------ */
+void orc_mxfp4_dequant_f64(const uint8_t* q, const uint8_t* e8, int64_t rows, int64_t cols,
+                           double* out)
+{
+    for (int64_t r = 0; r < rows; ++r)
+        for (int64_t c = 0; c < cols; ++c) {
+            uint8_t byte = q[r * (cols / 2) + c / 2];
+            uint8_t code = (c & 1) ? (uint8_t)(byte >> 4) : (uint8_t)(byte & 15);
+            out[r * cols + c] = ldexp(orc_e2m1_decode(code), (int)e8[r * (cols / 32) + c / 32] - 127);
+        }
+}
+
+int orc_mxfp4_gemm_rows(const uint8_t* qa, const uint8_t* e8a, const uint8_t* qb,
+                        const uint8_t* e8b, int64_t M, int64_t N, int64_t K,
+                        const int64_t* rows_sel, int64_t n_sel, double* out, double* absout)
+{
+    if (K % 32) return ORC_EINVAL;
+    double* a = (double*)malloc(sizeof(double) * (size_t)K);
+    double* bt = (double*)malloc(sizeof(double) * (size_t)(N * K));
+    if (!a || !bt) {
+        free(a);
+        free(bt);
+        return ORC_EINVAL;
+    }
+    orc_mxfp4_dequant_f64(qb, e8b, N, K, bt);
+    for (int64_t s = 0; s < n_sel; ++s) {
+        int64_t i = rows_sel[s];
+        if (i < 0 || i >= M) {
+            free(a);
+            free(bt);
+            return ORC_EINVAL;
+        }
+        orc_mxfp4_dequant_f64(qa + i * (K / 2), e8a + i * (K / 32), 1, K, a);
+        for (int64_t j = 0; j < N; ++j) {
+            double acc = 0.0, aacc = 0.0;
+            for (int64_t k = 0; k < K; ++k) {
+                double pr = a[k] * bt[j * K + k];
+                acc += pr;
+                aacc += fabs(pr);
+            }
+            out[s * N + j] = acc;
+            absout[s * N + j] = aacc;
+        }
+    }
+    free(a);
+    free(bt);
+    return ORC_OK;
+}

@@ -120,16 +120,16 @@ def test_mxfp8_and_dequant_argument_errors(nv):
 
 def test_mxfp4_argument_errors(nv):
     L = nv._lib
-    assert L.mxfp4_quantize(None, 32, 32, 32, 1, FAKE, FAKE, None, None, None) == 1
-    assert L.mxfp4_quantize(FAKE, 32, 32, 32, 0, FAKE, FAKE, FAKE, FAKE, None) == 1   # no direction
-    assert L.mxfp4_quantize(FAKE, 32, 32, 32, 4, FAKE, FAKE, FAKE, FAKE, None) == 1   # unknown bit
-    assert L.mxfp4_quantize(FAKE, 32, 32, 32, 2, FAKE, FAKE, None, FAKE, None) == 1   # col output NULL
-    assert L.mxfp4_quantize(FAKE, 48, 32, 32, 1, FAKE, FAKE, None, None, None) == 2   # rows % 32
-    assert L.mxfp4_quantize(FAKE, 32, 48, 48, 1, FAKE, FAKE, None, None, None) == 2   # cols % 32
-    assert L.mxfp4_quantize(FAKE, 32, 64, 32, 1, FAKE, FAKE, None, None, None) == 2   # ld < cols
-    assert L.mxfp4_quantize(FAKE + 8, 32, 32, 32, 1, FAKE, FAKE, None, None, None) == 3
-    assert L.mxfp4_quantize(FAKE, 32, 32, 36, 1, FAKE, FAKE, None, None, None) == 3   # ld % 8
-    assert L.mxfp4_quantize(FAKE, 32, 32, 32, 2, None, None, FAKE + 4, FAKE, None) == 3
+    assert L.mxfp4_quantize(None, 32, 32, 32, 1, 0, FAKE, FAKE, None, None, None) == 1
+    assert L.mxfp4_quantize(FAKE, 32, 32, 32, 0, 0, FAKE, FAKE, FAKE, FAKE, None) == 1   # no direction
+    assert L.mxfp4_quantize(FAKE, 32, 32, 32, 4, 0, FAKE, FAKE, FAKE, FAKE, None) == 1   # unknown bit
+    assert L.mxfp4_quantize(FAKE, 32, 32, 32, 2, 0, FAKE, FAKE, None, FAKE, None) == 1   # col output NULL
+    assert L.mxfp4_quantize(FAKE, 48, 32, 32, 1, 0, FAKE, FAKE, None, None, None) == 2   # rows % 32
+    assert L.mxfp4_quantize(FAKE, 32, 48, 48, 1, 0, FAKE, FAKE, None, None, None) == 2   # cols % 32
+    assert L.mxfp4_quantize(FAKE, 32, 64, 32, 1, 0, FAKE, FAKE, None, None, None) == 2   # ld < cols
+    assert L.mxfp4_quantize(FAKE + 8, 32, 32, 32, 1, 0, FAKE, FAKE, None, None, None) == 3
+    assert L.mxfp4_quantize(FAKE, 32, 32, 36, 1, 0, FAKE, FAKE, None, None, None) == 3   # ld % 8
+    assert L.mxfp4_quantize(FAKE, 32, 32, 32, 2, 0, None, None, FAKE + 4, FAKE, None) == 3
 
 
 def test_mxfp8_gemm_argument_errors(nv):
@@ -155,3 +155,15 @@ def test_mxfp8_gemm_argument_errors(nv):
     assert q(nv, 32, 96, 96, p) == 2                    # tiled MXFP8 scales need K % 128
     p.mx_sf_layout = 3
     assert q(nv, 32, 128, 128, p) == 1
+
+
+def test_mxfp4_gemm_and_layout_argument_errors(nv):
+    L = nv._lib
+    g = L.mxfp4_gemm
+    args = (FAKE,) * 4
+    assert g(None, FAKE, FAKE, FAKE, 128, 128, 256, 0, FAKE, 128, None, FAKE, 256, None) == 1
+    assert g(*args, 128, 128, 128, 0, FAKE, 128, None, FAKE, 256, None) == 2      # K % 256
+    assert g(*args, 120, 128, 256, 0, FAKE, 128, None, FAKE, 256, None) == 2     # M % 16
+    assert g(*args, 128, 128, 256, 0, FAKE, 128, None, None, 0, None) == 7       # workspace
+    assert L.mxfp4_quantize(FAKE, 32, 64, 64, 1, 5, FAKE, FAKE, None, None, None) == 1  # layout
+    assert L.mxfp4_quantize(FAKE, 32, 64, 64, 1, 1, FAKE, FAKE, None, None, None) == 2  # K % 128

@@ -128,3 +128,32 @@ def test_gemm_sampled_entries(orc, layer, out, spec_a, spec_b, M, N):
             Dr, Ar = orc.nvfp4_gemm_rows(qa, sa, ga, qb, sb, gb, rows_sel=[i - i0])
             got = W.bf16_bits_to_f32(host(D[i:i + 1, j0:j0 + 16].contiguous()))
             check_gemm(got, Dr, Ar, True)
+
+
+@pytest.mark.parametrize("out,spec_a,spec_b,M,N", GEMMS, ids=[g[0] for g in GEMMS])
+def test_gemm_every_output_tile(orc, layer, out, spec_a, spec_b, M, N):
+    """One row x 16 columns inside every 256 x 256 output tile (the pair's tile): the row
+    in M-tile mt sits at offset (37 mt + 5) % 256 and the 16 columns of N-tile nt at
+    16 ((5 nt + 3) % 16), so the checks move across both CTAs of the pair, every lane
+    quadrant and every epilogue warp's column range, and cover the band rasterisation
+    and the persistent multi-tile loop of the full-size launch."""
+    D = layer[out]
+    tiles_m, tiles_n = M // 256, N // 256
+    j0s = [256 * nt + 16 * ((5 * nt + 3) % 16) for nt in range(tiles_n)]
+    slices = [_oracle_rows(orc, layer, spec_b, j0) for j0 in j0s]
+    qb = np.concatenate([t[0] for t in slices])
+    sb = np.concatenate([t[1] for t in slices])
+    gb = slices[0][2]
+    assert all(t[2] == gb for t in slices)
+    import torch
+    cols = np.concatenate([np.arange(j0, j0 + 16) for j0 in j0s])
+    cols_d = torch.from_numpy(cols).to(D.device)
+    worst = 0.0
+    for mt in range(tiles_m):
+        i = 256 * mt + (37 * mt + 5) % 256
+        i0 = (i // 16) * 16
+        qa, sa, ga = _oracle_rows(orc, layer, spec_a, i0)
+        Dr, Ar = orc.nvfp4_gemm_rows(qa, sa, ga, qb, sb, gb, rows_sel=[i - i0])
+        got = W.bf16_bits_to_f32(host(D[i][cols_d]))[None, :]
+        worst = max(worst, check_gemm(got, Dr, Ar, True))
+    assert worst <= 1.0

@@ -132,3 +132,64 @@ def test_down_projection_full_shape(nv, orc, moe):
         Dr, Ar = orc.nvfp4_gemm_rows(qa[r:r + 1], sa[r:r + 1], float(ga), qb[e], sb[e],
                                      float(gb[e]), rows_sel=[0])
         check_gemm(D[r:r + 1], Dr, Ar, True)
+
+
+def test_up_projection_every_expert(nv, orc, moe):
+    """The first and last routed row of every non-empty expert (the group boundaries of
+    the device-built tile table), against 32 columns of that expert's output: the first
+    16 and 16 at an offset that moves with the expert."""
+    offsets, x, rt, w_up = moe["offsets"], moe["x"], moe["row_token"], moe["w_up"]
+    import torch
+    am = (orc.amax(x, 0), 0.0)
+    H = moe["H"]
+    checked = 0
+    for e in range(E):
+        lo, hi = int(offsets[e]), int(offsets[e + 1])
+        if hi == lo:
+            continue
+        c1 = 256 * (e % 6) + 16 * (e % 16)
+        amw = orc.amax(w_up[e], 0)
+        qs = [orc.nvfp4_quantize(np.ascontiguousarray(w_up[e][c:c + 16]), 0, amax=(amw, amw))
+              for c in (0, c1)]
+        qb = np.concatenate([t[0] for t in qs])
+        sb = np.concatenate([t[1] for t in qs])
+        cols = torch.from_numpy(np.concatenate([np.arange(16), np.arange(c1, c1 + 16)])).cuda()
+        for r in sorted({lo, hi - 1}):
+            qa, sa, ga = _token_row(orc, x, rt[r], am)
+            Dr, Ar = orc.nvfp4_gemm_rows(qa, sa, ga, qb, sb, qs[0][2], rows_sel=[0])
+            got = W.bf16_bits_to_f32(host(H[r][cols]))[None, :]
+            check_gemm(got, Dr, Ar, True)
+            checked += 1
+    assert checked >= 2 * int(np.count_nonzero(np.diff(offsets) > 1))
+
+
+def test_down_projection_every_expert(nv, orc, moe):
+    """The grouped down GEMM at its full shape on random codes and in-range scale bytes:
+    the first and last row of every non-empty expert, every output column."""
+    import torch
+    offsets = moe["offsets"]
+    R = int(offsets[-1])
+    rng = np.random.default_rng(22)
+    qa = rng.integers(0, 256, (R, FFN // 2), dtype=np.uint8)
+    sa = rng.integers(0x28, 0x48, (R, FFN // 16), dtype=np.uint8)
+    qb = rng.integers(0, 256, (E, HID, FFN // 2), dtype=np.uint8)
+    sb = rng.integers(0x28, 0x48, (E, HID, FFN // 16), dtype=np.uint8)
+    gb = (rng.random(E) + 0.5).astype(np.float32)
+    ga = np.float32(1.25)
+    pr = grouped_padded_rows(offsets)
+    total_padded = int(sum(((c + 127) // 128) * 128 for c in np.diff(offsets)))
+    dev = dict(device="cuda")
+    A = nv.NVFP4Tensor(torch.from_numpy(qa).to(**dev),
+                       torch.from_numpy(rowmajor_to_sf_mma(sa, R, FFN, pr, total_padded)).to(**dev),
+                       torch.tensor([ga], **dev), R, FFN, nv.NVFP4_SF_MMA)
+    sfb = np.concatenate([rowmajor_to_sf_mma(sb[e], HID, FFN) for e in range(E)])
+    off = torch.from_numpy(offsets.astype(np.int32)).to(**dev)
+    D = nv.grouped_gemm(off, A, torch.from_numpy(qb).to(**dev), torch.from_numpy(sfb).to(**dev),
+                        torch.from_numpy(gb).to(**dev), HID, nv.NVFP4_OUT_BF16)
+    D = W.bf16_bits_to_f32(host(D))
+    for e in range(E):
+        lo, hi = int(offsets[e]), int(offsets[e + 1])
+        for r in sorted({lo, hi - 1}) if hi > lo else ():
+            Dr, Ar = orc.nvfp4_gemm_rows(qa[r:r + 1], sa[r:r + 1], float(ga), qb[e], sb[e],
+                                         float(gb[e]), rows_sel=[0])
+            check_gemm(D[r:r + 1], Dr, Ar, True)

@@ -120,3 +120,46 @@ def test_nvfp4_error_below_mxfp4(orc):
     qm, em = orc.mxfp4_quantize(x, 0)
     err_mx = np.mean((orc.mxfp4_dequant(qm, em) - xf) ** 2)
     assert err_nv < 0.75 * err_mx, (err_nv, err_mx)
+
+
+def test_mxfp4_gemm_oracle_closed_form(orc):
+    """Hand-built MXFP4 operands with a closed-form product: A elements +-1 (code 2 /
+    10), B elements 3 (code 5); block b of A row i scaled 2^(i-b), of B row j 2^(j+b);
+    so D[i][j] = 3 * 32 * sum_b s_b * 2^(i+j), s_b the block's sign."""
+    M, N, K = 2, 3, 128
+    signs = [1, 1, -1, 1]
+    codes = np.concatenate([np.full(32, 2 if s > 0 else 10, dtype=np.uint8) for s in signs])
+    qa = np.tile(codes[0::2] | (codes[1::2] << 4), (M, 1))
+    e8a = np.array([[127 + i - b for b in range(4)] for i in range(M)], dtype=np.uint8)
+    qb = np.full((N, K // 2), 5 | (5 << 4), dtype=np.uint8)
+    e8b = np.array([[127 + j + b for b in range(4)] for j in range(N)], dtype=np.uint8)
+    D, A = orc.mxfp4_gemm_rows(qa, e8a, qb, e8b)
+    for i in range(M):
+        for j in range(N):
+            assert D[i, j] == 3 * 32 * sum(signs) * 2.0 ** (i + j)
+            assert A[i, j] == 3 * 32 * 4 * 2.0 ** (i + j)
+
+
+def test_mxfp4_gemm_oracle_vs_numpy(orc):
+    """The MXFP4 GEMM reference against numpy on the independent dequantisation of this
+    file's grid (E2M1 magnitude x 2^(byte - 127)), on quantised Gaussian data; and NVFP4's
+    product of the same data is closer to the bf16 product than MXFP4's."""
+    rng = np.random.default_rng(33)
+    x = W.f32_to_bf16_bits(W.normal(rng, (32, 256)))
+    w = W.f32_to_bf16_bits(W.normal(rng, (48, 256), 0.02))
+    qa, ea = orc.mxfp4_quantize(x, 0)
+    qb, eb = orc.mxfp4_quantize(w, 0)
+    D, A = orc.mxfp4_gemm_rows(qa, ea, qb, eb)
+
+    def hat(q, e):
+        mag = np.array(GRID + [-g for g in GRID])[codes_of(q)]
+        return mag * np.repeat(2.0 ** (e.astype(np.int64) - 127), 32, axis=1)
+
+    ah, bh = hat(qa, ea), hat(qb, eb)
+    np.testing.assert_allclose(D, ah @ bh.T, rtol=0, atol=1e-13 * A.max())
+    np.testing.assert_allclose(A, np.abs(ah) @ np.abs(bh).T, rtol=1e-13)
+    ref = W.bf16_bits_to_f32(x).astype(np.float64) @ W.bf16_bits_to_f32(w).astype(np.float64).T
+    na, sa_, ga = orc.nvfp4_quantize(x, 0)
+    nb, sb_, gb = orc.nvfp4_quantize(w, 0)
+    Dn, _ = orc.nvfp4_gemm_rows(na, sa_, ga, nb, sb_, gb)
+    assert np.linalg.norm(Dn - ref) < np.linalg.norm(D - ref)
