@@ -60,7 +60,12 @@ constexpr int BM = 128;                    // A rows per CTA; a CTA pair covers 
 constexpr int kMmaM = 2 * BM;              // M of the two-SM MMA
 constexpr int kMaxStages = 8;
 constexpr int kMaxAccStages = 2;
-constexpr int kGemmThreads = 448;  // producer, MMA, 4 scale writers, 8 epilogue warps
+#ifndef NVFP4_GEMM_EPI_WARPS
+#define NVFP4_GEMM_EPI_WARPS 8
+#endif
+constexpr int kEpiWarps = NVFP4_GEMM_EPI_WARPS;     // epilogue warps per CTA (8 or 16)
+constexpr int kGemmThreads = 32 * (6 + kEpiWarps);  // producer, MMA, 4 scale writers, epilogue
+static_assert(kEpiWarps == 8 || kEpiWarps == 16, "epilogue warps: 8 or 16");
 constexpr int kTmemCols = 512;
 constexpr int kMaxGemmGroups = 256;
 constexpr int kEpiStageBytes = 2048;  // per epilogue warp: 32 rows x 64 bytes of BF16
@@ -115,13 +120,13 @@ struct GemmCfg {
     static constexpr int kSfCols = kSfColsA + kSfAtoms * 4 * kBlocksN;  // written per stage
     static constexpr int kSfStride = (kSfCols + 15) / 16 * 16;            // columns per stage region
     static constexpr int kStagesBySmem =
-        (kSmemLimit - kSmemShared - 8 * kEpiStageBytes - 1024) / kStageBytes;
+        (kSmemLimit - kSmemShared - kEpiWarps * kEpiStageBytes - 1024) / kStageBytes;
     static constexpr int kStagesByTmem = (kTmemCols - kTmemSF) / kSfStride;
     static constexpr int kStages = kStagesBySmem < kStagesByTmem
                                        ? (kStagesBySmem < kMaxStages ? kStagesBySmem : kMaxStages)
                                        : (kStagesByTmem < kMaxStages ? kStagesByTmem : kMaxStages);
     static constexpr size_t kSmemBytes =
-        (size_t)kStages * kStageBytes + kSmemShared + 8 * kEpiStageBytes + 1024;
+        (size_t)kStages * kStageBytes + kSmemShared + kEpiWarps * kEpiStageBytes + 1024;
     static_assert(kStages >= 4, "pipeline too shallow");
     static_assert(kTmemSF + kStages * kSfStride <= kTmemCols, "tensor memory overflow");
     static_assert(kSmemBytes <= (size_t)kSmemLimit, "shared memory overflow");
@@ -144,7 +149,6 @@ struct GemmArgs {
     float* amax_out;  // optional: max |D| (as stored), atomically accumulated
     uint64_t wait_ns;  // limit of every barrier wait (2 s; shorter under the test hook)
     int no_copies;     // test hook: the producers issue no copy (see wait_test_hook)
-    int st32;          // D and its rows are 32-byte aligned: each lane stores 32-byte pieces
 };
 
 // ---------------------------------------------------------------- PTX wrappers
@@ -336,16 +340,6 @@ __device__ __forceinline__ void tmem_store_words(uint32_t taddr, const uint32_t*
     }
 }
 
-// 32 bytes (8 words) to global memory in one instruction, marked to leave L2
-// first: the output streams past while the operand tiles stay resident.
-__device__ __forceinline__ void st_global_v8_ef(void* p, const uint32_t* v)
-{
-    asm volatile("st.global.L2::evict_first.v8.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8};" ::"l"(p),
-                 "r"(v[0]), "r"(v[1]), "r"(v[2]), "r"(v[3]), "r"(v[4]), "r"(v[5]), "r"(v[6]),
-                 "r"(v[7])
-                 : "memory");
-}
-
 __device__ __forceinline__ void tmem_ld_wait() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory"); }
 
 // ---------------------------------------------------------------- scheduling
@@ -422,7 +416,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
         }
         for (int b = 0; b < kAcc; ++b) {
             mbar_init(&sh->acc_full[b], 1);
-            mbar_init(&sh->acc_empty[b], 16);  // leader: 8 epilogue warps of each CTA
+            mbar_init(&sh->acc_empty[b], 2 * kEpiWarps);  // leader: epilogue warps of both CTAs
         }
         fence_barrier_init();
         // tile table (both CTAs compute the same one)
@@ -607,7 +601,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
         }
     } else {
         // ------------------------------------------------ epilogue (warps 6..13, both CTAs)
-        constexpr int kCols = kBN / 2;     // accumulator columns per warp
+        constexpr int kCols = kBN / (kEpiWarps / 4);  // accumulator columns per warp
         constexpr int kChunks = kCols / 32;
         const int quad = warp & 3;                   // TMEM lanes 32*quad .. 32*quad+31
         const int col0 = ((warp - 6) >> 2) * kCols;
@@ -634,7 +628,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
                 // accumulator is released before any store.
                 uint32_t packed[16 * kChunks];
                 float m_all = 0.0f;  // max |x| over the warp's columns (before rounding)
-                constexpr int kPer = kChunks == 2 ? 2 : 1;
+                constexpr int kPer = (kChunks == 2 && kEpiWarps == 8) ? 2 : 1;
 #pragma unroll
                 for (int hh = 0; hh < kChunks; hh += kPer) {
                     uint32_t r[32 * kPer];
@@ -670,17 +664,6 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
                                 }
                             }
                     }
-                }
-                if (a.st32) {
-                    // each lane stores its own row in 32-byte pieces (16 columns):
-                    // whole sectors without a shared-memory turnaround
-                    if (row_ok) {
-                        uint16_t* drow = static_cast<uint16_t*>(a.D) + row * a.ldd + cbase;
-#pragma unroll
-                        for (int g = 0; g < 2 * kChunks; ++g)
-                            if (cbase + 16 * g < a.N) st_global_v8_ef(drow + 16 * g, packed + 8 * g);
-                    }
-                    continue;
                 }
                 const int64_t rowbase = c.row0 + (int64_t)BM * rank + 32 * quad;
                 // 32-column chunks through a 64-byte-swizzled 32x64-byte staging
@@ -727,21 +710,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
                     const float x1 = __fmul_rn(__uint_as_float(r[4 * v + 1]), alpha);
                     const float x2 = __fmul_rn(__uint_as_float(r[4 * v + 2]), alpha);
                     const float x3 = __fmul_rn(__uint_as_float(r[4 * v + 3]), alpha);
-                    r[4 * v] = __float_as_uint(x0), r[4 * v + 1] = __float_as_uint(x1);
-                    r[4 * v + 2] = __float_as_uint(x2), r[4 * v + 3] = __float_as_uint(x3);
-                    if (cbase + 4 * v < a.N) out_max = absmax3(out_max, absmax3(x0, x1, x2), x3);
-                }
-                // N is a multiple of 16, so an 8-column piece is stored whole or not at all
-#pragma unroll
-                for (int v = 0; v < 4; ++v) {
-                    if (cbase + 8 * v >= a.N) continue;
-                    if (a.st32) {
-                        st_global_v8_ef(drow + 8 * v, r + 8 * v);
-                    } else {
-                        reinterpret_cast<uint4*>(drow + 8 * v)[0] =
-                            make_uint4(r[8 * v], r[8 * v + 1], r[8 * v + 2], r[8 * v + 3]);
-                        reinterpret_cast<uint4*>(drow + 8 * v)[1] =
-                            make_uint4(r[8 * v + 4], r[8 * v + 5], r[8 * v + 6], r[8 * v + 7]);
+                    if (cbase + 4 * v < a.N) {
+                        *reinterpret_cast<float4*>(drow + 4 * v) = make_float4(x0, x1, x2, x3);
+                        out_max = absmax3(out_max, absmax3(x0, x1, x2), x3);
                     }
                 }
             }
@@ -852,7 +823,6 @@ static GemmDevice& gemm_device(int dev)
 }
 
 static bool al16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
-static bool al32(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 31u) == 0; }
 
 constexpr size_t kGemmWorkspace = 256;
 
@@ -960,7 +930,6 @@ extern "C" nvfp4_status nvfp4_gemm(const uint8_t* qa, const uint8_t* sfa, const 
     a.G = 1;
     a.status = static_cast<uint32_t*>(workspace) + 2;
     a.amax_out = amax_out;
-    a.st32 = al32(D) && (ldd * (a.bf16_out ? 2 : 4)) % 32 == 0;
     return launch_gemm<kFmtNVFP4>(qa, qb, a, M, N, (M + kMmaM - 1) / kMmaM,
                                   static_cast<cudaStream_t>(stream));
 }
@@ -986,7 +955,6 @@ extern "C" nvfp4_status mxfp8_gemm(const uint8_t* qa, const uint8_t* sfa, const 
     a.G = 1;
     a.status = static_cast<uint32_t*>(workspace) + 2;
     a.amax_out = amax_out;
-    a.st32 = al32(D) && (ldd * (a.bf16_out ? 2 : 4)) % 32 == 0;
     return launch_gemm<kFmtMXFP8>(qa, qb, a, M, N, (M + kMmaM - 1) / kMmaM,
                                   static_cast<cudaStream_t>(stream));
 }
@@ -1012,7 +980,6 @@ extern "C" nvfp4_status mxfp4_gemm(const uint8_t* qa, const uint8_t* sfa, const 
     a.G = 1;
     a.status = static_cast<uint32_t*>(workspace) + 2;
     a.amax_out = amax_out;
-    a.st32 = al32(D) && (ldd * (a.bf16_out ? 2 : 4)) % 32 == 0;
     return launch_gemm<kFmtMXFP4>(qa, qb, a, M, N, (M + kMmaM - 1) / kMmaM,
                                   static_cast<cudaStream_t>(stream));
 }
@@ -1052,7 +1019,6 @@ extern "C" nvfp4_status nvfp4_grouped_gemm(int G, const int32_t* group_offsets, 
     a.total_rows = total_rows;
     a.status = static_cast<uint32_t*>(workspace) + 2;
     a.amax_out = amax_out;
-    a.st32 = al32(D);  // ldd = N, a multiple of 128
     // upper bound on M tiles: every group may add one partial tile
     return launch_gemm<kFmtNVFP4>(qa, qb, a, total_rows, (int64_t)G * N,
                                   (total_rows + kMmaM - 1) / kMmaM + G,

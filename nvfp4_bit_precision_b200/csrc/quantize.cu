@@ -224,6 +224,22 @@ __device__ __forceinline__ void unpack8(const uint4& p, float* v)
     v[7] = bf16_hi(p.w);
 }
 
+// RN(a / 6) for a >= 0.  Markstein's corrected quotient (P. Markstein,
+// "Computation of elementary functions on the IBM RISC System/6000 processor",
+// IBM J. Res. Develop. 34(1), 1990): q0 = RN(a z) with z = RN(1/6), the
+// remainder a - 6 q0 exactly in one fused multiply-add, then RN(q0 + r z).
+// Checked against the IEEE division for every non-negative float: equal for
+// every a >= 2^-120; below that (quotients near the subnormal range) the
+// division itself is used.
+__device__ __forceinline__ float div6_rn(float a)
+{
+    if (a < 7.52316384526264005100e-37f) return __fdiv_rn(a, 6.0f);  // 2^-120
+    const float z = 0.16666667163372039794921875f;                    // RN(1/6)
+    const float q0 = __fmul_rn(a, z);
+    const float r = __fmaf_rn(-q0, 6.0f, a);
+    return __fmaf_rn(r, z, q0);
+}
+
 // Quantisation of 16-value blocks given their (possibly 2D-reduced) amax:
 // scale byte = E4M3_RNE((amax_b / 6) * S), r = RN(S / d) from the per-CTA table,
 // codes = RNE or SR of x * r.  times4: v and amax_b hold 4x the values (Hadamard
@@ -245,8 +261,8 @@ __device__ __forceinline__ uint32_t quant_block16x2(float (&v)[16], float (&w)[1
         am_v = __fmul_rn(am_v, 0.25f);
         am_w = __fmul_rn(am_w, 0.25f);
     }
-    const float sv = __fmul_rn(__fdiv_rn(am_v, 6.0f), S);
-    const float sw = __fmul_rn(__fdiv_rn(am_w, 6.0f), S);
+    const float sv = __fmul_rn(div6_rn(am_v), S);
+    const float sw = __fmul_rn(div6_rn(am_w), S);
     const uint32_t bytes = e4m3x2_rne_sat(sw, sv) & 0xFFFFu;
     float rv = rtab[bytes & 0xFFu], rw = rtab[bytes >> 8];  // RN(S / d); 0 when d = 0
     if (times4) {
