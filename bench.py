@@ -543,6 +543,52 @@ def time_mxfp4_gemm(step, steps, warmup, fp4_peak):
             "unit": "TFLOP/s", "frac": round(tf / fp4_peak, 4)}
 
 
+def time_moe_combine(step, steps, warmup, pk):
+    """The MXFP8 return trip of the MoE expert outputs without the network: the down
+    projection's output Out [65536, 4096] (rows in expert order) quantised to MXFP8
+    rowwise, then each token's 4 rows combined with weights 1/4 into [16384, 4096] bf16
+    (mxfp8_combine).  Timed apart from the step with CUDA events; on one GPU there is no
+    all-to-all to time.  Link bytes: what an expert-parallel run would send per step."""
+    nv, torch = step.nv, step.torch
+    dev = step.Out.device
+    R, H = step.Out.shape
+    te = step.h["token_expert"]
+    order = np.argsort(te.reshape(-1), kind="stable")
+    pos = np.empty_like(order)
+    pos[order] = np.arange(order.size)
+    slot = torch.from_numpy(pos.reshape(te.shape).astype(np.int32)).to(dev)
+    w = torch.full(te.shape, 1.0 / TOPK, dtype=torch.float32, device=dev)
+    u8 = dict(dtype=torch.uint8, device=dev)
+    q, e8 = torch.empty((R, H), **u8), torch.empty((R, H // 32), **u8)
+    out = torch.empty((MOE_TOKENS, H), dtype=torch.bfloat16, device=dev)
+
+    def run():
+        nv.mxfp8_quantize(step.Out, R, H, H, nv.NVFP4_ROWWISE, 0, 0, 0, q, e8, None, None)
+        nv.mxfp8_combine(q, e8, R, H, slot, w, MOE_TOKENS, TOPK, out, step.ws[6], 256)
+
+    for _ in range(max(warmup, 3)):
+        run()
+    stream = torch.cuda.current_stream()
+    s_, e_ = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    torch.cuda.synchronize()
+    s_.record(stream)
+    for _ in range(steps):
+        run()
+    e_.record(stream)
+    torch.cuda.synchronize()
+    step.check_status()
+    ms = s_.elapsed_time(e_) / steps
+    nbytes = 2 * R * H + 2 * (R * H + R * H // 32) + MOE_TOKENS * H * 2
+    return {"kernel": "mxfp8_quantize (rowwise) + mxfp8_combine_kernel on the MoE output "
+                      "65536x4096 -> 16384x4096 bf16, top-4 weights 1/4", "bound": "hbm",
+            "us": round(ms * 1e3, 1), "algorithmic_bytes": nbytes,
+            "achieved": round(nbytes / (ms / 1e3) / 1e9, 1), "peak": pk["hbm_gbs"], "unit": "GB/s",
+            "frac": round(nbytes / (ms / 1e3) / 1e9 / pk["hbm_gbs"], 4),
+            "link_bytes_mxfp8": R * H + R * H // 32, "link_bytes_bf16": 2 * R * H,
+            "note": "one GPU: no all-to-all is timed; link bytes are what an expert-parallel "
+                    "run would send back per step"}
+
+
 def quant_algorithmic_bytes():
     """Bytes the dY quantisation must move: two reads of the bf16 input (amax pass and
     quantise pass), NVFP4 codes and scales in both directions, MXFP8 codes and scales."""
@@ -554,11 +600,11 @@ def host_inputs(seed_dense=4, seed_moe=3):
     d = W.dense_linear_layer(seed_dense, TOKENS, HIDDEN, FFN)
     rng = np.random.default_rng(seed_moe)
     tok = W.f32_to_bf16_bits(W.normal(rng, (MOE_TOKENS, MOE_HIDDEN)))
-    _, row_token, offsets = W.moe_routing(rng, MOE_TOKENS, EXPERTS, TOPK)
+    token_expert, row_token, offsets = W.moe_routing(rng, MOE_TOKENS, EXPERTS, TOPK)
     w_up = W.f32_to_bf16_bits(W.normal(rng, (EXPERTS, MOE_FFN, MOE_HIDDEN), 0.02))
     w_down = W.f32_to_bf16_bits(W.normal(rng, (EXPERTS, MOE_HIDDEN, MOE_FFN), 0.02))
     return dict(x=d["x"], w=d["w"], dy=d["dy"], tok=tok, row_token=row_token, offsets=offsets,
-                w_up=w_up, w_down=w_down)
+                w_up=w_up, w_down=w_down, token_expert=token_expert)
 
 
 # ----------------------------------------------------------------------------- clocks
@@ -932,6 +978,7 @@ def main():
     cfgs = time_configs(dev, max(args.steps, 10), args.warmup, pk, fp4_peak)
     mx8 = time_mxfp8_backward(step, args.steps, args.warmup, fp4_peak / 2)
     mx4g = time_mxfp4_gemm(step, args.steps, args.warmup, fp4_peak)
+    comb = time_moe_combine(step, args.steps, args.warmup, pk)
     gd = per_kernel["gemm_dense"]
     gemm_ms = sum(gd) / len(gd)
     gemm_tflops = DENSE_FLOP_PER_GEMM / (gemm_ms / 1e3) / 1e12
@@ -982,7 +1029,8 @@ def main():
             "grouped_gemm_roofline": grouped_roofline(per_kernel["gemm_grouped"], args.steps,
                                                       step, pk, fp4_peak),
             "configs": cfgs,
-            "next_rows": {"mxfp8_backward_gemm": mx8, "mxfp4_gemm": mx4g, "mxfp4_quantize": {
+            "next_rows": {"mxfp8_backward_gemm": mx8, "mxfp4_gemm": mx4g,
+                          "moe_combine_mxfp8": comb, "mxfp4_quantize": {
                 "bound": "hbm", "kernel": "mxfp4_kernel on dY 16384x20480, both directions "
                 "(timed apart from the step)", "ms": round(mx4_ms, 4),
                 "achieved": round(mx4_bytes / (mx4_ms / 1e3) / 1e9, 1), "peak": pk["hbm_gbs"],

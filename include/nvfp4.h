@@ -235,7 +235,8 @@ nvfp4_status nvfp4_quantize_noalloc_status(void* stream);
  * satfinite or SR (Philox stream 2).
  * directions: NVFP4_ROWWISE (codes [rows, cols], scales [rows, cols/32]) and/or
  * NVFP4_COLWISE (codes [cols, rows], scales [cols, rows/32]).  The block axis
- * must be a multiple of 32, the other a multiple of 16.
+ * must be a multiple of 32, the other a multiple of 16 (any row count for
+ * NVFP4_ROWWISE alone).
  */
 nvfp4_status mxfp8_quantize(const void* x_bf16, int64_t rows, int64_t cols, int64_t ld,
                             int directions, int rounding, uint64_t seed, uint32_t offset,
@@ -370,6 +371,24 @@ nvfp4_status nvfp4_grouped_gemm(int G, const int32_t* group_offsets, int64_t tot
                                 const uint8_t* qb, const uint8_t* sfb, const float* gb,
                                 int64_t N, int64_t K, int out_dtype, void* D, float* amax_out,
                                 void* workspace, size_t ws_bytes, void* stream);
+
+/*
+ * mxfp8_combine -- the receiving end of the MXFP8-compressed expert combine
+ * (iitak, "But": expert outputs travel at 8.25 bits per number instead of 16).
+ * q [rows, cols] E4M3 codes and e8 [rows, cols/32] row-major E8M0 scales are the
+ * expert-output rows this rank received (mxfp8_quantize rowwise on the sender);
+ * token t's k rows are slot_row[t*k + j] (device int32, -1 = no row) with
+ * routing weights weight[t*k + j] (device FP32).  Computes, in FP32 with one
+ * rounding per product and per sum, j in order,
+ *   out[t][c] = sum_j weight[t][j] * (e4m3(q[r][c]) * 2^(e8[r][c/32] - 127)),
+ * then RNE to bf16 into out_bf16 [tokens, cols].  cols a multiple of 32;
+ * 1 <= k <= 64; q 8-byte and out 16-byte aligned.  A row index >= rows is
+ * skipped and reported in the optional workspace's status word
+ * (NVFP4_ERR_INDEX).  Asynchronous on `stream`; allocates nothing.
+ */
+nvfp4_status mxfp8_combine(const uint8_t* q, const uint8_t* e8, int64_t rows, int64_t cols,
+                           const int32_t* slot_row, const float* weight, int64_t tokens, int k,
+                           void* out_bf16, void* workspace, size_t ws_bytes, void* stream);
 
 /* Synchronise `stream` and return the device status word of a workspace
  * (NVFP4_OK, NVFP4_ERR_TIMEOUT or NVFP4_ERR_INDEX); clears it. */

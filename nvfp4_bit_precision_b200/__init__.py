@@ -47,6 +47,7 @@ EXPORTED = [
     "nvfp4_sf_mma_grouped_bytes", "nvfp4_workspace_status", "nvfp4_status_string",
     "nvfp4_version", "nvfp4_quantize_noalloc", "nvfp4_quantize_noalloc_status",
     "nvfp4_gather_rows", "mxfp4_quantize", "mxfp8_gemm", "mxfp8_sf_mma_bytes", "mxfp4_gemm",
+    "mxfp8_combine",
 ]
 
 
@@ -82,6 +83,7 @@ _lib.nvfp4_gemm.argtypes = [_P, _P, _P, _P, _P, _P, _I64, _I64, _I64, ctypes.c_i
                             _P, _SZ, _P]
 _lib.mxfp8_gemm.argtypes = [_P, _P, _P, _P, _I64, _I64, _I64, ctypes.c_int, _P, _I64, _P, _P, _SZ,
                             _P]
+_lib.mxfp8_combine.argtypes = [_P, _P, _I64, _I64, _P, _P, _I64, ctypes.c_int, _P, _P, _SZ, _P]
 _lib.mxfp8_sf_mma_bytes.argtypes = [_I64, _I64]
 _lib.mxfp8_sf_mma_bytes.restype = _SZ
 _lib.nvfp4_grouped_gemm.argtypes = [ctypes.c_int, _P, _I64, _P, _P, _P, _P, _P, _P, _I64, _I64,
@@ -102,7 +104,7 @@ _lib.nvfp4_status_string.argtypes = [ctypes.c_int]
 _lib.nvfp4_status_string.restype = ctypes.c_char_p
 _lib.nvfp4_version.restype = ctypes.c_int
 for _n in ("nvfp4_quantize", "nvfp4_quantize_noalloc", "mxfp8_quantize", "mxfp4_quantize",
-           "nvfp4_dequantize", "nvfp4_gemm", "mxfp8_gemm", "mxfp4_gemm",
+           "nvfp4_dequantize", "nvfp4_gemm", "mxfp8_gemm", "mxfp4_gemm", "mxfp8_combine",
            "nvfp4_grouped_gemm", "nvfp4_gather_rows", "nvfp4_workspace_status",
            "nvfp4_quantize_noalloc_status"):
     getattr(_lib, _n).restype = ctypes.c_int
@@ -196,6 +198,13 @@ def mxfp8_gemm(qa, sfa, qb, sfb, M, N, K, out_dtype, D, ldd, amax_out, workspace
     _check(_lib.mxfp8_gemm(_ptr(qa), _ptr(sfa), _ptr(qb), _ptr(sfb), M, N, K, out_dtype, _ptr(D),
                            ldd, _ptr(amax_out), _ptr(workspace), ws_bytes, _stream(stream)),
            "mxfp8_gemm")
+
+
+def mxfp8_combine(q, e8, rows, cols, slot_row, weight, tokens, k, out, workspace=None,
+                  ws_bytes=0, stream=None) -> None:
+    _check(_lib.mxfp8_combine(_ptr(q), _ptr(e8), rows, cols, _ptr(slot_row), _ptr(weight), tokens,
+                              k, _ptr(out), _ptr(workspace), ws_bytes, _stream(stream)),
+           "mxfp8_combine")
 
 
 def nvfp4_grouped_gemm(G, group_offsets, total_rows, qa, sfa, ga, qb, sfb, gb, N, K, out_dtype, D,

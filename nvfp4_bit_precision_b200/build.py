@@ -13,7 +13,7 @@ ROOT = os.path.dirname(PKG)
 CSRC = os.path.join(PKG, "csrc")
 INCLUDE = os.path.join(ROOT, "include")
 LIB = os.path.join(PKG, "libnvfp4.so")
-SOURCES = ["quantize.cu", "gemm.cu", "mxfp4.cu"]
+SOURCES = ["quantize.cu", "gemm.cu", "mxfp4.cu", "moe_comm.cu"]
 HEADERS = ["common.cuh"]
 
 NVCC_FLAGS = [

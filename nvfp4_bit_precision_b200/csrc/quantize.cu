@@ -1325,7 +1325,10 @@ extern "C" nvfp4_status nvfp4_quantize(const void* x_bf16, int64_t rows, int64_t
                                        size_t ws_bytes, void* stream)
 {
     if (!x_bf16 || !p) return NVFP4_ERR_INVALID_ARG;
-    if (rows <= 0 || cols <= 0 || rows % 16 || cols % 16 || ld < cols) return NVFP4_ERR_SHAPE;
+    // MXFP8 rowwise alone quantises every row on its own: any row count will do
+    const bool mx_rows_only = p->outputs == 0 && p->mx_outputs == NVFP4_ROWWISE;
+    if (rows <= 0 || cols <= 0 || (rows % 16 && !mx_rows_only) || cols % 16 || ld < cols)
+        return NVFP4_ERR_SHAPE;
     if (!aligned16(x_bf16) || (ld * 2) % 16) return NVFP4_ERR_ALIGN;
     if (p->rounding != NVFP4_RNE && p->rounding != NVFP4_SR) return NVFP4_ERR_INVALID_ARG;
     if (p->mx_rounding != NVFP4_RNE && p->mx_rounding != NVFP4_SR) return NVFP4_ERR_INVALID_ARG;

@@ -91,6 +91,8 @@ def lib():
         L.orc_mxfp4_dequant_f64.argtypes = [P, P, i64, i64, P]
         L.orc_mxfp4_gemm_rows.argtypes = [P, P, P, P, i64, i64, i64, P, i64, P, P]
         L.orc_mxfp4_gemm_rows.restype = ctypes.c_int
+        L.orc_mxfp8_combine.argtypes = [P, P, i64, i64, P, P, i64, ctypes.c_int, P]
+        L.orc_mxfp8_combine.restype = ctypes.c_int
         _lib = L
     return _lib
 
@@ -339,3 +341,19 @@ def mxfp4_gemm_rows(qa, e8a, qb, e8b, rows_sel=None):
     if rc != 0:
         raise ValueError("oracle mxfp4 gemm: invalid arguments")
     return out, absout
+
+
+def mxfp8_combine(q, e8, slot_row, weight):
+    """bf16 bits [tokens, cols] of sum_j weight[t, j] * xhat(slot_row[t, j]) (binary32, one
+    rounding per product and per sum, j in order; slot_row -1 = none)."""
+    q = np.ascontiguousarray(q, dtype=np.uint8)
+    e8 = np.ascontiguousarray(e8, dtype=np.uint8)
+    sr = np.ascontiguousarray(slot_row, dtype=np.int32)
+    w = np.ascontiguousarray(weight, dtype=np.float32)
+    rows, cols = q.shape
+    tokens, k = sr.shape
+    out = np.zeros((tokens, cols), dtype=np.uint16)
+    rc = lib().orc_mxfp8_combine(_p(q), _p(e8), rows, cols, _p(sr), _p(w), tokens, k, _p(out))
+    if rc != 0:
+        raise ValueError("oracle mxfp8_combine: invalid arguments")
+    return out

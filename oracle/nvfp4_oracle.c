@@ -765,3 +765,41 @@ int orc_mxfp4_gemm_rows(const uint8_t* qa, const uint8_t* e8a, const uint8_t* qb
     free(bt);
     return ORC_OK;
 }
+
+/* ------------------------------------------------------------------------ */
+/* Combine of MXFP8 expert outputs [iitak, "But": expert outputs cross the   */
+/* link at 8.25 bits per number].  out[t][c] = sum_j w[t][j] * xhat(r, c),   */
+/* r = slot_row[t][j] (-1: none), xhat = e4m3(code) * 2^(e8 - 127); binary32 */
+/* with one rounding per product and per sum, j in order, as the receiving   */
+/* rank computes it; the result is rounded to bf16 (nearest even) and its    */
+/* bits returned.  The sum order is the build's definition (the pages give   */
+/* none).                                                                     */
+/* ------------------------------------------------------------------------ */
+static uint16_t f32_to_bf16_rne(float f)
+{
+    uint32_t u;
+    memcpy(&u, &f, 4);
+    uint32_t bias = ((u >> 16) & 1u) + 0x7FFFu;
+    return (uint16_t)((u + bias) >> 16);
+}
+
+int orc_mxfp8_combine(const uint8_t* q, const uint8_t* e8, int64_t rows, int64_t cols,
+                      const int32_t* slot_row, const float* w, int64_t tokens, int k,
+                      uint16_t* out)
+{
+    if (cols % 32 || k < 1) return ORC_EINVAL;
+    for (int64_t t = 0; t < tokens; ++t)
+        for (int64_t c = 0; c < cols; ++c) {
+            float acc = 0.0f;
+            for (int j = 0; j < k; ++j) {
+                int32_t r = slot_row[t * k + j];
+                if (r < 0 || r >= rows) continue;
+                float scale = (float)ldexp(1.0, (int)e8[r * (cols / 32) + c / 32] - 127);
+                float xhat = (float)orc_e4m3_decode(q[r * cols + c]) * scale;
+                float prod = w[t * k + j] * xhat;
+                acc = acc + prod;
+            }
+            out[t * cols + c] = f32_to_bf16_rne(acc);
+        }
+    return ORC_OK;
+}

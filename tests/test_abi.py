@@ -167,3 +167,17 @@ def test_mxfp4_gemm_and_layout_argument_errors(nv):
     assert g(*args, 128, 128, 256, 0, FAKE, 128, None, None, 0, None) == 7       # workspace
     assert L.mxfp4_quantize(FAKE, 32, 64, 64, 1, 5, FAKE, FAKE, None, None, None) == 1  # layout
     assert L.mxfp4_quantize(FAKE, 32, 64, 64, 1, 1, FAKE, FAKE, None, None, None) == 2  # K % 128
+
+
+def test_mxfp8_rowwise_alone_takes_any_row_count(nv):
+    """MXFP8 rowwise without NVFP4 outputs quantises rows independently, so 17 rows pass
+    validation (the call then fails only for want of a GPU); other requests keep the
+    16-row rule.  And the combine validates its shapes."""
+    L = nv._lib
+    assert L.mxfp8_quantize(FAKE, 17, 64, 64, 1, 0, 0, 0, FAKE, FAKE, None, None, None) != 2
+    assert L.mxfp8_quantize(FAKE, 17, 64, 64, 2, 0, 0, 0, None, None, FAKE, FAKE, None) == 2
+    c = L.mxfp8_combine
+    assert c(FAKE, FAKE, 4, 48, FAKE, FAKE, 2, 4, FAKE, None, 0, None) == 2      # cols % 32
+    assert c(FAKE, FAKE, 4, 64, FAKE, FAKE, 2, 0, FAKE, None, 0, None) == 1      # k
+    assert c(FAKE + 4, FAKE, 4, 64, FAKE, FAKE, 2, 4, FAKE, None, 0, None) == 3  # q alignment
+    assert c(FAKE, FAKE, 4, 64, FAKE, FAKE, 0, 4, FAKE, None, 0, None) == 0      # no tokens
