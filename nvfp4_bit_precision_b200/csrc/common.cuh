@@ -370,12 +370,15 @@ __device__ __forceinline__ float absmax3(float a, float b, float c)
     return d;
 }
 
-// max |v_i| over 16 values, starting from m (m >= 0).
+// max |v_i| over 16 values, starting from m (m >= 0).  A tree of three-input
+// maxima (depth 3 instead of a chain of 8); max is exact, so the order does not
+// change the result.
 __device__ __forceinline__ float absmax16(const float* v, float m)
 {
-#pragma unroll
-    for (int i = 0; i < 16; i += 2) m = absmax3(m, v[i], v[i + 1]);
-    return m;
+    const float a = absmax3(v[0], v[1], v[2]), b = absmax3(v[3], v[4], v[5]);
+    const float c = absmax3(v[6], v[7], v[8]), d = absmax3(v[9], v[10], v[11]);
+    const float e = absmax3(v[12], v[13], v[14]), f = absmax3(v[15], m, 0.0f);
+    return absmax3(absmax3(a, b, c), absmax3(d, e, f), 0.0f);
 }
 
 // Butterfly stages h = 1, 2, 4, 8 of the 16-point Hadamard (IEEE add/sub in a

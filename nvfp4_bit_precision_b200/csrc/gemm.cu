@@ -66,6 +66,7 @@ constexpr int kMaxAccStages = 2;
 constexpr int kEpiWarps = NVFP4_GEMM_EPI_WARPS;     // epilogue warps per CTA (8 or 16)
 constexpr int kGemmThreads = 32 * (6 + kEpiWarps);  // producer, MMA, 4 scale writers, epilogue
 static_assert(kEpiWarps == 8 || kEpiWarps == 16, "epilogue warps: 8 or 16");
+
 constexpr int kTmemCols = 512;
 constexpr int kMaxGemmGroups = 256;
 constexpr int kEpiStageBytes = 2048;  // per epilogue warp: 32 rows x 64 bytes of BF16
@@ -183,48 +184,17 @@ __device__ __forceinline__ void mbar_arrive_cluster(uint32_t bar_cluster_addr)
                  : "memory");
 }
 
-#ifndef NVFP4_GEMM_LOAD_HINT
-#define NVFP4_GEMM_LOAD_HINT 0
-#endif
-#ifndef NVFP4_GEMM_STORE_HINT
-#define NVFP4_GEMM_STORE_HINT 0
-#endif
-
 // Pair-form TMA load: the box lands in this CTA's shared memory and its bytes
 // are counted on the barrier at `bar` (a cluster address: the leader's).  No
 // multicast.  x is a multiple of 128 bytes at every call site.
 __device__ __forceinline__ void tma_load_2d_pair(void* dst, const CUtensorMap* map, int32_t x,
                                                  int32_t y, uint32_t bar)
 {
-#if NVFP4_GEMM_LOAD_HINT
-    uint64_t pol;
-    asm volatile("createpolicy.fractional.L2::evict_last.b64 %0, 1.0;" : "=l"(pol));
-    asm volatile(
-        "cp.async.bulk.tensor.2d.cta_group::2.shared::cluster.global.mbarrier::complete_tx::bytes.L2::cache_hint "
-        "[%0], [%1, {%2, %3}], [%4], %5;" ::"r"(smem_addr(dst)),
-        "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(bar), "l"(pol)
-        : "memory");
-#else
     asm volatile(
         "cp.async.bulk.tensor.2d.cta_group::2.shared::cluster.global.mbarrier::complete_tx::bytes "
         "[%0], [%1, {%2, %3}], [%4];" ::"r"(smem_addr(dst)),
         "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(bar)
         : "memory");
-#endif
-}
-
-// 16-byte store of output data.
-__device__ __forceinline__ void st_out_v4(void* p, uint4 v)
-{
-#if NVFP4_GEMM_STORE_HINT
-    uint64_t pol;
-    asm volatile("createpolicy.fractional.L2::evict_first.b64 %0, 1.0;" : "=l"(pol));
-    asm volatile("st.global.L2::cache_hint.v4.u32 [%0], {%1,%2,%3,%4}, %5;" ::"l"(p), "r"(v.x),
-                 "r"(v.y), "r"(v.z), "r"(v.w), "l"(pol)
-                 : "memory");
-#else
-    *reinterpret_cast<uint4*>(p) = v;
-#endif
 }
 
 // Four-dimensional TMA tile load completing on `bar` (x = 0 at every call site).
@@ -714,7 +684,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
                         const uint4 v = lds128(stg + r * 64 + 16 * (q ^ ((r >> 1) & 3)));
                         const int64_t grow = rowbase + r, col = cbase + 32 * hh + 8 * q;
                         if (grow < c.row_end && col < a.N)
-                            st_out_v4(static_cast<uint16_t*>(a.D) + grow * a.ldd + col, v);
+                            *reinterpret_cast<uint4*>(static_cast<uint16_t*>(a.D) + grow * a.ldd + col) = v;
                     }
                     __syncwarp();
                 }

@@ -557,19 +557,21 @@ __global__ void __launch_bounds__(256, 2) amax_rows_kernel(QArgs a, uint32_t* am
 //   2 activations: rowwise RNE, columnwise Hadamard RNE
 //   3 weights:     16x16 2D scales, both directions, RNE
 //   4 MoE rows:    rowwise RNE only (gather and groups at run time)
+//   5 MXFP8 rows:  MXFP8 rowwise only (the expert outputs of the MoE combine)
 // Fixed switches let the compiler drop the unused branches and the registers
 // they hold; results are identical to variant 0.
 enum : int8_t { kOff = 0, kOn = 1, kRt = 2 };
 struct QSpec {
     int8_t nv_row, nv_col, mx_row, mx_col, sr, mx_sr, rht, two_d, groups;
 };
-constexpr int kNumSpecs = 5;
+constexpr int kNumSpecs = 6;
 constexpr QSpec kSpecs[kNumSpecs] = {
     {kRt, kRt, kRt, kRt, kRt, kRt, kRt, kRt, kRt},
     {kOn, kOn, kOff, kOn, kOn, kOff, kOn, kOff, kOff},
     {kOn, kOn, kOff, kOff, kOff, kRt, kOn, kOff, kOff},
     {kOn, kOn, kOff, kOff, kOff, kRt, kOff, kOn, kOff},
     {kOn, kOff, kOff, kOff, kOff, kRt, kRt, kOff, kRt},
+    {kOff, kOff, kOn, kOff, kOff, kRt, kOff, kOff, kOff},
 };
 __host__ __device__ constexpr bool spec_pick(int8_t s, bool run_time)
 {
@@ -1148,6 +1150,7 @@ static QuantKernel quant_variant(bool tma, int spec)
     case 2: return tma ? quant_kernel<true, 2> : nullptr;
     case 3: return tma ? quant_kernel<true, 3> : nullptr;
     case 4: return tma ? quant_kernel<true, 4> : quant_kernel<false, 4>;
+    case 5: return tma ? quant_kernel<true, 5> : nullptr;
     }
     return nullptr;
 }
