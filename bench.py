@@ -931,6 +931,12 @@ def main():
     step.check_status()
     clocks = clk.summary()
     per_kernel = {k: [s.elapsed_time(e) for s, e in v] for k, v in ev.items()}
+    # The SM clock the dense GEMMs of the last timed step ran at: each call's own
+    # cycle count (longest CTA, entry to exit) over its CUDA-event time.  The event
+    # also spans the launch gap, so this slightly underestimates the clock.
+    kernel_mhz = [step.nv.nvfp4_gemm_cycles(step.ws[i]) / (s.elapsed_time(e) * 1e3)
+                  for i, (s, e) in zip((2, 4, 5), ev["gemm_dense"][-3:])]
+    kernel_mhz = sum(kernel_mhz) / len(kernel_mhz)
 
     # ---------------- end to end: pinned host inputs -> device, results -> host
     barrier()
@@ -1012,6 +1018,14 @@ def main():
                          "peak_note": f"dense FP4 tensor rate of the chip (ncu: 32768 FLOP per "
                                       f"SM per cycle, 148 SMs) at the median SM clock of the "
                                       f"timed region, {fp4_mhz} MHz",
+                         "sm_mhz_in_kernel": round(kernel_mhz, 1),
+                         "frac_at_kernel_clock": round(gemm_tflops / hw_fp4_peak(
+                             {"sm_mhz": kernel_mhz})[0], 4),
+                         "kernel_clock_note": "SM cycles counted inside the GEMM (clock64 of the "
+                                              "longest CTA, nvfp4_gemm_cycles) over its CUDA-event "
+                                              "time, mean of the last step's three launches: the "
+                                              "clock the power limit holds the kernel at, which "
+                                              "the NVML reading in `clocks` does not show",
                          "frac_of_4x_bf16_burst": round(gemm_tflops / derived_peak, 4),
                          "note_4x_bf16_burst": f"4 x {pk['bf16_tflops']} burst bf16 of "
                                                f"{pk['source']} (nominal fp4/bf16 ratio): "

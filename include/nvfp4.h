@@ -296,8 +296,21 @@ nvfp4_status nvfp4_dequantize(const uint8_t* q, const uint8_t* sf, const float* 
                               int64_t cols, int sf_layout, int out_dtype, void* out,
                               void* stream);
 
-/* Workspace bytes nvfp4_gemm / nvfp4_grouped_gemm need (status word). */
+/* Workspace bytes nvfp4_gemm / nvfp4_grouped_gemm / mxfp8_gemm / mxfp4_gemm
+ * need: the status word (bytes 8..11) and the call's SM cycle count (bytes
+ * 16..23), both cleared by every call. */
 size_t nvfp4_gemm_workspace_size(int64_t M, int64_t N, int64_t K);
+
+/*
+ * nvfp4_gemm_cycles -- measurement aid (no counterpart in the pages): the SM
+ * clock cycles, kernel entry to exit, of the longest-running CTA of the last
+ * GEMM call that used `workspace`.  Divided by that call's CUDA-event time it
+ * gives the SM clock the call actually ran at (the power limit lowers it under
+ * dense FP4 work, which the driver's clock readout does not show).
+ * Synchronises `stream`; *cycles is host memory.  NVFP4_ERR_INVALID_ARG for a
+ * null workspace or output pointer.
+ */
+nvfp4_status nvfp4_gemm_cycles(void* workspace, void* stream, uint64_t* cycles);
 
 /*
  * nvfp4_gemm -- block-scaled NVFP4 GEMM on the tcgen05 tensor cores

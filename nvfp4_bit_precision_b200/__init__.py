@@ -47,7 +47,7 @@ EXPORTED = [
     "nvfp4_sf_mma_grouped_bytes", "nvfp4_workspace_status", "nvfp4_status_string",
     "nvfp4_version", "nvfp4_quantize_noalloc", "nvfp4_quantize_noalloc_status",
     "nvfp4_gather_rows", "mxfp4_quantize", "mxfp8_gemm", "mxfp8_sf_mma_bytes", "mxfp4_gemm",
-    "mxfp8_combine",
+    "mxfp8_combine", "nvfp4_gemm_cycles",
 ]
 
 
@@ -99,6 +99,7 @@ _lib.nvfp4_sf_mma_bytes.restype = _SZ
 _lib.nvfp4_sf_mma_grouped_bytes.argtypes = [_I64, ctypes.c_int, _I64]
 _lib.nvfp4_sf_mma_grouped_bytes.restype = _SZ
 _lib.nvfp4_workspace_status.argtypes = [_P, _P]
+_lib.nvfp4_gemm_cycles.argtypes = [_P, _P, ctypes.POINTER(ctypes.c_uint64)]
 _lib.nvfp4_quantize_noalloc_status.argtypes = [_P]
 _lib.nvfp4_status_string.argtypes = [ctypes.c_int]
 _lib.nvfp4_status_string.restype = ctypes.c_char_p
@@ -106,7 +107,7 @@ _lib.nvfp4_version.restype = ctypes.c_int
 for _n in ("nvfp4_quantize", "nvfp4_quantize_noalloc", "mxfp8_quantize", "mxfp4_quantize",
            "nvfp4_dequantize", "nvfp4_gemm", "mxfp8_gemm", "mxfp4_gemm", "mxfp8_combine",
            "nvfp4_grouped_gemm", "nvfp4_gather_rows", "nvfp4_workspace_status",
-           "nvfp4_quantize_noalloc_status"):
+           "nvfp4_quantize_noalloc_status", "nvfp4_gemm_cycles"):
     getattr(_lib, _n).restype = ctypes.c_int
 
 
@@ -226,6 +227,15 @@ def nvfp4_gather_rows(q_src, sf_src, src_rows, k, row_index, rows, group_offsets
 
 def nvfp4_workspace_status(workspace, stream=None) -> int:
     return int(_lib.nvfp4_workspace_status(_ptr(workspace), _stream(stream)))
+
+
+def nvfp4_gemm_cycles(workspace, stream=None) -> int:
+    """SM cycles (entry to exit) of the longest CTA of the last GEMM call on
+    `workspace`; synchronises the stream."""
+    v = ctypes.c_uint64(0)
+    _check(_lib.nvfp4_gemm_cycles(_ptr(workspace), _stream(stream), ctypes.byref(v)),
+           "nvfp4_gemm_cycles")
+    return int(v.value)
 
 
 def nvfp4_quantize_noalloc_status(stream=None) -> int:

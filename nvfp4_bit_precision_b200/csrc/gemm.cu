@@ -147,6 +147,7 @@ struct GemmArgs {
     const int32_t* group_offsets;
     int64_t total_rows;
     uint32_t* status;
+    unsigned long long* cycles;  // workspace: SM cycles of the longest CTA of this call
     float* amax_out;  // optional: max |D| (as stored), atomically accumulated
     uint64_t wait_ns;  // limit of every barrier wait (2 s; shorter under the test hook)
     int no_copies;     // test hook: the producers issue no copy (see wait_test_hook)
@@ -407,6 +408,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
     const bool leader = rank == 0;
     const int pair = blockIdx.x >> 1, n_pairs = gridDim.x >> 1;
     uint8_t* epi_stage = smem + kS * C::kStageBytes + kSmemShared;
+    const long long t_entry = clock64();
 
     if (threadIdx.x == 0) {
         for (int s = 0; s < kS; ++s) {
@@ -735,6 +737,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
     cluster_sync();
     tc_fence_after();
     if (warp == 1) tmem_dealloc_pair(tmem, kTmemCols);
+    if (threadIdx.x == 0) atomicMax(a.cycles, (unsigned long long)(clock64() - t_entry));
 }
 
 // ---------------------------------------------------------------- host side
@@ -863,8 +866,8 @@ static nvfp4_status launch_variant(const void* qa, const void* qb, GemmArgs& a, 
     if (kBN == 256 &&
         !make_sfb_map(&msf, a.sfb, a.G, a.N, a.K, C::kKStage, C::kKAtom, C::kSfAtoms))
         return NVFP4_ERR_CUDA;
-    // the status word reports this call only; the output amax starts at 0
-    if (cudaMemsetAsync(a.status, 0, 4, st) != cudaSuccess) return NVFP4_ERR_CUDA;
+    // the status word and the cycle count report this call only; the output amax starts at 0
+    if (cudaMemsetAsync(a.status, 0, 16, st) != cudaSuccess) return NVFP4_ERR_CUDA;
     if (a.amax_out && cudaMemsetAsync(a.amax_out, 0, 4, st) != cudaSuccess) return NVFP4_ERR_CUDA;
     const int64_t tiles = max_tiles_m * ((a.N + kBN - 1) / kBN);
     const int pairs = (int)std::max<int64_t>(1, std::min<int64_t>(tiles, info.pairs));
@@ -886,6 +889,21 @@ static nvfp4_status launch_gemm(const void* qa, const void* qb, GemmArgs& a, int
 using namespace nvfp4;
 
 extern "C" size_t nvfp4_gemm_workspace_size(int64_t, int64_t, int64_t) { return kGemmWorkspace; }
+
+// SM clock cycles, from entry to exit, of the longest-running CTA of the last
+// GEMM call given this workspace (bytes 16..23).  Divided by the call's
+// CUDA-event time it gives the SM clock the call ran at.
+extern "C" nvfp4_status nvfp4_gemm_cycles(void* workspace, void* stream, uint64_t* cycles)
+{
+    if (!workspace || !cycles) return NVFP4_ERR_INVALID_ARG;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    unsigned long long v = 0;
+    const unsigned long long* src = static_cast<const unsigned long long*>(workspace) + 2;
+    if (cudaMemcpyAsync(&v, src, 8, cudaMemcpyDeviceToHost, st) != cudaSuccess) return NVFP4_ERR_CUDA;
+    if (cudaStreamSynchronize(st) != cudaSuccess) return NVFP4_ERR_CUDA;
+    *cycles = v;
+    return NVFP4_OK;
+}
 
 // Checks shared by the dense GEMMs; k_mult is the K granularity of a stage.
 static nvfp4_status check_dense(const uint8_t* qa, const uint8_t* sfa, const uint8_t* qb,
@@ -930,6 +948,7 @@ extern "C" nvfp4_status nvfp4_gemm(const uint8_t* qa, const uint8_t* sfa, const 
     a.grouped = 0;
     a.G = 1;
     a.status = static_cast<uint32_t*>(workspace) + 2;
+    a.cycles = static_cast<unsigned long long*>(workspace) + 2;
     a.amax_out = amax_out;
     return launch_gemm<kFmtNVFP4>(qa, qb, a, M, N, (M + kMmaM - 1) / kMmaM,
                                   static_cast<cudaStream_t>(stream));
@@ -955,6 +974,7 @@ extern "C" nvfp4_status mxfp8_gemm(const uint8_t* qa, const uint8_t* sfa, const 
     a.grouped = 0;
     a.G = 1;
     a.status = static_cast<uint32_t*>(workspace) + 2;
+    a.cycles = static_cast<unsigned long long*>(workspace) + 2;
     a.amax_out = amax_out;
     return launch_gemm<kFmtMXFP8>(qa, qb, a, M, N, (M + kMmaM - 1) / kMmaM,
                                   static_cast<cudaStream_t>(stream));
@@ -980,6 +1000,7 @@ extern "C" nvfp4_status mxfp4_gemm(const uint8_t* qa, const uint8_t* sfa, const 
     a.grouped = 0;
     a.G = 1;
     a.status = static_cast<uint32_t*>(workspace) + 2;
+    a.cycles = static_cast<unsigned long long*>(workspace) + 2;
     a.amax_out = amax_out;
     return launch_gemm<kFmtMXFP4>(qa, qb, a, M, N, (M + kMmaM - 1) / kMmaM,
                                   static_cast<cudaStream_t>(stream));
@@ -1019,6 +1040,7 @@ extern "C" nvfp4_status nvfp4_grouped_gemm(int G, const int32_t* group_offsets, 
     a.group_offsets = group_offsets;
     a.total_rows = total_rows;
     a.status = static_cast<uint32_t*>(workspace) + 2;
+    a.cycles = static_cast<unsigned long long*>(workspace) + 2;
     a.amax_out = amax_out;
     // upper bound on M tiles: every group may add one partial tile
     return launch_gemm<kFmtNVFP4>(qa, qb, a, total_rows, (int64_t)G * N,

@@ -41,7 +41,14 @@ def test_size_helpers(nv):
     assert nv.nvfp4_sf_mma_bytes(130, 256) == 256 * 16
     assert nv.nvfp4_sf_mma_grouped_bytes(300, 4, 512) == (384 + 512) * 32
     assert nv.nvfp4_quantize_workspace_size() >= 16
-    assert nv.nvfp4_gemm_workspace_size() >= 16
+    assert nv.nvfp4_gemm_workspace_size() >= 24  # status word + the call's cycle count
+
+
+def test_gemm_cycles_argument_errors(nv):
+    c = ctypes.c_uint64(7)
+    assert nv._lib.nvfp4_gemm_cycles(None, None, ctypes.byref(c)) == 1
+    assert nv._lib.nvfp4_gemm_cycles(FAKE, None, None) == 1
+    assert c.value == 7
 
 
 FAKE = 1 << 20  # a 16-byte aligned non-null address that validation never dereferences

@@ -258,3 +258,38 @@ def test_all_zero_operands(nv, orc):
     am = torch.full((1,), 7.0, dtype=torch.float32, device="cuda")
     D = host(nv.gemm(out["row"], out["row"], nv.NVFP4_OUT_F32, amax_out=am))
     assert not np.any(D) and host(am)[0] == 0.0
+
+
+def test_gemm_cycle_count(nv):
+    """The workspace's cycle count of a GEMM call: positive, cleared by the next
+    call, and divided by the call's CUDA-event time a clock between 0.5 and 2.2 GHz
+    (the B200's SM clock range)."""
+    import torch
+    dev = torch.device("cuda")
+    M, N, K = 4096, 4096, 4096
+    g = torch.Generator(device=dev)
+    g.manual_seed(0)
+    u8 = dict(dtype=torch.uint8, device=dev)
+    qa = torch.randint(0, 256, (M, K // 2), generator=g, **u8)
+    qb = torch.randint(0, 256, (N, K // 2), generator=g, **u8)
+    sa = torch.randint(0x30, 0x40, (nv.nvfp4_sf_mma_bytes(M, K),), generator=g, **u8)
+    sb = torch.randint(0x30, 0x40, (nv.nvfp4_sf_mma_bytes(N, K),), generator=g, **u8)
+    one = torch.ones(1, dtype=torch.float32, device=dev)
+    D = torch.empty((M, N), dtype=torch.bfloat16, device=dev)
+    ws = torch.zeros(nv.nvfp4_gemm_workspace_size(M, N, K), **u8)
+    for _ in range(3):
+        nv.nvfp4_gemm(qa, sa, one, qb, sb, one, M, N, K, nv.NVFP4_OUT_BF16, D, N, None, ws, ws.numel())
+    s, e = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    s.record()
+    nv.nvfp4_gemm(qa, sa, one, qb, sb, one, M, N, K, nv.NVFP4_OUT_BF16, D, N, None, ws, ws.numel())
+    e.record()
+    e.synchronize()
+    cycles = nv.nvfp4_gemm_cycles(ws)
+    mhz = cycles / (s.elapsed_time(e) * 1e3)
+    assert nv.nvfp4_workspace_status(ws) == 0
+    assert 500 < mhz < 2200, (cycles, mhz)
+    # the next call restarts the count
+    nv.nvfp4_gemm(qa, sa, one, qb, sb, one, 256, 256, 256, nv.NVFP4_OUT_BF16, D, N, None, ws,
+                  ws.numel())
+    small = nv.nvfp4_gemm_cycles(ws)
+    assert 0 < small < cycles
