@@ -46,7 +46,7 @@ DENSE_FLOP_PER_GEMM = 2 * TOKENS * FFN * HIDDEN
 # ncu --set full capture of each kernel as it stands -- the forward GEMM
 # 16384x20480x5120, and the amax + fused pass on dY 16384x20480; set to None
 # whenever the kernel changes.
-TRAFFIC_BYTES = {"gemm_dense_fwd": 1147.7e6, "quant_dy": 2076.1e6}
+TRAFFIC_BYTES = {"gemm_dense_fwd": 1147.2e6, "quant_dy": 2076.1e6}
 
 
 def peaks():
@@ -95,9 +95,11 @@ class Step:
         self.Dr, self.Dc = mk(T, F), mk(F, T)
         self.mx_q = torch.empty((F, T), **u8)
         self.mx_e = torch.empty((F, T // 32), **u8)
-        self.Y = torch.empty((T, F), **bf)
-        self.dX = torch.empty((T, H), **bf)
-        self.dW = torch.empty((F, H), **bf)
+        # Two output slots, so the end-to-end loop can read step i's results back
+        # while step i+1 computes; self.Y etc. are slot 0's.
+        self.outs = [dict(Y=torch.empty((T, F), **bf), dX=torch.empty((T, H), **bf),
+                          dW=torch.empty((F, H), **bf)) for _ in range(2)]
+        self.Y, self.dX, self.dW = (self.outs[0][k] for k in ("Y", "dX", "dW"))
         self.ws = [torch.zeros(256, **u8) for _ in range(8)]
         # MoE: expert weights are quantised once (outside the step), activations every step
         R = self.routed
@@ -112,7 +114,9 @@ class Step:
         self.A_dn = nv.NVFP4Tensor(torch.empty((R, MOE_FFN // 2), **u8),
                                    torch.zeros(gsf(R, EXPERTS, MOE_FFN), **u8),
                                    torch.empty(1, **f32), R, MOE_FFN, nv.NVFP4_SF_MMA)
-        self.Out = torch.empty((R, MOE_HIDDEN), **bf)
+        for o in self.outs:
+            o["Out"] = torch.empty((R, MOE_HIDDEN), **bf)
+        self.Out = self.outs[0]["Out"]
         self.wup = self._quantize_experts(h["w_up"], MOE_FFN, MOE_HIDDEN)
         self.wdn = self._quantize_experts(h["w_down"], MOE_HIDDEN, MOE_FFN)
         torch.cuda.synchronize(dev)
@@ -186,13 +190,14 @@ class Step:
 
         ws = self.ws
         inp = self.inputs[slot]
+        out = self.outs[slot]
         timed("quant_x", lambda: self._q(inp["x"], T, H, H, self.Xr, self.Xc, ws[0], rht=1))
         timed("quant_w", lambda: self._q(inp["w"], F, H, H, self.Wr, self.Wc, ws[1], scaling=1))
-        timed("gemm_dense", lambda: self._g(self.Xr, self.Wr, self.Y, ws[2]))
+        timed("gemm_dense", lambda: self._g(self.Xr, self.Wr, out["Y"], ws[2]))
         timed("quant_dy", lambda: self._q(inp["dy"], T, F, F, self.Dr, self.Dc, ws[3], rounding=1,
                                           rht=1, mx_col=(self.mx_q, self.mx_e)))
-        timed("gemm_dense", lambda: self._g(self.Dr, self.Wc, self.dX, ws[4]))
-        timed("gemm_dense", lambda: self._g(self.Dc, self.Xc, self.dW, ws[5]))
+        timed("gemm_dense", lambda: self._g(self.Dr, self.Wc, out["dX"], ws[4]))
+        timed("gemm_dense", lambda: self._g(self.Dc, self.Xc, out["dW"], ws[5]))
         # MoE expert forward
         R = self.routed
         timed("quant_tok", lambda: self._q(inp["tok"], MOE_TOKENS, MOE_HIDDEN, MOE_HIDDEN, self.Tq,
@@ -209,7 +214,7 @@ class Step:
         qd, sd, gd = self.wdn
         timed("gemm_grouped", lambda: nv.nvfp4_grouped_gemm(
             EXPERTS, self.offsets, R, self.A_dn.q, self.A_dn.sf, self.A_dn.g, qd, sd, gd,
-            MOE_HIDDEN, MOE_FFN, nv.NVFP4_OUT_BF16, self.Out, None, ws[7], 256))
+            MOE_HIDDEN, MOE_FFN, nv.NVFP4_OUT_BF16, out["Out"], None, ws[7], 256))
 
     # dense: 3 quantise calls x (amax + fused pass) + 3 GEMMs; MoE: token quantise (amax +
     # fused pass), dispatch, 2 grouped GEMMs, H quantise (fused pass only: amax from the GEMM)
@@ -218,14 +223,15 @@ class Step:
     def flops(self):
         return DENSE_FLOP + 2 * 2 * self.routed * MOE_FFN * MOE_HIDDEN
 
-    def _outputs(self):
-        return [self.Y, self.dX, self.dW, self.Out]
+    def _outputs(self, slot=0):
+        o = self.outs[slot]
+        return [o["Y"], o["dX"], o["dW"], o["Out"]]
 
-    def results_d2h(self, host_bufs):
-        """Copy every output of the step in full (Y, dX, dW and the MoE output, 1.58 GB of
-        bf16) into pinned host buffers, asynchronously on the current stream; returns the
-        bytes copied."""
-        outs = self._outputs()
+    def results_d2h(self, host_bufs, slot=0):
+        """Copy every output of the step in output slot `slot` in full (Y, dX, dW and the
+        MoE output, 1.58 GB of bf16) into pinned host buffers, asynchronously on the
+        current stream; returns the bytes copied."""
+        outs = self._outputs(slot)
         for h, o in zip(host_bufs, outs):
             h.copy_(o, non_blocking=True)
         return sum(o.numel() * o.element_size() for o in outs)
@@ -947,13 +953,17 @@ def main():
     # ---------------- end to end: pinned host inputs -> device, results -> host
     barrier()
     torch.cuda.synchronize()
-    # Step i+1's inputs are copied (from pinned host memory, on a copy stream) while
-    # step i computes; every step copies its own inputs and reads its results back.
+    # Step i+1's inputs are copied in (from pinned host memory, on a copy stream) and
+    # step i-1's results are read back (into pinned host memory, on a second copy
+    # stream) while step i computes; every step copies its own inputs in and all of
+    # its results out.  Inputs and outputs have two slots each.
     e0 = torch.cuda.Event(enable_timing=True)
     e1 = torch.cuda.Event(enable_timing=True)
     copy_stream = torch.cuda.Stream(device=dev)
-    landed = [torch.cuda.Event(), torch.cuda.Event()]   # slot's inputs copied
-    consumed = [torch.cuda.Event(), torch.cuda.Event()]  # slot's step done with its inputs
+    d2h_stream = torch.cuda.Stream(device=dev)
+    landed = [torch.cuda.Event(), torch.cuda.Event()]    # slot's inputs copied in
+    consumed = [torch.cuda.Event(), torch.cuda.Event()]   # slot's step done (inputs free)
+    read_back = [torch.cuda.Event(), torch.cuda.Event()]  # slot's outputs copied out
     host_out = [step.result_host_buffers() for _ in range(2)]
     e0.record(stream)
     copy_stream.wait_event(e0)
@@ -971,9 +981,16 @@ def main():
                 step.upload_inputs(nxt, non_blocking=True)
             landed[nxt].record(copy_stream)
         stream.wait_event(landed[slot])
+        if i >= 2:
+            stream.wait_event(read_back[slot])  # step i-2's results are out of this slot
         step.run(slot=slot)
         consumed[slot].record(stream)
-        d2h = step.results_d2h(host_out[slot])
+        d2h_stream.wait_event(consumed[slot])
+        with torch.cuda.stream(d2h_stream):
+            d2h = step.results_d2h(host_out[slot], slot)
+        read_back[slot].record(d2h_stream)
+    stream.wait_stream(d2h_stream)
+    stream.wait_stream(copy_stream)
     e1.record(stream)
     torch.cuda.synchronize()
     barrier()
@@ -1068,7 +1085,12 @@ def main():
                     "value": round(3 * DENSE_FLOP_PER_GEMM / (lin_ms / 1e3) / 1e12, 1),
                     "unit": "TFLOP/s"}},
             "e2e": {"value": round(value_e2e, 2), "unit": "TFLOP/s",
-                    "h2d_bytes_per_step": step.h2d_bytes(), "d2h_bytes_per_step": d2h},
+                    "h2d_bytes_per_step": step.h2d_bytes(), "d2h_bytes_per_step": d2h,
+                    "ms_per_step": round(ms_e2e / args.steps, 3),
+                    "note": "every step copies all its bf16 inputs in from pinned host memory "
+                            "and all its bf16 outputs out in full; copies in, kernels and "
+                            "copies out of consecutive steps overlap on three streams (two "
+                            "input and two output slots): PCIe bounds it"},
             "gpu_launches": Step.LAUNCHES_PER_STEP * args.steps,
             "clocks": clocks,
         }
