@@ -630,7 +630,6 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
                 // arrive (two loads in flight per wait for 64-column warps): the
                 // accumulator is released before any store.
                 uint32_t packed[16 * kChunks];
-                float m_all = 0.0f;  // max |x| over the warp's columns (before rounding)
                 constexpr int kPer = (kChunks == 2 && kEpiWarps == 8) ? 2 : 1;
 #pragma unroll
                 for (int hh = 0; hh < kChunks; hh += kPer) {
@@ -640,9 +639,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
                     tmem_ld_wait();
 #pragma unroll
                     for (int i = 0; i < 16 * kPer; ++i) {
-                        const float x0 = __fmul_rn(__uint_as_float(r[2 * i]), alpha);
-                        const float x1 = __fmul_rn(__uint_as_float(r[2 * i + 1]), alpha);
-                        m_all = absmax3(m_all, x0, x1);
+                        float x0, x1;  // two IEEE products, as two __fmul_rn
+                        mul2(x0, x1, __uint_as_float(r[2 * i]), __uint_as_float(r[2 * i + 1]), alpha, alpha);
                         const __nv_bfloat162 p = __floats2bfloat162_rn(x0, x1);
                         packed[16 * hh + i] = *reinterpret_cast<const uint32_t*>(&p);
                     }
@@ -651,22 +649,19 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
                 __syncwarp();
                 if (lane == 0) mbar_arrive_cluster(cluster_addr(&sh->acc_empty[buf], 0));  // accumulator drained
                 const int64_t cbase = c.n0 + col0;
-                // max |D| of this lane's row (rounded values where the N tail cuts the row)
-                if (row_ok) {
-                    if (cbase + kCols <= a.N) {
-                        out_max = fmaxf(out_max, m_all);
-                    } else {
+                // max |D| of this lane's stored (rounded) values, after the accumulator
+                // is released: only when asked for, and off the drain's critical path
+                if (a.amax_out && row_ok) {
 #pragma unroll
-                        for (int g = 0; g < 4 * kChunks; ++g)
-                            if (cbase + 8 * g < a.N) {
+                    for (int g = 0; g < 4 * kChunks; ++g)
+                        if (cbase + 8 * g < a.N) {
 #pragma unroll
-                                for (int i = 0; i < 4; ++i) {
-                                    const uint32_t w = packed[4 * g + i];
-                                    out_max = absmax3(out_max, __uint_as_float(w << 16),
-                                                      __uint_as_float(w & 0xFFFF0000u));
-                                }
+                            for (int i = 0; i < 4; ++i) {
+                                const uint32_t w = packed[4 * g + i];
+                                out_max = absmax3(out_max, __uint_as_float(w << 16),
+                                                  __uint_as_float(w & 0xFFFF0000u));
                             }
-                    }
+                        }
                 }
                 const int64_t rowbase = c.row0 + (int64_t)BM * rank + 32 * quad;
                 // 32-column chunks through a 64-byte-swizzled 32x64-byte staging
