@@ -486,7 +486,7 @@ def time_mxfp8_backward(step, steps, warmup, fp8_peak, hw_fp8_peak):
                                            nv.NVFP4_OUT_BF16, step.dX, H, None, step.ws[4], 256),
             "wgrad": lambda: nv.mxfp8_gemm(dyc[0], dyc[1], xc[0], xc[1], F, H, T,
                                            nv.NVFP4_OUT_BF16, step.dW, H, None, step.ws[5], 256)}
-    ms = {}
+    ms, mhz = {}, {}
     for name, fn in runs.items():
         for _ in range(max(warmup, 3)):
             fn()
@@ -499,6 +499,9 @@ def time_mxfp8_backward(step, steps, warmup, fp8_peak, hw_fp8_peak):
             evs.append((s_, e_))
         torch.cuda.synchronize()
         ms[name] = sum(a.elapsed_time(b) for a, b in evs) / steps
+        if name != "quant_dy":  # the last launch's own SM clock
+            ws_i = step.ws[4] if name == "dgrad" else step.ws[5]
+            mhz[name] = nv.nvfp4_gemm_cycles(ws_i) / (evs[-1][0].elapsed_time(evs[-1][1]) * 1e3)
     step.check_status()
     flop = 2 * T * H * F
     tf = {k: flop / (ms[k] / 1e3) / 1e12 for k in ("dgrad", "wgrad")}
@@ -517,6 +520,7 @@ def time_mxfp8_backward(step, steps, warmup, fp8_peak, hw_fp8_peak):
             "hw_fp8_peak": round(hw_fp8_peak, 1),
             "hw_peak_note": "dense FP8 tensor rate of the chip (16384 FLOP per SM per cycle) at the "
                             "sampled SM clock",
+            "sm_mhz_in_kernel": round((mhz["dgrad"] + mhz["wgrad"]) / 2, 1),
             "quant_dy_mxfp8_both_us": round(ms["quant_dy"] * 1e3, 1),
             "quant_dy_mxfp8_both_gbs": round(qbytes / (ms["quant_dy"] / 1e3) / 1e9, 1)}
 
@@ -547,12 +551,14 @@ def time_mxfp4_gemm(step, steps, warmup, fp4_peak, hw_fp4):
     step.check_status()
     ms = sum(a.elapsed_time(b) for a, b in evs) / steps
     tf = DENSE_FLOP_PER_GEMM / (ms / 1e3) / 1e12
+    mhz = nv.nvfp4_gemm_cycles(step.ws[2]) / (evs[-1][0].elapsed_time(evs[-1][1]) * 1e3)
     return {"kernel": "gemm_kernel<MXFP4> (tcgen05 kind::mxf4, UE8M0 block-32 scales), "
                       "16384x20480x5120, bf16 out, timed apart from the step", "bound": "tensor",
             "us": round(ms * 1e3, 1), "achieved": round(tf, 1), "peak": round(fp4_peak, 1),
             "unit": "TFLOP/s", "frac": round(tf / fp4_peak, 4),
             "peak_note": "4 x the measured bf16 burst rate (nominal fp4/bf16 ratio)",
-            "frac_of_hw_fp4_peak": round(tf / hw_fp4, 4)}
+            "frac_of_hw_fp4_peak": round(tf / hw_fp4, 4),
+            "sm_mhz_in_kernel": round(mhz, 1)}
 
 
 def time_moe_combine(step, steps, warmup, pk):
@@ -994,6 +1000,12 @@ def main():
     e1.record(stream)
     torch.cuda.synchronize()
     barrier()
+    if args.steps >= 2:
+        # Both slots computed the same inputs (a fixed seed): their read-back results
+        # must agree bit for bit, or the overlap of copies and kernels raced.
+        for a_, b_ in zip(host_out[0], host_out[1]):
+            if not torch.equal(a_, b_):
+                raise RuntimeError("end-to-end results differ between the two slots")
     ms_e2e = e0.elapsed_time(e1)
 
     mx4_ms, mx4_bytes = time_mxfp4(step, args.steps, args.warmup)
