@@ -633,7 +633,8 @@ class ClockSampler:
     REASONS = (("hw_slowdown", "nvmlClocksEventReasonHwSlowdown", 0x8),
                ("hw_thermal_slowdown", "nvmlClocksEventReasonHwThermalSlowdown", 0x40),
                ("sw_thermal_slowdown", "nvmlClocksEventReasonSwThermalSlowdown", 0x20),
-               ("sw_power_cap", "nvmlClocksEventReasonSwPowerCap", 0x4))
+               ("sw_power_cap", "nvmlClocksEventReasonSwPowerCap", 0x4),
+               ("hw_power_brake_slowdown", "nvmlClocksEventReasonHwPowerBrakeSlowdown", 0x80))
 
     def __init__(self, device):
         self.device = device
@@ -665,7 +666,11 @@ class ClockSampler:
             try:
                 mhz = N.nvmlDeviceGetClockInfo(self.handle, N.NVML_CLOCK_SM)
                 bits = get_reasons(self.handle) if get_reasons else 0
-                self.samples.append((mhz, bits))
+                try:
+                    watts = N.nvmlDeviceGetPowerUsage(self.handle) / 1000.0
+                except Exception:
+                    watts = None
+                self.samples.append((mhz, bits, watts))
             except Exception:
                 pass
             self.stop.wait(0.005)
@@ -696,13 +701,18 @@ class ClockSampler:
         if not self.samples:
             return {"sm_mhz": None, "sm_max_mhz": self.max_mhz, "reasons": ["unsampled"]}
         reasons = set()
-        for _, bits in self.samples:
+        for smp in self.samples:
             for name, attr, default in self.REASONS:
-                if bits & getattr(self.nvml, attr, default):
+                if smp[1] & getattr(self.nvml, attr, default):
                     reasons.add(name)
-        return {"sm_mhz": statistics.median(m for m, _ in self.samples),
-                "sm_max_mhz": self.max_mhz, "reasons": sorted(reasons),
-                "samples": len(self.samples), "source": "nvml, 5 ms"}
+        watts = [smp[2] for smp in self.samples if len(smp) > 2 and smp[2] is not None]
+        out = {"sm_mhz": statistics.median(smp[0] for smp in self.samples),
+               "sm_max_mhz": self.max_mhz, "reasons": sorted(reasons),
+               "samples": len(self.samples), "source": "nvml, 5 ms"}
+        if watts:
+            out["power_w_median"] = round(statistics.median(watts), 1)
+            out["power_w_max"] = round(max(watts), 1)
+        return out
 
 
 # ----------------------------------------------------------------------------- CPU oracle
