@@ -46,7 +46,7 @@ DENSE_FLOP_PER_GEMM = 2 * TOKENS * FFN * HIDDEN
 # ncu --set full capture of each kernel as it stands -- the forward GEMM
 # 16384x20480x5120, and the amax + fused pass on dY 16384x20480; set to None
 # whenever the kernel changes.
-TRAFFIC_BYTES = {"gemm_dense_fwd": 1147.2e6, "quant_dy": 2076.1e6}
+TRAFFIC_BYTES = {"gemm_dense_fwd": 1147.3e6, "quant_dy": 2076.1e6}
 
 
 def peaks():
@@ -666,11 +666,7 @@ class ClockSampler:
             try:
                 mhz = N.nvmlDeviceGetClockInfo(self.handle, N.NVML_CLOCK_SM)
                 bits = get_reasons(self.handle) if get_reasons else 0
-                try:
-                    watts = N.nvmlDeviceGetPowerUsage(self.handle) / 1000.0
-                except Exception:
-                    watts = None
-                self.samples.append((mhz, bits, watts))
+                self.samples.append((mhz, bits))
             except Exception:
                 pass
             self.stop.wait(0.005)
@@ -705,14 +701,9 @@ class ClockSampler:
             for name, attr, default in self.REASONS:
                 if smp[1] & getattr(self.nvml, attr, default):
                     reasons.add(name)
-        watts = [smp[2] for smp in self.samples if len(smp) > 2 and smp[2] is not None]
-        out = {"sm_mhz": statistics.median(smp[0] for smp in self.samples),
-               "sm_max_mhz": self.max_mhz, "reasons": sorted(reasons),
-               "samples": len(self.samples), "source": "nvml, 5 ms"}
-        if watts:
-            out["power_w_median"] = round(statistics.median(watts), 1)
-            out["power_w_max"] = round(max(watts), 1)
-        return out
+        return {"sm_mhz": statistics.median(smp[0] for smp in self.samples),
+                "sm_max_mhz": self.max_mhz, "reasons": sorted(reasons),
+                "samples": len(self.samples), "source": "nvml, 5 ms"}
 
 
 # ----------------------------------------------------------------------------- CPU oracle
