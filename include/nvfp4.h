@@ -395,7 +395,7 @@ nvfp4_status nvfp4_grouped_gemm(int G, const int32_t* group_offsets, int64_t tot
  * rounding per product and per sum, j in order,
  *   out[t][c] = sum_j weight[t][j] * (e4m3(q[r][c]) * 2^(e8[r][c/32] - 127)),
  * then RNE to bf16 into out_bf16 [tokens, cols].  cols a multiple of 32;
- * 1 <= k <= 64; q 8-byte and out 16-byte aligned.  A row index >= rows is
+ * 1 <= k <= 64; q and out 16-byte aligned.  A row index >= rows is
  * skipped and reported in the optional workspace's status word
  * (NVFP4_ERR_INDEX).  Asynchronous on `stream`; allocates nothing.
  */

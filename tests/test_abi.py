@@ -187,4 +187,5 @@ def test_mxfp8_rowwise_alone_takes_any_row_count(nv):
     assert c(FAKE, FAKE, 4, 48, FAKE, FAKE, 2, 4, FAKE, None, 0, None) == 2      # cols % 32
     assert c(FAKE, FAKE, 4, 64, FAKE, FAKE, 2, 0, FAKE, None, 0, None) == 1      # k
     assert c(FAKE + 4, FAKE, 4, 64, FAKE, FAKE, 2, 4, FAKE, None, 0, None) == 3  # q alignment
+    assert c(FAKE + 8, FAKE, 4, 64, FAKE, FAKE, 2, 4, FAKE, None, 0, None) == 3  # 16 bytes
     assert c(FAKE, FAKE, 4, 64, FAKE, FAKE, 0, 4, FAKE, None, 0, None) == 0      # no tokens
