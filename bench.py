@@ -580,26 +580,33 @@ def time_moe_combine(step, steps, warmup, pk):
     q, e8 = torch.empty((R, H), **u8), torch.empty((R, H // 32), **u8)
     out = torch.empty((MOE_TOKENS, H), dtype=torch.bfloat16, device=dev)
 
-    def run():
-        nv.mxfp8_quantize(step.Out, R, H, H, nv.NVFP4_ROWWISE, 0, 0, 0, q, e8, None, None)
-        nv.mxfp8_combine(q, e8, R, H, slot, w, MOE_TOKENS, TOPK, out, step.ws[6], 256)
+    quant = lambda: nv.mxfp8_quantize(step.Out, R, H, H, nv.NVFP4_ROWWISE, 0, 0, 0, q, e8, None, None)
+    comb = lambda: nv.mxfp8_combine(q, e8, R, H, slot, w, MOE_TOKENS, TOPK, out, step.ws[6], 256)
 
     for _ in range(max(warmup, 3)):
-        run()
+        quant()
+        comb()
     stream = torch.cuda.current_stream()
-    s_, e_ = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    evs = []
     torch.cuda.synchronize()
-    s_.record(stream)
     for _ in range(steps):
-        run()
-    e_.record(stream)
+        ev3 = [torch.cuda.Event(enable_timing=True) for _ in range(3)]
+        ev3[0].record(stream)
+        quant()
+        ev3[1].record(stream)
+        comb()
+        ev3[2].record(stream)
+        evs.append(ev3)
     torch.cuda.synchronize()
     step.check_status()
-    ms = s_.elapsed_time(e_) / steps
+    q_ms = sum(a.elapsed_time(b) for a, b, _ in evs) / steps
+    c_ms = sum(b.elapsed_time(c) for _, b, c in evs) / steps
+    ms = q_ms + c_ms
     nbytes = 2 * R * H + 2 * (R * H + R * H // 32) + MOE_TOKENS * H * 2
     return {"kernel": "mxfp8_quantize (rowwise) + mxfp8_combine_kernel on the MoE output "
                       "65536x4096 -> 16384x4096 bf16, top-4 weights 1/4", "bound": "hbm",
-            "us": round(ms * 1e3, 1), "algorithmic_bytes": nbytes,
+            "us": round(ms * 1e3, 1), "quantize_us": round(q_ms * 1e3, 1),
+            "combine_us": round(c_ms * 1e3, 1), "algorithmic_bytes": nbytes,
             "achieved": round(nbytes / (ms / 1e3) / 1e9, 1), "peak": pk["hbm_gbs"], "unit": "GB/s",
             "frac": round(nbytes / (ms / 1e3) / 1e9 / pk["hbm_gbs"], 4),
             "link_bytes_mxfp8": R * H + R * H // 32, "link_bytes_bf16": 2 * R * H,
