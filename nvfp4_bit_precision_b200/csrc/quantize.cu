@@ -1038,17 +1038,29 @@ __global__ void __launch_bounds__(256) gather_rows_kernel(
         s_src[i] = s;
     }
     __syncthreads();
-    // codes: 16-byte vectors, one row after another
-    for (int64_t idx = threadIdx.x; idx < (int64_t)nr * chunks; idx += blockDim.x) {
-        const int i = (int)(idx / chunks);
-        const int64_t c = idx - (int64_t)i * chunks;
-        const uint4 v = *reinterpret_cast<const uint4*>(q_src + s_src[i] * (k / 2) + c * 16);
-        *reinterpret_cast<uint4*>(q_dst + (r0 + i) * (k / 2) + c * 16) = v;
+    // codes: one warp per row at a time, its lanes on consecutive 16-byte
+    // vectors, four loads in flight per lane before their stores
+    {
+        const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+        const int nwarps = blockDim.x >> 5;
+        for (int i = warp; i < nr; i += nwarps) {
+            const uint4* __restrict__ src = reinterpret_cast<const uint4*>(q_src + s_src[i] * (k / 2));
+            uint4* __restrict__ dst = reinterpret_cast<uint4*>(q_dst + (r0 + i) * (k / 2));
+            int64_t c = lane;
+            for (; c + 96 < chunks; c += 128) {
+                const uint4 v0 = src[c], v1 = src[c + 32], v2 = src[c + 64], v3 = src[c + 96];
+                dst[c] = v0;
+                dst[c + 32] = v1;
+                dst[c + 64] = v2;
+                dst[c + 96] = v3;
+            }
+            for (; c < chunks; c += 32) dst[c] = src[c];
+        }
     }
     // scales: 4 bytes (one row's four 16-blocks of a 64-column group) at a time
-    for (int64_t idx = threadIdx.x; idx < (int64_t)nr * k64; idx += blockDim.x) {
-        const int64_t j = idx / nr;
-        const int i = (int)(idx - j * nr);
+    for (int idx = threadIdx.x; idx < nr * (int)k64; idx += blockDim.x) {  // < 2^31: k <= 2^30
+        const int j = idx / nr;
+        const int i = idx - j * nr;
         const int64_t s = s_src[i];
         const uint32_t v = *reinterpret_cast<const uint32_t*>(sf_src + sf_mma_offset(s, 4 * j, k16));
         *reinterpret_cast<uint32_t*>(sf_dst + sf_mma_offset(dst_blk * 128 + i, 4 * j, k16)) = v;
@@ -1493,7 +1505,7 @@ extern "C" nvfp4_status nvfp4_gather_rows(const uint8_t* q_src, const uint8_t* s
                                           void* workspace, size_t ws_bytes, void* stream)
 {
     if (!q_src || !sf_src || !row_index || !q_dst || !sf_dst) return NVFP4_ERR_INVALID_ARG;
-    if (src_rows <= 0 || rows <= 0 || k <= 0 || k % 64) return NVFP4_ERR_SHAPE;
+    if (src_rows <= 0 || rows <= 0 || k <= 0 || k % 64 || k > (int64_t(1) << 30)) return NVFP4_ERR_SHAPE;
     if (group_offsets && (num_groups < 1 || num_groups > kMaxGroups)) return NVFP4_ERR_INVALID_ARG;
     if (!aligned16(q_src) || !aligned16(q_dst) || (reinterpret_cast<uintptr_t>(sf_src) & 3) ||
         (reinterpret_cast<uintptr_t>(sf_dst) & 3))
