@@ -989,34 +989,53 @@ __global__ void __launch_bounds__(kQuantThreads, 2)
 // the grouped tiled layout.  One CTA per (group, 128-row block), the blocks the
 // grouped GEMM tiles over, so each CTA writes whole 512-byte scale atoms.
 // --------------------------------------------------------------------------
-__global__ void __launch_bounds__(256) gather_rows_kernel(
+__global__ void __launch_bounds__(512) gather_rows_kernel(
     const uint8_t* q_src, const uint8_t* sf_src, int64_t src_rows, int64_t k,
     const int32_t* row_index, int64_t rows, const int32_t* group_offsets, int G, uint8_t* q_dst,
     uint8_t* sf_dst, uint32_t* status)
 {
-    // locate this CTA's (group, block): group e has ceil(count/128) blocks
+    // locate this CTA's (group, block): group e has ceil(count/128) blocks.
+    // The offsets come into shared memory in one parallel load; warp 0 then
+    // scans 32 groups per step (block counts, inclusive shuffle scan, ballot).
     __shared__ int s_e, s_t, s_pad_blk;
-    if (threadIdx.x == 0) {
-        int64_t b = blockIdx.x, pad_blk = 0;
-        int e = -1, t = 0;
+    __shared__ int32_t s_off[kMaxGroups + 1];
+    if (group_offsets) {
+        for (int g = threadIdx.x; g <= G; g += blockDim.x) s_off[g] = group_offsets[g];
+        __syncthreads();
+    }
+    if (threadIdx.x < 32) {
+        const int lane = threadIdx.x;
+        int e = -1, t = 0, pad_blk = 0;
+        const int b = blockIdx.x;
         if (!group_offsets) {
-            if (b * 128 < rows) e = 0, t = (int)b, pad_blk = 0;
+            if ((int64_t)b * 128 < rows) e = 0, t = b;
         } else {
-            for (int g = 0; g < G; ++g) {
-                const int64_t cnt = group_offsets[g + 1] - group_offsets[g];
-                const int64_t nb = (cnt + 127) / 128;
-                if (b < nb) {
-                    e = g;
-                    t = (int)b;
+            int before = 0;  // blocks of the groups already scanned
+            for (int g0 = 0; g0 < G; g0 += 32) {
+                const int g = g0 + lane;
+                const int nb = g < G ? (s_off[g + 1] - s_off[g] + 127) / 128 : 0;
+                int incl = nb;
+                for (int d = 1; d < 32; d <<= 1) {
+                    const int v = __shfl_up_sync(0xffffffffu, incl, d);
+                    if (lane >= d) incl += v;
+                }
+                const unsigned hit = __ballot_sync(0xffffffffu, b < before + incl && b >= before + incl - nb && nb > 0);
+                if (hit) {
+                    const int src = __ffs(hit) - 1;
+                    const int excl = before + __shfl_sync(0xffffffffu, incl - nb, src);
+                    e = g0 + src;
+                    t = b - excl;
+                    pad_blk = excl;
                     break;
                 }
-                b -= nb;
-                pad_blk += nb;
+                before += __shfl_sync(0xffffffffu, incl, 31);
             }
         }
-        s_e = e;
-        s_t = t;
-        s_pad_blk = (int)pad_blk;
+        if (lane == 0) {
+            s_e = e;
+            s_t = t;
+            s_pad_blk = pad_blk;
+        }
     }
     __syncthreads();
     const int e = s_e;
@@ -1057,13 +1076,26 @@ __global__ void __launch_bounds__(256) gather_rows_kernel(
             for (; c < chunks; c += 32) dst[c] = src[c];
         }
     }
-    // scales: 4 bytes (one row's four 16-blocks of a 64-column group) at a time
-    for (int idx = threadIdx.x; idx < nr * (int)k64; idx += blockDim.x) {  // < 2^31: k <= 2^30
-        const int j = idx / nr;
-        const int i = idx - j * nr;
-        const int64_t s = s_src[i];
-        const uint32_t v = *reinterpret_cast<const uint32_t*>(sf_src + sf_mma_offset(s, 4 * j, k16));
-        *reinterpret_cast<uint32_t*>(sf_dst + sf_mma_offset(dst_blk * 128 + i, 4 * j, k16)) = v;
+    // scales: 4 bytes (one row's four 16-blocks of a 64-column group) per
+    // word; consecutive threads write consecutive words of a destination atom
+    // (word w holds row (w >> 2) + 32 * (w & 3)), eight loads in flight each
+    const int total = 128 * (int)k64;  // < 2^31: k <= 2^30
+    for (int base = threadIdx.x; base < total; base += 8 * blockDim.x) {
+        uint32_t v[8];
+#pragma unroll
+        for (int u = 0; u < 8; ++u) {
+            const int idx = base + u * blockDim.x;
+            const int w = idx & 127, i = (w >> 2) | ((w & 3) << 5);
+            if (idx < total && i < nr)
+                v[u] = *reinterpret_cast<const uint32_t*>(sf_src + sf_mma_offset(s_src[i], 4 * (idx >> 7), k16));
+        }
+#pragma unroll
+        for (int u = 0; u < 8; ++u) {
+            const int idx = base + u * blockDim.x;
+            const int w = idx & 127, i = (w >> 2) | ((w & 3) << 5);
+            if (idx < total && i < nr)
+                *reinterpret_cast<uint32_t*>(sf_dst + sf_mma_offset(dst_blk * 128 + i, 4 * (idx >> 7), k16)) = v[u];
+        }
     }
 }
 
@@ -1518,7 +1550,7 @@ extern "C" nvfp4_status nvfp4_gather_rows(const uint8_t* q_src, const uint8_t* s
     uint32_t* status = workspace ? static_cast<uint32_t*>(workspace) + 2 : nullptr;
     if (status && cudaMemsetAsync(status, 0, 4, st) != cudaSuccess) return NVFP4_ERR_CUDA;
     const int64_t blocks = (rows + 127) / 128 + (group_offsets ? num_groups : 0);
-    gather_rows_kernel<<<(int)blocks, 256, 0, st>>>(q_src, sf_src, src_rows, k, row_index, rows,
+    gather_rows_kernel<<<(int)blocks, 512, 0, st>>>(q_src, sf_src, src_rows, k, row_index, rows,
                                                     group_offsets, num_groups, q_dst, sf_dst,
                                                     status);
     return cudaGetLastError() == cudaSuccess ? NVFP4_OK : NVFP4_ERR_CUDA;
