@@ -673,27 +673,36 @@ class ClockSampler:
             try:
                 mhz = N.nvmlDeviceGetClockInfo(self.handle, N.NVML_CLOCK_SM)
                 bits = get_reasons(self.handle) if get_reasons else 0
-                self.samples.append((mhz, bits))
+                self.raw.append((time.perf_counter(), mhz, bits))
+                self.first.set()
             except Exception:
                 pass
             self.stop.wait(0.005)
 
     def __enter__(self):
+        # NVML is opened and the thread has taken its first sample before the
+        # timed region starts; only samples taken inside the region are kept.
         import threading
         try:
             self._open()
         except Exception:
             self.handle = None
             return self
+        self.raw = []
         self.stop = threading.Event()
+        self.first = threading.Event()
         self.thread = threading.Thread(target=self._run, daemon=True)
         self.thread.start()
+        self.first.wait(timeout=2.0)
+        self.t_begin = time.perf_counter()
         return self
 
     def __exit__(self, *a):
         if self.thread is not None:
+            t_end = time.perf_counter()
             self.stop.set()
             self.thread.join(timeout=5)
+            self.samples = [(m, b) for t, m, b in self.raw if self.t_begin <= t <= t_end]
         if self.nvml is not None:
             try:
                 self.nvml.nvmlShutdown()

@@ -71,6 +71,34 @@ def test_clock_summary_decodes_reasons():
     assert c.summary()["reasons"] == ["hw_power_brake_slowdown"]
 
 
+def test_clock_sampler_keeps_only_the_timed_region(monkeypatch):
+    """The sampler's thread has taken a sample before the region starts, and only the
+    samples taken between entering and leaving the region are summarised (a fake NVML
+    whose clock reads 1000 MHz until the region starts, 1965 MHz inside it)."""
+    import time
+    import types
+    import bench
+    state = {"inside": False}
+    fake = types.SimpleNamespace(
+        NVML_CLOCK_SM=0, nvmlClocksEventReasonSwPowerCap=0x4,
+        nvmlDeviceGetClockInfo=lambda h, c: 1965 if state["inside"] else 1000,
+        nvmlDeviceGetCurrentClocksEventReasons=lambda h: 0x4 if state["inside"] else 0x40,
+        nvmlShutdown=lambda: None)
+
+    def fake_open(self):
+        self.nvml, self.handle, self.max_mhz = fake, object(), 1965
+        time.sleep(0.02)  # a slow NVML start
+
+    monkeypatch.setattr(bench.ClockSampler, "_open", fake_open)
+    with bench.ClockSampler("cpu") as c:
+        assert c.raw, "no sample before the region"
+        state["inside"] = True
+        time.sleep(0.1)
+    s = c.summary()
+    assert s["samples"] >= 3
+    assert s["sm_mhz"] == 1965 and s["reasons"] == ["sw_power_cap"]
+
+
 def test_hw_fp4_peak_uses_the_sampled_clock():
     """The GEMM roofline's peak: 32768 FP4 FLOP per SM per cycle on 148 SMs at the
     median clock of the timed region, falling back to the maximum clock (then 1965

@@ -241,6 +241,40 @@ def test_gather_rows_matches_oracle(nv, orc, grouped):
     assert np.array_equal(host(fused.sf), host(got.sf))
 
 
+def test_gather_rows_256_groups(nv, orc):
+    """Dispatch into the 256-group limit: runs of more than 32 empty groups, groups of
+    1, 127, 128, 129 and 256 rows, the last group non-empty after 39 empty ones.  Every
+    dispatched row's codes and scale bytes equal the oracle's quantisation of the
+    gathered rows; the padding rows' scale bytes are left as they were (zero here)."""
+    import torch
+    rng = np.random.default_rng(57)
+    tokens, k, G = 704, 128, 256
+    counts = np.zeros(G, dtype=np.int64)
+    sizes = {0: 3, 1: 1, 2: 127, 40: 128, 41: 129, 73: 256, 74: 5, 150: 64, 215: 33}
+    for e, c in sizes.items():
+        counts[e] = c
+    counts[255] = 134
+    offsets = np.concatenate([[0], np.cumsum(counts)]).astype(np.int32)
+    total = int(offsets[-1])
+    x = W.f32_to_bf16_bits(W.student_t(rng, (tokens, k), 4.0, 1.0))
+    row_index = np.concatenate([rng.permutation(tokens),
+                                rng.integers(0, tokens, total - tokens)]).astype(np.int32)
+    src = nv.quantize(to_dev(x), sf_layout=nv.NVFP4_SF_MMA)["row"]
+    got = nv.gather_rows(src, torch.from_numpy(row_index).cuda(), torch.from_numpy(offsets).cuda())
+    xg = np.ascontiguousarray(x[row_index])
+    qo, so, go = orc.nvfp4_quantize(xg, 0, amax=(orc.amax(x, 0), 0.0))
+    assert np.array_equal(host(got.q), qo)
+    pr = grouped_padded_rows(offsets)
+    assert np.array_equal(sf_mma_to_rowmajor(host(got.sf), total, k, pr), so)
+    sf_all = host(got.sf).reshape(-1)
+    mask = np.ones(sf_all.size, dtype=bool)
+    k16 = k // 16
+    r = pr[:, None]
+    b = np.arange(k16)[None, :]
+    mask[((r // 128) * (k16 // 4) + b // 4) * 512 + (r % 32) * 16 + ((r % 128) // 32) * 4 + b % 4] = False
+    assert not sf_all[mask].any()
+
+
 def test_gather_rows_bad_index_reports(nv):
     import torch
     x = torch.zeros((64, 64), dtype=torch.bfloat16, device="cuda")
