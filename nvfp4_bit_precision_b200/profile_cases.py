@@ -4,6 +4,8 @@
     python -m nvfp4_bit_precision_b200.profile_cases mxfp8-gemm M N K [--warm W]
     python -m nvfp4_bit_precision_b200.profile_cases grouped-gemm N K [--warm W]
     python -m nvfp4_bit_precision_b200.profile_cases quant-grad ROWS COLS [--warm W]
+    python -m nvfp4_bit_precision_b200.profile_cases quant-act ROWS COLS [--warm W]
+    python -m nvfp4_bit_precision_b200.profile_cases quant-weight ROWS COLS [--warm W]
     python -m nvfp4_bit_precision_b200.profile_cases mxfp4 ROWS COLS [--warm W]
 
 Each runs W untimed launches of the case, then one more, on synthetic operands
@@ -90,6 +92,31 @@ def _quant_grad(nv, torch, rows, cols, warm):
     return ws
 
 
+def _quant_act(nv, torch, rows, cols, warm):
+    """The activation recipe: rowwise and columnwise Hadamard, both RNE."""
+    dev = torch.device("cuda")
+    g = torch.Generator(device=dev)
+    g.manual_seed(3)
+    x = torch.randn((rows, cols), generator=g, device=dev).to(torch.bfloat16)
+    ws = torch.zeros(256, dtype=torch.uint8, device=dev)
+    for _ in range(warm + 1):
+        nv.quantize(x, rowwise=True, colwise=True, rht=True, sf_layout=nv.NVFP4_SF_MMA, workspace=ws)
+    return ws
+
+
+def _quant_weight(nv, torch, rows, cols, warm):
+    """The weight recipe: 16x16 2D scales, both directions, RNE."""
+    dev = torch.device("cuda")
+    g = torch.Generator(device=dev)
+    g.manual_seed(4)
+    x = (torch.randn((rows, cols), generator=g, device=dev) * 0.02).to(torch.bfloat16)
+    ws = torch.zeros(256, dtype=torch.uint8, device=dev)
+    for _ in range(warm + 1):
+        nv.quantize(x, rowwise=True, colwise=True, scaling=nv.NVFP4_2D16x16, sf_layout=nv.NVFP4_SF_MMA,
+                    workspace=ws)
+    return ws
+
+
 def _mxfp4(nv, torch, rows, cols, warm):
     """MXFP4 of a bf16 ~N(0, 1) tensor, both directions."""
     dev = torch.device("cuda")
@@ -103,7 +130,8 @@ def _mxfp4(nv, torch, rows, cols, warm):
 
 def main(argv=None) -> int:
     ap = argparse.ArgumentParser()
-    ap.add_argument("case", choices=["gemm", "mxfp8-gemm", "grouped-gemm", "quant-grad", "mxfp4"])
+    ap.add_argument("case", choices=["gemm", "mxfp8-gemm", "grouped-gemm", "quant-grad", "quant-act",
+                                         "quant-weight", "mxfp4"])
     ap.add_argument("dims", type=int, nargs="+")
     ap.add_argument("--warm", type=int, default=3)
     args = ap.parse_args(argv)
@@ -118,6 +146,10 @@ def main(argv=None) -> int:
         ws = _grouped(nv, torch, *args.dims[:2], args.warm)
     elif args.case == "quant-grad":
         ws = _quant_grad(nv, torch, *args.dims[:2], args.warm)
+    elif args.case == "quant-act":
+        ws = _quant_act(nv, torch, *args.dims[:2], args.warm)
+    elif args.case == "quant-weight":
+        ws = _quant_weight(nv, torch, *args.dims[:2], args.warm)
     else:
         ws = _mxfp4(nv, torch, *args.dims[:2], args.warm)
     torch.cuda.synchronize()
