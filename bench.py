@@ -263,11 +263,25 @@ def hw_fp4_peak(clocks):
     return HW_FP4_FLOP_PER_SM_CYCLE * NUM_SMS * mhz * 1e6 / 1e12, mhz
 
 
+# Measured on this machine: right after a loop of dense GEMMs, HBM-bound kernels can run
+# about 20% slower for several milliseconds (the MXFP8 quantise and combine of the MoE
+# output: 174 and 129 us against 142 and 108 us), and 250 ms of idle brings them back.
+# The lines timed apart from the step start after such a pause, so that none inherits
+# the state the GEMM loop before it left.
+SETTLE_S = 0.25
+
+
+def settle(torch):
+    torch.cuda.synchronize()
+    time.sleep(SETTLE_S)
+
+
 def time_mxfp4(step, steps, warmup):
     """MXFP4 (OCP: 32-blocks, E8M0, E2M1) of the resident dY, both directions from one
     call, timed apart from the step: mean ms per launch over `steps` launches after
     `warmup`, CUDA events on the launching stream.  dY (671 MB) is larger than L2."""
     nv, torch = step.nv, step.torch
+    settle(torch)
     dy = step.inputs[0]["dy"]
     R, C = dy.shape
     u8 = dict(dtype=torch.uint8, device=dy.device)
@@ -360,6 +374,7 @@ def time_configs(dev, reps, warmup, pk, fp4_peak):
     (3) 2D weight quantisation, activation quantisation and the 8192x4096x4096 GEMM."""
     import torch
     import nvfp4_bit_precision_b200 as nv
+    settle(torch)
     flush = L2Flush(dev)
     bf = lambda a: torch.from_numpy(np.ascontiguousarray(a).view(np.int16)).to(dev).view(
         torch.bfloat16)
@@ -583,6 +598,7 @@ def time_moe_combine(step, steps, warmup, pk):
     quant = lambda: nv.mxfp8_quantize(step.Out, R, H, H, nv.NVFP4_ROWWISE, 0, 0, 0, q, e8, None, None)
     comb = lambda: nv.mxfp8_combine(q, e8, R, H, slot, w, MOE_TOKENS, TOPK, out, step.ws[6], 256)
 
+    settle(torch)
     for _ in range(max(warmup, 3)):
         quant()
         comb()
@@ -611,7 +627,8 @@ def time_moe_combine(step, steps, warmup, pk):
             "frac": round(nbytes / (ms / 1e3) / 1e9 / pk["hbm_gbs"], 4),
             "link_bytes_mxfp8": R * H + R * H // 32, "link_bytes_bf16": 2 * R * H,
             "note": "one GPU: no all-to-all is timed; link bytes are what an expert-parallel "
-                    "run would send back per step"}
+                    "run would send back per step; timed after a 250 ms pause that follows the "
+                    "GEMM lines"}
 
 
 def quant_algorithmic_bytes():
