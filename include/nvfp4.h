@@ -274,7 +274,7 @@ nvfp4_status mxfp4_quantize(const void* x_bf16, int64_t rows, int64_t cols, int6
  * 1 <= num_groups <= 256), or into the dense layout when group_offsets is NULL.
  * Quantising the tokens once and gathering gives the same bytes as quantising
  * the gathered rows whenever every token is routed at least once (the global
- * scale then comes from the same amax).  k a multiple of 64, at most 2^30; q_src, q_dst
+ * scale then comes from the same amax).  k a multiple of 64, at most 2^28; q_src, q_dst
  * 16-byte aligned, scale pointers 4-byte aligned.  Out-of-range indices are
  * reported in the workspace status word (optional workspace).
  */

@@ -1079,7 +1079,7 @@ __global__ void __launch_bounds__(512) gather_rows_kernel(
     // scales: 4 bytes (one row's four 16-blocks of a 64-column group) per
     // word; consecutive threads write consecutive words of a destination atom
     // (word w holds row (w >> 2) + 32 * (w & 3)), eight loads in flight each
-    const int total = 128 * (int)k64;  // < 2^31: k <= 2^30
+    const int total = 128 * (int)k64;  // <= 2^29 (k <= 2^28): no index below overflows
     for (int base = threadIdx.x; base < total; base += 8 * blockDim.x) {
         uint32_t v[8];
 #pragma unroll
@@ -1537,7 +1537,7 @@ extern "C" nvfp4_status nvfp4_gather_rows(const uint8_t* q_src, const uint8_t* s
                                           void* workspace, size_t ws_bytes, void* stream)
 {
     if (!q_src || !sf_src || !row_index || !q_dst || !sf_dst) return NVFP4_ERR_INVALID_ARG;
-    if (src_rows <= 0 || rows <= 0 || k <= 0 || k % 64 || k > (int64_t(1) << 30)) return NVFP4_ERR_SHAPE;
+    if (src_rows <= 0 || rows <= 0 || k <= 0 || k % 64 || k > (int64_t(1) << 28)) return NVFP4_ERR_SHAPE;
     if (group_offsets && (num_groups < 1 || num_groups > kMaxGroups)) return NVFP4_ERR_INVALID_ARG;
     if (!aligned16(q_src) || !aligned16(q_dst) || (reinterpret_cast<uintptr_t>(sf_src) & 3) ||
         (reinterpret_cast<uintptr_t>(sf_dst) & 3))

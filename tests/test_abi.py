@@ -109,6 +109,7 @@ def test_gather_rows_argument_errors(nv):
     L = nv._lib.nvfp4_gather_rows
     assert L(None, FAKE, 64, 64, FAKE, 64, None, 0, FAKE, FAKE, FAKE, 256, None) == 1
     assert L(FAKE, FAKE, 64, 48, FAKE, 64, None, 0, FAKE, FAKE, FAKE, 256, None) == 2  # k % 64
+    assert L(FAKE, FAKE, 64, (1 << 28) + 64, FAKE, 64, None, 0, FAKE, FAKE, FAKE, 256, None) == 2
     assert L(FAKE, FAKE, 0, 64, FAKE, 64, None, 0, FAKE, FAKE, FAKE, 256, None) == 2   # no source
     assert L(FAKE, FAKE, 64, 64, FAKE, 64, FAKE, 0, FAKE, FAKE, FAKE, 256, None) == 1  # 0 groups
     assert L(FAKE, FAKE, 64, 64, FAKE, 64, FAKE, 300, FAKE, FAKE, FAKE, 256, None) == 1
