@@ -279,10 +279,17 @@ __device__ __forceinline__ uint32_t quant_block16x2(float (&v)[16], float (&w)[1
             for (int i = 0; i < 16; ++i) w[i] = __fmul_rn(w[i], 0.25f);
         }
     }
+    if (times4) {
+        // after the Hadamard butterflies the values sit in (v_i, w_i) register
+        // pairs: one packed multiply per such pair needs no re-pairing
 #pragma unroll
-    for (int i = 0; i < 16; i += 2) {
-        mul2(v[i], v[i + 1], v[i], v[i + 1], rv, rv);
-        mul2(w[i], w[i + 1], w[i], w[i + 1], rw, rw);
+        for (int i = 0; i < 16; ++i) mul2(v[i], w[i], v[i], w[i], rv, rw);
+    } else {
+#pragma unroll
+        for (int i = 0; i < 16; i += 2) {
+            mul2(v[i], v[i + 1], v[i], v[i + 1], rv, rv);
+            mul2(w[i], w[i + 1], w[i], w[i + 1], rw, rw);
+        }
     }
     if (sr) {
         // one Philox call per 16-element block: word q drives elements 4q..4q+3
