@@ -799,8 +799,25 @@ __global__ void __launch_bounds__(kQuantThreads, 2)
             const bool cvalid = cg0 < a.cols;        // cols is even: the pair is whole
             const int64_t rbase = r0 + 32 * rgrp;
             // the pair's 4 bytes: chunk cp/4 of each row, byte 4*(cp%4) within it
+            // shared addresses of the pair's word in rows j = 0..7 of the group (TMA
+            // tiles: the swizzle depends on row & 7); row i is row i & 7 plus
+            // (i >> 3) * 8 rows, a constant offset
+            uint32_t pw_base[8];
+            {
+                const int q = cp >> 2;
+                const uint32_t b0 = smem_addr(T) + 4u * (cp & 3);
+#pragma unroll
+                for (int j = 0; j < 8; ++j)
+                    pw_base[j] = kTma ? b0 + (q >> 3) * (kTileRows * 128) + (32 * rgrp + j) * 128 +
+                                            (((q & 7) ^ j) << 4)
+                                      : b0 + (32 * rgrp + j) * kPitch + q * 16;
+            }
             auto pair_word = [&](int i) -> uint32_t {
-                return ld_shared_u32(chunk_addr<kTma>(T, 32 * rgrp + i, cp >> 2) + 4 * (cp & 3));
+                uint32_t r;
+                asm volatile("ld.shared.u32 %0, [%1];"
+                             : "=r"(r)
+                             : "r"(pw_base[i & 7] + (i >> 3) * (kTma ? 8 * 128 : 8 * kPitch)));
+                return r;
             };
             // MXFP8 columnwise: the 32-row block's amax of each column is
             // gathered while the NVFP4 pass below unpacks the rows (the
