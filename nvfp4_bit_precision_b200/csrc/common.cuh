@@ -286,6 +286,35 @@ __device__ __forceinline__ void philox4x32_10_keyed_x2(uint32_t a0, uint32_t a1,
     rb = U4{y0, y1, y2, y3};
 }
 
+// Four Philox4x32-10 blocks with consecutive 64-bit counters j .. j+3 in the
+// first two words, computed round by round side by side.
+__device__ __forceinline__ void philox4x32_10_keyed_x4(uint64_t j, uint32_t c2, uint32_t c3,
+                                                       const PhiloxKeys& k, U4 (&r)[4])
+{
+    uint32_t x0[4], x1[4], x2[4], x3[4];
+#pragma unroll
+    for (int b = 0; b < 4; ++b) {
+        x0[b] = static_cast<uint32_t>(j + b);
+        x1[b] = static_cast<uint32_t>((j + b) >> 32);
+        x2[b] = c2;
+        x3[b] = c3;
+    }
+#pragma unroll
+    for (int rd = 0; rd < 10; ++rd) {
+#pragma unroll
+        for (int b = 0; b < 4; ++b) {
+            const uint64_t p0 = static_cast<uint64_t>(x0[b]) * 0xD2511F53u;
+            const uint64_t p1 = static_cast<uint64_t>(x2[b]) * 0xCD9E8D57u;
+            x0[b] = static_cast<uint32_t>(p1 >> 32) ^ x1[b] ^ k.k0[rd];
+            x2[b] = static_cast<uint32_t>(p0 >> 32) ^ x3[b] ^ k.k1[rd];
+            x1[b] = static_cast<uint32_t>(p1);
+            x3[b] = static_cast<uint32_t>(p0);
+        }
+    }
+#pragma unroll
+    for (int b = 0; b < 4; ++b) r[b] = U4{x0[b], x1[b], x2[b], x3[b]};
+}
+
 // MXFP8 stream: random bits for elements idx8*8 .. idx8*8+7; element j takes
 // the 16-bit half (j % 2) of word j / 2.
 __device__ __forceinline__ U4 sr_block8(const PhiloxKeys& k, uint32_t offset, uint32_t stream,

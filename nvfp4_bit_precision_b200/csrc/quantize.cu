@@ -249,13 +249,16 @@ __device__ __forceinline__ float div6_rn(float a)
 // Two blocks at once (v and w, with their amax): both scale bytes from one
 // paired E4M3 conversion and both Philox blocks computed side by side.  Returns
 // the scale bytes (v's in bits 0..7, w's in bits 8..15); the codes go to
-// cv0/cv1 and cw0/cw1.
+// cv0/cv1 and cw0/cw1.  With use_pre the two blocks' Philox words are given (pre_v,
+// pre_w: the same words the call would compute from idx_v and idx_w).
 __device__ __forceinline__ uint32_t quant_block16x2(float (&v)[16], float (&w)[16], float am_v,
                                                     float am_w, float S, const float* rtab,
                                                     bool times4, bool sr, const PhiloxKeys& pk,
                                                     uint32_t offset, uint32_t stream,
                                                     uint64_t idx_v, uint64_t idx_w, uint32_t& cv0,
-                                                    uint32_t& cv1, uint32_t& cw0, uint32_t& cw1)
+                                                    uint32_t& cv1, uint32_t& cw0, uint32_t& cw1,
+                                                    bool use_pre = false, U4 pre_v = U4{},
+                                                    U4 pre_w = U4{})
 {
     if (times4) {
         am_v = __fmul_rn(am_v, 0.25f);
@@ -294,10 +297,15 @@ __device__ __forceinline__ uint32_t quant_block16x2(float (&v)[16], float (&w)[1
     if (sr) {
         // one Philox call per 16-element block: word q drives elements 4q..4q+3
         U4 a, b;
-        const uint64_t jv = idx_v >> 4, jw = idx_w >> 4;
-        philox4x32_10_keyed_x2(static_cast<uint32_t>(jv), static_cast<uint32_t>(jv >> 32),
-                               static_cast<uint32_t>(jw), static_cast<uint32_t>(jw >> 32), stream,
-                               offset, pk, a, b);
+        if (use_pre) {
+            a = pre_v;
+            b = pre_w;
+        } else {
+            const uint64_t jv = idx_v >> 4, jw = idx_w >> 4;
+            philox4x32_10_keyed_x2(static_cast<uint32_t>(jv), static_cast<uint32_t>(jv >> 32),
+                                   static_cast<uint32_t>(jw), static_cast<uint32_t>(jw >> 32), stream,
+                                   offset, pk, a, b);
+        }
         cv0 = e2m1x4_sr(v + 0, a.x) | (e2m1x4_sr(v + 4, a.y) << 16);
         cv1 = e2m1x4_sr(v + 8, a.z) | (e2m1x4_sr(v + 12, a.w) << 16);
         cw0 = e2m1x4_sr(w + 0, b.x) | (e2m1x4_sr(w + 4, b.y) << 16);
@@ -724,6 +732,10 @@ __global__ void __launch_bounds__(kQuantThreads, 2)
                 uint32_t codes[8];
                 uint32_t sfw = 0;
                 bool all_valid = true;
+                // the random words of the thread's four blocks (consecutive
+                // counters), four Philox chains side by side
+                U4 rnd[4] = {};
+                if (sr) philox4x32_10_keyed_x4((uint64_t)(rg * a.cols + cbase) >> 4, 0u, a.offset, a.pk, rnd);
 #pragma unroll
                 for (int bp = 0; bp < 4; bp += 2) {  // two 16-blocks at a time
                     const int64_t cg = cbase + 16 * bp;
@@ -742,7 +754,7 @@ __global__ void __launch_bounds__(kQuantThreads, 2)
                     const uint32_t bytes = quant_block16x2(
                         v, w, amv, amw, S_row, sh->rtab[0], false, sr && rvalid && cg < a.cols, a.pk,
                         a.offset, 0u, idx, idx + 16, codes[2 * bp], codes[2 * bp + 1],
-                        codes[2 * bp + 2], codes[2 * bp + 3]);
+                        codes[2 * bp + 2], codes[2 * bp + 3], sr, rnd[bp], rnd[bp + 1]);
                     sfw |= bytes << (8 * bp);
                 }
                 if (all_valid) {
