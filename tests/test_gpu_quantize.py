@@ -172,6 +172,34 @@ def test_gather_grouped_layout(nv, orc):
     assert nv.nvfp4_workspace_status(out["workspace"]) == 0
 
 
+def test_gather_gradient_recipe(nv, orc):
+    """Gathered input (rows copied one by one into the staged tile, not TMA boxes)
+    with every output of the gradient recipe: rowwise SR, columnwise Hadamard + SR and
+    MXFP8 columnwise, on a ragged tile edge in both directions (320 x 320).  Each
+    output equals the oracle's quantisation of the gathered matrix."""
+    import torch
+    rng = np.random.default_rng(71)
+    tokens, cols, total = 96, 320, 320
+    x = W.heavy_tailed(2, tokens, cols)
+    row_index = np.concatenate([rng.permutation(tokens),
+                                rng.integers(0, tokens, total - tokens)]).astype(np.int32)
+    out = nv.quantize(to_dev(x), rows=total, row_index=torch.from_numpy(row_index).cuda(),
+                      src_rows=tokens, rowwise=True, colwise=True, rounding=1, rht=True, seed=3,
+                      mx_outputs=nv.NVFP4_COLWISE, sf_layout=nv.NVFP4_SF_MMA)
+    xg = np.ascontiguousarray(x[row_index])
+    qr, sr, gr = orc.nvfp4_quantize(xg, 0, 1, 0, 0, 3)
+    qc, sc, gc = orc.nvfp4_quantize(xg, 1, 1, 0, 1, 3)
+    mq, me = orc.mxfp8_quantize(xg, 1, 0, 3)
+    np.testing.assert_array_equal(host(out["row"].q), qr)
+    np.testing.assert_array_equal(sf_mma_to_rowmajor(host(out["row"].sf), total, cols), sr)
+    np.testing.assert_array_equal(host(out["col"].q), qc)
+    np.testing.assert_array_equal(sf_mma_to_rowmajor(host(out["col"].sf), cols, total), sc)
+    np.testing.assert_array_equal(host(out["mx_col"][0]), mq)
+    np.testing.assert_array_equal(host(out["mx_col"][1]), me)
+    assert float(host(out["row"].g)[0]) == gr and float(host(out["col"].g)[0]) == gc
+    assert nv.nvfp4_workspace_status(out["workspace"]) == 0
+
+
 def test_gather_bad_index_reports(nv):
     import torch
     x = torch.zeros((32, 64), dtype=torch.bfloat16, device="cuda")
