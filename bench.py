@@ -886,6 +886,16 @@ def grouped_roofline(times, steps, step, pk, fp4_peak):
     return out
 
 
+def bench_config(world):
+    """The workload's `config`, the same on both arms.  Every token is routed to
+    TOPK experts, so the routed row count is fixed."""
+    return {"workload": WORKLOAD, "tokens": TOKENS, "hidden": HIDDEN, "ffn": FFN,
+            "moe": {"experts": EXPERTS, "hidden": MOE_HIDDEN, "ffn": MOE_FFN,
+                    "tokens": MOE_TOKENS, "top_k": TOPK, "routed_rows": MOE_TOKENS * TOPK},
+            "parallelism": f"replicas x{world}",
+            "l2": "inputs larger than L2 (dY 671 MB, X 168 MB, W 210 MB > 126 MB)"}
+
+
 def run_reference(args, rank, world):
     if rank != 0:
         return
@@ -899,7 +909,7 @@ def run_reference(args, rank, world):
     line = {"impl": "reference", "metric": METRIC, "value": v, "unit": "TFLOP/s", "n_gpus": 1,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": None,
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
-            "data": "synthetic", "config": {"workload": WORKLOAD, "parallelism": "replicas"},
+            "data": "synthetic", "config": bench_config(world),
             "cpu_baseline": {"value": v, "unit": "TFLOP/s", "cores": info["cores"],
                              "kind": "oracle", "sample": info["sample"]},
             "e2e": {"value": v, "unit": "TFLOP/s", "h2d_bytes_per_step": 0,
@@ -1071,11 +1081,7 @@ def main():
             "scaling": "weak", "vs_baseline": None, "dtype": "fp4",
             "data": "synthetic (seeded numpy: N(0,1) activations, N(0,0.02) weights, "
                     "Student-t df=3 gradients, Zipf(1.1) top-4 routing)",
-            "config": {"workload": WORKLOAD, "tokens": TOKENS, "hidden": HIDDEN, "ffn": FFN,
-                       "moe": {"experts": EXPERTS, "hidden": MOE_HIDDEN, "ffn": MOE_FFN,
-                               "tokens": MOE_TOKENS, "top_k": TOPK, "routed_rows": step.routed},
-                       "parallelism": f"replicas x{world}",
-                       "l2": "inputs larger than L2 (dY 671 MB, X 168 MB, W 210 MB > 126 MB)"},
+            "config": bench_config(world),
             "roofline": {"bound": "tensor", "kernel": "gemm_kernel (dense NVFP4 GEMM, "
                          "16384x20480x5120 class, mean of fwd/dgrad/wgrad launches)",
                          "achieved": round(gemm_tflops, 1), "peak": round(derived_peak, 1),

@@ -127,3 +127,15 @@ def test_grouped_roofline_bytes_and_flops():
     up_roof = max(2 * 65536 * 1536 * 4096 / 9529.6e12, 578813952 / 6550.4e9) * 1e6
     assert abs(r["up"]["roofline_us"] - round(up_roof, 1)) < 0.11
     assert abs(r["up"]["frac"] - up_roof / 100.0) < 1e-4
+
+
+def test_both_arms_report_the_same_config():
+    """The reference arm's line carries the workload `config` of the measured arm,
+    built by the same function (routed rows: every token goes to TOPK experts)."""
+    import inspect
+    import bench
+    c = bench.bench_config(2)
+    assert c["parallelism"] == "replicas x2"
+    assert c["moe"]["routed_rows"] == bench.MOE_TOKENS * bench.TOPK
+    assert "bench_config(world)" in inspect.getsource(bench.run_reference)
+    assert "bench_config(world)" in inspect.getsource(bench.main)
