@@ -7,6 +7,8 @@
     python -m nvfp4_bit_precision_b200.profile_cases quant-act ROWS COLS [--warm W]
     python -m nvfp4_bit_precision_b200.profile_cases quant-weight ROWS COLS [--warm W]
     python -m nvfp4_bit_precision_b200.profile_cases mxfp4 ROWS COLS [--warm W]
+    python -m nvfp4_bit_precision_b200.profile_cases dispatch TOKENS HIDDEN [--warm W]
+    python -m nvfp4_bit_precision_b200.profile_cases combine TOKENS HIDDEN [--warm W]
 
 Each runs W untimed launches of the case, then one more, on synthetic operands
 (codes and in-range scale bytes drawn on the device; bf16 inputs ~N(0, 1e-3)),
@@ -128,10 +130,54 @@ def _mxfp4(nv, torch, rows, cols, warm):
     return None
 
 
+def _dispatch(nv, torch, tokens, hidden, warm):
+    """MoE dispatch of quantised token rows (top-4 Zipf(1.1) routing over 64 experts)
+    into the grouped layout."""
+    import numpy as np
+
+    import workloads as W
+    dev = torch.device("cuda")
+    _, row_token, offsets = W.moe_routing(np.random.default_rng(3), tokens, 64, 4)
+    R = int(offsets[-1])
+    g = torch.Generator(device=dev)
+    g.manual_seed(5)
+    x = torch.randn((tokens, hidden), generator=g, device=dev).to(torch.bfloat16)
+    t = nv.quantize(x, sf_layout=nv.NVFP4_SF_MMA)["row"]
+    u8 = dict(dtype=torch.uint8, device=dev)
+    qd = torch.empty((R, hidden // 2), **u8)
+    sd = torch.zeros(nv.nvfp4_sf_mma_grouped_bytes(R, 64, hidden), **u8)
+    rt = torch.from_numpy(row_token.astype(np.int32)).to(dev)
+    off = torch.from_numpy(offsets.astype(np.int32)).to(dev)
+    ws = torch.zeros(256, **u8)
+    for _ in range(warm + 1):
+        nv.nvfp4_gather_rows(t.q, t.sf, tokens, hidden, rt, R, off, 64, qd, sd, ws, 256)
+    return ws
+
+
+def _combine(nv, torch, tokens, hidden, warm):
+    """MXFP8 combine of top-4 expert rows (in expert order) into tokens x hidden bf16."""
+    import numpy as np
+    dev = torch.device("cuda")
+    R, k = 4 * tokens, 4
+    g = torch.Generator(device=dev)
+    g.manual_seed(6)
+    out_rows = torch.randn((R, hidden), generator=g, device=dev).to(torch.bfloat16)
+    u8 = dict(dtype=torch.uint8, device=dev)
+    q, e8 = torch.empty((R, hidden), **u8), torch.empty((R, hidden // 32), **u8)
+    nv.mxfp8_quantize(out_rows, R, hidden, hidden, nv.NVFP4_ROWWISE, 0, 0, 0, q, e8, None, None)
+    slot = torch.from_numpy(np.random.default_rng(7).permutation(R).reshape(tokens, k).astype(np.int32)).to(dev)
+    w = torch.full((tokens, k), 1.0 / k, dtype=torch.float32, device=dev)
+    out = torch.empty((tokens, hidden), dtype=torch.bfloat16, device=dev)
+    ws = torch.zeros(256, **u8)
+    for _ in range(warm + 1):
+        nv.mxfp8_combine(q, e8, R, hidden, slot, w, tokens, k, out, ws, 256)
+    return ws
+
+
 def main(argv=None) -> int:
     ap = argparse.ArgumentParser()
     ap.add_argument("case", choices=["gemm", "mxfp8-gemm", "grouped-gemm", "quant-grad", "quant-act",
-                                         "quant-weight", "mxfp4"])
+                                         "quant-weight", "mxfp4", "dispatch", "combine"])
     ap.add_argument("dims", type=int, nargs="+")
     ap.add_argument("--warm", type=int, default=3)
     args = ap.parse_args(argv)
@@ -150,6 +196,10 @@ def main(argv=None) -> int:
         ws = _quant_act(nv, torch, *args.dims[:2], args.warm)
     elif args.case == "quant-weight":
         ws = _quant_weight(nv, torch, *args.dims[:2], args.warm)
+    elif args.case == "dispatch":
+        ws = _dispatch(nv, torch, *args.dims[:2], args.warm)
+    elif args.case == "combine":
+        ws = _combine(nv, torch, *args.dims[:2], args.warm)
     else:
         ws = _mxfp4(nv, torch, *args.dims[:2], args.warm)
     torch.cuda.synchronize()
