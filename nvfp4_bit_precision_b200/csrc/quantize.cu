@@ -1093,23 +1093,40 @@ __global__ void __launch_bounds__(512) gather_rows_kernel(
         s_src[i] = s;
     }
     __syncthreads();
-    // codes: one warp per row at a time, its lanes on consecutive 16-byte
-    // vectors, four loads in flight per lane before their stores
+    // codes: one warp per two rows at a time, its lanes on consecutive 16-byte
+    // vectors, four loads per row in flight per lane before their stores
     {
         const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
         const int nwarps = blockDim.x >> 5;
-        for (int i = warp; i < nr; i += nwarps) {
+        for (int i = warp; i < nr; i += 2 * nwarps) {
+            // rows i and i + nwarps: both rows' loads in flight before their stores
+            const int i2 = i + nwarps;
+            const bool two = i2 < nr;
             const uint4* __restrict__ src = reinterpret_cast<const uint4*>(q_src + s_src[i] * (k / 2));
             uint4* __restrict__ dst = reinterpret_cast<uint4*>(q_dst + (r0 + i) * (k / 2));
+            const uint4* __restrict__ src2 =
+                reinterpret_cast<const uint4*>(q_src + s_src[two ? i2 : i] * (k / 2));
+            uint4* __restrict__ dst2 = reinterpret_cast<uint4*>(q_dst + (r0 + (two ? i2 : i)) * (k / 2));
             int64_t c = lane;
             for (; c + 96 < chunks; c += 128) {
                 const uint4 v0 = src[c], v1 = src[c + 32], v2 = src[c + 64], v3 = src[c + 96];
+                uint4 u0, u1, u2, u3;
+                if (two) u0 = src2[c], u1 = src2[c + 32], u2 = src2[c + 64], u3 = src2[c + 96];
                 dst[c] = v0;
                 dst[c + 32] = v1;
                 dst[c + 64] = v2;
                 dst[c + 96] = v3;
+                if (two) {
+                    dst2[c] = u0;
+                    dst2[c + 32] = u1;
+                    dst2[c + 64] = u2;
+                    dst2[c + 96] = u3;
+                }
             }
-            for (; c < chunks; c += 32) dst[c] = src[c];
+            for (; c < chunks; c += 32) {
+                dst[c] = src[c];
+                if (two) dst2[c] = src2[c];
+            }
         }
     }
     // scales: 4 bytes (one row's four 16-blocks of a 64-column group) per
