@@ -588,6 +588,11 @@ constexpr QSpec kSpecs[kNumSpecs] = {
     {kOn, kOff, kOff, kOff, kOff, kRt, kRt, kOff, kRt},
     {kOff, kOff, kOn, kOff, kOff, kRt, kOff, kOff, kOff},
 };
+template <bool B>
+struct BoolC {
+    static constexpr bool value = B;
+};
+
 __host__ __device__ constexpr bool spec_pick(int8_t s, bool run_time)
 {
     return s == kRt ? run_time : s == kOn;
@@ -716,295 +721,306 @@ __global__ void __launch_bounds__(kQuantThreads, 2)
         const int64_t tile = tile_of(k);
         const int64_t tr = tile_row(a, tile), tc = tile - tr * a.tiles_c;
         const int64_t r0 = tr * kTileRows, c0 = tc * kTileCols;
+        // A tile wholly inside the tensor runs a copy of the body compiled
+        // without the edge predicates (every check below is then a constant);
+        // tiles on an edge run the general copy.  Same results either way.
+        const bool full_tile = r0 + kTileRows <= a.rows && c0 + kTileCols <= a.cols;
+        auto tile_body = [&](auto full_c) {
+            constexpr bool kFull = decltype(full_c)::value;
 
-        // ---------------- rowwise: thread = (row, 64-column half) ----------
-        if (nv_row || mx_row) {
-            const int rl = 16 * warp + (lane & 15);
-            const int h = lane >> 4;
-            const int64_t rg = r0 + rl;
-            const bool rvalid = rg < a.rows;
-            const int64_t cbase = c0 + 64 * h;
-            // Shared-memory reads are unconditional: positions past the tensor
-            // hold zeros (TMA) or stale bytes (gather), and blocks made of them
-            // are never stored; 1D blocks and 16x16 tiles never mix valid and
-            // invalid elements because rows and cols are multiples of 16.
-            if (nv_row) {
-                uint32_t codes[8];
-                uint32_t sfw = 0;
-                bool all_valid = true;
-                // the random words of the thread's four blocks (consecutive
-                // counters), four Philox chains side by side
-                U4 rnd[4] = {};
-                if (sr) philox4x32_10_keyed_x4((uint64_t)(rg * a.cols + cbase) >> 4, 0u, a.offset, a.pk, rnd);
-#pragma unroll
-                for (int bp = 0; bp < 4; bp += 2) {  // two 16-blocks at a time
-                    const int64_t cg = cbase + 16 * bp;
-                    all_valid &= rvalid && cg + 16 < a.cols;
-                    float v[16], w[16];
-                    unpack8(ld_shared_v4(chunk_addr<kTma>(T, rl, 8 * h + 2 * bp)), v);
-                    unpack8(ld_shared_v4(chunk_addr<kTma>(T, rl, 8 * h + 2 * bp + 1)), v + 8);
-                    unpack8(ld_shared_v4(chunk_addr<kTma>(T, rl, 8 * h + 2 * bp + 2)), w);
-                    unpack8(ld_shared_v4(chunk_addr<kTma>(T, rl, 8 * h + 2 * bp + 3)), w + 8);
-                    float amv = absmax16(v, 0.0f), amw = absmax16(w, 0.0f);
-                    if (two_d) {
-                        amv = warp_max16(amv);
-                        amw = warp_max16(amw);
+            // ---------------- rowwise: thread = (row, 64-column half) ----------
+            if (nv_row || mx_row) {
+                const int rl = 16 * warp + (lane & 15);
+                const int h = lane >> 4;
+                const int64_t rg = r0 + rl;
+                const bool rvalid = kFull || rg < a.rows;
+                const int64_t cbase = c0 + 64 * h;
+                // Shared-memory reads are unconditional: positions past the tensor
+                // hold zeros (TMA) or stale bytes (gather), and blocks made of them
+                // are never stored; 1D blocks and 16x16 tiles never mix valid and
+                // invalid elements because rows and cols are multiples of 16.
+                if (nv_row) {
+                    uint32_t codes[8];
+                    uint32_t sfw = 0;
+                    bool all_valid = true;
+                    // the random words of the thread's four blocks (consecutive
+                    // counters), four Philox chains side by side
+                    U4 rnd[4] = {};
+                    if (sr) philox4x32_10_keyed_x4((uint64_t)(rg * a.cols + cbase) >> 4, 0u, a.offset, a.pk, rnd);
+    #pragma unroll
+                    for (int bp = 0; bp < 4; bp += 2) {  // two 16-blocks at a time
+                        const int64_t cg = cbase + 16 * bp;
+                        all_valid &= kFull || (rvalid && cg + 16 < a.cols);
+                        float v[16], w[16];
+                        unpack8(ld_shared_v4(chunk_addr<kTma>(T, rl, 8 * h + 2 * bp)), v);
+                        unpack8(ld_shared_v4(chunk_addr<kTma>(T, rl, 8 * h + 2 * bp + 1)), v + 8);
+                        unpack8(ld_shared_v4(chunk_addr<kTma>(T, rl, 8 * h + 2 * bp + 2)), w);
+                        unpack8(ld_shared_v4(chunk_addr<kTma>(T, rl, 8 * h + 2 * bp + 3)), w + 8);
+                        float amv = absmax16(v, 0.0f), amw = absmax16(w, 0.0f);
+                        if (two_d) {
+                            amv = warp_max16(amv);
+                            amw = warp_max16(amw);
+                        }
+                        const uint64_t idx = (uint64_t)(rg * a.cols + cg);
+                        const uint32_t bytes = quant_block16x2(
+                            v, w, amv, amw, S_row, sh->rtab[0], false, sr && (kFull || (rvalid && cg < a.cols)), a.pk,
+                            a.offset, 0u, idx, idx + 16, codes[2 * bp], codes[2 * bp + 1],
+                            codes[2 * bp + 2], codes[2 * bp + 3], sr, rnd[bp], rnd[bp + 1]);
+                        sfw |= bytes << (8 * bp);
                     }
-                    const uint64_t idx = (uint64_t)(rg * a.cols + cg);
-                    const uint32_t bytes = quant_block16x2(
-                        v, w, amv, amw, S_row, sh->rtab[0], false, sr && rvalid && cg < a.cols, a.pk,
-                        a.offset, 0u, idx, idx + 16, codes[2 * bp], codes[2 * bp + 1],
-                        codes[2 * bp + 2], codes[2 * bp + 3], sr, rnd[bp], rnd[bp + 1]);
-                    sfw |= bytes << (8 * bp);
+                    if (all_valid) {
+                        store_codes32(a.q_row + rg * (a.cols / 2) + cbase / 2, codes, q_row_vec);
+                        const int64_t b0 = cbase / 16;
+                        const int64_t off = mma_sf ? sf_mma_offset(padded_row(sh, grouped, rg), b0, a.cols / 16)
+                                                   : rg * (a.cols / 16) + b0;
+                        if (sf_row_vec) {
+                            *reinterpret_cast<uint32_t*>(a.sf_row + off) = sfw;
+                        } else {
+    #pragma unroll
+                            for (int blk = 0; blk < 4; ++blk) a.sf_row[off + blk] = (sfw >> (8 * blk)) & 0xFFu;
+                        }
+                    } else if (rvalid) {
+    #pragma unroll
+                        for (int blk = 0; blk < 4; ++blk) {
+                            const int64_t cg = cbase + 16 * blk;
+                            if (cg >= a.cols) continue;
+                            *reinterpret_cast<uint2*>(a.q_row + rg * (a.cols / 2) + cg / 2) =
+                                make_uint2(codes[2 * blk], codes[2 * blk + 1]);
+                            const int64_t off = mma_sf ? sf_mma_offset(padded_row(sh, grouped, rg), cg / 16, a.cols / 16)
+                                                       : rg * (a.cols / 16) + cg / 16;
+                            a.sf_row[off] = (sfw >> (8 * blk)) & 0xFFu;
+                        }
+                    }
                 }
-                if (all_valid) {
-                    store_codes32(a.q_row + rg * (a.cols / 2) + cbase / 2, codes, q_row_vec);
-                    const int64_t b0 = cbase / 16;
-                    const int64_t off = mma_sf ? sf_mma_offset(padded_row(sh, grouped, rg), b0, a.cols / 16)
-                                               : rg * (a.cols / 16) + b0;
-                    if (sf_row_vec) {
-                        *reinterpret_cast<uint32_t*>(a.sf_row + off) = sfw;
-                    } else {
-#pragma unroll
-                        for (int blk = 0; blk < 4; ++blk) a.sf_row[off + blk] = (sfw >> (8 * blk)) & 0xFFu;
-                    }
-                } else if (rvalid) {
-#pragma unroll
-                    for (int blk = 0; blk < 4; ++blk) {
-                        const int64_t cg = cbase + 16 * blk;
-                        if (cg >= a.cols) continue;
-                        *reinterpret_cast<uint2*>(a.q_row + rg * (a.cols / 2) + cg / 2) =
-                            make_uint2(codes[2 * blk], codes[2 * blk + 1]);
-                        const int64_t off = mma_sf ? sf_mma_offset(padded_row(sh, grouped, rg), cg / 16, a.cols / 16)
-                                                   : rg * (a.cols / 16) + cg / 16;
-                        a.sf_row[off] = (sfw >> (8 * blk)) & 0xFFu;
+                if (mx_row && rvalid) {
+    #pragma unroll 1
+                    for (int part = 0; part < 2; ++part) {
+                        const int64_t cg = cbase + 32 * part;
+                        if (!kFull && cg >= a.cols) continue;
+                        float v[32];
+    #pragma unroll
+                        for (int q = 0; q < 4; ++q)
+                            unpack8(ld_shared_v4(chunk_addr<kTma>(T, rl, 8 * h + 4 * part + q)), v + 8 * q);
+                        uint32_t out[8];
+                        const uint32_t e8 = mx_block32(v, mx_sr, a.pk, a.offset,
+                                                       (uint64_t)(rg * a.cols + cg), out);
+                        uint4* dst = reinterpret_cast<uint4*>(a.mx_q_row + rg * a.cols + cg);
+                        dst[0] = make_uint4(out[0], out[1], out[2], out[3]);
+                        dst[1] = make_uint4(out[4], out[5], out[6], out[7]);
+                        a.mx_sf_row[mx_sf_off(a, rg, cg / 32, a.cols / 32)] = (uint8_t)e8;
                     }
                 }
             }
-            if (mx_row && rvalid) {
-#pragma unroll 1
-                for (int part = 0; part < 2; ++part) {
-                    const int64_t cg = cbase + 32 * part;
-                    if (cg >= a.cols) continue;
-                    float v[32];
-#pragma unroll
-                    for (int q = 0; q < 4; ++q)
-                        unpack8(ld_shared_v4(chunk_addr<kTma>(T, rl, 8 * h + 4 * part + q)), v + 8 * q);
-                    uint32_t out[8];
-                    const uint32_t e8 = mx_block32(v, mx_sr, a.pk, a.offset,
-                                                   (uint64_t)(rg * a.cols + cg), out);
-                    uint4* dst = reinterpret_cast<uint4*>(a.mx_q_row + rg * a.cols + cg);
-                    dst[0] = make_uint4(out[0], out[1], out[2], out[3]);
-                    dst[1] = make_uint4(out[4], out[5], out[6], out[7]);
-                    a.mx_sf_row[mx_sf_off(a, rg, cg / 32, a.cols / 32)] = (uint8_t)e8;
-                }
-            }
-        }
 
-        // ---------------- columnwise: thread = (column pair, 32-row group) --
-        // One 32-bit shared load per row gives both columns of the pair; the
-        // pair's two Hadamard transforms run in the two lanes of f32x2.
-        if (nv_col || mx_col) {
-            const int cp = 32 * (warp & 1) + lane;  // column pair 0..63
-            const int rgrp = warp >> 1;              // 32-row group 0..3
-            const int64_t cg0 = c0 + 2 * cp;         // columns cg0, cg0 + 1
-            const bool cvalid = cg0 < a.cols;        // cols is even: the pair is whole
-            const int64_t rbase = r0 + 32 * rgrp;
-            // the pair's 4 bytes: chunk cp/4 of each row, byte 4*(cp%4) within it
-            // shared addresses of the pair's word in rows j = 0..7 of the group (TMA
-            // tiles: the swizzle depends on row & 7); row i is row i & 7 plus
-            // (i >> 3) * 8 rows, a constant offset
-            uint32_t pw_base[8];
-            {
-                const int q = cp >> 2;
-                const uint32_t b0 = smem_addr(T) + 4u * (cp & 3);
-#pragma unroll
-                for (int j = 0; j < 8; ++j)
-                    pw_base[j] = kTma ? b0 + (q >> 3) * (kTileRows * 128) + (32 * rgrp + j) * 128 +
-                                            (((q & 7) ^ j) << 4)
-                                      : b0 + (32 * rgrp + j) * kPitch + q * 16;
-            }
-            auto pair_word = [&](int i) -> uint32_t {
-                uint32_t r;
-                asm volatile("ld.shared.u32 %0, [%1];"
-                             : "=r"(r)
-                             : "r"(pw_base[i & 7] + (i >> 3) * (kTma ? 8 * 128 : 8 * kPitch)));
-                return r;
-            };
-            // MXFP8 columnwise: the 32-row block's amax of each column is
-            // gathered while the NVFP4 pass below unpacks the rows (the
-            // Hadamard's sign flips leave |x| alone); the conversion then
-            // re-reads the rows 8 at a time.  rows is a multiple of 32 here.
-            float mxa = 0.0f, mxb = 0.0f;
-            const int64_t cwarp = c0 + 64 * (warp & 1);  // first column of the warp
-            uint8_t* stg_qc = qc_stage_all + warp * kQcStageBytes;
-            const bool qc_staged = kTma && nv_col && a.qc_staged;
-            if (kTma && (a.mx_staged || qc_staged)) {
-                if (lane == 0) bulk_wait_read0();  // this warp's previous stores have read its staging
-                __syncwarp();
-            }
-            if (rbase < a.rows) {
-                // rows is a multiple of 16: both 16-row blocks exist, or (at the
-                // bottom edge) only the first.  The first block's codes wait in
-                // registers so each column gets one 16-byte store.
-                const bool two = rbase + 32 <= a.rows;
-                const int64_t b0 = rbase / 16;
-                uint32_t keep0 = 0, keep1 = 0, keep2 = 0, keep3 = 0, keep_sf = 0;
-#pragma unroll
-                for (int sub = 0; sub < 2; ++sub) {
-                    if (sub == 1 && !two) break;
-                    const int64_t rg = rbase + 16 * sub;
-                    float va[16], vb[16];
-#pragma unroll
-                    for (int i = 0; i < 16; ++i)
-                        unpack_bf16x2(pair_word(16 * sub + i), rht ? ((signs >> i) & 1u) << 31 : 0u,
-                                      va[i], vb[i]);
-                    if (mx_col) {
-                        mxa = absmax16(va, mxa);
-                        mxb = absmax16(vb, mxb);
-                    }
-                    if (!nv_col) continue;
-                    if (rht) hadamard16x2_times4(va, vb);
-                    float ama = absmax16(va, 0.0f), amb = absmax16(vb, 0.0f);
-                    if (two_d) {  // 16x16 tile = 8 column pairs (lanes) x 16 rows
-                        float m = fmaxf(ama, amb);
-#pragma unroll
-                        for (int o = 1; o < 8; o <<= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
-                        ama = amb = m;
-                    }
-                    uint32_t ca0, ca1, cb0, cb1;
-                    const uint32_t bab = quant_block16x2(
-                        va, vb, ama, amb, S_col, sh->rtab[1], rht, sr && cvalid, a.pk, a.offset, 1u,
-                        (uint64_t)(cg0 * a.rows + rg), (uint64_t)((cg0 + 1) * a.rows + rg), ca0, ca1,
-                        cb0, cb1);
-                    const uint32_t ba = bab & 0xFFu, bb = bab >> 8;
-                    if (!cvalid) continue;
-                    if (two && sub == 0) {
-                        keep0 = ca0, keep1 = ca1, keep2 = cb0, keep3 = cb1;
-                        keep_sf = ba | (bb << 8);
-                        continue;
-                    }
-                    uint8_t* da = a.q_col + cg0 * (a.rows / 2) + rbase / 2;
-                    uint8_t* db = da + a.rows / 2;
-                    const int64_t offa = mma_sf ? sf_mma_offset(cg0, b0, a.rows / 16)
-                                                : cg0 * (a.rows / 16) + b0;
-                    const int64_t offb = mma_sf ? sf_mma_offset(cg0 + 1, b0, a.rows / 16)
-                                                : offa + a.rows / 16;
-                    if (!two) {  // a lone 16-row block: 8 code bytes and one scale per column
-                        *reinterpret_cast<uint2*>(da) = make_uint2(ca0, ca1);
-                        *reinterpret_cast<uint2*>(db) = make_uint2(cb0, cb1);
-                        a.sf_col[offa] = (uint8_t)ba;
-                        a.sf_col[offb] = (uint8_t)bb;
-                    } else {
-                        if (qc_staged) {  // buffer row 2*lane + h = column cg0 + h
-                            st_shared_v4(stg_qc + (2 * lane) * 16, make_uint4(keep0, keep1, ca0, ca1));
-                            st_shared_v4(stg_qc + (2 * lane + 1) * 16, make_uint4(keep2, keep3, cb0, cb1));
-                        } else if (q_col_vec) {
-                            *reinterpret_cast<uint4*>(da) = make_uint4(keep0, keep1, ca0, ca1);
-                            *reinterpret_cast<uint4*>(db) = make_uint4(keep2, keep3, cb0, cb1);
-                        } else {
-                            reinterpret_cast<uint2*>(da)[0] = make_uint2(keep0, keep1);
-                            reinterpret_cast<uint2*>(da)[1] = make_uint2(ca0, ca1);
-                            reinterpret_cast<uint2*>(db)[0] = make_uint2(keep2, keep3);
-                            reinterpret_cast<uint2*>(db)[1] = make_uint2(cb0, cb1);
+            // ---------------- columnwise: thread = (column pair, 32-row group) --
+            // One 32-bit shared load per row gives both columns of the pair; the
+            // pair's two Hadamard transforms run in the two lanes of f32x2.
+            if (nv_col || mx_col) {
+                const int cp = 32 * (warp & 1) + lane;  // column pair 0..63
+                const int rgrp = warp >> 1;              // 32-row group 0..3
+                const int64_t cg0 = c0 + 2 * cp;         // columns cg0, cg0 + 1
+                const bool cvalid = kFull || cg0 < a.cols;  // cols is even: the pair is whole
+                const int64_t rbase = r0 + 32 * rgrp;
+                // the pair's 4 bytes: chunk cp/4 of each row, byte 4*(cp%4) within it
+                // shared addresses of the pair's word in rows j = 0..7 of the group (TMA
+                // tiles: the swizzle depends on row & 7); row i is row i & 7 plus
+                // (i >> 3) * 8 rows, a constant offset
+                uint32_t pw_base[8];
+                {
+                    const int q = cp >> 2;
+                    const uint32_t b0 = smem_addr(T) + 4u * (cp & 3);
+    #pragma unroll
+                    for (int j = 0; j < 8; ++j)
+                        pw_base[j] = kTma ? b0 + (q >> 3) * (kTileRows * 128) + (32 * rgrp + j) * 128 +
+                                                (((q & 7) ^ j) << 4)
+                                          : b0 + (32 * rgrp + j) * kPitch + q * 16;
+                }
+                auto pair_word = [&](int i) -> uint32_t {
+                    uint32_t r;
+                    asm volatile("ld.shared.u32 %0, [%1];"
+                                 : "=r"(r)
+                                 : "r"(pw_base[i & 7] + (i >> 3) * (kTma ? 8 * 128 : 8 * kPitch)));
+                    return r;
+                };
+                // MXFP8 columnwise: the 32-row block's amax of each column is
+                // gathered while the NVFP4 pass below unpacks the rows (the
+                // Hadamard's sign flips leave |x| alone); the conversion then
+                // re-reads the rows 8 at a time.  rows is a multiple of 32 here.
+                float mxa = 0.0f, mxb = 0.0f;
+                const int64_t cwarp = c0 + 64 * (warp & 1);  // first column of the warp
+                uint8_t* stg_qc = qc_stage_all + warp * kQcStageBytes;
+                const bool qc_staged = kTma && nv_col && a.qc_staged;
+                if (kTma && (a.mx_staged || qc_staged)) {
+                    if (lane == 0) bulk_wait_read0();  // this warp's previous stores have read its staging
+                    __syncwarp();
+                }
+                if (kFull || rbase < a.rows) {
+                    // rows is a multiple of 16: both 16-row blocks exist, or (at the
+                    // bottom edge) only the first.  The first block's codes wait in
+                    // registers so each column gets one 16-byte store.
+                    const bool two = kFull || rbase + 32 <= a.rows;
+                    const int64_t b0 = rbase / 16;
+                    uint32_t keep0 = 0, keep1 = 0, keep2 = 0, keep3 = 0, keep_sf = 0;
+    #pragma unroll
+                    for (int sub = 0; sub < 2; ++sub) {
+                        if (sub == 1 && !two) break;
+                        const int64_t rg = rbase + 16 * sub;
+                        float va[16], vb[16];
+    #pragma unroll
+                        for (int i = 0; i < 16; ++i)
+                            unpack_bf16x2(pair_word(16 * sub + i), rht ? ((signs >> i) & 1u) << 31 : 0u,
+                                          va[i], vb[i]);
+                        if (mx_col) {
+                            mxa = absmax16(va, mxa);
+                            mxb = absmax16(vb, mxb);
                         }
-                        const uint32_t sfa = (keep_sf & 0xFFu) | (ba << 8);
-                        const uint32_t sfb = (keep_sf >> 8) | (bb << 8);
-                        if (sf_col_vec) {
-                            *reinterpret_cast<uint16_t*>(a.sf_col + offa) = (uint16_t)sfa;
-                            *reinterpret_cast<uint16_t*>(a.sf_col + offb) = (uint16_t)sfb;
+                        if (!nv_col) continue;
+                        if (rht) hadamard16x2_times4(va, vb);
+                        float ama = absmax16(va, 0.0f), amb = absmax16(vb, 0.0f);
+                        if (two_d) {  // 16x16 tile = 8 column pairs (lanes) x 16 rows
+                            float m = fmaxf(ama, amb);
+    #pragma unroll
+                            for (int o = 1; o < 8; o <<= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+                            ama = amb = m;
+                        }
+                        uint32_t ca0, ca1, cb0, cb1;
+                        const uint32_t bab = quant_block16x2(
+                            va, vb, ama, amb, S_col, sh->rtab[1], rht, sr && cvalid, a.pk, a.offset, 1u,
+                            (uint64_t)(cg0 * a.rows + rg), (uint64_t)((cg0 + 1) * a.rows + rg), ca0, ca1,
+                            cb0, cb1);
+                        const uint32_t ba = bab & 0xFFu, bb = bab >> 8;
+                        if (!cvalid) continue;
+                        if (two && sub == 0) {
+                            keep0 = ca0, keep1 = ca1, keep2 = cb0, keep3 = cb1;
+                            keep_sf = ba | (bb << 8);
+                            continue;
+                        }
+                        uint8_t* da = a.q_col + cg0 * (a.rows / 2) + rbase / 2;
+                        uint8_t* db = da + a.rows / 2;
+                        const int64_t offa = mma_sf ? sf_mma_offset(cg0, b0, a.rows / 16)
+                                                    : cg0 * (a.rows / 16) + b0;
+                        const int64_t offb = mma_sf ? sf_mma_offset(cg0 + 1, b0, a.rows / 16)
+                                                    : offa + a.rows / 16;
+                        if (!two) {  // a lone 16-row block: 8 code bytes and one scale per column
+                            *reinterpret_cast<uint2*>(da) = make_uint2(ca0, ca1);
+                            *reinterpret_cast<uint2*>(db) = make_uint2(cb0, cb1);
+                            a.sf_col[offa] = (uint8_t)ba;
+                            a.sf_col[offb] = (uint8_t)bb;
                         } else {
-                            a.sf_col[offa] = (uint8_t)sfa;
-                            a.sf_col[offa + 1] = (uint8_t)(sfa >> 8);
-                            a.sf_col[offb] = (uint8_t)sfb;
-                            a.sf_col[offb + 1] = (uint8_t)(sfb >> 8);
+                            if (qc_staged) {  // buffer row 2*lane + h = column cg0 + h
+                                st_shared_v4(stg_qc + (2 * lane) * 16, make_uint4(keep0, keep1, ca0, ca1));
+                                st_shared_v4(stg_qc + (2 * lane + 1) * 16, make_uint4(keep2, keep3, cb0, cb1));
+                            } else if (q_col_vec) {
+                                *reinterpret_cast<uint4*>(da) = make_uint4(keep0, keep1, ca0, ca1);
+                                *reinterpret_cast<uint4*>(db) = make_uint4(keep2, keep3, cb0, cb1);
+                            } else {
+                                reinterpret_cast<uint2*>(da)[0] = make_uint2(keep0, keep1);
+                                reinterpret_cast<uint2*>(da)[1] = make_uint2(ca0, ca1);
+                                reinterpret_cast<uint2*>(db)[0] = make_uint2(keep2, keep3);
+                                reinterpret_cast<uint2*>(db)[1] = make_uint2(cb0, cb1);
+                            }
+                            const uint32_t sfa = (keep_sf & 0xFFu) | (ba << 8);
+                            const uint32_t sfb = (keep_sf >> 8) | (bb << 8);
+                            if (sf_col_vec) {
+                                *reinterpret_cast<uint16_t*>(a.sf_col + offa) = (uint16_t)sfa;
+                                *reinterpret_cast<uint16_t*>(a.sf_col + offb) = (uint16_t)sfb;
+                            } else {
+                                a.sf_col[offa] = (uint8_t)sfa;
+                                a.sf_col[offa + 1] = (uint8_t)(sfa >> 8);
+                                a.sf_col[offb] = (uint8_t)sfb;
+                                a.sf_col[offb + 1] = (uint8_t)(sfb >> 8);
+                            }
                         }
                     }
                 }
-            }
-            if (qc_staged && rbase < a.rows && cwarp < a.cols) {
-                // this warp's 64 columns x 32 rows of NVFP4 codes (16 bytes per
-                // column) out with one TMA store, clipped at the tensor edge
-                fence_proxy_async_smem();
-                __syncwarp();
-                if (lane == 0) {
-                    tma_store_2d(&map_qc, stg_qc, (int32_t)(rbase / 2), (int32_t)cwarp);
-                    bulk_commit();
-                }
-            }
-            if (kTma && mx_col && a.mx_staged) {
-                // This warp's 64 columns x 32 rows of codes go to its staging
-                // buffer (row 2*lane + h of the buffer = column cg0 + h) and out
-                // with one TMA store; the store clips what lies past the tensor.
-                if (rbase < a.rows && cwarp < a.cols) {
-                    uint8_t* stg = mx_stage_all + warp * kMxStageBytes;
-                    float sa, sb;
-                    const int ea = mx_exponent(mxa, sa), eb = mx_exponent(mxb, sb);
-                    const int64_t ia = cg0 * a.rows + rbase, ib = ia + a.rows;  // element indices
-#pragma unroll
-                    for (int g2 = 0; g2 < 2; ++g2) {  // 16 rows per pass
-                        uint2 ca[2], cb[2];
-#pragma unroll
-                        for (int gg = 0; gg < 2; ++gg) {
-                            const int g = 2 * g2 + gg;
-                            float va[8], vb[8];
-#pragma unroll
-                            for (int i = 0; i < 8; ++i) {
-                                const uint32_t w = pair_word(8 * g + i);
-                                va[i] = bf16_lo(w);
-                                vb[i] = bf16_hi(w);
-                            }
-                            U4 wa{}, wb{};
-                            if (mx_sr) {
-                                wa = sr_block8(a.pk, a.offset, 2u, (uint64_t)(ia >> 3) + g);
-                                wb = sr_block8(a.pk, a.offset, 2u, (uint64_t)(ib >> 3) + g);
-                            }
-                            ca[gg] = mx_convert8(va, sa, mx_sr, wa);
-                            cb[gg] = mx_convert8(vb, sb, mx_sr, wb);
-                        }
-                        st_shared_v4(stg + (2 * lane) * 32 + 16 * g2,
-                                     make_uint4(ca[0].x, ca[0].y, ca[1].x, ca[1].y));
-                        st_shared_v4(stg + (2 * lane + 1) * 32 + 16 * g2,
-                                     make_uint4(cb[0].x, cb[0].y, cb[1].x, cb[1].y));
-                    }
-                    if (cvalid) {
-                        a.mx_sf_col[mx_sf_off(a, cg0, rbase / 32, a.rows / 32)] = (uint8_t)(ea + 127);
-                        a.mx_sf_col[mx_sf_off(a, cg0 + 1, rbase / 32, a.rows / 32)] = (uint8_t)(eb + 127);
-                    }
+                if (qc_staged && (kFull || (rbase < a.rows && cwarp < a.cols))) {
+                    // this warp's 64 columns x 32 rows of NVFP4 codes (16 bytes per
+                    // column) out with one TMA store, clipped at the tensor edge
                     fence_proxy_async_smem();
                     __syncwarp();
                     if (lane == 0) {
-                        tma_store_2d(&map_mx, stg, (int32_t)rbase, (int32_t)cwarp);
+                        tma_store_2d(&map_qc, stg_qc, (int32_t)(rbase / 2), (int32_t)cwarp);
                         bulk_commit();
                     }
                 }
-            } else if (mx_col && cvalid && rbase < a.rows) {
-                float sa, sb;
-                const int ea = mx_exponent(mxa, sa), eb = mx_exponent(mxb, sb);
-                const int64_t ia = cg0 * a.rows + rbase, ib = ia + a.rows;  // element indices
-                uint8_t* qa = a.mx_q_col + ia;
-                uint8_t* qb = a.mx_q_col + ib;
-#pragma unroll 2
-                for (int g = 0; g < 4; ++g) {
-                    float va[8], vb[8];
-#pragma unroll
-                    for (int i = 0; i < 8; ++i) {
-                        const uint32_t w = pair_word(8 * g + i);
-                        va[i] = bf16_lo(w);
-                        vb[i] = bf16_hi(w);
+                if (kTma && mx_col && a.mx_staged) {
+                    // This warp's 64 columns x 32 rows of codes go to its staging
+                    // buffer (row 2*lane + h of the buffer = column cg0 + h) and out
+                    // with one TMA store; the store clips what lies past the tensor.
+                    if (kFull || (rbase < a.rows && cwarp < a.cols)) {
+                        uint8_t* stg = mx_stage_all + warp * kMxStageBytes;
+                        float sa, sb;
+                        const int ea = mx_exponent(mxa, sa), eb = mx_exponent(mxb, sb);
+                        const int64_t ia = cg0 * a.rows + rbase, ib = ia + a.rows;  // element indices
+    #pragma unroll
+                        for (int g2 = 0; g2 < 2; ++g2) {  // 16 rows per pass
+                            uint2 ca[2], cb[2];
+    #pragma unroll
+                            for (int gg = 0; gg < 2; ++gg) {
+                                const int g = 2 * g2 + gg;
+                                float va[8], vb[8];
+    #pragma unroll
+                                for (int i = 0; i < 8; ++i) {
+                                    const uint32_t w = pair_word(8 * g + i);
+                                    va[i] = bf16_lo(w);
+                                    vb[i] = bf16_hi(w);
+                                }
+                                U4 wa{}, wb{};
+                                if (mx_sr) {
+                                    wa = sr_block8(a.pk, a.offset, 2u, (uint64_t)(ia >> 3) + g);
+                                    wb = sr_block8(a.pk, a.offset, 2u, (uint64_t)(ib >> 3) + g);
+                                }
+                                ca[gg] = mx_convert8(va, sa, mx_sr, wa);
+                                cb[gg] = mx_convert8(vb, sb, mx_sr, wb);
+                            }
+                            st_shared_v4(stg + (2 * lane) * 32 + 16 * g2,
+                                         make_uint4(ca[0].x, ca[0].y, ca[1].x, ca[1].y));
+                            st_shared_v4(stg + (2 * lane + 1) * 32 + 16 * g2,
+                                         make_uint4(cb[0].x, cb[0].y, cb[1].x, cb[1].y));
+                        }
+                        if (cvalid) {
+                            a.mx_sf_col[mx_sf_off(a, cg0, rbase / 32, a.rows / 32)] = (uint8_t)(ea + 127);
+                            a.mx_sf_col[mx_sf_off(a, cg0 + 1, rbase / 32, a.rows / 32)] = (uint8_t)(eb + 127);
+                        }
+                        fence_proxy_async_smem();
+                        __syncwarp();
+                        if (lane == 0) {
+                            tma_store_2d(&map_mx, stg, (int32_t)rbase, (int32_t)cwarp);
+                            bulk_commit();
+                        }
                     }
-                    U4 wa{}, wb{};
-                    if (mx_sr) {
-                        wa = sr_block8(a.pk, a.offset, 2u, (uint64_t)(ia >> 3) + g);
-                        wb = sr_block8(a.pk, a.offset, 2u, (uint64_t)(ib >> 3) + g);
+                } else if (mx_col && cvalid && (kFull || rbase < a.rows)) {
+                    float sa, sb;
+                    const int ea = mx_exponent(mxa, sa), eb = mx_exponent(mxb, sb);
+                    const int64_t ia = cg0 * a.rows + rbase, ib = ia + a.rows;  // element indices
+                    uint8_t* qa = a.mx_q_col + ia;
+                    uint8_t* qb = a.mx_q_col + ib;
+    #pragma unroll 2
+                    for (int g = 0; g < 4; ++g) {
+                        float va[8], vb[8];
+    #pragma unroll
+                        for (int i = 0; i < 8; ++i) {
+                            const uint32_t w = pair_word(8 * g + i);
+                            va[i] = bf16_lo(w);
+                            vb[i] = bf16_hi(w);
+                        }
+                        U4 wa{}, wb{};
+                        if (mx_sr) {
+                            wa = sr_block8(a.pk, a.offset, 2u, (uint64_t)(ia >> 3) + g);
+                            wb = sr_block8(a.pk, a.offset, 2u, (uint64_t)(ib >> 3) + g);
+                        }
+                        *reinterpret_cast<uint2*>(qa + 8 * g) = mx_convert8(va, sa, mx_sr, wa);
+                        *reinterpret_cast<uint2*>(qb + 8 * g) = mx_convert8(vb, sb, mx_sr, wb);
                     }
-                    *reinterpret_cast<uint2*>(qa + 8 * g) = mx_convert8(va, sa, mx_sr, wa);
-                    *reinterpret_cast<uint2*>(qb + 8 * g) = mx_convert8(vb, sb, mx_sr, wb);
+                    a.mx_sf_col[mx_sf_off(a, cg0, rbase / 32, a.rows / 32)] = (uint8_t)(ea + 127);
+                    a.mx_sf_col[mx_sf_off(a, cg0 + 1, rbase / 32, a.rows / 32)] = (uint8_t)(eb + 127);
                 }
-                a.mx_sf_col[mx_sf_off(a, cg0, rbase / 32, a.rows / 32)] = (uint8_t)(ea + 127);
-                a.mx_sf_col[mx_sf_off(a, cg0 + 1, rbase / 32, a.rows / 32)] = (uint8_t)(eb + 127);
             }
-        }
+        };
+        if (full_tile)
+            tile_body(BoolC<true>{});
+        else
+            tile_body(BoolC<false>{});
         __syncwarp();
         if (lane == 0) mbar_arrive(&empty[stage]);  // this warp is done with the stage
     }
